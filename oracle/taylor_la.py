@@ -1,0 +1,212 @@
+"""Causal Taylor linear attention, float64, written from its definition.
+
+Test infrastructure only (see the package docstring).
+
+Notation follows "Simple linear attention language models balance the
+recall-throughput tradeoff" (BASED): q, k in R^{d'} (the projected feature
+dimension of §4 "Taylor Linear Attention"), v in R^{dv}, feature map phi,
+state S = sum_j phi(k_j) v_j^T, normaliser z = sum_j phi(k_j) (the "K-state" of
+App. D.4 "State size").
+
+Layouts: q, k are [B, H, N, d'], v is [B, H, N, dv]; S is [B, H, D, dv] and z
+is [B, H, D] with D = 1 + d' + d'^2. Feature order: index 0 is the constant 1,
+indices 1..d' are x_a, index 1 + d' + a*d' + b is x_a*x_b/sqrt(2) (row-major
+vec of the outer product).
+
+Readings of points the pages leave open:
+* the quadratic block is the full d'^2 outer product (widths 273 / 1057);
+* phi carries no extra scale: callers pre-scale q and k;
+* the output is normalised by the K-state, with no epsilon: every causal term
+  is 1 + s + s^2/2 = ((s+1)^2 + 1)/2 >= 1/2, so row i's denominator is at
+  least (i+1)/2 (asserted below);
+* causality is inclusive: token i attends to keys j <= i.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+_SQRT_HALF = np.sqrt(0.5)
+
+
+def feature_dim(d_feat: int) -> int:
+    """Width D = 1 + d' + d'^2 of the Taylor feature map."""
+    return 1 + d_feat + d_feat * d_feat
+
+
+def feature_map(x: np.ndarray) -> np.ndarray:
+    """phi(x) = [1, x, vec(x (x) x)/sqrt(2)] along the last axis, float64.
+
+    BASED §4 "Taylor Linear Attention": the 2nd-order Taylor approximation of
+    exp(q.k) written as a feature map; phi(q).phi(k) = 1 + q.k + (q.k)^2/2.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    outer = x[..., :, None] * x[..., None, :]             # [..., d', d'], (a, b)
+    second = outer.reshape(*x.shape[:-1], d * d) * _SQRT_HALF
+    ones = np.ones(x.shape[:-1] + (1,), dtype=np.float64)
+    return np.concatenate([ones, x, second], axis=-1)
+
+
+def _check_den(den: np.ndarray, n_keys: np.ndarray) -> None:
+    # Each causal weight is ((s+1)^2 + 1)/2 >= 1/2, so den >= (#keys)/2.
+    if not np.all(den >= 0.5 * n_keys * (1.0 - 1e-12)):
+        raise AssertionError("denominator below its lower bound (#keys)/2")
+
+
+def la_quadratic_parts(q, k, v, row_block: int = 1024):
+    """Numerator and denominator of the masked quadratic form.
+
+    num_i = sum_{j<=i} a_ij v_j, den_i = sum_{j<=i} a_ij, a_ij = 1 + s_ij + s_ij^2/2,
+    s_ij = q_i . k_j (BASED §2 "Efficient attentions": linear attention replaces
+    exp(q^T k) by phi(q)^T phi(k); §4 fixes phi to the 2nd-order Taylor map, whose
+    product is this polynomial). Computed in blocks of query rows; each block is
+    a dense matmul followed by the causal mask -- no reordering of the sum.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    *lead, n, _ = q.shape
+    dv = v.shape[-1]
+    num = np.empty(tuple(lead) + (n, dv), dtype=np.float64)
+    den = np.empty(tuple(lead) + (n,), dtype=np.float64)
+    for r0 in range(0, n, row_block):
+        r1 = min(n, r0 + row_block)
+        s = q[..., r0:r1, :] @ np.swapaxes(k[..., :r1, :], -1, -2)   # [..., rows, r1]
+        a = 1.0 + s + 0.5 * s * s
+        rows = np.arange(r0, r1)[:, None]
+        cols = np.arange(r1)[None, :]
+        a = np.where(cols <= rows, a, 0.0)
+        num[..., r0:r1, :] = a @ v[..., :r1, :]
+        den[..., r0:r1] = a.sum(axis=-1)
+    _check_den(den, np.arange(1, n + 1, dtype=np.float64))
+    return num, den
+
+
+def la_quadratic(q, k, v, row_block: int = 1024) -> np.ndarray:
+    """y_i = num_i / den_i of the causal Taylor linear attention (quadratic form)."""
+    num, den = la_quadratic_parts(q, k, v, row_block)
+    return num / den[..., None]
+
+
+def la_rows(q, k, v, rows) -> np.ndarray:
+    """y at selected query rows of one head: q [N, d'], k [N, d'], v [N, dv].
+
+    Same definition as la_quadratic, evaluated row by row (cost O(i) per row), for
+    checking sampled outputs of large problems.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    out = np.empty((len(rows), v.shape[-1]), dtype=np.float64)
+    for r, i in enumerate(rows):
+        s = k[: i + 1] @ q[i]
+        a = 1.0 + s + 0.5 * s * s
+        den = a.sum()
+        _check_den(np.array([den]), np.array([i + 1.0]))
+        out[r] = (a @ v[: i + 1]) / den
+    return out
+
+
+def la_state(k, v):
+    """S = sum_j phi(k_j) v_j^T and z = sum_j phi(k_j) over all tokens.
+
+    The recurrent state of linear attention ("Gated Slot Attention", App. A: an
+    additive matrix-valued state of key-value outer products) together with the
+    K-state for the denominator (BASED App. D.4). phi is built explicitly, so the
+    feature order and the 1/sqrt(2) are part of what this pins.
+    """
+    fk = feature_map(k)                                            # [..., N, D]
+    v = np.asarray(v, dtype=np.float64)
+    S = np.swapaxes(fk, -1, -2) @ v                                # [..., D, dv]
+    z = fk.sum(axis=-2)                                            # [..., D]
+    return S, z
+
+
+def la_recurrent(q, k, v, S0=None, z0=None):
+    """Token-by-token recurrent form (BASED §2: recurrent generation).
+
+    For t = 0..N-1: S += phi(k_t) v_t^T; z += phi(k_t);
+    y_t = phi(q_t)^T S / phi(q_t)^T z   (the output includes token t itself).
+    Starts from S0, z0 (zeros when omitted). Returns (y, S, z).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    *lead, n, d_feat = q.shape
+    dv = v.shape[-1]
+    D = feature_dim(d_feat)
+    S = np.zeros(tuple(lead) + (D, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    z = np.zeros(tuple(lead) + (D,)) if z0 is None else np.array(z0, dtype=np.float64)
+    y = np.empty(tuple(lead) + (n, dv), dtype=np.float64)
+    fq = feature_map(q)
+    fk = feature_map(k)
+    for t in range(n):
+        S += fk[..., t, :, None] * v[..., t, None, :]
+        z += fk[..., t, :]
+        num = np.einsum("...f,...fe->...e", fq[..., t, :], S)
+        den = np.einsum("...f,...f->...", fq[..., t, :], z)
+        y[..., t, :] = num / den[..., None]
+    return y, S, z
+
+
+def la_chunked(q, k, v, chunk: int):
+    """Chunkwise form: on-diagonal masked quadratic part + off-diagonal state part.
+
+    For chunk c holding tokens [cC, (c+1)C):
+      y_c = (A_c V_c + phi(Q_c) S_{c-1}) / (rowsum(A_c) + phi(Q_c) z_{c-1}),
+      A_c = (1 + Q_c K_c^T + (Q_c K_c^T)^2/2) with the causal mask inside the chunk,
+      S_c = S_{c-1} + phi(K_c)^T V_c,  z_c = z_{c-1} + colsum(phi(K_c)).
+    BASED App. B (Algorithm 1: quadratic on-diagonal tiles with local causal
+    masking plus linear off-diagonal cumulative state) and "Gated Slot
+    Attention" App. A.1 (inter-chunk and intra-chunk terms). Returns (y, S, z).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    *lead, n, d_feat = q.shape
+    dv = v.shape[-1]
+    D = feature_dim(d_feat)
+    S = np.zeros(tuple(lead) + (D, dv))
+    z = np.zeros(tuple(lead) + (D,))
+    y = np.empty(tuple(lead) + (n, dv))
+    for c0 in range(0, n, chunk):
+        c1 = min(n, c0 + chunk)
+        qc, kc, vc = q[..., c0:c1, :], k[..., c0:c1, :], v[..., c0:c1, :]
+        s = qc @ np.swapaxes(kc, -1, -2)
+        a = 1.0 + s + 0.5 * s * s
+        m = np.tril(np.ones((c1 - c0, c1 - c0), dtype=bool))
+        a = np.where(m, a, 0.0)
+        fq = feature_map(qc)
+        fk = feature_map(kc)
+        num = a @ vc + fq @ S
+        den = a.sum(axis=-1) + np.einsum("...tf,...f->...t", fq, z)
+        y[..., c0:c1, :] = num / den[..., None]
+        S = S + np.swapaxes(fk, -1, -2) @ vc
+        z = z + fk.sum(axis=-2)
+    return y, S, z
+
+
+def la_taylor_terms(q, k, v):
+    """Order-0, order-1 and order-2 Taylor terms of the causal numerator and denominator.
+
+    BASED App. B (Algorithm 1) writes the output as y = T0 + T1 + T2, one term
+    per Taylor order. With the K-state normalisation each order contributes to
+    both the numerator and the denominator:
+      T0_i = sum_{j<=i} v_j,              d0_i = i + 1,
+      T1_i = sum_{j<=i} (q_i.k_j) v_j,    d1_i = sum_{j<=i} q_i.k_j,
+      T2_i = sum_{j<=i} (q_i.k_j)^2/2 v_j, d2_i = sum_{j<=i} (q_i.k_j)^2/2,
+    and y_i = (T0 + T1 + T2)_i / (d0 + d1 + d2)_i. Returns ((T0, T1, T2), (d0, d1, d2)).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n = q.shape[-2]
+    mask = np.tril(np.ones((n, n), dtype=bool))
+    s = q @ np.swapaxes(k, -1, -2)
+    w0 = np.where(mask, 1.0, 0.0) * np.ones_like(s)
+    w1 = np.where(mask, s, 0.0)
+    w2 = np.where(mask, 0.5 * s * s, 0.0)
+    terms = tuple(w @ v for w in (w0, w1, w2))
+    dens = tuple(w.sum(axis=-1) for w in (w0, w1, w2))
+    return terms, dens

@@ -1,0 +1,316 @@
+"""Pins for the CPU oracle (CPU only, no GPU).
+
+The oracle is checked against things other than itself: hand-derived golden
+values, a mathematical identity of the feature map, a library softmax-attention
+routine (torch scaled_dot_product_attention in float64), textbook special cases,
+the O(eps^3) convergence of the Taylor weights to exp, equivalence of
+independently written formulations, and pure-Python brute force on N <= 8.
+The mutation tests at the end plant plausible mistakes in copies of the oracle
+and check that at least one pin rejects each of them.
+"""
+
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import brute
+
+RNG = np.random.default_rng(1234)
+
+
+def _qkv(B, H, N, d, dv, scale=None, seed=0):
+    rng = np.random.default_rng(seed)
+    s = d ** -0.25 if scale is None else scale
+    q = rng.standard_normal((B, H, N, d)) * s
+    k = rng.standard_normal((B, H, N, d)) * s
+    v = rng.standard_normal((B, H, N, dv))
+    return q, k, v
+
+
+def _golden(golden_dir, name):
+    with open(os.path.join(golden_dir, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- feature map
+
+@pytest.mark.parametrize("d", [1, 2, 3, 16, 32])
+def test_phi_product_is_taylor_polynomial(d):
+    # phi(q).phi(k) must equal 1 + s + s^2/2 with s = q.k for every q, k.
+    q = RNG.standard_normal((50, d))
+    k = RNG.standard_normal((50, d))
+    lhs = np.einsum("nf,nf->n", oracle.feature_map(q), oracle.feature_map(k))
+    s = np.einsum("nd,nd->n", q, k)
+    np.testing.assert_allclose(lhs, 1 + s + s * s / 2, rtol=1e-12, atol=1e-12)
+
+
+def test_phi_width():
+    assert oracle.feature_dim(16) == 273 and oracle.feature_dim(32) == 1057
+    assert oracle.feature_map(np.zeros((4, 16))).shape == (4, 273)
+
+
+def test_phi_golden_order(golden_dir):
+    g = _golden(golden_dir, "phi_d2.json")
+    np.testing.assert_allclose(oracle.feature_map(np.array(g["x"])), g["phi"], rtol=0, atol=1e-15)
+    np.testing.assert_allclose(brute.phi(g["x"]), g["phi"], rtol=0, atol=1e-15)
+
+
+def test_taylor_weight_minimum():
+    # 1 + s + s^2/2 = ((s+1)^2 + 1)/2 has its minimum 1/2 at s = -1.
+    s = np.linspace(-5, 5, 100001)
+    w = 1 + s + s * s / 2
+    assert abs(w.min() - 0.5) < 1e-9 and abs(s[w.argmin()] + 1) < 1e-4
+
+
+# ---------------------------------------------------------------- linear attention
+
+def test_la_hand_example(golden_dir):
+    g = _golden(golden_dir, "la_hand_d1.json")
+    q = np.array(g["q"])[None, None, :, None]
+    k = np.array(g["k"])[None, None, :, None]
+    v = np.array(g["v"])[None, None, :, None]
+    np.testing.assert_allclose(oracle.la_quadratic(q, k, v)[0, 0, :, 0], g["y"], rtol=1e-14)
+    y, S, z = oracle.la_recurrent(q, k, v)
+    np.testing.assert_allclose(y[0, 0, :, 0], g["y"], rtol=1e-14)
+    S2, z2 = oracle.la_state(k, v)
+    np.testing.assert_allclose(S2[0, 0, :, 0], g["S"], rtol=1e-14)
+    np.testing.assert_allclose(z2[0, 0], g["z"], rtol=1e-14)
+    np.testing.assert_allclose(S[0, 0, :, 0], g["S"], rtol=1e-14)
+
+
+@pytest.mark.parametrize("d,dv,N", [(1, 1, 5), (2, 3, 7), (3, 2, 8)])
+def test_la_brute_force(d, dv, N):
+    q, k, v = _qkv(1, 1, N, d, dv, scale=0.8, seed=d * 10 + N)
+    yb, Sb, zb = brute.la(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist())
+    np.testing.assert_allclose(oracle.la_quadratic(q, k, v)[0, 0], yb, rtol=1e-12, atol=1e-13)
+    S, z = oracle.la_state(k, v)
+    np.testing.assert_allclose(S[0, 0], Sb, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(z[0, 0], zb, rtol=1e-12, atol=1e-13)
+
+
+def test_la_quadratic_equals_recurrent():
+    q, k, v = _qkv(2, 3, 97, 16, 8, seed=1)
+    yq = oracle.la_quadratic(q, k, v, row_block=32)
+    yr, Sr, zr = oracle.la_recurrent(q, k, v)
+    np.testing.assert_allclose(yq, yr, rtol=1e-10, atol=1e-12)
+    S, z = oracle.la_state(k, v)
+    np.testing.assert_allclose(S, Sr, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(z, zr, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("chunk", [1, 5, 16, 64, 200])
+def test_la_chunked_equals_quadratic(chunk):
+    q, k, v = _qkv(1, 2, 131, 16, 16, seed=2)
+    y, S, z = oracle.la_chunked(q, k, v, chunk)
+    np.testing.assert_allclose(y, oracle.la_quadratic(q, k, v), rtol=1e-10, atol=1e-12)
+    S2, z2 = oracle.la_state(k, v)
+    np.testing.assert_allclose(S, S2, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(z, z2, rtol=1e-10, atol=1e-10)
+
+
+def test_la_taylor_terms_compose():
+    q, k, v = _qkv(1, 1, 40, 4, 3, seed=3)
+    (t0, t1, t2), (d0, d1, d2) = oracle.la_taylor_terms(q, k, v)
+    y = (t0 + t1 + t2) / (d0 + d1 + d2)[..., None]
+    np.testing.assert_allclose(y, oracle.la_quadratic(q, k, v), rtol=1e-12, atol=1e-13)
+    # order 0 alone is the cumulative sum of v, order-0 denominator the count
+    np.testing.assert_allclose(t0, np.cumsum(v, axis=-2), rtol=1e-12)
+    np.testing.assert_allclose(d0[0, 0], np.arange(1, 41))
+
+
+def test_la_decode_continues_prefill():
+    q, k, v = _qkv(1, 2, 60, 16, 8, seed=4)
+    n0 = 45
+    S0, z0 = oracle.la_state(k[..., :n0, :], v[..., :n0, :])
+    y, S, z = oracle.la_recurrent(q[..., n0:, :], k[..., n0:, :], v[..., n0:, :], S0, z0)
+    np.testing.assert_allclose(y, oracle.la_quadratic(q, k, v)[..., n0:, :], rtol=1e-10, atol=1e-12)
+    S2, z2 = oracle.la_state(k, v)
+    np.testing.assert_allclose(S, S2, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(z, z2, rtol=1e-10)
+
+
+def test_la_rows_matches_quadratic():
+    q, k, v = _qkv(1, 1, 300, 16, 8, seed=5)
+    rows = [0, 1, 63, 64, 127, 128, 299]
+    np.testing.assert_allclose(oracle.la_rows(q[0, 0], k[0, 0], v[0, 0], rows),
+                               oracle.la_quadratic(q, k, v)[0, 0, rows], rtol=1e-12, atol=1e-13)
+
+
+def test_la_zero_query_is_cumulative_mean():
+    # q = 0 makes every weight 1: y_i = mean(v_0..v_i).
+    _, k, v = _qkv(1, 2, 50, 16, 5, seed=6)
+    q = np.zeros_like(k)
+    mean = np.cumsum(v, axis=-2) / np.arange(1, 51)[:, None]
+    np.testing.assert_allclose(oracle.la_quadratic(q, k, v), mean, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(oracle.la_recurrent(q, k, v)[0], mean, rtol=1e-12, atol=1e-13)
+
+
+def test_la_single_token_is_identity():
+    q, k, v = _qkv(3, 2, 1, 16, 7, seed=7)
+    np.testing.assert_allclose(oracle.la_quadratic(q, k, v), v, rtol=1e-14)
+
+
+def test_la_denominator_bound_attained():
+    # s = q.k = -1 for every pair gives weight 1/2: den_i = (i+1)/2 exactly.
+    n = 20
+    q = np.zeros((1, 1, n, 3)); q[..., 0] = 1.0
+    k = np.zeros((1, 1, n, 3)); k[..., 0] = -1.0
+    v = RNG.standard_normal((1, 1, n, 2))
+    _, den = oracle.la_quadratic_parts(q, k, v)
+    np.testing.assert_allclose(den[0, 0], 0.5 * np.arange(1, n + 1), rtol=1e-15)
+
+
+def test_la_denominator_bound_random():
+    q, k, v = _qkv(2, 2, 200, 16, 4, scale=1.5, seed=8)
+    _, den = oracle.la_quadratic_parts(q, k, v)
+    assert np.all(den >= 0.5 * np.arange(1, 201))
+
+
+def _softmax_causal_torch(q, k, v):
+    # library routine: causal softmax attention with unit scale
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    return torch.nn.functional.scaled_dot_product_attention(
+        t(q), t(k), t(v), is_causal=True, scale=1.0).numpy()
+
+
+def _taylor_error_ratio(la_fn):
+    q, k, v = _qkv(1, 2, 64, 16, 8, seed=9)
+    errs = []
+    for eps in (0.2, 0.1, 0.05):
+        y = la_fn(eps * q, k, v)
+        errs.append(np.abs(y - _softmax_causal_torch(eps * q, k, v)).max())
+    return errs[0] / errs[1], errs[1] / errs[2]
+
+
+def test_la_converges_to_softmax_at_third_order():
+    # 1 + s + s^2/2 = exp(s) - s^3/6 + ...: the gap to softmax attention is O(eps^3).
+    r1, r2 = _taylor_error_ratio(oracle.la_quadratic)
+    assert 6.5 < r1 < 9.5 and 7.0 < r2 < 9.0, (r1, r2)
+
+
+# ---------------------------------------------------------------- sliding window
+
+def test_swa_hand_example(golden_dir):
+    g = _golden(golden_dir, "swa_hand_w2.json")
+    a = lambda key: np.array(g[key])[None, None, :, None]
+    y = oracle.swa(a("q"), a("k"), a("v"), g["w"], g["scale"])
+    np.testing.assert_allclose(y[0, 0, :, 0], g["y"], rtol=1e-14)
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 8])
+def test_swa_brute_force(w):
+    q, k, v = _qkv(1, 1, 8, 4, 3, scale=1.0, seed=10 + w)
+    yb = brute.swa(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), w, 0.7)
+    np.testing.assert_allclose(oracle.swa(q, k, v, w, 0.7)[0, 0], yb, rtol=1e-12, atol=1e-13)
+
+
+def test_swa_full_window_is_causal_softmax_library():
+    q, k, v = _qkv(2, 2, 50, 64, 64, scale=0.6, seed=11)
+    scale = 1 / 8
+    ref = _softmax_causal_torch(q * scale, k, v)
+    np.testing.assert_allclose(oracle.swa(q, k, v, 64, scale, row_block=16), ref, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(oracle.swa(q, k, v, 50, scale), ref, rtol=1e-12, atol=1e-13)
+
+
+def test_swa_window_one_is_identity():
+    q, k, v = _qkv(1, 3, 30, 8, 8, seed=12)
+    np.testing.assert_allclose(oracle.swa(q, k, v, 1, 0.3), v, rtol=1e-14)
+
+
+def test_swa_rows_before_window_are_causal_prefix():
+    q, k, v = _qkv(1, 1, 200, 64, 64, scale=0.6, seed=13)
+    y = oracle.swa(q, k, v, 64, 0.125, row_block=37)
+    ref = _softmax_causal_torch(q[..., :64, :] * 0.125, k[..., :64, :], v[..., :64, :])
+    np.testing.assert_allclose(y[..., :64, :], ref, rtol=1e-12, atol=1e-13)
+    # row 150 sees exactly keys 87..150: one query, 64 keys, no mask
+    i = 150
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(a))
+    ref_i = torch.nn.functional.scaled_dot_product_attention(
+        t(q[..., i:i + 1, :]), t(k[..., i - 63:i + 1, :]), t(v[..., i - 63:i + 1, :]),
+        scale=0.125).numpy()
+    np.testing.assert_allclose(y[..., i:i + 1, :], ref_i, rtol=1e-12, atol=1e-13)
+    rows = [0, 5, 63, 64, 65, 150, 199]
+    np.testing.assert_allclose(oracle.swa_rows(q[0, 0], k[0, 0], v[0, 0], 64, 0.125, rows),
+                               y[0, 0, rows], rtol=1e-12, atol=1e-13)
+
+
+@pytest.mark.parametrize("n0", [0, 1, 30, 64, 100])
+def test_swa_ring_decode_continues_prefill(n0):
+    w, scale = 16, 0.25
+    q, k, v = _qkv(2, 2, n0 + 40, 8, 8, scale=0.7, seed=14 + n0)
+    full = oracle.swa(q, k, v, w, scale)
+    kc, vc = oracle.swa_ring_after_prefill(k[..., :n0, :], v[..., :n0, :], w)
+    for t in range(n0, n0 + 40):
+        y, kc, vc = oracle.swa_decode_step(kc, vc, t, q[..., t, :], k[..., t, :], v[..., t, :], w, scale)
+        np.testing.assert_allclose(y, full[..., t, :], rtol=1e-12, atol=1e-13)
+
+
+def test_swa_ring_contents():
+    k = np.arange(10, dtype=np.float64).reshape(1, 1, 10, 1)
+    kc, _ = oracle.swa_ring_after_prefill(k, k, 4)
+    # tokens 6..9 at slots 6%4=2, 7%4=3, 8%4=0, 9%4=1
+    np.testing.assert_array_equal(kc[0, 0, :, 0], [8, 9, 6, 7])
+    kc, _ = oracle.swa_ring_after_prefill(k[..., :2, :], k[..., :2, :], 4)
+    np.testing.assert_array_equal(kc[0, 0, :, 0], [0, 1, 0, 0])
+
+
+# ---------------------------------------------------------------- planted mistakes
+
+def _mut_phi_no_sqrt(x):
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    outer = (x[..., :, None] * x[..., None, :]).reshape(*x.shape[:-1], d * d)
+    return np.concatenate([np.ones(x.shape[:-1] + (1,)), x, outer], axis=-1)
+
+
+def _mut_la(coef1=1.0, coef2=0.5, strict=False):
+    def la(q, k, v):
+        s = q @ np.swapaxes(k, -1, -2)
+        a = 1.0 + coef1 * s + coef2 * s * s
+        n = s.shape[-1]
+        m = np.tril(np.ones((n, n), dtype=bool), k=-1 if strict else 0)
+        a = np.where(m, a, 0.0)
+        den = a.sum(-1)
+        den = np.where(den == 0, 1.0, den)
+        return (a @ v) / den[..., None]
+    return la
+
+
+def test_mutant_phi_without_sqrt_half_is_caught(golden_dir):
+    q = RNG.standard_normal((10, 16))
+    k = RNG.standard_normal((10, 16))
+    lhs = np.einsum("nf,nf->n", _mut_phi_no_sqrt(q), _mut_phi_no_sqrt(k))
+    s = np.einsum("nd,nd->n", q, k)
+    assert not np.allclose(lhs, 1 + s + s * s / 2)
+    g = _golden(golden_dir, "phi_d2.json")
+    assert not np.allclose(_mut_phi_no_sqrt(np.array(g["x"])), g["phi"])
+
+
+@pytest.mark.parametrize("mutant", [
+    _mut_la(coef2=1.0),          # wrong second-order coefficient
+    _mut_la(coef1=-1.0),         # wrong sign of the first-order term
+])
+def test_mutant_coefficients_caught_by_convergence(mutant):
+    r1, r2 = _taylor_error_ratio(mutant)
+    assert not (6.5 < r1 < 9.5 and 7.0 < r2 < 9.0)
+
+
+def test_mutant_exclusive_mask_caught(golden_dir):
+    g = _golden(golden_dir, "la_hand_d1.json")
+    a = lambda key: np.array(g[key])[None, None, :, None]
+    y = _mut_la(strict=True)(a("q"), a("k"), a("v"))
+    assert not np.allclose(y[0, 0, :, 0], g["y"])
+    np.testing.assert_allclose(_mut_la()(a("q"), a("k"), a("v"))[0, 0, :, 0], g["y"], rtol=1e-14)
+
+
+def test_mutant_window_off_by_one_caught(golden_dir):
+    g = _golden(golden_dir, "swa_hand_w2.json")
+    a = lambda key: np.array(g[key])[None, None, :, None]
+    # a window of w+1 keys (reading "preceding w keys" as excluding self)
+    y = oracle.swa(a("q"), a("k"), a("v"), g["w"] + 1, g["scale"])
+    assert not np.allclose(y[0, 0, :, 0], g["y"])
