@@ -1,0 +1,519 @@
+"""Throughput of the BASED hot path on B200: Taylor linear attention + sliding-window attention.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mine|reference]
+
+One step = one pass of the whole hot path over one batch of the 360M-shaped
+workload (B=8 sequences, N=2048 tokens, 16 linear-attention heads with d'=16,
+dv=64, 16 sliding-window heads of dim 64 with w=64, bf16 inputs):
+  1. Taylor linear-attention prefill (y, final S and z),
+  2. sliding-window prefill (y and the 64-slot ring KV cache),
+  3. one generated token per sequence: linear-attention decode step and
+     sliding-window decode step, continuing from the prefilled states.
+Tokens per step = B*N (prefill) + B (decode). `value` is whole-job tokens/s
+(all ranks) with inputs resident in HBM; `e2e` is the same through the public
+API with pinned host inputs copied in and outputs copied back inside the
+timed region. Multi-GPU: one process per GPU (torchrun), each rank runs its
+own batch (weak scaling, no data-path collective); time is the max over ranks.
+
+--impl reference times the CPU oracle (float64 NumPy) on a bounded sample of
+the same workload: the comparison arm on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "prefill & decode tokens/s (Taylor LA + SWA) and % of roofline on 1 B200"
+UNIT = "tokens/s"
+WORKLOAD = dict(B=8, H=16, N=2048, d_feat=16, d_v=64, swa_heads=16, swa_dim=64, w=64)
+N_INPUT_SETS = 3          # rotated so every step reads inputs last touched two steps earlier
+
+
+def _feature_dim(d):
+    return 1 + d + d * d
+
+
+# ---------------------------------------------------------------- algorithmic work per launch
+# Per head-token figures of the Taylor LA and SWA paths (bytes at bf16 inputs, fp32 state).
+
+def la_prefill_work(B, H, N, d_feat, d_v, chunk):
+    D = _feature_dim(d_feat)
+    flops = B * H * N * (2 * chunk * d_feat + 2 * chunk * d_v + 2 * chunk + 4 * D * d_v + 4 * D)
+    byts = B * H * N * (2 * d_feat + 2 * d_v) * 2 + B * H * (D * d_v + D) * 4
+    return flops, byts
+
+
+def swa_prefill_work(B, H, N, d, w):
+    flops = B * H * N * 4 * w * d
+    byts = B * H * N * 4 * d * 2 + B * H * 2 * w * d * 2      # q, k, v, y + ring cache
+    return flops, byts
+
+
+def la_decode_work(B, H, d_feat, d_v):
+    D = _feature_dim(d_feat)
+    flops = B * H * (4 * D * d_v + 4 * D + d_feat * d_feat)
+    byts = B * H * (2 * (D * d_v + D) * 4 + (2 * d_feat + 2 * d_v) * 2)
+    return flops, byts
+
+
+def swa_decode_work(B, H, d, w):
+    flops = B * H * 4 * w * d
+    byts = B * H * (2 * w * d * 2 + 2 * d * 2 + 4 * d * 2)   # ring read, slot write, q k v y
+    return flops, byts
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return dict(hbm_gbs=float(d["hbm_gbs"]), bf16_tflops=float(d["bf16_tflops"]),
+                    bf16_tflops_sustained=float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                    source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0, source="fallback")
+
+
+KERNEL_SOURCES = {
+    "la_prefill": ["la_prefill_tc.cu", "tcgen05.cuh", "common.cuh"],
+    "swa_prefill": ["swa.cu", "common.cuh"],
+    "la_decode": ["la_decode.cu", "common.cuh"],
+    "swa_decode": ["swa.cu", "common.cuh"],
+}
+
+
+def kernel_source_hash(kind):
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES[kind]:
+        with open(os.path.join(ROOT, "linear_attention_sequence_causal_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
+
+
+def measured_traffic(kind):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current source."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(p):
+        return None
+    pat = re.compile(r"^\|\s*%s\s*\|\s*([0-9a-f]{12})\s*\|\s*([0-9.eE+]+)\s*\|" % re.escape(kind))
+    with open(p) as f:
+        for line in f:
+            m = pat.match(line.strip())
+            if m and m.group(1) == kernel_source_hash(kind):
+                return float(m.group(2))
+    return None
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_id}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, val in zip(self.NAMES, parts[5:9]):
+                    if val.lower() == "active":
+                        reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+
+def dist_setup(n_gpus):
+    import torch
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"--gpus {n_gpus} but WORLD_SIZE={world}")
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, dev):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- the GPU arm
+
+def run_mine(args):
+    import torch
+
+    import linear_attention_sequence_causal_b200 as based
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    W = WORKLOAD
+    B, H, N, df, dv, Hs, ds, w = (W[k] for k in ("B", "H", "N", "d_feat", "d_v", "swa_heads", "swa_dim", "w"))
+    D = _feature_dim(df)
+    scale = 1.0 / math.sqrt(ds)
+    chunk = 128
+
+    # Inputs: N_INPUT_SETS seeded sets per rank, resident in HBM; one more token per
+    # sequence for the decode step.
+    sets = []
+    for s in range(N_INPUT_SETS):
+        seed = 1000 * rank + s
+        la = synthetic.la_inputs(B, H, N + 1, df, dv, "bf16", seed=seed)
+        sw = synthetic.swa_inputs(B, Hs, N + 1, ds, "bf16", seed=seed + 500)
+        d = {}
+        for name, t in (("q", la.q), ("k", la.k), ("v", la.v)):
+            d[name] = t[:, :, :N].contiguous().to(dev)
+            d[name + "1"] = t[:, :, N].contiguous().to(dev)
+        for name, t in (("sq", sw.q), ("sk", sw.k), ("sv", sw.v)):
+            d[name] = t[:, :, :N].contiguous().to(dev)
+            d[name + "1"] = t[:, :, N].contiguous().to(dev)
+        sets.append(d)
+    y = torch.empty((B, H, N, dv), dtype=torch.bfloat16, device=dev)
+    S = torch.empty((B, H, D, dv), dtype=torch.float32, device=dev)
+    z = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    ys = torch.empty((B, Hs, N, ds), dtype=torch.bfloat16, device=dev)
+    kc = torch.empty((B, Hs, w, ds), dtype=torch.bfloat16, device=dev)
+    vc = torch.empty_like(kc)
+    y1 = torch.empty((B, H, dv), dtype=torch.bfloat16, device=dev)
+    ys1 = torch.empty((B, Hs, ds), dtype=torch.bfloat16, device=dev)
+    ws_bytes = based.la_prefill_workspace(B, H, N, df, dv, torch.bfloat16, chunk)
+    ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(d, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        based.la_prefill(d["q"], d["k"], d["v"], chunk=chunk, y=y, S=S, z=z, workspace=ws)
+        if ev is not None:
+            ev[1].record(stream)
+        based.swa_prefill(d["sq"], d["sk"], d["sv"], w=w, scale=scale, y=ys, k_cache=kc, v_cache=vc)
+        if ev is not None:
+            ev[2].record(stream)
+        based.la_decode_step(S, z, d["q1"], d["k1"], d["v1"], y=y1)
+        if ev is not None:
+            ev[3].record(stream)
+        based.swa_decode(kc, vc, N, d["sq1"], d["sk1"], d["sv1"], w=w, scale=scale, y=ys1)
+        if ev is not None:
+            ev[4].record(stream)
+
+    launches_per_step = 1 + (1 if ws_bytes else 0) + 2 + 1 + 1
+
+    for i in range(args.warmup):
+        step(sets[i % N_INPUT_SETS])
+    torch.cuda.synchronize(dev)
+    if based.get_last_error(dev) != 0:
+        raise SystemExit("device status error after warm-up")
+
+    gpu_index = local
+    try:
+        p = torch.cuda.get_device_properties(dev)
+        gpu_index = f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+    except Exception:
+        pass
+    clocks = ClockSampler(gpu_index)
+    clocks.start()
+    # keep the GPU busy a moment so the sampler sees load before the timed region
+    for i in range(args.warmup):
+        step(sets[i % N_INPUT_SETS])
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(sets[i % N_INPUT_SETS], evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    per_kernel = {name: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
+                  for j, name in enumerate(("la_prefill", "swa_prefill", "la_decode", "swa_decode"))}
+    if based.get_last_error(dev) != 0:
+        raise SystemExit("device status error in the timed region")
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
+
+    tokens_per_step = B * N + B
+    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    ms_per_step = elapsed_ms / args.steps
+
+    # ---- roofline of the dominant kernel (algorithmic work / measured launch time)
+    peaks = load_peaks()
+    work = {
+        "la_prefill": la_prefill_work(B, H, N, df, dv, chunk),
+        "swa_prefill": swa_prefill_work(B, Hs, N, ds, w),
+        "la_decode": la_decode_work(B, H, df, dv),
+        "swa_decode": swa_decode_work(B, Hs, ds, w),
+    }
+    dom = max(per_kernel, key=per_kernel.get)
+    flops, byts = work[dom]
+    t_s = per_kernel[dom] / 1e3
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    t_byte = byts / (peaks["hbm_gbs"] * 1e9)
+    if t_flop > t_byte:
+        roof = {"bound": "tensor", "achieved": flops / t_s / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": byts / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(dom)
+    roof["kernel"] = dom
+    roof["peak_source"] = peaks["source"] + (" burst" if roof["bound"] == "tensor" else " copy")
+    roof["algorithmic_per_launch"] = {"flops": flops, "bytes": byts}
+
+    kernels = {}
+    for name, ms in per_kernel.items():
+        f_, b_ = work[name]
+        kernels[name] = {"us": round(ms * 1e3, 2), "GB_s": round(b_ / (ms / 1e3) / 1e9, 1),
+                         "TFLOP_s": round(f_ / (ms / 1e3) / 1e12, 1),
+                         "roofline_frac": round(max(f_ / (peaks["bf16_tflops"] * 1e12),
+                                                    b_ / (peaks["hbm_gbs"] * 1e9)) / (ms / 1e3), 3)}
+    prefill_ms = per_kernel["la_prefill"] + per_kernel["swa_prefill"]
+    decode_ms = per_kernel["la_decode"] + per_kernel["swa_decode"]
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = run_e2e(based, dev, stream, B, H, N, df, dv, Hs, ds, w, scale, chunk, y, S, z, ys, kc, vc, y1, ys1,
+                  ws, min(args.steps, 20), world)
+
+    result = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "360M-shaped: B=8, N=2048; Taylor LA 16 heads d'=16 dv=64; "
+                               "SWA 16 heads d=64 w=64; + 1 decode token per sequence",
+                   "B": B, "N": N, "la_heads": H, "d_feat": df, "d_v": dv, "swa_heads": Hs,
+                   "swa_head_dim": ds, "w": w, "chunk": chunk, "tokens_per_step": tokens_per_step,
+                   "l2": f"inputs rotated over {N_INPUT_SETS} sets (>{N_INPUT_SETS * 0.23:.1f} GB); "
+                         "each step's inputs were last read two steps earlier",
+                   "parallelism": f"dp{world}"},
+        "prefill": {"tokens_per_s": world * B * N / (prefill_ms / 1e3), "ms": prefill_ms},
+        "decode": {"tokens_per_s": world * B / (decode_ms / 1e3), "ms": decode_ms, "batch": B},
+        "kernels": kernels,
+        "roofline": roof,
+        "gpu_launches": launches_per_step * args.steps,
+        "e2e": e2e,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(based, dev, stream, B, H, N, df, dv, Hs, ds, w, scale, chunk, y, S, z, ys, kc, vc, y1, ys1, ws,
+            steps, world):
+    import torch
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    la = synthetic.la_inputs(B, H, N + 1, df, dv, "bf16", seed=77)
+    sw = synthetic.swa_inputs(B, Hs, N + 1, ds, "bf16", seed=78)
+    host = {}
+    for name, t in (("q", la.q), ("k", la.k), ("v", la.v), ("sq", sw.q), ("sk", sw.k), ("sv", sw.v)):
+        host[name] = t[:, :, :N].contiguous().pin_memory()
+        host[name + "1"] = t[:, :, N].contiguous().pin_memory()
+    devb = {n: torch.empty_like(t, device=dev) for n, t in host.items()}
+    out_y = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    out_ys = torch.empty(ys.shape, dtype=ys.dtype).pin_memory()
+    out_y1 = torch.empty(y1.shape, dtype=y1.dtype).pin_memory()
+    out_ys1 = torch.empty(ys1.shape, dtype=ys1.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in (out_y, out_ys, out_y1, out_ys1))
+
+    def step():
+        for n in host:
+            devb[n].copy_(host[n], non_blocking=True)
+        based.la_prefill(devb["q"], devb["k"], devb["v"], chunk=chunk, y=y, S=S, z=z, workspace=ws)
+        based.swa_prefill(devb["sq"], devb["sk"], devb["sv"], w=w, scale=scale, y=ys, k_cache=kc, v_cache=vc)
+        based.la_decode_step(S, z, devb["q1"], devb["k1"], devb["v1"], y=y1)
+        based.swa_decode(kc, vc, N, devb["sq1"], devb["sk1"], devb["sv1"], w=w, scale=scale, y=ys1)
+        out_y.copy_(y, non_blocking=True)
+        out_ys.copy_(ys, non_blocking=True)
+        out_y1.copy_(y1, non_blocking=True)
+        out_ys1.copy_(ys1, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(a.elapsed_time(b), world, dev)
+    return {"value": world * (B * N + B) * steps / (ms / 1e3), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+# ---------------------------------------------------------------- the CPU oracle arm
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n and n[0]:
+            return int(n[0])
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(n_heads, seed=0):
+    """Time the oracle on n_heads heads of one sequence (LA prefill + SWA prefill + decode
+    token for those heads). Returns (seconds, tokens) with tokens = n_heads * (N + 1) / H."""
+    import numpy as np
+
+    import oracle
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    W = WORKLOAD
+    N, df, dv, ds, w = W["N"], W["d_feat"], W["d_v"], W["swa_dim"], W["w"]
+    la = synthetic.la_inputs(1, n_heads, N + 1, df, dv, "bf16", seed=seed)
+    sw = synthetic.swa_inputs(1, n_heads, N + 1, ds, "bf16", seed=seed + 1)
+    scale = 1.0 / math.sqrt(ds)
+    t0 = time.perf_counter()
+    oracle.la_quadratic(la.q64[..., :N, :], la.k64[..., :N, :], la.v64[..., :N, :])
+    S, z = oracle.la_state(la.k64[..., :N, :], la.v64[..., :N, :])
+    oracle.la_recurrent(la.q64[..., N:, :], la.k64[..., N:, :], la.v64[..., N:, :], S, z)
+    oracle.swa(sw.q64[..., :N, :], sw.k64[..., :N, :], sw.v64[..., :N, :], w, scale)
+    kc, vc = oracle.swa_ring_after_prefill(sw.k64[..., :N, :], sw.v64[..., :N, :], w)
+    oracle.swa_decode_step(kc, vc, N, sw.q64[..., N, :], sw.k64[..., N, :], sw.v64[..., N, :], w, scale)
+    dt = time.perf_counter() - t0
+    return dt, n_heads * (N + 1) / W["H"]
+
+
+def cpu_baseline(seconds):
+    # calibrate on one head, then size the sample to about `seconds` of CPU work
+    dt1, _ = oracle_sample(1, seed=1)
+    heads = max(1, min(WORKLOAD["H"] * WORKLOAD["B"], int(seconds / max(dt1, 1e-3))))
+    dt, tokens = oracle_sample(heads, seed=2)
+    return {"value": tokens / dt, "unit": UNIT, "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{heads} of {WORKLOAD['B'] * WORKLOAD['H']} (sequence, head) pairs of the "
+                      f"workload (LA + SWA prefill of N={WORKLOAD['N']} plus one decode token each), "
+                      f"{dt:.1f} s; tokens = heads x (N+1) / {WORKLOAD['H']}"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = 150.0 / max(1, args.steps + args.warmup)          # seconds per step, whole run < ~3 min
+    dt1, _ = oracle_sample(1, seed=1)
+    heads = max(1, min(WORKLOAD["H"] * WORKLOAD["B"], int(budget / max(dt1, 1e-3))))
+    for i in range(args.warmup):
+        oracle_sample(heads, seed=10 + i)
+    tot_t, tot_tok = 0.0, 0.0
+    for i in range(args.steps):
+        dt, tok = oracle_sample(heads, seed=100 + i)
+        tot_t += dt
+        tot_tok += tok
+    value = tot_tok / tot_t
+    sample = (f"per step {heads} (sequence, head) pairs of the workload through the float64 oracle "
+              f"(LA + SWA prefill of N={WORKLOAD['N']} plus one decode token)")
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot_t / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": "360M-shaped: B=8, N=2048; Taylor LA 16 heads d'=16 dv=64; "
+                               "SWA 16 heads d=64 w=64; + 1 decode token per sequence",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "kind": "oracle", "cores": _blas_threads(),
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=("mine", "reference"), default="mine")
+    p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample size")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    args = p.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_mine(args)
+
+
+if __name__ == "__main__":
+    main()

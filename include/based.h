@@ -1,0 +1,185 @@
+/*
+ * based.h -- C ABI of the B200 (sm_100a) BASED hot path: causal Taylor linear
+ * attention and sliding-window softmax attention, prefill and decode.
+ *
+ * The method is that of "Simple linear attention language models balance the
+ * recall-throughput tradeoff" (BASED, arXiv 2402.18668v2):
+ *   - linear attention through a feature map, computed in a parallel form for
+ *     prompt processing and a recurrent form for generation (§2 "Efficient
+ *     attentions", §5 "Execution stages");
+ *   - the 2nd-order Taylor feature map with projected dimension d' (§4 "Taylor
+ *     Linear Attention"), used here in its explicit form
+ *         phi(x) = [1, x, vec(x (x) x)/sqrt(2)],  D = 1 + d' + d'^2 features,
+ *     so that phi(q).phi(k) = 1 + q.k + (q.k)^2/2;
+ *   - outputs normalised by the "K-state" z (App. D.4 "State size");
+ *   - exact softmax attention inside a small sliding window with a w-sized KV
+ *     cache (§4 "Local Exact Attention").
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensors are dense, contiguous, row-major, batch-major then head-major,
+ *   and live in device memory of the current CUDA device. Every pointer must
+ *   be 16-byte aligned. The library never allocates memory and keeps no
+ *   pointer after a call returns; the caller owns every buffer.
+ * - dtype selects the element type of q, k, v, y and the SWA caches:
+ *   BASED_F32 (float) or BASED_BF16 (__nv_bfloat16). S and z are always float.
+ *   Arithmetic is fp32 (fp32 accumulation of bf16 tensor-core products on the
+ *   bf16 prefill path).
+ * - Work is enqueued on `stream` (0 = legacy default stream); every call is
+ *   asynchronous. Argument errors are reported synchronously by the return
+ *   value and enqueue nothing. Errors detected on the device (a bounded
+ *   internal wait that expired) are recorded in a per-device status word read
+ *   by based_get_last_error().
+ * - Causality is inclusive: token i attends to keys j <= i.
+ * - Feature order of phi and of the rows of S and z: index 0 is the constant
+ *   1; 1..d' hold x_a; 1 + d' + a*d' + b holds x_a*x_b/sqrt(2).
+ */
+#ifndef BASED_H
+#define BASED_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define BASED_API __attribute__((visibility("default")))
+#else
+#define BASED_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BASED_OK = 0,
+    BASED_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, workspace too small */
+    BASED_ERR_UNSUPPORTED = 2,   /* valid but not built: d', dv, d, w, chunk or dtype outside the set */
+    BASED_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, device query, sync) */
+    BASED_ERR_TIMEOUT = 4        /* a bounded wait inside a kernel expired; outputs are undefined */
+} based_status_t;
+
+typedef enum {
+    BASED_F32 = 0,
+    BASED_BF16 = 1
+} based_dtype_t;
+
+/*
+ * based_la_prefill -- parallel (prompt-processing) form of causal Taylor linear
+ * attention over N tokens, starting from an empty state.
+ *
+ * Computes, for every batch b, head h and token i,
+ *     y_i = sum_{j<=i} a_ij v_j / sum_{j<=i} a_ij,   a_ij = 1 + q_i.k_j + (q_i.k_j)^2/2
+ *         = phi(q_i)^T S_i / phi(q_i)^T z_i,         S_i = sum_{j<=i} phi(k_j) v_j^T,
+ * and writes the final state S = S_{N-1} and z = z_{N-1}.
+ * BASED §4 "Taylor Linear Attention"; App. B "Forward / Generation Prefill"
+ * (Algorithm 1: y = T0 + T1 + T2, on-diagonal quadratic tiles with a local causal
+ * mask plus an off-diagonal cumulative state); App. D.4 (K-state z).
+ *
+ *   q, k    [B, H, N, d_feat]  dtype, read only
+ *   v       [B, H, N, d_v]     dtype, read only
+ *   y       [B, H, N, d_v]     dtype, written (round-to-nearest for bf16)
+ *   S       [B, H, D, d_v]     float, written; D = 1 + d_feat + d_feat^2
+ *   z       [B, H, D]          float, written
+ *           S and z may both be NULL (final state not wanted), not just one.
+ *   d_feat  16 or 32;  d_v  64 or 128;  N >= 1;  B, H >= 1
+ *   chunk   tokens per on-diagonal tile: 0 (library's choice) or one of the
+ *           values the dtype supports: BASED_F32 {16, 32, 64},
+ *           BASED_BF16 {64, 128, 256}. The result does not depend on it beyond
+ *           rounding.
+ *   workspace, workspace_bytes
+ *           device scratch of at least based_la_prefill_workspace(...) bytes
+ *           (NULL allowed when that size is 0). Used to split long sequences
+ *           into segments whose start states are summed from the preceding
+ *           segments' totals; its contents on entry do not matter.
+ * Returns BASED_ERR_INVALID_ARG for null or misaligned pointers, non-positive
+ * sizes, or a workspace smaller than required; BASED_ERR_UNSUPPORTED for a
+ * (d_feat, d_v, dtype, chunk) combination outside the built set.
+ */
+BASED_API based_status_t based_la_prefill(const void* q, const void* k, const void* v, void* y,
+                                float* S, float* z,
+                                int B, int H, int N, int d_feat, int d_v,
+                                based_dtype_t dtype, int chunk,
+                                void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/*
+ * based_la_prefill_workspace -- bytes of device scratch based_la_prefill needs
+ * for these arguments on the current device (0 when no segment split is used).
+ * Returns 0 for arguments based_la_prefill would reject.
+ */
+BASED_API size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int d_v,
+                                  based_dtype_t dtype, int chunk);
+
+/*
+ * based_la_decode_step -- recurrent (next-token) form: one generated token per
+ * sequence. In place, for every (b, h):
+ *     S += phi(k) v^T;  z += phi(k);  y = phi(q)^T S / phi(q)^T z
+ * (the output includes the current token). BASED §2 "Efficient attentions"
+ * (recurrent generation), App. B "Next Token Prediction" (KV-state update).
+ *
+ *   S       [B, H, D, d_v] float, read and written in place
+ *   z       [B, H, D]      float, read and written in place
+ *   q, k    [B, H, d_feat] dtype;  v [B, H, d_v] dtype
+ *   y       [B, H, d_v]    dtype, written
+ *   d_feat  16 or 32;  d_v 64 or 128
+ * A state produced by based_la_prefill over N tokens followed by M decode steps
+ * equals, up to rounding, the state of a prefill over N + M tokens.
+ */
+BASED_API based_status_t based_la_decode_step(float* S, float* z,
+                                    const void* q, const void* k, const void* v, void* y,
+                                    int B, int H, int d_feat, int d_v,
+                                    based_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * based_swa_prefill -- causal sliding-window softmax attention over N tokens:
+ *     y_i = sum_j softmax_j(scale * q_i.k_j) v_j  over  i - w < j <= i
+ * (w keys including the query's own position). BASED §4 "Local Exact
+ * Attention", App. A.1 (O(Nw) cost), App. C (TCWINDOW layers).
+ *
+ *   q, k, v, y  [B, H, N, d] dtype
+ *   k_cache, v_cache  [B, H, w, d] dtype, written with the ring state after the
+ *           prompt: slot t mod w holds token t for t in [max(0, N-w), N); slots
+ *           never written are set to zero. Both NULL to skip.
+ *   d 64;  1 <= w <= 64;  scale finite (the workloads use 1/sqrt(d))
+ */
+BASED_API based_status_t based_swa_prefill(const void* q, const void* k, const void* v, void* y,
+                                 void* k_cache, void* v_cache,
+                                 int B, int H, int N, int d, int w, float scale,
+                                 based_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * based_swa_decode -- one generated token per sequence over the w-slot ring
+ * KV cache (BASED §4 "Local Exact Attention": a w-sized KV cache; App. B
+ * "Next Token Prediction"). t is the number of tokens every sequence has seen
+ * before this one. Writes (k, v) into slot t mod w, then attends over the
+ * min(t+1, w) slots holding tokens max(0, t-w+1) .. t.
+ *
+ *   k_cache, v_cache [B, H, w, d] dtype, read and written in place
+ *   q, k, v, y       [B, H, d]    dtype
+ *   t >= 0;  d 64;  1 <= w <= 64
+ */
+BASED_API based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t,
+                                const void* q, const void* k, const void* v, void* y,
+                                int B, int H, int d, int w, float scale,
+                                based_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * based_get_last_error -- synchronises `stream`, then reports and clears the
+ * device status word of the current device: BASED_ERR_TIMEOUT if a bounded
+ * wait in a kernel expired since the last call, BASED_ERR_CUDA if the stream
+ * reported a CUDA error, else BASED_OK.
+ */
+BASED_API based_status_t based_get_last_error(cudaStream_t stream);
+
+/* Static, NUL-terminated name of a status code ("BASED_OK", ...). */
+BASED_API const char* based_status_string(based_status_t status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+BASED_API int based_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BASED_H */

@@ -1,0 +1,23 @@
+"""BASED hot path on B200: causal Taylor linear attention + sliding-window attention.
+
+The computation lives in libbased.so (hand-written sm_100a CUDA kernels behind
+the C ABI of include/based.h); this package is its ctypes binding. Importing it
+does not need a GPU; calling an op does.
+"""
+
+from .binding import (  # noqa: F401
+    BasedError,
+    SYMBOLS,
+    feature_dim,
+    get_last_error,
+    la_decode_step,
+    la_prefill,
+    la_prefill_workspace,
+    lib,
+    library_path,
+    status_string,
+    swa_decode,
+    swa_prefill,
+)
+
+__version__ = "0.1.0"

@@ -1,0 +1,214 @@
+"""Thin ctypes binding over libbased.so (argument marshalling only).
+
+Every function takes CUDA torch tensors, allocates outputs with torch on the
+inputs' device, and passes raw device pointers plus the current torch stream to
+the C ABI declared in include/based.h. All arithmetic runs in the library's CUDA
+kernels; there is no CPU path. If libbased.so is missing or cannot be loaded,
+every call raises BasedError.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libbased.so")
+
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, 1, 2, 3, 4
+F32, BF16 = 0, 1
+_DTYPES = {torch.float32: F32, torch.bfloat16: BF16}
+
+SYMBOLS = (
+    "based_la_prefill",
+    "based_la_prefill_workspace",
+    "based_la_decode_step",
+    "based_swa_prefill",
+    "based_swa_decode",
+    "based_get_last_error",
+    "based_status_string",
+    "based_version",
+)
+
+
+class BasedError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status) if _lib_or_none() else status}")
+
+
+_LIB = None
+
+
+def _declare(lib):
+    vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    lib.based_la_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.based_la_prefill.restype = i
+    lib.based_la_prefill_workspace.argtypes = [i, i, i, i, i, i, i]
+    lib.based_la_prefill_workspace.restype = sz
+    lib.based_la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.based_la_decode_step.restype = i
+    lib.based_swa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
+    lib.based_swa_prefill.restype = i
+    lib.based_swa_decode.argtypes = [vp, vp, ctypes.c_int64, vp, vp, vp, vp, i, i, i, i, f, i, vp]
+    lib.based_swa_decode.restype = i
+    lib.based_get_last_error.argtypes = [vp]
+    lib.based_get_last_error.restype = i
+    lib.based_status_string.argtypes = [i]
+    lib.based_status_string.restype = ctypes.c_char_p
+    lib.based_version.argtypes = []
+    lib.based_version.restype = i
+    return lib
+
+
+def _lib_or_none():
+    global _LIB
+    if _LIB is None and os.path.exists(_LIB_PATH):
+        try:
+            _LIB = _declare(ctypes.CDLL(_LIB_PATH))
+        except OSError:
+            _LIB = None
+    return _LIB
+
+
+def lib():
+    """The loaded libbased.so (ctypes.CDLL); raises BasedError when it is missing."""
+    L = _lib_or_none()
+    if L is None:
+        raise BasedError(ERR_CUDA, f"libbased.so not loadable at {_LIB_PATH}; build it with "
+                                   "python -m linear_attention_sequence_causal_b200.build")
+    return L
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def status_string(status: int) -> str:
+    return lib().based_status_string(int(status)).decode()
+
+
+def _check(status: int, what: str):
+    if status != OK:
+        raise BasedError(status, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(*ts: torch.Tensor) -> int:
+    dt = ts[0].dtype
+    for t in ts:
+        if not t.is_cuda:
+            raise BasedError(ERR_INVALID_ARG, "tensors must be on a CUDA device")
+        if t.dtype != dt:
+            raise BasedError(ERR_INVALID_ARG, "q, k, v must share one dtype")
+        if not t.is_contiguous():
+            raise BasedError(ERR_INVALID_ARG, "tensors must be contiguous")
+    if dt not in _DTYPES:
+        raise BasedError(ERR_UNSUPPORTED, f"dtype {dt} (float32 or bfloat16 only)")
+    return _DTYPES[dt]
+
+
+def feature_dim(d_feat: int) -> int:
+    return 1 + d_feat + d_feat * d_feat
+
+
+def la_prefill_workspace(B, H, N, d_feat, d_v, dtype=torch.bfloat16, chunk=0) -> int:
+    return int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, _DTYPES[dtype], chunk))
+
+
+def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None, z=None,
+               workspace=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
+    """Causal Taylor linear attention over [B,H,N,*] inputs; returns (y, S, z).
+
+    S [B,H,D,dv] and z [B,H,D] (float32) hold the final state when want_state.
+    """
+    dt = _dtype_code(q, k, v)
+    B, H, N, d_feat = q.shape
+    d_v = v.shape[-1]
+    D = feature_dim(d_feat)
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty((B, H, N, d_v), dtype=q.dtype, device=dev)
+        if want_state:
+            S = torch.empty((B, H, D, d_v), dtype=torch.float32, device=dev) if S is None else S
+            z = torch.empty((B, H, D), dtype=torch.float32, device=dev) if z is None else z
+        else:
+            S = z = None
+        ws_bytes = int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, dt, chunk))
+        if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = lib().based_la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z),
+                                    B, H, N, d_feat, d_v, dt, chunk,
+                                    _ptr(workspace) if ws_bytes else None, ws_bytes, _stream(dev))
+    _check(st, "based_la_prefill")
+    return y, S, z
+
+
+def la_decode_step(S, z, q, k, v, y=None) -> torch.Tensor:
+    """One recurrent step, S and z updated in place; q, k [B,H,d'], v [B,H,dv]."""
+    dt = _dtype_code(q, k, v)
+    B, H, d_feat = q.shape
+    d_v = v.shape[-1]
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty((B, H, d_v), dtype=q.dtype, device=dev)
+        st = lib().based_la_decode_step(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
+                                        B, H, d_feat, d_v, dt, _stream(dev))
+    _check(st, "based_la_decode_step")
+    return y
+
+
+def swa_prefill(q, k, v, w: int = 64, scale: Optional[float] = None, want_cache: bool = True,
+                y=None, k_cache=None, v_cache=None):
+    """Sliding-window softmax attention over [B,H,N,d]; returns (y, k_cache, v_cache)."""
+    dt = _dtype_code(q, k, v)
+    B, H, N, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(q)
+        if want_cache:
+            k_cache = torch.empty((B, H, w, d), dtype=q.dtype, device=dev) if k_cache is None else k_cache
+            v_cache = torch.empty((B, H, w, d), dtype=q.dtype, device=dev) if v_cache is None else v_cache
+        else:
+            k_cache = v_cache = None
+        st = lib().based_swa_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(k_cache), _ptr(v_cache),
+                                     B, H, N, d, w, scale, dt, _stream(dev))
+    _check(st, "based_swa_prefill")
+    return y, k_cache, v_cache
+
+
+def swa_decode(k_cache, v_cache, t: int, q, k, v, w: int = 64, scale: Optional[float] = None,
+               y=None) -> torch.Tensor:
+    """One step over the ring cache (updated in place); q, k, v [B,H,d]."""
+    dt = _dtype_code(q, k, v)
+    B, H, d = q.shape
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(q)
+        st = lib().based_swa_decode(_ptr(k_cache), _ptr(v_cache), int(t), _ptr(q), _ptr(k), _ptr(v),
+                                    _ptr(y), B, H, d, w, scale, dt, _stream(dev))
+    _check(st, "based_swa_decode")
+    return y
+
+
+def get_last_error(device=None) -> int:
+    """Synchronise the current stream and return the device status (0 = OK)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib().based_get_last_error(_stream(dev)))

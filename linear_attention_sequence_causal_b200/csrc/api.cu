@@ -1,0 +1,187 @@
+// C ABI of libbased: argument validation, kernel selection, device status word.
+// The declarations and the contract of every entry point are in include/based.h.
+#include <atomic>
+#include <cstdint>
+
+#include "../../include/based.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace {
+
+// Per-device status word written by kernels whose bounded waits expired.
+__device__ unsigned g_based_status;
+
+constexpr int kMaxDevices = 64;
+std::atomic<unsigned*> g_status_ptr[kMaxDevices];
+std::atomic<int> g_num_sms[kMaxDevices];
+
+bool current_device(int* dev) { return cudaGetDevice(dev) == cudaSuccess && *dev >= 0 && *dev < kMaxDevices; }
+
+unsigned* status_word(int dev) {
+    unsigned* p = g_status_ptr[dev].load(std::memory_order_acquire);
+    if (p == nullptr) {
+        void* addr = nullptr;
+        if (cudaGetSymbolAddress(&addr, g_based_status) != cudaSuccess) return nullptr;
+        p = static_cast<unsigned*>(addr);
+        g_status_ptr[dev].store(p, std::memory_order_release);
+    }
+    return p;
+}
+
+int num_sms(int dev) {
+    int n = g_num_sms[dev].load(std::memory_order_relaxed);
+    if (n <= 0) {
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+        g_num_sms[dev].store(n, std::memory_order_relaxed);
+    }
+    return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_dtype(based_dtype_t d) { return d == BASED_F32 || d == BASED_BF16; }
+bool la_dims_built(int d_feat, int d_v) {
+    return (d_feat == 16 || d_feat == 32) && (d_v == 64 || d_v == 128);
+}
+
+// SIMT chunk sizes (shared memory bound: d' = 32 stops at 32 tokens).
+bool simt_chunk_ok(int d_feat, int chunk) {
+    return chunk == 16 || chunk == 32 || (chunk == 64 && d_feat == 16);
+}
+
+enum class LaPath { None, Simt, TensorCore };
+
+// Kernel choice for a prefill: the tcgen05 kernel for the bf16 shapes it is
+// built for, the fp32 CUDA-core kernel otherwise.
+LaPath choose_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
+    const bool bf16 = dtype == BASED_BF16;
+    if (*chunk == 0) {
+        if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, 128)) { *chunk = 128; return LaPath::TensorCore; }
+        *chunk = d_feat == 16 ? 64 : 32;
+        return LaPath::Simt;
+    }
+    if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, *chunk)) return LaPath::TensorCore;
+    if (simt_chunk_ok(d_feat, *chunk)) return LaPath::Simt;
+    return LaPath::None;
+}
+
+}  // namespace
+
+extern "C" {
+
+int based_version(void) { return 100; }
+
+const char* based_status_string(based_status_t s) {
+    switch (s) {
+        case BASED_OK: return "BASED_OK";
+        case BASED_ERR_INVALID_ARG: return "BASED_ERR_INVALID_ARG";
+        case BASED_ERR_UNSUPPORTED: return "BASED_ERR_UNSUPPORTED";
+        case BASED_ERR_CUDA: return "BASED_ERR_CUDA";
+        case BASED_ERR_TIMEOUT: return "BASED_ERR_TIMEOUT";
+    }
+    return "BASED_ERR_UNKNOWN";
+}
+
+size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int d_v, based_dtype_t dtype, int chunk) {
+    if (B <= 0 || H <= 0 || N <= 0 || !ok_dtype(dtype) || !la_dims_built(d_feat, d_v)) return 0;
+    int dev;
+    if (!current_device(&dev)) return 0;
+    const LaPath path = choose_la_path(d_feat, d_v, dtype, &chunk);
+    if (path != LaPath::TensorCore) return 0;
+    return based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, num_sms(dev));
+}
+
+based_status_t based_la_prefill(const void* q, const void* k, const void* v, void* y, float* S,
+                                float* z, int B, int H, int N, int d_feat, int d_v,
+                                based_dtype_t dtype, int chunk, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
+    if ((S == nullptr) != (z == nullptr)) return BASED_ERR_INVALID_ARG;
+    if (S != nullptr && (!aligned16(S) || !aligned16(z))) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || chunk < 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (!la_dims_built(d_feat, d_v) || (long long)B * H > 65535) return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const int sms = num_sms(dev);
+    unsigned* status = status_word(dev);
+    if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
+    const LaPath path = choose_la_path(d_feat, d_v, dtype, &chunk);
+    if (path == LaPath::None) return BASED_ERR_UNSUPPORTED;
+
+    based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype == BASED_BF16, chunk,
+                           workspace, workspace_bytes, status};
+    cudaError_t e;
+    if (path == LaPath::TensorCore) {
+        const size_t need = based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms);
+        if (workspace_bytes < need || (need > 0 && !ok_ptr(workspace))) return BASED_ERR_INVALID_ARG;
+        e = based::launch_la_prefill_tc(a, sms, stream);
+    } else {
+        e = based::launch_la_prefill_simt(a, stream);
+    }
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+based_status_t based_la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
+                                    void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
+                                    cudaStream_t stream) {
+    if (!ok_ptr(S) || !ok_ptr(z) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y))
+        return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (!la_dims_built(d_feat, d_v) || (long long)B * H > (1LL << 30)) return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const int sms = num_sms(dev);
+    if (sms <= 0) return BASED_ERR_CUDA;
+    const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, B, H, d_feat, d_v,
+                                                  dtype == BASED_BF16, sms, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+based_status_t based_swa_prefill(const void* q, const void* k, const void* v, void* y, void* k_cache,
+                                 void* v_cache, int B, int H, int N, int d, int w, float scale,
+                                 based_dtype_t dtype, cudaStream_t stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
+    if ((k_cache == nullptr) != (v_cache == nullptr)) return BASED_ERR_INVALID_ARG;
+    if (k_cache != nullptr && (!aligned16(k_cache) || !aligned16(v_cache))) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || w <= 0 || d <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (!(scale == scale) || scale - scale != 0.0f) return BASED_ERR_INVALID_ARG;   // NaN or inf
+    if (d != 64 || w > 64 || (long long)B * H > 65535) return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (status == nullptr) return BASED_ERR_CUDA;
+    const cudaError_t e = based::launch_swa_prefill(q, k, v, y, k_cache, v_cache, B, H, N, d, w, scale,
+                                                    dtype == BASED_BF16, status, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
+                                const void* v, void* y, int B, int H, int d, int w, float scale,
+                                based_dtype_t dtype, cudaStream_t stream) {
+    if (!ok_ptr(k_cache) || !ok_ptr(v_cache) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y))
+        return BASED_ERR_INVALID_ARG;
+    if (t < 0 || B <= 0 || H <= 0 || w <= 0 || d <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (!(scale == scale) || scale - scale != 0.0f) return BASED_ERR_INVALID_ARG;
+    if (d != 64 || w > 64 || (long long)B * H > (1LL << 30)) return BASED_ERR_UNSUPPORTED;
+    const cudaError_t e = based::launch_swa_decode(k_cache, v_cache, t, q, k, v, y, B, H, d, w, scale,
+                                                   dtype == BASED_BF16, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+based_status_t based_get_last_error(cudaStream_t stream) {
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BASED_ERR_CUDA;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (status == nullptr) return BASED_ERR_CUDA;
+    unsigned word = 0;
+    if (cudaMemcpy(&word, status, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess) return BASED_ERR_CUDA;
+    if (word != 0) {
+        const unsigned zero = 0;
+        if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return BASED_ERR_CUDA;
+    }
+    return (word & based::DEV_ERR_TIMEOUT) ? BASED_ERR_TIMEOUT : BASED_OK;
+}
+
+}  // extern "C"

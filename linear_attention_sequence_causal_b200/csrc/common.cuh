@@ -1,0 +1,46 @@
+// Shared device helpers for the BASED kernels (sm_100a).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace based {
+
+// Bits of the per-device status word (read and cleared by based_get_last_error).
+enum : unsigned {
+    DEV_ERR_TIMEOUT = 1u,   // a bounded wait expired
+};
+
+// Inputs are read as fp32 regardless of storage type.
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Global nanosecond timer, used to bound every spin wait.
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Upper bound of any single wait inside a kernel. A wait that runs past it
+// records DEV_ERR_TIMEOUT and gives up; nothing ever spins without a bound.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
+
+// sqrt(1/2) as an fp32 literal: the order-2 Taylor features carry 1/sqrt(2).
+constexpr float kSqrtHalf = 0.70710678118654752440f;
+
+__host__ __device__ constexpr int feature_dim(int d_feat) { return 1 + d_feat + d_feat * d_feat; }
+// Distinct features of phi once the symmetric outer product is folded:
+// 1 + d' + d'(d'+1)/2 (153 at d' = 16, 561 at d' = 32).
+__host__ __device__ constexpr int sym_feature_dim(int d_feat) {
+    return 1 + d_feat + d_feat * (d_feat + 1) / 2;
+}
+
+}  // namespace based

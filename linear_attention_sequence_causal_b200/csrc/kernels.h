@@ -1,0 +1,41 @@
+// Host-side launchers of the BASED kernels (internal to libbased; not part of the C ABI).
+// Every launcher only enqueues work on `stream` and returns the launch's cudaError_t.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace based {
+
+struct LaPrefillArgs {
+    const void* q; const void* k; const void* v; void* y;
+    float* S; float* z;              // may both be null
+    int B, H, N, d_feat, d_v;
+    bool bf16;
+    int chunk;                       // resolved, never 0
+    void* workspace; size_t ws_bytes;
+    unsigned* status;                // device status word
+};
+
+// SIMT fp32-arithmetic path: any supported dtype, chunk in {16, 32, 64}.
+cudaError_t launch_la_prefill_simt(const LaPrefillArgs& a, cudaStream_t stream);
+
+// Tensor-core (tcgen05/TMEM) path: bf16 inputs, d' = 16, dv = 64, chunk = 128.
+bool la_prefill_tc_supported(int d_feat, int d_v, int chunk);
+size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms);
+cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
+                             void* y, int B, int H, int d_feat, int d_v, bool bf16,
+                             int num_sms, cudaStream_t stream);
+
+cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y,
+                               void* k_cache, void* v_cache, int B, int H, int N, int d, int w,
+                               float scale, bool bf16, unsigned* status, cudaStream_t stream);
+
+cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q,
+                              const void* k, const void* v, void* y, int B, int H, int d, int w,
+                              float scale, bool bf16, cudaStream_t stream);
+
+}  // namespace based

@@ -1,0 +1,239 @@
+// Causal sliding-window softmax attention: prefill over a sequence, decode over a ring cache.
+//
+// "Simple linear attention language models balance the recall-throughput
+// tradeoff" (BASED), §4 "Local Exact Attention": exact softmax over a window of
+// the most recent keys, O(Nw) time and a w-sized KV cache for generation; App. B
+// "Next Token Prediction" names the windowed decode as one of the generation
+// kernels. Window convention: token i sees keys i - w < j <= i (w keys including
+// itself), which is what a w-slot ring holds after token i is written.
+//
+// Prefill (CUDA-core path): a CTA takes 64 consecutive queries of one head and
+// stages those queries plus the 64 + w - 1 keys and values they can see in
+// shared memory (fp32), so every K/V row is read from global memory once per
+// tile. Four threads share a query, each owning 16 of the 64 dims: partial dot
+// products are combined with two butterfly shuffles and the softmax runs online
+// (running max and sum, rescaling the accumulator), in fp32 with expf.
+//
+// Decode: one CTA per (b, h). The new key/value go to slot t mod w; thread j
+// scores slot j, the CTA reduces max and sum, then thread e accumulates output
+// dim e over the valid slots (coalesced over e).
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace based {
+namespace {
+
+constexpr int kQTile = 64;
+constexpr int kHead = 64;        // head dim d
+constexpr int kMaxW = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(256)
+swa_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
+                        T* __restrict__ y, int N, int w, float scale) {
+    extern __shared__ float smem[];
+    constexpr int KR = kQTile + kMaxW - 1;                 // key rows a tile can see
+    float* sQ = smem;                                      // [64][64]
+    float* sK = sQ + kQTile * kHead;                       // [KR][64]
+    float* sV = sK + KR * kHead;                           // [KR][64]
+
+    const int tid = threadIdx.x;
+    const size_t bh = blockIdx.y;
+    const int i0 = blockIdx.x * kQTile;
+    const int j0 = i0 - (w - 1);                           // first key row (may be < 0)
+    const T* qb = q + bh * (size_t)N * kHead;
+    const T* kb = k + bh * (size_t)N * kHead;
+    const T* vb = v + bh * (size_t)N * kHead;
+
+    for (int e = tid; e < kQTile * kHead; e += 256) {
+        const int r = e / kHead;
+        sQ[e] = (i0 + r < N) ? to_f32(qb[(size_t)i0 * kHead + e]) : 0.f;
+    }
+    const int nk = kQTile + w - 1;
+    for (int e = tid; e < nk * kHead; e += 256) {
+        const int r = e / kHead, c = e % kHead;
+        const int j = j0 + r;
+        const bool ok = j >= 0 && j < N;
+        sK[e] = ok ? to_f32(kb[(size_t)j * kHead + c]) : 0.f;
+        sV[e] = ok ? to_f32(vb[(size_t)j * kHead + c]) : 0.f;
+    }
+    __syncthreads();
+
+    const int qi = tid >> 2;          // query within the tile
+    const int part = tid & 3;         // 16-dim slice
+    const int i = i0 + qi;
+    const float* qrow = sQ + qi * kHead + part * 16;
+    float qreg[16];
+#pragma unroll
+    for (int d = 0; d < 16; ++d) qreg[d] = qrow[d] * scale;
+
+    float m = -INFINITY, l = 0.f;
+    float acc[16];
+#pragma unroll
+    for (int d = 0; d < 16; ++d) acc[d] = 0.f;
+
+    // Same trip count for every lane (w), so the shuffles stay converged.
+    for (int jj = 0; jj < w; ++jj) {
+        const int j = i - jj;                              // key position
+        const int r = j - j0;                              // row in sK / sV
+        const bool valid = (j >= 0) && (i < N);
+        const float* krow = sK + (valid ? r : 0) * kHead + part * 16;
+        float s = 0.f;
+#pragma unroll
+        for (int d = 0; d < 16; ++d) s = fmaf(qreg[d], krow[d], s);
+        s += __shfl_xor_sync(0xffffffffu, s, 1);
+        s += __shfl_xor_sync(0xffffffffu, s, 2);
+        if (valid) {
+            const float mn = fmaxf(m, s);
+            const float corr = expf(m - mn);               // 0 on the first key (m = -inf)
+            const float p = expf(s - mn);
+            l = l * corr + p;
+            const float* vrow = sV + r * kHead + part * 16;
+#pragma unroll
+            for (int d = 0; d < 16; ++d) acc[d] = fmaf(p, vrow[d], acc[d] * corr);
+            m = mn;
+        }
+    }
+    if (i < N) {
+        const float inv = 1.f / l;
+        T* yrow = y + (bh * (size_t)N + i) * kHead + part * 16;
+#pragma unroll
+        for (int d = 0; d < 16; ++d) yrow[d] = from_f32<T>(acc[d] * inv);
+    }
+}
+
+// Ring cache after the prompt: slot t mod w holds token t for t in [max(0, N-w), N), others 0.
+template <typename T>
+__global__ void swa_fill_ring_kernel(const T* __restrict__ k, const T* __restrict__ v,
+                                     T* __restrict__ kc, T* __restrict__ vc, int N, int w) {
+    const size_t bh = blockIdx.x;
+    for (int e = threadIdx.x; e < w * kHead; e += blockDim.x) {
+        const int slot = e / kHead, c = e % kHead;
+        // newest token u < N with u mod w == slot
+        const int last = N - 1;
+        const int u = last - (((last - slot) % w) + w) % w;
+        T kv = from_f32<T>(0.f), vv = from_f32<T>(0.f);
+        if (u >= 0) {
+            kv = k[(bh * (size_t)N + u) * kHead + c];
+            vv = v[(bh * (size_t)N + u) * kHead + c];
+        }
+        kc[(bh * w + slot) * kHead + c] = kv;
+        vc[(bh * w + slot) * kHead + c] = vv;
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kMaxW)
+swa_decode_kernel(T* __restrict__ kc, T* __restrict__ vc, long long t, const T* __restrict__ q,
+                  const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y, int w,
+                  float scale) {
+    __shared__ float s_q[kHead], s_k[kHead], s_v[kHead];
+    __shared__ float s_p[kMaxW];
+    __shared__ float s_red[2][2];
+    const int tid = threadIdx.x;          // 64 threads
+    const size_t bh = blockIdx.x;
+    const int new_slot = (int)(t % w);
+
+    s_q[tid] = to_f32(q[bh * kHead + tid]) * scale;
+    const T knew = k[bh * kHead + tid];
+    const T vnew = v[bh * kHead + tid];
+    s_k[tid] = to_f32(knew);
+    s_v[tid] = to_f32(vnew);
+    __syncthreads();
+
+    float s = -INFINITY;
+    bool valid = false;
+    if (tid < w) {
+        // newest token u <= t held by slot tid; valid when u >= 0
+        const long long u = t - ((((t - tid) % w) + w) % w);
+        valid = u >= 0;
+        if (valid) {
+            float acc = 0.f;
+            if (tid == new_slot) {
+#pragma unroll 16
+                for (int d = 0; d < kHead; ++d) acc = fmaf(s_q[d], s_k[d], acc);
+            } else {
+                const T* krow = kc + (bh * w + tid) * kHead;
+#pragma unroll 16
+                for (int d = 0; d < kHead; ++d) acc = fmaf(s_q[d], to_f32(krow[d]), acc);
+            }
+            s = acc;
+        }
+    }
+    float m = s;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((tid & 31) == 0) s_red[0][tid >> 5] = m;
+    __syncthreads();
+    m = fmaxf(s_red[0][0], s_red[0][1]);
+    const float p = valid ? expf(s - m) : 0.f;
+    float sum = p;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    if ((tid & 31) == 0) s_red[1][tid >> 5] = sum;
+    s_p[tid] = p;
+    __syncthreads();
+    const float inv = 1.f / (s_red[1][0] + s_red[1][1]);
+
+    float acc = 0.f;
+    for (int j = 0; j < w; ++j) {
+        const float pj = s_p[j];
+        if (pj != 0.f) {
+            const float vj = (j == new_slot) ? s_v[tid] : to_f32(vc[(bh * w + j) * kHead + tid]);
+            acc = fmaf(pj, vj, acc);
+        }
+    }
+    y[bh * kHead + tid] = from_f32<T>(acc * inv);
+    kc[(bh * w + new_slot) * kHead + tid] = knew;
+    vc[(bh * w + new_slot) * kHead + tid] = vnew;
+}
+
+template <typename T>
+cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void* k_cache,
+                      void* v_cache, int B, int H, int N, int w, float scale, cudaStream_t stream) {
+    constexpr size_t smem = (size_t)(kQTile * kHead + 2 * (kQTile + kMaxW - 1) * kHead) * sizeof(float);
+    auto kern = swa_prefill_simt_kernel<T>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((N + kQTile - 1) / kQTile, B * H);
+    kern<<<grid, 256, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                     static_cast<const T*>(v), static_cast<T*>(y), N, w, scale);
+    e = cudaGetLastError();
+    if (e != cudaSuccess || k_cache == nullptr) return e;
+    swa_fill_ring_kernel<T><<<B * H, 256, 0, stream>>>(static_cast<const T*>(k), static_cast<const T*>(v),
+                                                      static_cast<T*>(k_cache), static_cast<T*>(v_cache), N, w);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y, void* k_cache,
+                               void* v_cache, int B, int H, int N, int d, int w, float scale,
+                               bool bf16, unsigned* status, cudaStream_t stream) {
+    (void)status;
+    if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
+    return bf16 ? prefill_t<__nv_bfloat16>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, stream)
+                : prefill_t<float>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, stream);
+}
+
+cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
+                              const void* v, void* y, int B, int H, int d, int w, float scale,
+                              bool bf16, cudaStream_t stream) {
+    if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
+    if (bf16) {
+        swa_decode_kernel<__nv_bfloat16><<<B * H, kMaxW, 0, stream>>>(
+            static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), (long long)t,
+            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w, scale);
+    } else {
+        swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(
+            static_cast<float*>(k_cache), static_cast<float*>(v_cache), (long long)t,
+            static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
+            static_cast<float*>(y), w, scale);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace based

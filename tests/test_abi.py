@@ -1,0 +1,108 @@
+"""The C ABI library loads and exports every symbol include/*.h declares (CPU only).
+
+Also checks the synchronous argument validation, which returns before any CUDA
+call and so runs without a GPU (no kernel is launched: every case here fails
+validation first).
+"""
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+import linear_attention_sequence_causal_b200 as based
+from linear_attention_sequence_causal_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        names |= set(re.findall(r"BASED_API\s+[\w\s\*]+?\b(based_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(binding.library_path()):
+        from linear_attention_sequence_causal_b200 import build
+        build.build()
+    return based.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_symbols()
+    for n in ("based_la_prefill", "based_la_decode_step", "based_swa_prefill", "based_swa_decode",
+              "based_get_last_error", "based_la_prefill_workspace"):
+        assert n in names
+    assert set(binding.SYMBOLS) <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(binding.library_path())
+    for name in sorted(_declared_symbols()):
+        assert hasattr(raw, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.based_version() >= 100
+    assert based.status_string(0) == "BASED_OK"
+    assert based.status_string(4) == "BASED_ERR_TIMEOUT"
+    assert based.status_string(99) == "BASED_ERR_UNKNOWN"
+
+
+FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: validation fails first
+MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
+
+
+def test_la_prefill_rejects_bad_arguments(lib):
+    f = lib.based_la_prefill
+    ok = dict(B=1, H=1, N=16, df=16, dv=64, dt=1, chunk=0)
+
+    def call(q=FAKE, S=FAKE, z=FAKE, **kw):
+        a = dict(ok, **kw)
+        return f(q, FAKE, FAKE, FAKE, S, z, a["B"], a["H"], a["N"], a["df"], a["dv"], a["dt"],
+                 a["chunk"], None, 0, None)
+
+    assert call(q=None) == binding.ERR_INVALID_ARG
+    assert call(q=MISALIGNED) == binding.ERR_INVALID_ARG
+    assert call(S=None) == binding.ERR_INVALID_ARG          # S without z
+    assert call(N=0) == binding.ERR_INVALID_ARG
+    assert call(B=-1) == binding.ERR_INVALID_ARG
+    assert call(dt=7) == binding.ERR_INVALID_ARG
+    assert call(chunk=-1) == binding.ERR_INVALID_ARG
+    assert call(df=8) == binding.ERR_UNSUPPORTED
+    assert call(dv=96) == binding.ERR_UNSUPPORTED
+
+
+def test_decode_and_swa_reject_bad_arguments(lib):
+    assert lib.based_la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 64, 1, None) \
+        == binding.ERR_INVALID_ARG
+    assert lib.based_la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 24, 64, 1, None) \
+        == binding.ERR_UNSUPPORTED
+    sp = lib.based_swa_prefill
+    assert sp(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 64, 0, 0.125, 1, None) == binding.ERR_INVALID_ARG
+    assert sp(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 8, 64, 64, 0.125, 1, None) == binding.ERR_INVALID_ARG
+    assert sp(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 64, 64, float("nan"), 1, None) \
+        == binding.ERR_INVALID_ARG
+    assert sp(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 128, 64, 0.1, 1, None) == binding.ERR_UNSUPPORTED
+    assert sp(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 64, 65, 0.1, 1, None) == binding.ERR_UNSUPPORTED
+    sd = lib.based_swa_decode
+    assert sd(FAKE, FAKE, -1, FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 64, 0.125, 1, None) == binding.ERR_INVALID_ARG
+    assert sd(FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 80, 0.125, 1, None) == binding.ERR_UNSUPPORTED
+
+
+def test_workspace_query_rejects_bad_arguments(lib):
+    assert lib.based_la_prefill_workspace(0, 1, 1, 16, 64, 1, 0) == 0
+    assert lib.based_la_prefill_workspace(1, 1, 1, 8, 64, 1, 0) == 0
+
+
+def test_python_binding_requires_cuda_tensors():
+    import torch
+    x = torch.zeros(1, 1, 4, 16)
+    with pytest.raises(based.BasedError):
+        based.la_prefill(x, x, torch.zeros(1, 1, 4, 64))

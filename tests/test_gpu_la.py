@@ -1,0 +1,227 @@
+"""GPU parity: causal Taylor linear attention (prefill + decode) against the CPU oracle.
+
+Every case runs the CUDA library through its C ABI (via the ctypes binding) on
+seeded synthetic inputs and compares element by element with the float64
+oracle evaluated on the same (bf16-rounded) inputs. Tolerances: y max-abs 1e-4
+(fp32 inputs) / 2e-2 (bf16 inputs); S, z max|diff|/max|ref| 1e-5 / 1e-2; the
+constant feature of z counts tokens and must equal N exactly.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import linear_attention_sequence_causal_b200 as based
+from linear_attention_sequence_causal_b200 import synthetic
+from parity_util import assert_state, assert_y, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+def _run_prefill(inp, chunk=0, want_state=True):
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y, S, z = based.la_prefill(q, k, v, chunk=chunk, want_state=want_state)
+    assert based.get_last_error() == 0
+    return y, S, z
+
+
+def _check_full(inp, dtype, y, S, z):
+    ref_y = oracle.la_quadratic(inp.q64, inp.k64, inp.v64)
+    assert_y(to64(y), ref_y, dtype)
+    if S is not None:
+        ref_S, ref_z = oracle.la_state(inp.k64, inp.v64)
+        assert_state(to64(S), ref_S, dtype, "S")
+        assert_state(to64(z), ref_z, dtype, "z")
+        assert np.all(to64(z)[..., 0] == inp.k64.shape[-2])
+
+
+# ------------------------------------------------------------ small / ragged cases
+
+@pytest.mark.parametrize("chunk", [0, 16, 32, 64])
+def test_tiny_fp32(chunk):
+    """B=1, H=1, N=256, d'=16, dv=64, fp32 inputs (the tiny workload)."""
+    inp = synthetic.la_inputs(1, 1, 256, 16, 64, "f32", seed=0)
+    y, S, z = _run_prefill(inp, chunk)
+    _check_full(inp, torch.float32, y, S, z)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [1, 7, 64, 65, 127, 128, 129, 300])
+def test_ragged_lengths(dtype, N):
+    inp = synthetic.la_inputs(2, 3, N, 16, 64, dtype, seed=N)
+    y, S, z = _run_prefill(inp)
+    _check_full(inp, DT[dtype], y, S, z)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("d_feat,d_v", [(16, 128), (32, 64), (32, 128)])
+def test_other_shapes(dtype, d_feat, d_v):
+    inp = synthetic.la_inputs(1, 2, 200, d_feat, d_v, dtype, seed=d_feat + d_v)
+    y, S, z = _run_prefill(inp)
+    _check_full(inp, DT[dtype], y, S, z)
+
+
+def test_bf16_chunks_agree_with_oracle():
+    inp = synthetic.la_inputs(1, 2, 777, 16, 64, "bf16", seed=5)
+    for chunk in (0, 16, 32, 64, 128, 256):
+        try:
+            y, S, z = _run_prefill(inp, chunk)
+        except based.BasedError as e:
+            assert e.status == 2, (chunk, e)     # chunk not built for this dtype
+            continue
+        _check_full(inp, torch.bfloat16, y, S, z)
+
+
+def test_no_state_output():
+    inp = synthetic.la_inputs(2, 2, 100, 16, 64, "bf16", seed=6)
+    y, S, z = _run_prefill(inp, want_state=False)
+    assert S is None and z is None
+    assert_y(to64(y), oracle.la_quadratic(inp.q64, inp.k64, inp.v64), torch.bfloat16)
+
+
+def test_zero_query_is_cumulative_mean():
+    inp = synthetic.la_inputs(1, 2, 150, 16, 64, "f32", seed=7)
+    q = torch.zeros_like(inp.q).to(DEV)
+    y, _, _ = based.la_prefill(q, inp.k.to(DEV), inp.v.to(DEV))
+    mean = np.cumsum(inp.v64, axis=-2) / np.arange(1, 151)[:, None]
+    assert_y(to64(y), mean, torch.float32)
+
+
+def test_outputs_stay_in_bounds_and_deterministic():
+    inp = synthetic.la_inputs(1, 2, 130, 16, 64, "bf16", seed=8)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    canary = torch.full((2 * 130 * 64 + 4096,), 7.0, dtype=torch.bfloat16, device=DEV)
+    y = canary[: 2 * 130 * 64].view(1, 2, 130, 64)
+    based.la_prefill(q, k, v, y=y)
+    torch.cuda.synchronize()
+    assert torch.all(canary[2 * 130 * 64:] == 7.0)
+    y2, _, _ = based.la_prefill(q, k, v)
+    assert torch.equal(y, y2)
+
+
+# ------------------------------------------------------------ full-size workloads (sampled)
+
+def _sampled_check(inp, dtype, y, S, z, heads, rows, state_heads):
+    y64, S64, z64 = to64(y), to64(S), to64(z)
+    for (b, h) in heads:
+        ref = oracle.la_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], rows)
+        assert_y(y64[b, h, rows], ref, dtype, f"y[{b},{h}]")
+    bs = [b for b, _ in state_heads]
+    hs = [h for _, h in state_heads]
+    ref_S, ref_z = oracle.la_state(inp.k64[bs, hs], inp.v64[bs, hs])
+    assert_state(S64[bs, hs], ref_S, dtype, "S")
+    assert_state(z64[bs, hs], ref_z, dtype, "z")
+    assert np.all(z64[..., 0] == inp.k64.shape[-2])
+
+
+def _rows(N, rng, n=48):
+    fixed = [0, 1, 63, 64, 127, 128, 255, 256, N // 2, N - 2, N - 1]
+    return sorted(set([r for r in fixed if r < N] + rng.integers(0, N, n).tolist()))
+
+
+def test_360m_prefill_sampled():
+    """B=8, H=16, N=2048, d'=16, dv=64, bf16, library's default chunk."""
+    inp = synthetic.la_inputs(8, 16, 2048, 16, 64, "bf16", seed=0)
+    y, S, z = _run_prefill(inp)
+    rng = np.random.default_rng(0)
+    heads = [(0, 0), (7, 15), (3, 9), (5, 2)]
+    _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(2048, rng),
+                   [(b, h) for b in range(8) for h in (0, 5, 11, 15)])
+    # all outputs finite, in a sane range (y is a convex-ish average of v)
+    assert torch.isfinite(y.float()).all()
+
+
+@pytest.mark.parametrize("chunk", [0, 64, 128, 256])
+def test_long_prefill_sampled(chunk):
+    """B=2, H=16, N=16384, chunk length swept; final S and z of sampled heads checked."""
+    inp = synthetic.la_inputs(2, 16, 16384, 16, 64, "bf16", seed=0)
+    try:
+        y, S, z = _run_prefill(inp, chunk)
+    except based.BasedError as e:
+        assert e.status == 2, e
+        pytest.skip(f"chunk {chunk} not built for bf16")
+    rng = np.random.default_rng(1)
+    _sampled_check(inp, torch.bfloat16, y, S, z, [(0, 0), (1, 15), (1, 7)], _rows(16384, rng, 24),
+                   [(0, 0), (0, 8), (1, 3), (1, 15)])
+
+
+def test_large_state_prefill_sampled():
+    """d'=32 (D=1057), H=8, dv=128, B=4, N=8192, bf16."""
+    inp = synthetic.la_inputs(4, 8, 8192, 32, 128, "bf16", seed=0)
+    y, S, z = _run_prefill(inp)
+    rng = np.random.default_rng(2)
+    _sampled_check(inp, torch.bfloat16, y, S, z, [(0, 0), (3, 7)], _rows(8192, rng, 16),
+                   [(0, 0), (2, 5), (3, 7)])
+
+
+# ------------------------------------------------------------ decode
+
+def _decode_run(B, H, d_feat, d_v, dtype, prompt, steps, seed, check_heads):
+    """Prefill `prompt` tokens, then `steps` decode steps; compare with the oracle."""
+    inp = synthetic.la_inputs(B, H, prompt + steps, d_feat, d_v, dtype, seed=seed)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    _, S, z = based.la_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                               v[:, :, :prompt].contiguous())
+    ys = torch.empty((B, H, steps, d_v), dtype=q.dtype, device=DEV)
+    # step-major copies so each step's q, k, v are contiguous [B, H, *] slices
+    qd, kd, vd = (x[:, :, prompt:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
+    for t in range(steps):
+        ys[:, :, t] = based.la_decode_step(S, z, qd[t], kd[t], vd[t])
+    assert based.get_last_error() == 0
+    dt = DT[dtype]
+    ys64, S64, z64 = to64(ys), to64(S), to64(z)
+    bs = [b for b, _ in check_heads]
+    hs = [h for _, h in check_heads]
+    ref = oracle.la_quadratic(inp.q64[bs, hs], inp.k64[bs, hs], inp.v64[bs, hs])
+    assert_y(ys64[bs, hs], ref[..., prompt:, :], dt, "decode y")
+    ref_S, ref_z = oracle.la_state(inp.k64[bs, hs], inp.v64[bs, hs])
+    assert_state(S64[bs, hs], ref_S, dt, "S")
+    assert_state(z64[bs, hs], ref_z, dt, "z")
+    assert np.all(z64[..., 0] == prompt + steps)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_decode_small(dtype):
+    _decode_run(2, 3, 16, 64, dtype, prompt=37, steps=40, seed=11,
+                check_heads=[(b, h) for b in range(2) for h in range(3)])
+
+
+@pytest.mark.parametrize("batch", [1, 16, 64, 128, 256])
+def test_decode_workload(batch):
+    """H=16, d'=16, dv=64, 512-token prompt then 1024 decode steps, bf16 q/k/v, fp32 state."""
+    rng = np.random.default_rng(batch)
+    heads = [(int(rng.integers(batch)), int(rng.integers(16))) for _ in range(4)] + [(batch - 1, 15)]
+    _decode_run(batch, 16, 16, 64, "bf16", prompt=512, steps=1024, seed=batch, check_heads=heads)
+
+
+def test_decode_large_state():
+    """d'=32, dv=128, H=8, batch 64, 256 decode steps after a 512-token prompt."""
+    _decode_run(64, 8, 32, 128, "bf16", prompt=512, steps=256, seed=3,
+                check_heads=[(0, 0), (31, 4), (63, 7)])
+
+
+def test_decode_resume_from_copied_state_is_bit_identical():
+    """The state (S, z) is the checkpoint: copying it out and back resumes exactly."""
+    inp = synthetic.la_inputs(2, 4, 80, 16, 64, "bf16", seed=12)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    _, S, z = based.la_prefill(q[:, :, :60].contiguous(), k[:, :, :60].contiguous(), v[:, :, :60].contiguous())
+    S_saved, z_saved = S.cpu().clone(), z.cpu().clone()
+    outs = []
+    for _ in range(2):
+        S2, z2 = S_saved.to(DEV), z_saved.to(DEV)
+        ys = [based.la_decode_step(S2, z2, q[:, :, t].contiguous(), k[:, :, t].contiguous(),
+                                   v[:, :, t].contiguous()) for t in range(60, 80)]
+        outs.append((torch.stack(ys), S2, z2))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_decode_rejects_unsupported():
+    S = torch.zeros(1, 1, 1 + 24 + 576, 64, device=DEV)
+    z = torch.zeros(1, 1, 1 + 24 + 576, device=DEV)
+    x = torch.zeros(1, 1, 24, device=DEV)
+    with pytest.raises(based.BasedError) as e:
+        based.la_decode_step(S, z, x, x, torch.zeros(1, 1, 64, device=DEV))
+    assert e.value.status == 2

@@ -1,0 +1,102 @@
+"""GPU parity: sliding-window softmax attention (prefill + ring decode) against the oracle.
+
+Tolerances: y max-abs 1e-4 (fp32 inputs) / 2e-2 (bf16 inputs). Ring-cache
+contents are copies of input values and must match bit for bit.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import linear_attention_sequence_causal_b200 as based
+from linear_attention_sequence_causal_b200 import synthetic
+from parity_util import assert_y, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+DT = {"f32": torch.float32, "bf16": torch.bfloat16}
+SCALE = 1.0 / math.sqrt(64)
+
+
+def _prefill(inp, w, scale=SCALE):
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    out = based.swa_prefill(q, k, v, w=w, scale=scale)
+    assert based.get_last_error() == 0
+    return out
+
+
+def test_tiny_fp32():
+    """One head, N=256, d=64, w=64, fp32."""
+    inp = synthetic.swa_inputs(1, 1, 256, 64, "f32", seed=0)
+    y, kc, vc = _prefill(inp, 64)
+    assert_y(to64(y), oracle.swa(inp.q64, inp.k64, inp.v64, 64, SCALE), torch.float32)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("w", [1, 2, 17, 64])
+@pytest.mark.parametrize("N", [1, 5, 64, 65, 130])
+def test_windows_and_lengths(dtype, w, N):
+    inp = synthetic.swa_inputs(2, 2, N, 64, dtype, seed=w * 1000 + N)
+    y, kc, vc = _prefill(inp, w)
+    assert_y(to64(y), oracle.swa(inp.q64, inp.k64, inp.v64, w, SCALE), DT[dtype])
+    rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, w)
+    assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
+
+
+def test_large_scores_stay_finite():
+    # scale 2 on unscaled N(0,1) inputs gives scores of order 100: max subtraction must hold
+    inp = synthetic.swa_inputs(1, 2, 200, 64, "f32", seed=3, qk_scale=1.0)
+    y, _, _ = _prefill(inp, 64, scale=2.0)
+    assert_y(to64(y), oracle.swa(inp.q64, inp.k64, inp.v64, 64, 2.0), torch.float32)
+
+
+def test_360m_prefill_sampled():
+    """16 heads x d=64, B=8, N=2048, w=64, bf16."""
+    inp = synthetic.swa_inputs(8, 16, 2048, 64, "bf16", seed=0)
+    y, kc, vc = _prefill(inp, 64)
+    y64 = to64(y)
+    rng = np.random.default_rng(0)
+    rows = sorted(set([0, 1, 62, 63, 64, 65, 127, 128, 1000, 2046, 2047] + rng.integers(0, 2048, 64).tolist()))
+    for b, h in [(0, 0), (7, 15), (2, 9), (5, 3)]:
+        ref = oracle.swa_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], 64, SCALE, rows)
+        assert_y(y64[b, h, rows], ref, torch.bfloat16, f"y[{b},{h}]")
+    rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, 64)
+    assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
+
+
+@pytest.mark.parametrize("dtype,batch,prompt,steps,w", [
+    ("f32", 2, 0, 70, 16), ("f32", 2, 10, 70, 64), ("bf16", 3, 100, 80, 64),
+    ("bf16", 64, 512, 1024, 64),
+])
+def test_decode_continues_prefill(dtype, batch, prompt, steps, w):
+    H = 16 if batch >= 64 else 2
+    inp = synthetic.swa_inputs(batch, H, prompt + steps, 64, dtype, seed=batch + prompt)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    if prompt > 0:
+        _, kc, vc = based.swa_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                                      v[:, :, :prompt].contiguous(), w=w, scale=SCALE)
+    else:
+        kc = torch.zeros((batch, H, w, 64), dtype=q.dtype, device=DEV)
+        vc = torch.zeros_like(kc)
+    qd, kd, vd = (x[:, :, prompt:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
+    ys = torch.empty((batch, H, steps, 64), dtype=q.dtype, device=DEV)
+    for t in range(steps):
+        ys[:, :, t] = based.swa_decode(kc, vc, prompt + t, qd[t], kd[t], vd[t], w=w, scale=SCALE)
+    assert based.get_last_error() == 0
+    heads = [(0, 0), (batch - 1, H - 1), (batch // 2, H // 2)]
+    bs = [b for b, _ in heads]
+    hs = [h for _, h in heads]
+    ref = oracle.swa(inp.q64[bs, hs], inp.k64[bs, hs], inp.v64[bs, hs], w, SCALE)
+    assert_y(to64(ys)[bs, hs], ref[..., prompt:, :], DT[dtype], "decode y")
+    rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, w)
+    assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
+
+
+def test_unsupported_head_dim():
+    x = torch.zeros(1, 1, 8, 128, device=DEV)
+    with pytest.raises(based.BasedError) as e:
+        based.swa_prefill(x, x, x, w=64)
+    assert e.value.status == 2
