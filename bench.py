@@ -498,6 +498,60 @@ def run_reference(args):
     }), flush=True)
 
 
+# ---------------------------------------------------------------- ncu capture cases
+
+PROFILE_CASES = {
+    # inputs larger than the 126 MB L2 so DRAM counters mean something; a few hundred MB at most
+    "la_prefill": "B=32 H=16 N=2048 d'=16 dv=64 bf16 (q,k,v,y 335 MB)",
+    "swa_prefill": "B=16 H=16 N=2048 d=64 w=64 bf16 (q,k,v,y 268 MB)",
+    "la_decode": "batch 256, H=16, d'=16, dv=64 (fp32 state 286 MB)",
+    "swa_decode": "batch 1024, H=16, d=64, w=64 (ring caches 268 MB)",
+}
+
+
+def run_profile(kind, reps):
+    """Launch one kernel `reps` times on its capture case (for ncu; prints timings only)."""
+    import torch
+
+    import linear_attention_sequence_causal_b200 as based
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    if kind == "la_prefill":
+        inp = synthetic.la_inputs(32, 16, 2048, 16, 64, "bf16", seed=0)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        fn = lambda: based.la_prefill(q, k, v)
+    elif kind == "swa_prefill":
+        inp = synthetic.swa_inputs(16, 16, 2048, 64, "bf16", seed=0)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        fn = lambda: based.swa_prefill(q, k, v, w=64)
+    elif kind == "la_decode":
+        S = torch.randn(256, 16, 273, 64, device=dev)
+        z = torch.rand(256, 16, 273, device=dev) + 300.0
+        x = torch.randn(256, 16, 16, device=dev).bfloat16()
+        vv = torch.randn(256, 16, 64, device=dev).bfloat16()
+        fn = lambda: based.la_decode_step(S, z, x, x, vv)
+    else:
+        kc = torch.randn(1024, 16, 64, 64, device=dev).bfloat16()
+        vc = torch.randn(1024, 16, 64, 64, device=dev).bfloat16()
+        x = torch.randn(1024, 16, 64, device=dev).bfloat16()
+        fn = lambda: based.swa_decode(kc, vc, 1000, x, x, x)
+    fn()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        fn()
+        b.record()
+        b.synchronize()
+        ts.append(a.elapsed_time(b))
+    if based.get_last_error() != 0:
+        raise SystemExit("device status error")
+    print(json.dumps({"profile": kind, "case": PROFILE_CASES[kind], "ms": ts}))
+
+
 def main(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
@@ -506,7 +560,12 @@ def main(argv=None):
     p.add_argument("--impl", choices=("mine", "reference"), default="mine")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample size")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--profile", choices=sorted(PROFILE_CASES), help="run one kernel on its ncu capture case")
+    p.add_argument("--profile-reps", type=int, default=3)
     args = p.parse_args(argv)
+    if args.profile:
+        run_profile(args.profile, args.profile_reps)
+        return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
