@@ -2,6 +2,7 @@
 // The declarations and the contract of every entry point are in include/based.h.
 #include <atomic>
 #include <cstdint>
+#include <cstdlib>
 
 #include "../../include/based.h"
 #include "common.cuh"
@@ -36,6 +37,15 @@ int num_sms(int dev) {
         g_num_sms[dev].store(n, std::memory_order_relaxed);
     }
     return n;
+}
+
+// BASED_DEBUG_SKIP_MMA=1 in the environment makes the tensor-core kernels issue
+// no MMA, so that their bounded waits expire: the failure-detection tests use it
+// to check that a stalled kernel reports BASED_ERR_TIMEOUT and leaves the
+// context usable. Read on every call; unset in normal use.
+unsigned debug_flags() {
+    const char* e = std::getenv("BASED_DEBUG_SKIP_MMA");
+    return (e != nullptr && e[0] == '1') ? based::DEBUG_SKIP_MMA : 0u;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -110,7 +120,7 @@ based_status_t based_la_prefill(const void* q, const void* k, const void* v, voi
     if (path == LaPath::None) return BASED_ERR_UNSUPPORTED;
 
     based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype == BASED_BF16, chunk,
-                           workspace, workspace_bytes, status};
+                           workspace, workspace_bytes, status, debug_flags()};
     cudaError_t e;
     if (path == LaPath::TensorCore) {
         const size_t need = based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms);
@@ -152,7 +162,7 @@ based_status_t based_swa_prefill(const void* q, const void* k, const void* v, vo
     unsigned* status = status_word(dev);
     if (status == nullptr) return BASED_ERR_CUDA;
     const cudaError_t e = based::launch_swa_prefill(q, k, v, y, k_cache, v_cache, B, H, N, d, w, scale,
-                                                    dtype == BASED_BF16, status, stream);
+                                                    dtype == BASED_BF16, status, debug_flags(), stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 

@@ -16,7 +16,12 @@ struct LaPrefillArgs {
     int chunk;                       // resolved, never 0
     void* workspace; size_t ws_bytes;
     unsigned* status;                // device status word
+    unsigned debug;                  // DEBUG_* bits (testing only)
 };
+
+// Testing aid: with this bit the tensor-core kernels issue no MMA, so their
+// bounded waits expire and report DEV_ERR_TIMEOUT (see debug_flags() in api.cu).
+constexpr unsigned DEBUG_SKIP_MMA = 1u;
 
 // SIMT fp32-arithmetic path: any supported dtype, chunk in {16, 32, 64}.
 cudaError_t launch_la_prefill_simt(const LaPrefillArgs& a, cudaStream_t stream);
@@ -32,7 +37,13 @@ cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, c
 
 cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y,
                                void* k_cache, void* v_cache, int B, int H, int N, int d, int w,
-                               float scale, bool bf16, unsigned* status, cudaStream_t stream);
+                               float scale, bool bf16, unsigned* status, unsigned debug,
+                               cudaStream_t stream);
+
+// Tensor-core path of the sliding-window prefill (bf16, d = 64, w <= 64), ring fill fused.
+cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, void* y, void* k_cache,
+                                  void* v_cache, int B, int H, int N, int w, float scale, unsigned* status,
+                                  unsigned debug, cudaStream_t stream);
 
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q,
                               const void* k, const void* v, void* y, int B, int H, int d, int w,

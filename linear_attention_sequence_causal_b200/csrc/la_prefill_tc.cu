@@ -5,35 +5,45 @@
 // the causal dot product are computed together, tile by tile; a tile's output is
 // a quadratic on-diagonal part under a local causal mask plus a linear
 // off-diagonal part read from the cumulative state of earlier tiles. With the
-// K-state normalisation (App. D.4), for a chunk of C = 128 tokens:
+// K-state normalisation (App. D.4), for a chunk c of C = 128 tokens:
 //
-//   s    = Q_c K_c^T                                  (tcgen05, M=128 N=128 K=16)
-//   A    = mask(1 + s + s^2/2)                        (CUDA cores, from TMEM)
-//   Y    = A [V_c | 1]  +  phi(Q_c) [S | z]           (tcgen05, N = 64 + 16)
-//   y_c  = Y[:, :64] / Y[:, 64]                       (epilogue)
-//   dS   = phi(K_c)^T [V_c | 1]                       (tcgen05, two 128-row tiles)
-//   [S | z] += dS                                     (fp32, in registers)
+//   s      = Q_c K_c^T                                MMA1  M=128 N=128 K=16
+//   Y      = phi(Q_c) [S | z]_{c-1}                   MMA3  M=128 N=80 K=160 (A from TMEM)
+//   [S|z] += phi(K_c)^T [V_c | 1]                     MMA4  two 128-row tiles, N=80, K=128,
+//                                                           accumulated in TMEM across chunks (fp32)
+//   A      = mask(1 + s + s^2/2)                      CUDA cores, from TMEM
+//   Y     += A [V_c | 1]                              MMA2  M=128 N=80 K=128
+//   y_c    = Y[:, :64] / Y[:, 64]                     epilogue
 //
 // The ones column appended to V makes every product carry its own
-// denominator: A [V | 1] yields the row sums of A, phi(Q)[S | z] yields
-// phi(q).z, and phi(K)^T [V | 1] yields the increment of z.
+// denominator: A [V | 1] gives the row sums of A, phi(Q)[S | z] gives phi(q).z,
+// and phi(K)^T [V | 1] gives the increment of z.
 //
-// phi is never written to HBM: each token's thread forms phi(q_t) and phi(k_t)
-// in registers and stores them (bf16) straight into the shared-memory operand
-// tiles. The order-2 block is folded by symmetry, (q.k)^2/2 =
-// sum_a (q_a^2/sqrt2)(k_a^2/sqrt2) + sum_{a<b} (q_a q_b)(k_a k_b), giving
-// 1 + 16 + 136 = 153 features (padded to 160) instead of 273; the final state
-// is expanded back to the 273-row layout on the way out.
+// phi never reaches HBM: each token's thread forms phi(q_t) and phi(k_t) in
+// registers; phi(Q) goes straight into tensor memory (the A operand of MMA3),
+// phi(K)^T into shared memory. The order-2 block is folded by symmetry,
+// (q.k)^2/2 = sum_a (q_a^2/sqrt2)(k_a^2/sqrt2) + sum_{a<b} (q_a q_b)(k_a k_b),
+// giving 1 + 16 + 136 = 153 features (padded to 160) instead of 273; the final
+// state is expanded back to the 273-row layout on the way out.
 //
-// CTA roles (288 threads, one CTA per (b, h), TMEM fully owned):
-//   warps 0-3  token threads: thread t owns token t of the chunk (TMEM lane t):
-//              loads q, k, v, builds the operand tiles, turns s into A and
-//              finishes y.
-//   warps 4-7  state threads: own the rows of dS (TMEM lanes), keep the running
-//              fp32 state [S | z] in registers and publish it as the bf16 B
-//              operand of the next chunk's inter-chunk product.
-//   warp 8     allocates TMEM; lane 0 issues every MMA and commit.
-// All hand-offs go through mbarriers whose waits are bounded.
+// One CTA per (b, h) with four roles (416 threads), so that the tensor pipe,
+// the CUDA cores and the memory system work on different chunks at once:
+//   warps 0-3   producers: thread t loads token t of chunk c+1 (prefetched in
+//               registers a chunk ahead) and writes Q, K, [V|1] and phi(K)^T
+//               into the free half of the double-buffered shared-memory tiles,
+//               then phi(Q) into tensor memory once MMA3 of the previous chunk
+//               has consumed it.
+//   warps 4-7   state: after each chunk, read the fp32 state rows 0..127 from
+//               TMEM in one batch and publish them as the bf16 B operand of the
+//               next MMA3 (double-buffered in shared memory); write the final
+//               state.
+//   warps 8-11  intra + epilogue: turn s into A and Y into y (TMEM lane = token);
+//               warp 8, whose rows of A are the shortest, also publishes state
+//               rows 128..159.
+//   warp 12     allocates TMEM; lane 0 issues every MMA and commit in the order
+//               MMA1, MMA3, MMA4, MMA2 so the CUDA-core stages (A, state
+//               publication) overlap the long MMAs.
+// Every hand-off is an mbarrier; every wait is bounded.
 //
 // Shared-memory operands use the canonical no-swizzle layouts (8-row x 16-byte
 // core matrices, each a contiguous 128-byte block); each thread writes whole
@@ -53,37 +63,41 @@ constexpr int C = 128;           // tokens per chunk
 constexpr int DS = 153;          // distinct (symmetric) features
 constexpr int KF = 160;          // DS padded to the MMA K step
 constexpr int NV = 80;           // [V | 1] padded to the MMA N step
-constexpr int kThreads = 288;
+constexpr int kThreads = 416;
 
-// Shared memory map (bytes). The update's second 128-row tile of phi(K)^T reads
-// feature rows 128..255 of which only 128..159 exist; the rows beyond alias the
-// next region (their products land in TMEM lanes that are never read).
-constexpr uint32_t OFF_PK = 0;                          // phi(K)^T: M=feature, K=token, MN-major
-constexpr uint32_t OFF_PQ = OFF_PK + KF * C * 2;        // phi(Q):   M=token, K=feature, K-major
-constexpr uint32_t OFF_A = OFF_PQ + C * KF * 2;         // A:        M=token i, K=token j, K-major
-constexpr uint32_t OFF_VA = OFF_A + C * C * 2;          // [V|1]:    N=column, K=token, MN-major
-constexpr uint32_t OFF_SB = OFF_VA + C * NV * 2;        // [S|z]:    N=column, K=feature, MN-major
-constexpr uint32_t OFF_Q = OFF_SB + KF * NV * 2;        // Q:        M=token, K=d', K-major
-constexpr uint32_t OFF_K = OFF_Q + C * DF * 2;          // K:        N=token, K=d', K-major
-constexpr uint32_t OFF_S1 = OFF_K + C * DF * 2;         // fp32 state rows 128..159 (warp 4)
-constexpr uint32_t OFF_BAR = OFF_S1 + 32 * NV * 4;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 128;
-static_assert(OFF_PK + (2 * C / 8 - 1) * 128 + (C / 8 - 1) * (KF / 8) * 128 + 128 <= SMEM_BYTES,
+// Shared memory map (bytes); [b] tiles are double-buffered by chunk parity.
+// MMA4's second 128-row tile of phi(K)^T reads feature rows 128..255 of which
+// only 128..159 exist; the rows beyond alias the next region (their products
+// land in TMEM lanes that are never read).
+constexpr uint32_t PK_BYTES = KF * C * 2;
+constexpr uint32_t VA_BYTES = C * NV * 2;
+constexpr uint32_t QK_BYTES = C * DF * 2;
+constexpr uint32_t OFF_PK = 0;                                  // [2] phi(K)^T: M=feature, K=token, MN-major
+constexpr uint32_t OFF_VA = OFF_PK + 2 * PK_BYTES;              // [2] [V|1]: N=column, K=token, MN-major
+constexpr uint32_t OFF_Q = OFF_VA + 2 * VA_BYTES;               // [2] Q: M=token, K=d', K-major
+constexpr uint32_t OFF_K = OFF_Q + 2 * QK_BYTES;                // [2] K: N=token, K=d', K-major
+constexpr uint32_t OFF_A = OFF_K + 2 * QK_BYTES;                // A: M=token i, K=token j, K-major
+constexpr uint32_t SB_BYTES = KF * NV * 2;
+constexpr uint32_t OFF_SB = OFF_A + C * C * 2;                  // [2] [S|z] bf16: N=column, K=feature, MN-major
+constexpr uint32_t OFF_BAR = OFF_SB + 2 * SB_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
+static_assert(OFF_PK + PK_BYTES + (2 * C / 8 - 1) * 128 + (C / 8 - 1) * (KF / 8) * 128 + 128 <= SMEM_BYTES,
               "second update tile must stay inside shared memory");
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
 // Core-matrix strides (bytes) of each operand: {K direction, M/N direction}.
 constexpr uint32_t PK_LBO = (KF / 8) * 128, PK_SBO = 128;
-constexpr uint32_t PQ_LBO = 128, PQ_SBO = (KF / 8) * 128;
 constexpr uint32_t A_LBO = 128, A_SBO = (C / 8) * 128;
 constexpr uint32_t VA_LBO = (NV / 8) * 128, VA_SBO = 128;
 constexpr uint32_t SB_LBO = (NV / 8) * 128, SB_SBO = 128;
 constexpr uint32_t QK_LBO = 128, QK_SBO = (DF / 8) * 128;
 
-// TMEM columns.
-constexpr uint32_t COL_S = 0;      // s = Q K^T, 128 columns
-constexpr uint32_t COL_Y = 128;    // Y, 80 columns
-constexpr uint32_t COL_D0 = 256;   // dS rows 0..127, 80 columns
-constexpr uint32_t COL_D1 = 384;   // dS rows 128..255, 80 columns
+// TMEM columns (all regions start on a multiple of 32).
+constexpr uint32_t COL_S = 0;      // s = Q K^T, 128 fp32 columns
+constexpr uint32_t COL_Y = 128;    // Y, 80 fp32 columns
+constexpr uint32_t COL_PQ = 224;   // phi(Q), 160 bf16 = 80 columns
+constexpr uint32_t COL_D0 = 320;   // [S|z] rows 0..127, 80 fp32 columns
+constexpr uint32_t COL_D1 = 416;   // [S|z] rows 128..255, 80 fp32 columns
 constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t ID_QK = idesc_bf16_f32(128, 128, false, false);
@@ -91,7 +105,22 @@ constexpr uint32_t ID_AV = idesc_bf16_f32(128, NV, false, true);
 constexpr uint32_t ID_UPD = idesc_bf16_f32(128, NV, true, true);
 constexpr uint32_t ID_INT = idesc_bf16_f32(128, NV, false, true);
 
-enum { BAR_IN, BAR_S, BAR_A, BAR_Y, BAR_SB, NUM_BARS };
+// Barriers: IN/FREE per shared-memory buffer, the rest once per chunk.
+enum {
+    BAR_IN0, BAR_IN1,        // producers -> MMA: Q, K, [V|1], phi(K)^T of a chunk are in buffer b
+    BAR_FREE0, BAR_FREE1,    // MMA commit: every MMA reading buffer b has completed
+    BAR_PQIN,                // producers -> MMA: phi(Q) is in TMEM
+    BAR_PQF,                 // MMA commit: MMA3 done (phi(Q) free)
+    BAR_SBF0, BAR_SBF1,      // MMA commit: MMA3 done reading [S|z] bf16 buffer b
+    BAR_S,                   // MMA commit: s ready
+    BAR_A,                   // epilogue warps -> MMA: A written
+    BAR_DS,                  // MMA commit: MMA4 done, [S|z] in TMEM is the state after chunk c
+    BAR_DSF,                 // state readers -> MMA: [S|z] read from TMEM
+    BAR_SBR,                 // state readers -> MMA: [S|z] bf16 written
+    BAR_Y,                   // MMA commit: Y complete
+    BAR_YF,                  // epilogue warps -> MMA: Y read
+    NUM_BARS
+};
 
 // Emit phi_sym(x) as 20 packed 16-byte pieces of 8 features, in feature order
 // [1, x_0..x_15, x_a x_b (a <= b, a-major; x_a^2 carries 1/sqrt2), 0 x 7].
@@ -134,10 +163,91 @@ __device__ __forceinline__ void pair_of(int p, int& a, int& b) {
     b = a + p;
 }
 
+
+// Feature rows of the final state: folded row f maps to one or two rows of the
+// 1 + d' + d'^2 layout (off-diagonal pairs are split evenly, each times 1/sqrt2).
+__device__ __forceinline__ void write_state_row(float* S, float* z, size_t bh, int f, const float* Sr) {
+    if (f >= DS) return;
+    int rows[2], nrows = 1;
+    float coef = 1.0f;
+    if (f <= DF) {
+        rows[0] = f;
+    } else {
+        int a, b;
+        pair_of(f - 1 - DF, a, b);
+        rows[0] = 1 + DF + a * DF + b;
+        if (a != b) { rows[1] = 1 + DF + b * DF + a; nrows = 2; coef = kSqrtHalf; }
+    }
+    for (int i = 0; i < nrows; ++i) {
+        float4* dst = reinterpret_cast<float4*>(S + (bh * feature_dim(DF) + rows[i]) * DV);
+#pragma unroll
+        for (int j = 0; j < DV / 4; ++j)
+            dst[j] = make_float4(Sr[4 * j] * coef, Sr[4 * j + 1] * coef, Sr[4 * j + 2] * coef, Sr[4 * j + 3] * coef);
+        z[bh * feature_dim(DF) + rows[i]] = Sr[DV] * coef;
+    }
+}
+
+// After MMA4 of chunk c: read one 80-column state row (fp32, TMEM lane of the
+// calling thread) in a single batch, release it to MMA4 of chunk c+1, then
+// publish it as bf16 row f of [S|z] buffer c&1 for MMA3 of chunk c+1 -- or, after
+// the last chunk, write it out as the final state. Whole-warp call.
+__device__ __forceinline__ bool publish_state(int c, int nchunks, int f, uint32_t taddr, uint64_t* bars,
+                                              uint32_t sbase, volatile int* abort_flag, unsigned* status,
+                                              float* S, float* z, size_t bh) {
+    if (!mbar_wait(&bars[BAR_DS], c & 1, abort_flag, status)) return false;
+    tc_fence_after();
+    float r[NV];
+#pragma unroll
+    for (int m = 0; m < NV / 16; ++m) tmem_ld16(taddr + 16 * m, r + 16 * m);
+    tmem_ld_wait();
+    tc_fence_before();
+    mbar_arrive(&bars[BAR_DSF]);
+    if (c + 1 < nchunks) {
+        const int b = c & 1;
+        // buffer b last held the state read by MMA3 of chunk c-1
+        if (c >= 2 && !mbar_wait(&bars[BAR_SBF0 + b], ((c >> 1) - 1) & 1, abort_flag, status)) return false;
+        const uint32_t row = sbase + OFF_SB + b * SB_BYTES + (f & 7) * 16 + (f >> 3) * SB_LBO;
+        const bool real = f < DS;
+#pragma unroll
+        for (int j = 0; j < NV / 8; ++j) {
+            float t8[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t8[e] = real ? r[8 * j + e] : 0.f;
+            st_shared_v4(row + j * SB_SBO, pack_bf16x8(t8));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&bars[BAR_SBR]);
+    } else if (S != nullptr && !*abort_flag) {
+        write_state_row(S, z, bh, f, r);
+    }
+    return true;
+}
+
+struct Raw {          // one token's inputs: q, k (2 x 16 B each), v (8 x 16 B)
+    uint4 q[2], k[2], v[8];
+};
+
+__device__ __forceinline__ void load_token(Raw& r, const __nv_bfloat16* q, const __nv_bfloat16* k,
+                                           const __nv_bfloat16* v, size_t row, bool valid) {
+    if (valid) {
+        const uint4* qp = reinterpret_cast<const uint4*>(q + row * DF);
+        const uint4* kp = reinterpret_cast<const uint4*>(k + row * DF);
+        const uint4* vp = reinterpret_cast<const uint4*>(v + row * DV);
+        r.q[0] = __ldg(qp); r.q[1] = __ldg(qp + 1);
+        r.k[0] = __ldg(kp); r.k[1] = __ldg(kp + 1);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r.v[i] = __ldg(vp + i);
+    } else {
+        r.q[0] = r.q[1] = r.k[0] = r.k[1] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) r.v[i] = make_uint4(0, 0, 0, 0);
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
-                     float* __restrict__ S, float* __restrict__ z, int N, unsigned* status) {
+                     float* __restrict__ S, float* __restrict__ z, int N, unsigned* status, unsigned debug) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * NUM_BARS);
@@ -151,117 +261,153 @@ la_prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     const int nchunks = (N + C - 1) / C;
 
     if (tid == 0) {
-        mbar_init(&bars[BAR_IN], 128);
-        mbar_init(&bars[BAR_S], 1);
-        mbar_init(&bars[BAR_A], 128);
-        mbar_init(&bars[BAR_Y], 1);
-        mbar_init(&bars[BAR_SB], 128);
+        for (int i = 0; i < NUM_BARS; ++i) {
+            const bool per_warpgroup = i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A || i == BAR_YF;
+            const bool state = i == BAR_DSF || i == BAR_SBR;          // warps 4-7 plus warp 8
+            mbar_init(&bars[i], per_warpgroup ? 128 : state ? 160 : 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 8) tmem_alloc(tmem_base_slot, TMEM_COLS);
+    if (warp == 12) tmem_alloc(tmem_base_slot, TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
 
     if (warp < 4) {
-        // ------------------------------------------------------------ token threads
+        // ------------------------------------------------------------ producers
         const int t = tid;                                   // token within chunk == TMEM lane
         const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
         const uint32_t cm = (t & 7) * 16;                    // row within a core matrix
+        Raw nxt;
+        load_token(nxt, q, k, v, bh * (size_t)N + t, t < N);
         for (int c = 0; c < nchunks; ++c) {
+            const int b = c & 1;
             const int t0 = c * C;
-            const int nv = min(C, N - t0);
-            const bool valid = t < nv;
-            const size_t row = bh * (size_t)N + t0 + t;
-            uint4 qr[2], kr[2], vr[8];
-            if (valid) {
-                const uint4* qp = reinterpret_cast<const uint4*>(q + row * DF);
-                const uint4* kp = reinterpret_cast<const uint4*>(k + row * DF);
-                const uint4* vp = reinterpret_cast<const uint4*>(v + row * DV);
-                qr[0] = __ldg(qp); qr[1] = __ldg(qp + 1);
-                kr[0] = __ldg(kp); kr[1] = __ldg(kp + 1);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) vr[i] = __ldg(vp + i);
-            } else {
-                qr[0] = qr[1] = kr[0] = kr[1] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-                for (int i = 0; i < 8; ++i) vr[i] = make_uint4(0, 0, 0, 0);
+            const bool valid = t < min(C, N - t0);
+            const Raw cur = nxt;
+            if (c + 1 < nchunks) {
+                const int tn = t0 + C + t;
+                load_token(nxt, q, k, v, bh * (size_t)N + tn, tn < N);
             }
-            // Q, K tiles (K-major, 2 core matrices along d')
-            const uint32_t qk_off = cm + (t >> 3) * QK_SBO;
-            st_shared_v4(sbase + OFF_Q + qk_off, qr[0]);
-            st_shared_v4(sbase + OFF_Q + qk_off + QK_LBO, qr[1]);
-            st_shared_v4(sbase + OFF_K + qk_off, kr[0]);
-            st_shared_v4(sbase + OFF_K + qk_off + QK_LBO, kr[1]);
-            // [V | 1] (MN-major: 16-byte piece = 8 columns of token t)
-            const uint32_t va_off = OFF_VA + cm + (t >> 3) * VA_LBO;
+            if (c >= 2 && !mbar_wait(&bars[BAR_FREE0 + b], ((c >> 1) - 1) & 1, abort_flag, status)) break;
+            // [V | 1] (MN-major: a 16-byte piece is 8 columns of token t)
+            const uint32_t va = sbase + OFF_VA + b * VA_BYTES + cm + (t >> 3) * VA_LBO;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) st_shared_v4(sbase + va_off + i * VA_SBO, vr[i]);
-            st_shared_v4(sbase + va_off + 8 * VA_SBO,
-                         make_uint4(valid ? 0x3F80u : 0u, 0u, 0u, 0u));   // bf16 1.0 in column 64
-            st_shared_v4(sbase + va_off + 9 * VA_SBO, make_uint4(0, 0, 0, 0));
-            // phi(Q) (K-major rows) and phi(K)^T (MN-major columns); padded tokens get phi(k) = 0
-            float xq[DF], xk[DF];
-            unpack_bf16x8(qr[0], xq);
-            unpack_bf16x8(qr[1], xq + 8);
-            unpack_bf16x8(kr[0], xk);
-            unpack_bf16x8(kr[1], xk + 8);
-            const uint32_t pq_off = OFF_PQ + cm + (t >> 3) * PQ_SBO;
-            emit_phi(xq, [&](int j, uint4 u) { st_shared_v4(sbase + pq_off + j * PQ_LBO, u); });
-            const uint32_t pk_off = OFF_PK + cm + (t >> 3) * PK_LBO;
+            for (int i = 0; i < 8; ++i) st_shared_v4(va + i * VA_SBO, cur.v[i]);
+            st_shared_v4(va + 8 * VA_SBO, make_uint4(valid ? 0x3F80u : 0u, 0u, 0u, 0u));  // bf16 1.0, column 64
+            st_shared_v4(va + 9 * VA_SBO, make_uint4(0, 0, 0, 0));
+            // Q, K (K-major, 2 core matrices along d')
+            const uint32_t qk = cm + (t >> 3) * QK_SBO + b * QK_BYTES;
+            st_shared_v4(sbase + OFF_Q + qk, cur.q[0]);
+            st_shared_v4(sbase + OFF_Q + qk + QK_LBO, cur.q[1]);
+            st_shared_v4(sbase + OFF_K + qk, cur.k[0]);
+            st_shared_v4(sbase + OFF_K + qk + QK_LBO, cur.k[1]);
+            // phi(K)^T (MN-major columns); padded tokens contribute nothing
+            const uint32_t pk = sbase + OFF_PK + b * PK_BYTES + cm + (t >> 3) * PK_LBO;
             if (valid) {
-                emit_phi(xk, [&](int j, uint4 u) { st_shared_v4(sbase + pk_off + j * PK_SBO, u); });
+                float xk[DF];
+                unpack_bf16x8(cur.k[0], xk);
+                unpack_bf16x8(cur.k[1], xk + 8);
+                emit_phi(xk, [&](int j, uint4 u) { st_shared_v4(pk + j * PK_SBO, u); });
             } else {
 #pragma unroll
-                for (int j = 0; j < KF / 8; ++j) st_shared_v4(sbase + pk_off + j * PK_SBO, make_uint4(0, 0, 0, 0));
+                for (int j = 0; j < KF / 8; ++j) st_shared_v4(pk + j * PK_SBO, make_uint4(0, 0, 0, 0));
             }
             fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[BAR_IN]);
+            mbar_arrive(&bars[BAR_IN0 + b]);
 
-            // s -> A (rows of s live in this thread's TMEM lane)
+            // phi(Q) -> TMEM lane t, once MMA3 of the previous chunk has read it
+            float xq[DF];
+            unpack_bf16x8(cur.q[0], xq);
+            unpack_bf16x8(cur.q[1], xq + 8);
+            if (c >= 1 && !mbar_wait(&bars[BAR_PQF], (c - 1) & 1, abort_flag, status)) break;
+            tc_fence_after();
+            uint32_t pkt[16];
+            emit_phi(xq, [&](int j, uint4 u) {
+                pkt[(j & 3) * 4 + 0] = u.x;
+                pkt[(j & 3) * 4 + 1] = u.y;
+                pkt[(j & 3) * 4 + 2] = u.z;
+                pkt[(j & 3) * 4 + 3] = u.w;
+                if ((j & 3) == 3) tmem_st16(lane_base + COL_PQ + (j >> 2) * 16, pkt);
+            });
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_PQIN]);
+        }
+    } else if (warp < 8) {
+        // ------------------------------------------------------------ state rows 0..127
+        const int f = (warp - 4) * 32 + lane;                // folded feature row == TMEM lane
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp - 4) * 32) << 16);
+        for (int c = 0; c < nchunks; ++c) {
+            if (!publish_state(c, nchunks, f, lane_base + COL_D0, bars, sbase, abort_flag, status, S, z, bh)) break;
+        }
+    } else if (warp < 12) {
+        // ------------------------------------------------------------ intra + epilogue
+        const int wq = warp - 8;
+        const int t = wq * 32 + lane;                        // token within chunk == TMEM lane
+        const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+        const uint32_t a_off = OFF_A + (t & 7) * 16 + (t >> 3) * A_SBO;
+        for (int c = 0; c < nchunks; ++c) {
             if (!mbar_wait(&bars[BAR_S], c & 1, abort_flag, status)) break;
             tc_fence_after();
-            const uint32_t a_off = OFF_A + cm + (t >> 3) * A_SBO;
+            // Row t of A: columns above the warp's diagonal block are zero; the rest
+            // come from TMEM in at most two batches of 64 columns.
 #pragma unroll
-            for (int b = 0; b < C / 32; ++b) {
-                if (b > warp) {                              // whole 32-column block above the diagonal
+            for (int half = 0; half < 2; ++half) {
+                if (2 * half > wq) {
 #pragma unroll
-                    for (int j = 0; j < 4; ++j) st_shared_v4(sbase + a_off + (4 * b + j) * A_LBO, make_uint4(0, 0, 0, 0));
+                    for (int j = 0; j < 8; ++j)
+                        st_shared_v4(sbase + a_off + (8 * half + j) * A_LBO, make_uint4(0, 0, 0, 0));
                     continue;
                 }
-                float s[32];
-                tmem_ld16(lane_base + COL_S + 32 * b, s);
-                tmem_ld16(lane_base + COL_S + 32 * b + 16, s + 16);
+                const bool two = 2 * half + 1 <= wq;         // second 32-column block also needed
+                float s[64];
+#pragma unroll
+                for (int m = 0; m < 2; ++m) tmem_ld16(lane_base + COL_S + 64 * half + 16 * m, s + 16 * m);
+                if (two) {
+#pragma unroll
+                    for (int m = 2; m < 4; ++m) tmem_ld16(lane_base + COL_S + 64 * half + 16 * m, s + 16 * m);
+                }
                 tmem_ld_wait();
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
+                for (int j = 0; j < 8; ++j) {
+                    if (j >= 4 && !two) {
+                        st_shared_v4(sbase + a_off + (8 * half + j) * A_LBO, make_uint4(0, 0, 0, 0));
+                        continue;
+                    }
                     float a8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int col = 32 * b + 8 * j + e;
+                        const int col = 64 * half + 8 * j + e;
                         const float sv = s[8 * j + e];
                         a8[e] = col <= t ? fmaf(sv, fmaf(0.5f, sv, 1.0f), 1.0f) : 0.0f;
                     }
-                    st_shared_v4(sbase + a_off + (4 * b + j) * A_LBO, pack_bf16x8(a8));
+                    st_shared_v4(sbase + a_off + (8 * half + j) * A_LBO, pack_bf16x8(a8));
                 }
             }
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&bars[BAR_A]);
 
-            // y = Y[:, :64] / Y[:, 64]
+            // state rows 128..159 (TMEM lanes 0..31 of the second tile): warp 8
+            if (wq == 0 &&
+                !publish_state(c, nchunks, 128 + lane, lane_base + COL_D1, bars, sbase, abort_flag, status, S, z, bh))
+                break;
+
             if (!mbar_wait(&bars[BAR_Y], c & 1, abort_flag, status)) break;
             tc_fence_after();
             float yv[NV];
 #pragma unroll
             for (int m = 0; m < NV / 16; ++m) tmem_ld16(lane_base + COL_Y + 16 * m, yv + 16 * m);
             tmem_ld_wait();
-            if (valid) {
+            tc_fence_before();
+            mbar_arrive(&bars[BAR_YF]);
+            const int tok = c * C + t;
+            if (tok < N) {
                 const float inv = 1.0f / yv[DV];
-                uint4* yp = reinterpret_cast<uint4*>(y + row * DV);
+                uint4* yp = reinterpret_cast<uint4*>(y + (bh * (size_t)N + tok) * DV);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     float o[8];
@@ -270,138 +416,68 @@ la_prefill_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
                     yp[i] = pack_bf16x8(o);
                 }
             }
-            tc_fence_before();
-        }
-    } else if (warp < 8) {
-        // ------------------------------------------------------------ state threads
-        const int wq = warp - 4;
-        const int f0 = wq * 32 + lane;                       // feature row of tile 0
-        const bool has_tile1 = (wq == 0);                    // rows 128..159 live in lanes 0..31
-        const int f1 = 128 + lane;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-        float S0[NV];
-#pragma unroll
-        for (int i = 0; i < NV; ++i) S0[i] = 0.f;
-        // Rows 128..159 (folded features 128..152 plus zero padding) are few: they
-        // stay in shared memory, one 80-float row per lane of warp 4.
-        float* S1 = reinterpret_cast<float*>(smem + OFF_S1) + lane * NV;
-        if (has_tile1) {
-            for (int i = 0; i < NV; ++i) S1[i] = 0.f;
-        }
-        for (int c = 0; c < nchunks; ++c) {
-            if (!mbar_wait(&bars[BAR_Y], c & 1, abort_flag, status)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int m = 0; m < NV / 16; ++m) {
-                float d[16];
-                tmem_ld16(lane_base + COL_D0 + 16 * m, d);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) S0[16 * m + i] += d[i];
-            }
-            if (has_tile1) {
-#pragma unroll
-                for (int m = 0; m < NV / 16; ++m) {
-                    float d[16];
-                    tmem_ld16(lane_base + COL_D1 + 16 * m, d);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) S1[16 * m + i] += (f1 < DS) ? d[i] : 0.f;
-                }
-            }
-            if (c + 1 < nchunks) {
-                const uint32_t sb0 = sbase + OFF_SB + (f0 & 7) * 16 + (f0 >> 3) * SB_LBO;
-#pragma unroll
-                for (int j = 0; j < NV / 8; ++j) st_shared_v4(sb0 + j * SB_SBO, pack_bf16x8(S0 + 8 * j));
-                if (has_tile1) {
-                    const uint32_t sb1 = sbase + OFF_SB + (f1 & 7) * 16 + (f1 >> 3) * SB_LBO;
-#pragma unroll
-                    for (int j = 0; j < NV / 8; ++j) {
-                        float t8[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) t8[e] = S1[8 * j + e];
-                        st_shared_v4(sb1 + j * SB_SBO, pack_bf16x8(t8));
-                    }
-                }
-                fence_proxy_async_smem();
-            }
-            tc_fence_before();
-            mbar_arrive(&bars[BAR_SB]);
-        }
-        if (S != nullptr && !*abort_flag) {
-            // Expand the folded state to the 1 + d' + d'^2 row layout.
-            auto write_rows = [&](const float* Sr, int f) {
-                if (f >= DS) return;
-                int rows[2], nrows = 1;
-                float coef = 1.0f;
-                if (f <= DF) {
-                    rows[0] = f;
-                } else {
-                    int a, b;
-                    pair_of(f - 1 - DF, a, b);
-                    rows[0] = 1 + DF + a * DF + b;
-                    if (a != b) { rows[1] = 1 + DF + b * DF + a; nrows = 2; coef = kSqrtHalf; }
-                }
-                for (int i = 0; i < nrows; ++i) {
-                    float4* dst = reinterpret_cast<float4*>(S + (bh * feature_dim(DF) + rows[i]) * DV);
-#pragma unroll
-                    for (int j = 0; j < DV / 4; ++j)
-                        dst[j] = make_float4(Sr[4 * j] * coef, Sr[4 * j + 1] * coef, Sr[4 * j + 2] * coef,
-                                             Sr[4 * j + 3] * coef);
-                    z[bh * feature_dim(DF) + rows[i]] = Sr[DV] * coef;
-                }
-            };
-            write_rows(S0, f0);
-            if (has_tile1) write_rows(S1, f1);
         }
     } else if (lane == 0) {
         // ------------------------------------------------------------ MMA issuer
-        const uint64_t dq = smem_desc(sbase + OFF_Q, QK_LBO, QK_SBO);
-        const uint64_t dk = smem_desc(sbase + OFF_K, QK_LBO, QK_SBO);
-        int issued = 0;
-        for (int c = 0; c < nchunks; ++c) {
-            if (!mbar_wait(&bars[BAR_IN], c & 1, abort_flag, status)) break;
+        int last_y = -1;
+        // testing: issue nothing, so every waiter times out
+        for (int c = 0; c < ((debug & DEBUG_SKIP_MMA) ? 0 : nchunks); ++c) {
+            const int b = c & 1;
+            if (!mbar_wait(&bars[BAR_IN0 + b], (c >> 1) & 1, abort_flag, status)) break;
             tc_fence_after();
-            mma_bf16(tmem + COL_S, dq, dk, ID_QK, 0);
+            // MMA1: s = Q K^T
+            mma_bf16(tmem + COL_S, smem_desc(sbase + OFF_Q + b * QK_BYTES, QK_LBO, QK_SBO),
+                     smem_desc(sbase + OFF_K + b * QK_BYTES, QK_LBO, QK_SBO), ID_QK, 0);
             mma_commit(&bars[BAR_S]);
-
-            if (!mbar_wait(&bars[BAR_A], c & 1, abort_flag, status)) break;
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < C / 16; ++j)
-                mma_bf16(tmem + COL_Y, smem_desc(sbase + OFF_A + j * 2 * A_LBO, A_LBO, A_SBO),
-                         smem_desc(sbase + OFF_VA + j * 2 * VA_LBO, VA_LBO, VA_SBO), ID_AV, j > 0);
-            if (c > 0) {                                     // state threads done with dS and [S|z] of c-1
-                if (!mbar_wait(&bars[BAR_SB], (c - 1) & 1, abort_flag, status)) break;
+            // MMA3: Y = phi(Q) [S|z]_{c-1}
+            if (!mbar_wait(&bars[BAR_PQIN], c & 1, abort_flag, status)) break;
+            if (c > 0) {
+                if (!mbar_wait(&bars[BAR_YF], (c - 1) & 1, abort_flag, status)) break;
+                if (!mbar_wait(&bars[BAR_SBR], (c - 1) & 1, abort_flag, status)) break;
                 tc_fence_after();
+                const uint32_t sb = sbase + OFF_SB + ((c - 1) & 1) * SB_BYTES;
+#pragma unroll
+                for (int j = 0; j < KF / 16; ++j)
+                    mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j,
+                                smem_desc(sb + j * 2 * SB_LBO, SB_LBO, SB_SBO), ID_INT, j > 0);
             }
+            mma_commit(&bars[BAR_PQF]);
+            if (c > 0) mma_commit(&bars[BAR_SBF0 + ((c - 1) & 1)]);
+            // MMA4: [S|z] += phi(K)^T [V|1], once the state readers are done with the previous state
+            if (c > 0 && !mbar_wait(&bars[BAR_DSF], (c - 1) & 1, abort_flag, status)) break;
+            tc_fence_after();
+            const uint32_t pk = sbase + OFF_PK + b * PK_BYTES;
+            const uint32_t va = sbase + OFF_VA + b * VA_BYTES;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
 #pragma unroll
                 for (int j = 0; j < C / 16; ++j)
                     mma_bf16(tmem + (r == 0 ? COL_D0 : COL_D1),
-                             smem_desc(sbase + OFF_PK + r * 16 * PK_SBO + j * 2 * PK_LBO, PK_LBO, PK_SBO),
-                             smem_desc(sbase + OFF_VA + j * 2 * VA_LBO, VA_LBO, VA_SBO), ID_UPD, j > 0);
+                             smem_desc(pk + r * 16 * PK_SBO + j * 2 * PK_LBO, PK_LBO, PK_SBO),
+                             smem_desc(va + j * 2 * VA_LBO, VA_LBO, VA_SBO), ID_UPD, (c > 0 || j > 0) ? 1u : 0u);
             }
-            if (c > 0) {
+            mma_commit(&bars[BAR_DS]);
+            // MMA2: Y += A [V|1]
+            if (!mbar_wait(&bars[BAR_A], c & 1, abort_flag, status)) break;
+            tc_fence_after();
 #pragma unroll
-                for (int j = 0; j < KF / 16; ++j)
-                    mma_bf16(tmem + COL_Y, smem_desc(sbase + OFF_PQ + j * 2 * PQ_LBO, PQ_LBO, PQ_SBO),
-                             smem_desc(sbase + OFF_SB + j * 2 * SB_LBO, SB_LBO, SB_SBO), ID_INT, 1);
-            }
+            for (int j = 0; j < C / 16; ++j)
+                mma_bf16(tmem + COL_Y, smem_desc(sbase + OFF_A + j * 2 * A_LBO, A_LBO, A_SBO),
+                         smem_desc(va + j * 2 * VA_LBO, VA_LBO, VA_SBO), ID_AV, (c > 0 || j > 0) ? 1u : 0u);
             mma_commit(&bars[BAR_Y]);
-            issued = c + 1;
+            mma_commit(&bars[BAR_FREE0 + b]);
+            last_y = c;
         }
-        // Never free TMEM under an MMA still in flight: wait (bounded) for the last commit.
-        if (issued > 0 && *abort_flag) {
+        // Never free TMEM under an MMA still in flight: on abort, wait (bounded) for the last commit.
+        if (*abort_flag && last_y >= 0) {
             const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&bars[BAR_Y], (issued - 1) & 1) && global_ns() - t0 < kWaitLimitNs) {}
+            while (!mbar_try_wait(&bars[BAR_Y], last_y & 1) && global_ns() - t0 < kWaitLimitNs) {}
         }
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
@@ -424,7 +500,8 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
     if (e != cudaSuccess) return e;
     la_prefill_tc_kernel<<<a.B * a.H, kThreads, SMEM_BYTES, stream>>>(
         static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.k),
-        static_cast<const __nv_bfloat16*>(a.v), static_cast<__nv_bfloat16*>(a.y), a.S, a.z, a.N, a.status);
+        static_cast<const __nv_bfloat16*>(a.v), static_cast<__nv_bfloat16*>(a.y), a.S, a.z, a.N, a.status,
+        a.debug);
     return cudaGetLastError();
 }
 

@@ -7,16 +7,17 @@
 // kernels. Window convention: token i sees keys i - w < j <= i (w keys including
 // itself), which is what a w-slot ring holds after token i is written.
 //
-// Prefill (CUDA-core path): a CTA takes 64 consecutive queries of one head and
+// Prefill: bf16 inputs go to the tensor-core kernel (swa_tc.cu). The fp32
+// path below runs on the CUDA cores: a CTA takes 64 consecutive queries of one head and
 // stages those queries plus the 64 + w - 1 keys and values they can see in
 // shared memory (fp32), so every K/V row is read from global memory once per
 // tile. Four threads share a query, each owning 16 of the 64 dims: partial dot
 // products are combined with two butterfly shuffles and the softmax runs online
 // (running max and sum, rescaling the accumulator), in fp32 with expf.
 //
-// Decode: one CTA per (b, h). The new key/value go to slot t mod w; thread j
-// scores slot j, the CTA reduces max and sum, then thread e accumulates output
-// dim e over the valid slots (coalesced over e).
+// Decode: one CTA per (b, h); the new key/value go to slot t mod w. bf16 uses
+// 16-byte loads (see swa_decode_bf16_kernel); the fp32 kernel scores slot j on
+// thread j, reduces max and sum, then accumulates output dim e on thread e.
 #include <math.h>
 
 #include "common.cuh"
@@ -192,30 +193,141 @@ swa_decode_kernel(T* __restrict__ kc, T* __restrict__ vc, long long t, const T* 
 
 template <typename T>
 cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void* k_cache,
-                      void* v_cache, int B, int H, int N, int w, float scale, cudaStream_t stream) {
-    constexpr size_t smem = (size_t)(kQTile * kHead + 2 * (kQTile + kMaxW - 1) * kHead) * sizeof(float);
-    auto kern = swa_prefill_simt_kernel<T>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const dim3 grid((N + kQTile - 1) / kQTile, B * H);
-    kern<<<grid, 256, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
-                                     static_cast<const T*>(v), static_cast<T*>(y), N, w, scale);
-    e = cudaGetLastError();
-    if (e != cudaSuccess || k_cache == nullptr) return e;
-    swa_fill_ring_kernel<T><<<B * H, 256, 0, stream>>>(static_cast<const T*>(k), static_cast<const T*>(v),
-                                                      static_cast<T*>(k_cache), static_cast<T*>(v_cache), N, w);
-    return cudaGetLastError();
+                      void* v_cache, int B, int H, int N, int w, float scale, unsigned* status,
+                      unsigned debug, cudaStream_t stream) {
+    if constexpr (sizeof(T) == 2) {
+        return launch_swa_prefill_tc(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, status, debug, stream);
+    } else {
+        constexpr size_t smem = (size_t)(kQTile * kHead + 2 * (kQTile + kMaxW - 1) * kHead) * sizeof(float);
+        auto kern = swa_prefill_simt_kernel<T>;
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        const dim3 grid((N + kQTile - 1) / kQTile, B * H);
+        kern<<<grid, 256, smem, stream>>>(static_cast<const T*>(q), static_cast<const T*>(k),
+                                         static_cast<const T*>(v), static_cast<T*>(y), N, w, scale);
+        e = cudaGetLastError();
+        if (e != cudaSuccess || k_cache == nullptr) return e;
+        swa_fill_ring_kernel<T><<<B * H, 256, 0, stream>>>(static_cast<const T*>(k), static_cast<const T*>(v),
+                                                          static_cast<T*>(k_cache), static_cast<T*>(v_cache), N, w);
+        return cudaGetLastError();
+    }
+}
+
+// bf16 decode: 128 threads per (b, h). Scores: eight lanes share a slot, each
+// taking one 16-byte piece of its 64-dim key (a warp scores four slots at a
+// time), combined by shuffles within the eight-lane group. Output: thread
+// (piece c, group g) sums slots g, g+16, g+32, g+48 for dims 8c..8c+7; the 16
+// groups' partial sums are then added through shared memory.
+__global__ void __launch_bounds__(128)
+swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
+                       const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                       const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, float scale) {
+    __shared__ float s_p[kMaxW];
+    __shared__ float s_part[16][kHead];
+    __shared__ uint4 s_new[2][8];           // new key / value, 8 pieces each
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const size_t bh = blockIdx.x;
+    const int new_slot = (int)(t % w);
+    if (tid < 16) {
+        const uint4* src = reinterpret_cast<const uint4*>((tid < 8 ? k : v) + bh * kHead) + (tid & 7);
+        const uint4 u = __ldg(src);
+        s_new[tid >> 3][tid & 7] = u;
+        reinterpret_cast<uint4*>((tid < 8 ? kc : vc) + (bh * w + new_slot) * kHead)[tid & 7] = u;
+    }
+    const int c = lane & 7;                  // 16-byte piece of a row: dims 8c..8c+7
+    float qv[8];
+    {
+        const uint4 u = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
+        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            qv[2 * e] = __uint_as_float(wd[e] << 16) * scale;
+            qv[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u) * scale;
+        }
+    }
+    __syncthreads();
+    // scores: pass p covers slots 16p .. 16p+15; warp `warp` takes 4 of them
+#pragma unroll
+    for (int pass = 0; pass < kMaxW / 16; ++pass) {
+        const int slot = pass * 16 + warp * 4 + (lane >> 3);
+        float part = 0.f;
+        bool valid = false;
+        if (slot < w) {
+            const long long u = t - ((((t - slot) % w) + w) % w);   // newest token held by the slot
+            valid = u >= 0;
+            if (valid) {
+                const uint4 kr = slot == new_slot ? s_new[0][c]
+                                                  : __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
+                const uint32_t wd[4] = {kr.x, kr.y, kr.z, kr.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    part = fmaf(qv[2 * e], __uint_as_float(wd[e] << 16), part);
+                    part = fmaf(qv[2 * e + 1], __uint_as_float(wd[e] & 0xFFFF0000u), part);
+                }
+            }
+        }
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        if (c == 0) s_p[slot] = valid ? part : -INFINITY;
+    }
+    __syncthreads();
+    if (warp == 0) {
+        const float a = s_p[lane], b = s_p[lane + 32];
+        float m = fmaxf(a, b);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        const float pa = a == -INFINITY ? 0.f : expf(a - m);
+        const float pb = b == -INFINITY ? 0.f : expf(b - m);
+        float sum = pa + pb;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        const float inv = 1.f / sum;
+        s_p[lane] = pa * inv;
+        s_p[lane + 32] = pb * inv;
+    }
+    __syncthreads();
+    {
+        const int g = tid >> 3;              // slot group 0..15
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+        for (int r = 0; r < kMaxW / 16; ++r) {
+            const int slot = g + 16 * r;
+            const float p = slot < w ? s_p[slot] : 0.f;
+            if (p != 0.f) {
+                const uint4 vr = slot == new_slot ? s_new[1][c]
+                                                  : __ldg(reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead) + c);
+                const uint32_t wd[4] = {vr.x, vr.y, vr.z, vr.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    acc[2 * e] = fmaf(p, __uint_as_float(wd[e] << 16), acc[2 * e]);
+                    acc[2 * e + 1] = fmaf(p, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_part[g][8 * c + e] = acc[e];
+    }
+    __syncthreads();
+    if (tid < kHead) {
+        float sum = 0.f;
+#pragma unroll
+        for (int g = 0; g < 16; ++g) sum += s_part[g][tid];
+        y[bh * kHead + tid] = __float2bfloat16_rn(sum);
+    }
 }
 
 }  // namespace
 
 cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y, void* k_cache,
                                void* v_cache, int B, int H, int N, int d, int w, float scale,
-                               bool bf16, unsigned* status, cudaStream_t stream) {
-    (void)status;
+                               bool bf16, unsigned* status, unsigned debug, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
-    return bf16 ? prefill_t<__nv_bfloat16>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, stream)
-                : prefill_t<float>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, stream);
+    return bf16 ? prefill_t<__nv_bfloat16>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, status, debug, stream)
+                : prefill_t<float>(q, k, v, y, k_cache, v_cache, B, H, N, w, scale, status, debug, stream);
 }
 
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
@@ -223,7 +335,7 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                               bool bf16, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
     if (bf16) {
-        swa_decode_kernel<__nv_bfloat16><<<B * H, kMaxW, 0, stream>>>(
+        swa_decode_bf16_kernel<<<B * H, 128, 0, stream>>>(
             static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), (long long)t,
             static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
             static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w, scale);

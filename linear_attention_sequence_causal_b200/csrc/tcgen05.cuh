@@ -171,3 +171,82 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
 
 }  // namespace tc
 }  // namespace based
+
+namespace based {
+namespace tc {
+
+// ------------------------------------------------------------------ 128-byte swizzled operands
+
+// Descriptor of a tile stored as 8-row x 128-byte atoms (1024 B, 1024-aligned)
+// with the 16-byte pieces of row r XOR-permuted by (r mod 8): the layout a TMA
+// load with 128-byte swizzle produces. K-major operands step along K inside the
+// 128-byte row by advancing `saddr`; `sbo` is the distance between 8-row atoms
+// along M/N (K-major) or along K (MN-major); `lbo` is the distance between atoms
+// along MN for MN-major operands wider than 64 bf16 (unused otherwise).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFFu) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;           // descriptor version for sm_100
+    d |= static_cast<uint64_t>(2) << 61;           // 128-byte swizzle
+    return d;
+}
+
+// Byte offset of 16-byte piece `chunk` (0..7) of row `row` inside a 128B-swizzled atom column.
+__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {
+    return row * 128u + ((chunk ^ (row & 7u)) << 4);
+}
+
+// ------------------------------------------------------------------ TMA
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+// 3-D tiled TMA load into shared memory, completing `bar`'s transaction count.
+// Coordinates: x innermost (elements), then y, z; y may be negative or past the
+// end (the box is zero-filled there); x must keep 16-byte alignment.
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint64_t* bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
+}  // namespace tc
+}  // namespace based
+
+namespace based {
+namespace tc {
+
+// D[tmem] (+)= A[tmem] * B[smem]: the A operand (M rows = TMEM lanes, K packed
+// two bf16 per 32-bit column, lower k in the low half) is read from tensor memory.
+__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns from registers: thread i writes lane (lane0 + i).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(
+            taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+}  // namespace tc
+}  // namespace based

@@ -1,0 +1,49 @@
+"""Failure detection on the GPU without a fault: a kernel whose bounded waits
+expire reports BASED_ERR_TIMEOUT through based_get_last_error, and the CUDA
+context stays usable for the next call.
+
+BASED_DEBUG_SKIP_MMA=1 makes the tensor-core kernels issue no MMA, so the
+waits on their completion barriers run out (after about two seconds); the
+kernels then free their tensor memory and return.
+"""
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import linear_attention_sequence_causal_b200 as based
+from linear_attention_sequence_causal_b200 import synthetic
+from parity_util import assert_y, to64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+TIMEOUT = 4
+
+
+def test_stalled_la_prefill_reports_timeout(monkeypatch):
+    import torch
+    inp = synthetic.la_inputs(1, 1, 300, 16, 64, "bf16", seed=3)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    monkeypatch.setenv("BASED_DEBUG_SKIP_MMA", "1")
+    based.la_prefill(q, k, v)                       # the launch itself succeeds
+    assert based.get_last_error() == TIMEOUT
+    assert based.get_last_error() == 0              # the word was cleared
+    monkeypatch.delenv("BASED_DEBUG_SKIP_MMA")
+    y, S, z = based.la_prefill(q, k, v)
+    assert based.get_last_error() == 0
+    assert_y(to64(y), oracle.la_quadratic(inp.q64, inp.k64, inp.v64), torch.bfloat16)
+
+
+def test_stalled_swa_prefill_reports_timeout(monkeypatch):
+    import torch
+    inp = synthetic.swa_inputs(1, 2, 200, 64, "bf16", seed=4)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    monkeypatch.setenv("BASED_DEBUG_SKIP_MMA", "1")
+    based.swa_prefill(q, k, v, w=64)
+    assert based.get_last_error() == TIMEOUT
+    monkeypatch.delenv("BASED_DEBUG_SKIP_MMA")
+    y, _, _ = based.swa_prefill(q, k, v, w=64)
+    assert based.get_last_error() == 0
+    assert_y(to64(y), oracle.swa(inp.q64, inp.k64, inp.v64, 64, 1 / math.sqrt(64)), torch.bfloat16)
