@@ -225,3 +225,33 @@ def test_decode_rejects_unsupported():
     with pytest.raises(based.BasedError) as e:
         based.la_decode_step(S, z, x, x, torch.zeros(1, 1, 64, device=DEV))
     assert e.value.status == 2
+
+
+# ------------------------------------------------------------ segments (few heads, long sequences)
+
+@pytest.mark.parametrize("B,H,N", [(1, 1, 300), (1, 2, 3000), (2, 3, 1000), (1, 1, 129)])
+def test_segmented_prefill_full(B, H, N):
+    """Few (b, h) pairs: each sequence is split into segments whose start states come
+    from a totals pass through the workspace; every output and the final state checked."""
+    inp = synthetic.la_inputs(B, H, N, 16, 64, "bf16", seed=N + H)
+    assert based.la_prefill_workspace(B, H, N, 16, 64) > 0 or N <= 128
+    y, S, z = _run_prefill(inp)
+    _check_full(inp, torch.bfloat16, y, S, z)
+
+
+def test_workspace_too_small_is_rejected():
+    import ctypes
+    from linear_attention_sequence_causal_b200 import binding
+    inp = synthetic.la_inputs(1, 2, 3000, 16, 64, "bf16", seed=1)
+    need = based.la_prefill_workspace(1, 2, 3000, 16, 64)
+    assert need > 0
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y = torch.empty(1, 2, 3000, 64, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(need, dtype=torch.uint8, device=DEV)
+    P = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = based.lib().based_la_prefill(P(q), P(k), P(v), P(y), None, None, 1, 2, 3000, 16, 64, binding.BF16, 0,
+                                      P(ws), need - 16, None)
+    assert st == binding.ERR_INVALID_ARG
+    st = based.lib().based_la_prefill(P(q), P(k), P(v), P(y), None, None, 1, 2, 3000, 16, 64, binding.BF16, 0,
+                                      None, 0, None)
+    assert st == binding.ERR_INVALID_ARG
