@@ -112,6 +112,34 @@ BASED_API size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int
                                   based_dtype_t dtype, int chunk);
 
 /*
+ * based_la_prefill_noalloc -- the same prefill as based_la_prefill, for callers
+ * that cannot allocate device memory themselves: code running inside a memory
+ * manager that owns every device buffer (a framework's caching allocator, a
+ * serving runtime with a fixed pool, a plugin host that hands out only its own
+ * tensors), or code on a latency-critical path where an allocation would stall
+ * the device. It takes no workspace: the segment totals live in one fixed
+ * 8 MiB array inside the library's device image, which every GPU that loads the
+ * library keeps until the process exits. The paper has no counterpart; this is
+ * a service of this library.
+ *
+ * Arguments, results and errors are those of based_la_prefill, minus the
+ * workspace. It calls no cudaMalloc, cudaFree or other allocating routine. It
+ * returns BASED_ERR_UNSUPPORTED when the call would need more scratch than the
+ * fixed array holds (not the case on a B200 for the shapes this library builds).
+ *
+ * The first call on a device looks up the array's device address with that
+ * device current, once per device; make that first call before any stream
+ * capture. All calls share the one array, which keeps the last call's contents
+ * (nothing in it needs to start at zero): calls that overlap on the GPU, for
+ * example on two streams at once, race on it and must be serialised by the caller.
+ */
+BASED_API based_status_t based_la_prefill_noalloc(const void* q, const void* k, const void* v, void* y,
+                                                  float* S, float* z,
+                                                  int B, int H, int N, int d_feat, int d_v,
+                                                  based_dtype_t dtype, int chunk,
+                                                  cudaStream_t stream);
+
+/*
  * based_la_decode_step -- recurrent (next-token) form: one generated token per
  * sequence. In place, for every (b, h):
  *     S += phi(k) v^T;  z += phi(k);  y = phi(q)^T S / phi(q)^T z

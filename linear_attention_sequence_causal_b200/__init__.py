@@ -12,6 +12,7 @@ from .binding import (  # noqa: F401
     get_last_error,
     la_decode_step,
     la_prefill,
+    la_prefill_noalloc,
     la_prefill_workspace,
     lib,
     library_path,

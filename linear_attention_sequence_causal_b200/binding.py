@@ -25,6 +25,7 @@ _DTYPES = {torch.float32: F32, torch.bfloat16: BF16}
 SYMBOLS = (
     "based_la_prefill",
     "based_la_prefill_workspace",
+    "based_la_prefill_noalloc",
     "based_la_decode_step",
     "based_swa_prefill",
     "based_swa_decode",
@@ -47,6 +48,8 @@ def _declare(lib):
     vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     lib.based_la_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
     lib.based_la_prefill.restype = i
+    lib.based_la_prefill_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp]
+    lib.based_la_prefill_noalloc.restype = i
     lib.based_la_prefill_workspace.argtypes = [i, i, i, i, i, i, i]
     lib.based_la_prefill_workspace.restype = sz
     lib.based_la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
@@ -152,6 +155,28 @@ def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None,
                                     B, H, N, d_feat, d_v, dt, chunk,
                                     _ptr(workspace) if ws_bytes else None, ws_bytes, _stream(dev))
     _check(st, "based_la_prefill")
+    return y, S, z
+
+
+def la_prefill_noalloc(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None, z=None):
+    """la_prefill without a workspace: the library's fixed device scratch is used
+    instead (for callers that must not allocate; calls must not overlap on the GPU)."""
+    dt = _dtype_code(q, k, v)
+    B, H, N, d_feat = q.shape
+    d_v = v.shape[-1]
+    D = feature_dim(d_feat)
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty((B, H, N, d_v), dtype=q.dtype, device=dev)
+        if want_state:
+            S = torch.empty((B, H, D, d_v), dtype=torch.float32, device=dev) if S is None else S
+            z = torch.empty((B, H, D), dtype=torch.float32, device=dev) if z is None else z
+        else:
+            S = z = None
+        st = lib().based_la_prefill_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z),
+                                            B, H, N, d_feat, d_v, dt, chunk, _stream(dev))
+    _check(st, "based_la_prefill_noalloc")
     return y, S, z
 
 

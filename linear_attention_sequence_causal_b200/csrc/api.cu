@@ -78,6 +78,22 @@ LaPath choose_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
 
 }  // namespace
 
+namespace based {
+
+// Lookups shared with the allocation-free prefill entry point (noalloc.cu).
+unsigned* device_status_word(int dev) { return status_word(dev); }
+int device_sm_count(int dev) { return num_sms(dev); }
+unsigned current_debug_flags() { return debug_flags(); }
+int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
+    switch (choose_la_path(d_feat, d_v, dtype, chunk)) {
+        case LaPath::TensorCore: return 2;
+        case LaPath::Simt: return 1;
+        default: return 0;
+    }
+}
+
+}  // namespace based
+
 extern "C" {
 
 int based_version(void) { return 100; }
