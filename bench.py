@@ -172,7 +172,8 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- distributed plumbing
 
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """Join the job launched by torchrun (one process per GPU); returns (rank, world, local rank)."""
     import torch
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -182,9 +183,12 @@ def dist_setup(n_gpus):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        timeout = datetime.timedelta(seconds=120)
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=timeout, device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=timeout)
     return rank, world, local
 
 
@@ -195,6 +199,7 @@ def barrier(world):
 
 
 def max_over_ranks(x, world, dev):
+    """The slowest rank's value (timing is the max over ranks)."""
     if world == 1:
         return x
     import torch
@@ -202,6 +207,16 @@ def max_over_ranks(x, world, dev):
     t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(rank, input_set):
+    """Seed of one rank's input set: every rank draws its own batch (weak scaling)."""
+    return 1000 * rank + input_set
+
+
+def whole_job_rate(world, units_per_step, steps, max_elapsed_ms):
+    """Units of all ranks per second over the slowest rank's time."""
+    return world * units_per_step * steps / (max_elapsed_ms / 1e3)
 
 
 # ---------------------------------------------------------------- the GPU arm
@@ -225,7 +240,7 @@ def run_mine(args):
     # sequence for the decode step.
     sets = []
     for s in range(N_INPUT_SETS):
-        seed = 1000 * rank + s
+        seed = rank_seed(rank, s)
         la = synthetic.la_inputs(B, H, N + 1, df, dv, "bf16", seed=seed)
         sw = synthetic.swa_inputs(B, Hs, N + 1, ds, "bf16", seed=seed + 500)
         d = {}
@@ -331,7 +346,7 @@ def run_mine(args):
     del graphs
 
     tokens_per_step = B * N + B
-    value = world * tokens_per_step * args.steps / (elapsed_ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, args.steps, elapsed_ms)
     ms_per_step = elapsed_ms / args.steps
 
     # ---- roofline of the dominant kernel (algorithmic work / measured launch time)
