@@ -274,35 +274,29 @@ def run_mine(args):
     launches_per_step = 1 + (1 if ws_bytes else 0) + 1 + 1 + 1
 
     # Eager warm-up (also the first use of each kernel), then one CUDA graph per
-    # API call and input set: replaying them keeps host launch overhead out of
-    # the device timeline of the small decode kernels.
+    # input set holding the whole step (the four API calls): replaying it keeps
+    # host launch overhead out of the device timeline of the small decode kernels.
     for i in range(args.warmup):
         for f in calls(sets[i % N_INPUT_SETS]):
             f()
     torch.cuda.synchronize(dev)
     if based.get_last_error(dev) != 0:
         raise SystemExit("device status error after warm-up")
-    graphs = []
     side = torch.cuda.Stream(dev)
-    for d in sets:
-        gs = []
-        for f in calls(d):
-            g = torch.cuda.CUDAGraph()
-            side.wait_stream(torch.cuda.current_stream(dev))
-            with torch.cuda.graph(g, stream=side):
-                f()
-            torch.cuda.current_stream(dev).wait_stream(side)
-            gs.append(g)
-        graphs.append(gs)
 
-    def step(i, ev=None):
-        gs = graphs[i % N_INPUT_SETS]
-        for j, g in enumerate(gs):
-            if ev is not None:
-                ev[j].record(stream)
-            g.replay()
-        if ev is not None:
-            ev[len(gs)].record(stream)
+    def capture(fns):
+        g = torch.cuda.CUDAGraph()
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.graph(g, stream=side):
+            for f in fns:
+                f()
+        torch.cuda.current_stream(dev).wait_stream(side)
+        return g
+
+    step_graphs = [capture(calls(d)) for d in sets]
+
+    def step(i):
+        step_graphs[i % N_INPUT_SETS].replay()
 
     for i in range(args.warmup):
         step(i)
@@ -324,26 +318,45 @@ def run_mine(args):
         i += 1
         if i % 64 == 0:
             torch.cuda.synchronize(dev)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize(dev)
     t_start.record(stream)
     for i in range(args.steps):
-        step(i, evs[i])
+        step(i)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
-    clk = clocks.stop()
-    clk["window"] = f"{args.preroll_s:.1f} s pre-roll of identical steps + the timed region"
     elapsed_ms = t_start.elapsed_time(t_end)
-    per_kernel = {name: sum(e[j].elapsed_time(e[j + 1]) for e in evs) / args.steps
-                  for j, name in enumerate(("la_prefill", "swa_prefill", "la_decode", "swa_decode"))}
     if based.get_last_error(dev) != 0:
         raise SystemExit("device status error in the timed region")
+
+    # Per-kernel launch durations: one graph per API call holding its launches
+    # over the rotated input sets, replayed back to back; CUDA events on the
+    # launching stream around the replays.
+    names = ("la_prefill", "swa_prefill", "la_decode", "swa_decode")
+    per_kernel = {}
+    reps = max(3, min(args.steps, 50))
+    for j, name in enumerate(names):
+        g = capture([calls(d)[j] for d in sets])
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        per_kernel[name] = a.elapsed_time(b) / (reps * N_INPUT_SETS)
+        del g
+    clk = clocks.stop()
+    clk["window"] = f"{args.preroll_s:.1f} s pre-roll of identical steps + the timed region + per-kernel replays"
+    if based.get_last_error(dev) != 0:
+        raise SystemExit("device status error in the per-kernel replays")
     elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
-    del graphs
+    del step_graphs
 
     tokens_per_step = B * N + B
     value = whole_job_rate(world, tokens_per_step, args.steps, elapsed_ms)

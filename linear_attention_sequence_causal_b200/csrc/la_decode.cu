@@ -7,17 +7,34 @@
 //
 // The step is bound by HBM: each (b, h) reads and writes its fp32 state once
 // (D x dv + D floats, 70 KB at d' = 16, dv = 64) while doing ~0.5 flop per byte.
-// One CTA streams one head's S with 128-bit loads and stores; consecutive
-// threads cover consecutive 16-byte pieces of a row, so a warp touches whole
-// row segments. phi(q) and phi(k) are formed once per CTA in shared memory and
-// never reach HBM. A head is never split across CTAs: z is updated in place and
-// every CTA that read it would race with the one writing it. Small batches get
-// larger CTAs (up to 1024 threads) instead, to keep enough loads in flight.
+//
+// Work split: a head's D feature rows are cut into P contiguous row ranges,
+// one CTA each, and the P CTAs of a head form one thread-block cluster
+// (P in {1, 2, 4, 8}, chosen so the grid covers every SM several times even at
+// batch 1). Rows of S and z are disjoint between the CTAs, so the in-place
+// update never races; each CTA produces a partial numerator phi(q)_rows . S_rows
+// (dv values) and a partial denominator phi(q)_rows . z_rows, and rank 0 of the
+// cluster sums the P partials through distributed shared memory and writes y.
+//
+// Streaming: a thread owns one 16-byte column group of every (kThreads / G)-th
+// row of its range. It issues the loads of a batch of kBatch rows before it
+// needs any of them, and the first batch is in flight before q, k and v have
+// even arrived, so the load latency overlaps the feature-map setup. phi(q) and
+// phi(k) are formed per row from q and k held in shared memory (two multiplies)
+// and never reach HBM.
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
 namespace based {
 namespace {
+
+namespace cg = cooperative_groups;
+
+constexpr int kThreads = 256;
+constexpr int kBatch = 8;        // rows in flight per thread
+constexpr int kMaxRanks = 8;     // portable cluster size
 
 template <int DF>
 __device__ __forceinline__ float phi_entry(const float* x, int f) {
@@ -27,102 +44,152 @@ __device__ __forceinline__ float phi_entry(const float* x, int f) {
     return (x[p / DF] * x[p % DF]) * kSqrtHalf;
 }
 
-template <typename T, int DF, int DV, int NT>
-__global__ void __launch_bounds__(NT)
+__device__ __forceinline__ void fma4(float4& acc, float s, const float4& x) {
+    acc.x = fmaf(s, x.x, acc.x);
+    acc.y = fmaf(s, x.y, acc.y);
+    acc.z = fmaf(s, x.z, acc.z);
+    acc.w = fmaf(s, x.w, acc.w);
+}
+
+template <typename T, int DF, int DV>
+__global__ void __launch_bounds__(kThreads)
 la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restrict__ q,
-                 const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y) {
+                 const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y, int P) {
     constexpr int D = feature_dim(DF);
-    constexpr int CW = DV;
-    constexpr int G = CW / 4;          // float4 pieces per row
-    constexpr int R = NT / G;          // rows in flight per sweep
-    constexpr int kThreads = NT;
-    static_assert(NT % G == 0 && NT >= CW, "thread layout");
+    constexpr int G = DV / 4;              // float4 column groups per row
+    constexpr int RPS = kThreads / G;      // rows per sweep of the CTA
+    constexpr int NW = kThreads / 32;
+    static_assert(kThreads % G == 0 && G <= 32 && 32 % G == 0, "thread layout");
 
     __shared__ float s_x[2][DF];
-    __shared__ float s_fq[D];
-    __shared__ float s_fk[D];
-    __shared__ float s_v[CW];
-    __shared__ float4 s_red[R][G];
-    __shared__ float s_dred[kThreads / 32];
+    __shared__ float s_v[DV];
+    __shared__ float4 s_red[NW][G];
+    __shared__ float s_dred[NW];
+    __shared__ float s_out[DV + 1];        // this CTA's partial numerator and denominator
 
     const int tid = threadIdx.x;
-    const size_t bh = blockIdx.x;
+    const int rank = (int)(blockIdx.x % (unsigned)P);
+    const size_t bh = blockIdx.x / (unsigned)P;
+    const int f0 = (rank * D) / P;
+    const int f1 = ((rank + 1) * D) / P;
+    const int g = tid % G;
+    const int r_thr = tid / G;
+
+    float* Sp = S + (bh * D) * (size_t)DV + 4 * g;
+
+    // First batch of state rows: in flight before anything else.
+    float4 buf[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+        const int f = f0 + r_thr + u * RPS;
+        if (f < f1) buf[u] = *reinterpret_cast<const float4*>(Sp + (size_t)f * DV);
+    }
 
     if (tid < DF) {
         s_x[0][tid] = to_f32(q[bh * DF + tid]);
         s_x[1][tid] = to_f32(k[bh * DF + tid]);
     }
-    if (tid < CW) s_v[tid] = to_f32(v[bh * DV + tid]);
-    __syncthreads();
-    for (int f = tid; f < D; f += kThreads) {
-        s_fq[f] = phi_entry<DF>(s_x[0], f);
-        s_fk[f] = phi_entry<DF>(s_x[1], f);
-    }
+    if (tid < DV) s_v[tid] = to_f32(v[bh * DV + tid]);
     __syncthreads();
 
-    // Denominator phi(q).z_new over all D features; z_new written back in place.
+    // Denominator part over this CTA's rows; z updated in place.
     float dpart = 0.f;
     float* zbh = z + bh * D;
-    for (int f = tid; f < D; f += kThreads) {
-        const float zn = zbh[f] + s_fk[f];
+    for (int f = f0 + tid; f < f1; f += kThreads) {
+        const float zn = zbh[f] + phi_entry<DF>(s_x[1], f);
         zbh[f] = zn;
-        dpart = fmaf(s_fq[f], zn, dpart);
+        dpart = fmaf(phi_entry<DF>(s_x[0], f), zn, dpart);
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, o);
-    if ((tid & 31) == 0) s_dred[tid >> 5] = dpart;
 
-    // Stream the state: one read, one write per element.
-    const int g = tid % G;
-    const int r0 = tid / G;
     const float4 vv = make_float4(s_v[4 * g], s_v[4 * g + 1], s_v[4 * g + 2], s_v[4 * g + 3]);
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    float* Sp = S + bh * (size_t)D * DV + 4 * g;
-#pragma unroll 4
-    for (int f = r0; f < D; f += R) {
-        float4* p = reinterpret_cast<float4*>(Sp + (size_t)f * DV);
-        float4 s = __ldcs(p);
-        const float kf = s_fk[f];
-        const float qf = s_fq[f];
-        s.x = fmaf(kf, vv.x, s.x);
-        s.y = fmaf(kf, vv.y, s.y);
-        s.z = fmaf(kf, vv.z, s.z);
-        s.w = fmaf(kf, vv.w, s.w);
-        __stcs(p, s);
-        acc.x = fmaf(qf, s.x, acc.x);
-        acc.y = fmaf(qf, s.y, acc.y);
-        acc.z = fmaf(qf, s.z, acc.z);
-        acc.w = fmaf(qf, s.w, acc.w);
+    for (int base = f0 + r_thr;; base += kBatch * RPS) {
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int f = base + u * RPS;
+            if (f < f1) {
+                float4 s = buf[u];
+                fma4(s, phi_entry<DF>(s_x[1], f), vv);
+                *reinterpret_cast<float4*>(Sp + (size_t)f * DV) = s;
+                fma4(acc, phi_entry<DF>(s_x[0], f), s);
+            }
+        }
+        const int next = base + kBatch * RPS;
+        if (next >= f1) break;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+            const int f = next + u * RPS;
+            if (f < f1) buf[u] = *reinterpret_cast<const float4*>(Sp + (size_t)f * DV);
+        }
     }
-    s_red[r0][g] = acc;
+
+    // CTA reduction: lanes of a warp that share a column group, then warps.
+    const int warp = tid >> 5, lane = tid & 31;
+#pragma unroll
+    for (int o = G; o < 32; o <<= 1) {
+        acc.x += __shfl_xor_sync(0xffffffffu, acc.x, o);
+        acc.y += __shfl_xor_sync(0xffffffffu, acc.y, o);
+        acc.z += __shfl_xor_sync(0xffffffffu, acc.z, o);
+        acc.w += __shfl_xor_sync(0xffffffffu, acc.w, o);
+    }
+    if (lane < G) s_red[warp][lane] = acc;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dpart += __shfl_xor_sync(0xffffffffu, dpart, o);
+    if (lane == 0) s_dred[warp] = dpart;
     __syncthreads();
-    if (tid < CW) {
+    if (tid < DV) {
+        float num = 0.f;
+#pragma unroll
+        for (int w = 0; w < NW; ++w) num += reinterpret_cast<const float*>(&s_red[w][tid >> 2])[tid & 3];
+        s_out[tid] = num;
+    } else if (tid == DV) {
         float den = 0.f;
 #pragma unroll
-        for (int i = 0; i < kThreads / 32; ++i) den += s_dred[i];
-        const int gg = tid >> 2, comp = tid & 3;
-        float num = 0.f;
-#pragma unroll 8
-        for (int r = 0; r < R; ++r) num += reinterpret_cast<const float*>(&s_red[r][gg])[comp];
+        for (int w = 0; w < NW; ++w) den += s_dred[w];
+        s_out[DV] = den;
+    }
+
+    // Cluster reduction through distributed shared memory; rank 0 writes y.
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster.sync();
+    if (rank == 0 && tid < DV) {
+        float num = 0.f, den = 0.f;
+        for (int r = 0; r < P; ++r) {
+            const float* o = cluster.map_shared_rank(s_out, r);
+            num += o[tid];
+            den += o[DV];
+        }
         y[bh * DV + tid] = from_f32<T>(num / den);
     }
+    cluster.sync();   // keep every rank's shared memory alive until rank 0 has read it
+}
+
+// Ranks per head: enough CTAs to cover every SM about four times, at least 16
+// rows per CTA, a power of two up to the portable cluster size.
+int ranks_per_head(int BH, int D, int num_sms) {
+    int P = 1;
+    while (P < kMaxRanks && (long long)BH * P < 4LL * num_sms && D / (2 * P) >= 16) P *= 2;
+    return P;
 }
 
 template <typename T, int DF, int DV>
 cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const void* v, void* y,
                          int BH, int num_sms, cudaStream_t stream) {
-    auto qq = static_cast<const T*>(q);
-    auto kk = static_cast<const T*>(k);
-    auto vv = static_cast<const T*>(v);
-    auto yy = static_cast<T*>(y);
-    // One CTA per head; fewer heads than ~2 waves of SMs get wider CTAs.
-    if ((long long)BH >= 2LL * num_sms)
-        la_decode_kernel<T, DF, DV, 256><<<BH, 256, 0, stream>>>(S, z, qq, kk, vv, yy);
-    else if ((long long)BH >= num_sms / 2)
-        la_decode_kernel<T, DF, DV, 512><<<BH, 512, 0, stream>>>(S, z, qq, kk, vv, yy);
-    else
-        la_decode_kernel<T, DF, DV, 1024><<<BH, 1024, 0, stream>>>(S, z, qq, kk, vv, yy);
-    return cudaGetLastError();
+    const int P = ranks_per_head(BH, feature_dim(DF), num_sms);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)BH * P);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = P;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV>, S, z, static_cast<const T*>(q),
+                              static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), P);
 }
 
 template <typename T>

@@ -30,6 +30,12 @@ constexpr int kQTile = 64;
 constexpr int kHead = 64;        // head dim d
 constexpr int kMaxW = 64;
 
+// Two floats as a bf16x2 word (round to nearest even), low half first.
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256)
 swa_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -213,110 +219,119 @@ cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void
     }
 }
 
-// bf16 decode: 128 threads per (b, h). Scores: eight lanes share a slot, each
-// taking one 16-byte piece of its 64-dim key (a warp scores four slots at a
-// time), combined by shuffles within the eight-lane group. Output: thread
-// (piece c, group g) sums slots g, g+16, g+32, g+48 for dims 8c..8c+7; the 16
-// groups' partial sums are then added through shared memory.
+// bf16 decode: 128 threads per (b, h), one memory round trip. Thread (warp,
+// lane) owns the 16-byte piece c = lane % 8 (dims 8c..8c+7) of slots
+// 16p + 4*warp + lane/8, p = 0..3, and loads that piece of both the key and the
+// value of its four slots up front, together with q and the new key/value. The
+// eight lanes of a slot combine their partial dot products by shuffles; every
+// warp then reduces the 64 scores itself (max, exp, sum) from shared memory, so
+// the weights are applied to values already in registers; the four warps'
+// partial outputs are added through shared memory.
 __global__ void __launch_bounds__(128)
 swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, float scale) {
-    __shared__ float s_p[kMaxW];
-    __shared__ float s_part[16][kHead];
-    __shared__ uint4 s_new[2][8];           // new key / value, 8 pieces each
+    __shared__ float s_sc[kMaxW];
+    __shared__ float s_part[4][kHead];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
+    const int c = lane & 7;
     const size_t bh = blockIdx.x;
     const int new_slot = (int)(t % w);
-    if (tid < 16) {
-        const uint4* src = reinterpret_cast<const uint4*>((tid < 8 ? k : v) + bh * kHead) + (tid & 7);
-        const uint4 u = __ldg(src);
-        s_new[tid >> 3][tid & 7] = u;
-        reinterpret_cast<uint4*>((tid < 8 ? kc : vc) + (bh * w + new_slot) * kHead)[tid & 7] = u;
+
+    const uint4 knew = __ldg(reinterpret_cast<const uint4*>(k + bh * kHead) + c);
+    const uint4 vnew = __ldg(reinterpret_cast<const uint4*>(v + bh * kHead) + c);
+    const uint4 qu = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
+    uint4 kr[4], vr[4];
+    bool valid[4];
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        // newest token held by the slot: u = t - ((t - slot) mod w); empty while u < 0
+        valid[p] = slot < w && t - ((((t - slot) % w) + w) % w) >= 0;
+        kr[p] = vr[p] = make_uint4(0, 0, 0, 0);
+        if (valid[p]) {
+            if (slot == new_slot) {
+                kr[p] = knew;
+                vr[p] = vnew;
+            } else {
+                kr[p] = __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
+                vr[p] = __ldg(reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead) + c);
+            }
+        }
     }
-    const int c = lane & 7;                  // 16-byte piece of a row: dims 8c..8c+7
+    if (tid < 8) {
+        reinterpret_cast<uint4*>(kc + (bh * w + new_slot) * kHead)[c] = knew;
+        reinterpret_cast<uint4*>(vc + (bh * w + new_slot) * kHead)[c] = vnew;
+    }
     float qv[8];
     {
-        const uint4 u = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
-        const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
+        const uint32_t wd[4] = {qu.x, qu.y, qu.z, qu.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             qv[2 * e] = __uint_as_float(wd[e] << 16) * scale;
             qv[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u) * scale;
         }
     }
-    __syncthreads();
-    // scores: pass p covers slots 16p .. 16p+15; warp `warp` takes 4 of them
 #pragma unroll
-    for (int pass = 0; pass < kMaxW / 16; ++pass) {
-        const int slot = pass * 16 + warp * 4 + (lane >> 3);
+    for (int p = 0; p < 4; ++p) {
+        const uint32_t wd[4] = {kr[p].x, kr[p].y, kr[p].z, kr[p].w};
         float part = 0.f;
-        bool valid = false;
-        if (slot < w) {
-            const long long u = t - ((((t - slot) % w) + w) % w);   // newest token held by the slot
-            valid = u >= 0;
-            if (valid) {
-                const uint4 kr = slot == new_slot ? s_new[0][c]
-                                                  : __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
-                const uint32_t wd[4] = {kr.x, kr.y, kr.z, kr.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    part = fmaf(qv[2 * e], __uint_as_float(wd[e] << 16), part);
-                    part = fmaf(qv[2 * e + 1], __uint_as_float(wd[e] & 0xFFFF0000u), part);
-                }
-            }
+        for (int e = 0; e < 4; ++e) {
+            part = fmaf(qv[2 * e], __uint_as_float(wd[e] << 16), part);
+            part = fmaf(qv[2 * e + 1], __uint_as_float(wd[e] & 0xFFFF0000u), part);
         }
         part += __shfl_xor_sync(0xffffffffu, part, 1);
         part += __shfl_xor_sync(0xffffffffu, part, 2);
         part += __shfl_xor_sync(0xffffffffu, part, 4);
-        if (c == 0) s_p[slot] = valid ? part : -INFINITY;
+        if (c == 0) s_sc[16 * p + 4 * warp + (lane >> 3)] = valid[p] ? part : -INFINITY;
     }
     __syncthreads();
-    if (warp == 0) {
-        const float a = s_p[lane], b = s_p[lane + 32];
-        float m = fmaxf(a, b);
+    // Softmax statistics, computed by every warp (slot 0 always holds a token).
+    const float a = s_sc[lane], b = s_sc[lane + 32];
+    float m = fmaxf(a, b);
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        const float pa = a == -INFINITY ? 0.f : expf(a - m);
-        const float pb = b == -INFINITY ? 0.f : expf(b - m);
-        float sum = pa + pb;
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = (a == -INFINITY ? 0.f : expf(a - m)) + (b == -INFINITY ? 0.f : expf(b - m));
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
-        const float inv = 1.f / sum;
-        s_p[lane] = pa * inv;
-        s_p[lane + 32] = pb * inv;
-    }
-    __syncthreads();
-    {
-        const int g = tid >> 3;              // slot group 0..15
-        float acc[8];
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.f / sum;
+    float acc[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
 #pragma unroll
-        for (int r = 0; r < kMaxW / 16; ++r) {
-            const int slot = g + 16 * r;
-            const float p = slot < w ? s_p[slot] : 0.f;
-            if (p != 0.f) {
-                const uint4 vr = slot == new_slot ? s_new[1][c]
-                                                  : __ldg(reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead) + c);
-                const uint32_t wd[4] = {vr.x, vr.y, vr.z, vr.w};
+    for (int p = 0; p < 4; ++p) {
+        if (!valid[p]) continue;
+        const float pr = expf(s_sc[16 * p + 4 * warp + (lane >> 3)] - m) * inv;
+        const uint32_t wd[4] = {vr[p].x, vr[p].y, vr[p].z, vr[p].w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    acc[2 * e] = fmaf(p, __uint_as_float(wd[e] << 16), acc[2 * e]);
-                    acc[2 * e + 1] = fmaf(p, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
-                }
-            }
+        for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(pr, __uint_as_float(wd[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(pr, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
         }
+    }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) s_part[g][8 * c + e] = acc[e];
+    for (int e = 0; e < 8; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_part[warp][8 * c + e] = acc[e];
     }
     __syncthreads();
-    if (tid < kHead) {
-        float sum = 0.f;
+    if (tid < 8) {
+        float o[8];
 #pragma unroll
-        for (int g = 0; g < 16; ++g) sum += s_part[g][tid];
-        y[bh * kHead + tid] = __float2bfloat16_rn(sum);
+        for (int e = 0; e < 8; ++e)
+            o[e] = s_part[0][8 * tid + e] + s_part[1][8 * tid + e] + s_part[2][8 * tid + e] + s_part[3][8 * tid + e];
+        uint4 packed;
+        packed.x = pack2(o[0], o[1]);
+        packed.y = pack2(o[2], o[3]);
+        packed.z = pack2(o[4], o[5]);
+        packed.w = pack2(o[6], o[7]);
+        reinterpret_cast<uint4*>(y + bh * kHead)[tid] = packed;
     }
 }
 
