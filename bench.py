@@ -608,6 +608,83 @@ def run_profile(kind, reps):
     print(json.dumps({"profile": kind, "case": PROFILE_CASES[kind], "ms": ts}))
 
 
+def run_sweep(reps):
+    """Extra lines beside the headline: the decode batch sweep (a CUDA graph of 32
+    steps per replay) and the long-prefill workload, each against its roofline."""
+    import torch
+
+    import linear_attention_sequence_causal_b200 as based
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    def timed(fn, n_inner):
+        fn()
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.graph(g, stream=side):
+            for _ in range(n_inner):
+                fn()
+        stream.wait_stream(side)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / (reps * n_inner)
+
+    H, df, dv, D = 16, 16, 64, _feature_dim(16)
+    for batch in (1, 16, 64, 128, 256):
+        S = torch.randn(batch, H, D, dv, device=dev) * 0.01
+        z = torch.rand(batch, H, D, device=dev) + 600.0
+        inp = synthetic.la_inputs(batch, H, 1, df, dv, "bf16", seed=batch)
+        q, k, v = (t[:, :, 0].contiguous().to(dev) for t in (inp.q, inp.k, inp.v))
+        y = torch.empty(batch, H, dv, dtype=torch.bfloat16, device=dev)
+        ms = timed(lambda: based.la_decode_step(S, z, q, k, v, y=y), 32)
+        _, byts = la_decode_work(batch, H, df, dv)
+        print(json.dumps({"sweep": "la_decode", "batch": batch, "us_per_step": ms * 1e3,
+                          "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                          "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+        kc = torch.randn(batch, H, 64, 64, device=dev).bfloat16()
+        vc = torch.randn(batch, H, 64, 64, device=dev).bfloat16()
+        sq = torch.randn(batch, H, 64, device=dev).bfloat16()
+        ys = torch.empty_like(sq)
+        ms = timed(lambda: based.swa_decode(kc, vc, 1000, sq, sq, sq, w=64, scale=0.125, y=ys), 32)
+        _, byts = swa_decode_work(batch, H, 64, 64)
+        print(json.dumps({"sweep": "swa_decode", "batch": batch, "us_per_step": ms * 1e3,
+                          "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                          "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+        del S, z, kc, vc
+    # long prefill: B=2, H=16, N=16384
+    B, N = 2, 16384
+    inp = synthetic.la_inputs(B, H, N, df, dv, "bf16", seed=0)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    for chunk in (64, 128, 256):
+        try:
+            ws_bytes = based.la_prefill_workspace(B, H, N, df, dv, torch.bfloat16, chunk)
+            ws = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=dev)
+            y = torch.empty(B, H, N, dv, dtype=torch.bfloat16, device=dev)
+            S = torch.empty(B, H, D, dv, device=dev)
+            z = torch.empty(B, H, D, device=dev)
+            ms = timed(lambda: based.la_prefill(q, k, v, chunk=chunk, y=y, S=S, z=z, workspace=ws), 1)
+        except based.BasedError as e:
+            print(json.dumps({"sweep": "la_prefill_long", "chunk": chunk, "unsupported": str(e)}), flush=True)
+            continue
+        flops, byts = la_prefill_work(B, H, N, df, dv, chunk)
+        print(json.dumps({"sweep": "la_prefill_long", "chunk": chunk, "us": ms * 1e3,
+                          "tokens_per_s": B * N / (ms / 1e3), "TFLOP_s": flops / (ms / 1e3) / 1e12,
+                          "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                          "GB_s": byts / (ms / 1e3) / 1e9}), flush=True)
+
+
 def main(argv=None):
     p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     p.add_argument("--gpus", type=int, default=1)
@@ -619,9 +696,13 @@ def main(argv=None):
     p.add_argument("--preroll-s", type=float, default=1.0, help="loaded seconds before the timed region")
     p.add_argument("--profile", choices=sorted(PROFILE_CASES), help="run one kernel on its ncu capture case")
     p.add_argument("--profile-reps", type=int, default=3)
+    p.add_argument("--sweep", action="store_true", help="decode batch sweep and long-prefill lines")
     args = p.parse_args(argv)
     if args.profile:
         run_profile(args.profile, args.profile_reps)
+        return
+    if args.sweep:
+        run_sweep(max(3, min(args.steps, 20)))
         return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -85,6 +85,15 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
         if (f < f1) buf[u] = *reinterpret_cast<const float4*>(Sp + (size_t)f * DV);
     }
 
+    // This thread's z rows (at most two: a CTA holds at most 2 * kThreads rows).
+    float* zbh = z + bh * D;
+    float zr[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int f = f0 + tid + i * kThreads;
+        if (f < f1) zr[i] = zbh[f];
+    }
+
     if (tid < DF) {
         s_x[0][tid] = to_f32(q[bh * DF + tid]);
         s_x[1][tid] = to_f32(k[bh * DF + tid]);
@@ -94,11 +103,14 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
 
     // Denominator part over this CTA's rows; z updated in place.
     float dpart = 0.f;
-    float* zbh = z + bh * D;
-    for (int f = f0 + tid; f < f1; f += kThreads) {
-        const float zn = zbh[f] + phi_entry<DF>(s_x[1], f);
-        zbh[f] = zn;
-        dpart = fmaf(phi_entry<DF>(s_x[0], f), zn, dpart);
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const int f = f0 + tid + i * kThreads;
+        if (f < f1) {
+            const float zn = zr[i] + phi_entry<DF>(s_x[1], f);
+            zbh[f] = zn;
+            dpart = fmaf(phi_entry<DF>(s_x[0], f), zn, dpart);
+        }
     }
 
     const float4 vv = make_float4(s_v[4 * g], s_v[4 * g + 1], s_v[4 * g + 2], s_v[4 * g + 3]);
@@ -169,6 +181,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
 int ranks_per_head(int BH, int D, int num_sms) {
     int P = 1;
     while (P < kMaxRanks && (long long)BH * P < 4LL * num_sms && D / (2 * P) >= 16) P *= 2;
+    while ((D + P - 1) / P > 2 * kThreads) P *= 2;    // z rows per thread: at most two
     return P;
 }
 
