@@ -22,8 +22,9 @@
 // registers; phi(Q) goes straight into tensor memory, phi(K) into shared
 // memory. The order-2 block is folded by symmetry,
 // (q.k)^2/2 = sum_a (q_a^2/sqrt2)(k_a^2/sqrt2) + sum_{a<b} (q_a q_b)(k_a k_b),
-// giving 1 + 16 + 136 = 153 features (padded to 160) instead of 273; the final
-// state is expanded back to the 273-row layout on the way out.
+// giving 1 + 16 + 136 = 153 features (padded to 160) instead of 273, in an
+// order that suits packed bf16x2 multiplies (see phi_word); the final state is
+// expanded back to the 273-row layout on the way out.
 //
 // Issue structure. One thread can keep only about one tcgen05.mma per ~117
 // cycles in flight (measured on B200 for any N <= 144), while MMAs from two
@@ -148,45 +149,69 @@ enum {
     NUM_BARS
 };
 
-// Emit phi_sym(x) and phi_sym(y) together (one copy of the code, which keeps
-// the kernel's instruction footprint small) as 20 packed 16-byte pieces of 8
-// features each, in feature order
-// [c0, x_0..x_15, x_a x_b (a <= b, a-major; x_a^2 carries 1/sqrt2), 0 x 7];
-// c0 is the constant feature (1, or 0 to emit an all-zero phi for x = 0).
+// ------------------------------------------------------------------ feature map
+// Kernel-internal order of the 153 distinct features (padded to 160), chosen so
+// that the order-2 products come out of packed bf16x2 multiplies of the bf16
+// inputs (a product of two bf16 values is exact in fp32, so one bf16x2 multiply
+// rounds exactly like an fp32 multiply followed by a bf16 conversion):
+//   0..15    x_a                                   (the input words themselves)
+//   16..31   x_a^2 / sqrt2                         (fp32, then bf16)
+//   32..143  x_a x_b for b = 2..15, a < 2 floor(b/2), by column b, pairs (a, a+1)
+//   144..151 x_{b-1} x_b for odd b                 (the pairs the columns leave over)
+//   152      the constant feature;  153..159 zero
+// The 1 + d' + d'^2 layout of the final state is rebuilt from this order in
+// write_final_state.
+__device__ __forceinline__ uint32_t bmul2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+__device__ __forceinline__ uint32_t bcast_bf16(uint32_t w, int hi) {
+    return __byte_perm(w, w, hi ? 0x3232 : 0x1010);
+}
+
+// phi(x) and phi(y) word by word (word w holds features 2w, 2w+1); one copy of
+// the code serves both operands, which keeps the kernel's instruction footprint
+// small. store(g, wx, wy) receives words 16g..16g+15 of each. Every loop is
+// unrolled, so all indices are compile-time constants.
 template <typename Store>
-__device__ __forceinline__ void emit_phi2(const float* x, float cx, const float* y, float cy, Store store) {
-    float bx[8], by[8];
-    int n = 0, piece = 0;
-    auto push = [&](float vx, float vy) {
-        bx[n] = vx;
-        by[n++] = vy;
-        if (n == 8) {
-            store(piece++, pack_bf16x8(bx), pack_bf16x8(by));
+__device__ __forceinline__ void emit_phi2(const uint4* xin, uint32_t cx, const uint4* yin, uint32_t cy, Store store) {
+    const uint32_t X[8] = {xin[0].x, xin[0].y, xin[0].z, xin[0].w, xin[1].x, xin[1].y, xin[1].z, xin[1].w};
+    const uint32_t Y[8] = {yin[0].x, yin[0].y, yin[0].z, yin[0].w, yin[1].x, yin[1].y, yin[1].z, yin[1].w};
+    uint32_t bx[16], by[16];
+    int n = 0, g = 0;
+    auto push = [&](uint32_t wx, uint32_t wy) {
+        bx[n] = wx;
+        by[n++] = wy;
+        if (n == 16) {
+            store(g++, bx, by);
             n = 0;
         }
     };
-    push(cx, cy);
 #pragma unroll
-    for (int a = 0; a < DF; ++a) push(x[a], y[a]);
+    for (int i = 0; i < 8; ++i) push(X[i], Y[i]);                      // x_a
 #pragma unroll
-    for (int a = 0; a < DF; ++a) {
-#pragma unroll
-        for (int b = a; b < DF; ++b) {
-            if (a == b) push((x[a] * x[a]) * kSqrtHalf, (y[a] * y[a]) * kSqrtHalf);
-            else push(x[a] * x[b], y[a] * y[b]);
-        }
+    for (int i = 0; i < 8; ++i) {                                       // x_a^2 / sqrt2
+        const float x0 = __uint_as_float(X[i] << 16), x1 = __uint_as_float(X[i] & 0xFFFF0000u);
+        const float y0 = __uint_as_float(Y[i] << 16), y1 = __uint_as_float(Y[i] & 0xFFFF0000u);
+        push(pack_bf16x2((x0 * x0) * kSqrtHalf, (x1 * x1) * kSqrtHalf),
+             pack_bf16x2((y0 * y0) * kSqrtHalf, (y1 * y1) * kSqrtHalf));
     }
 #pragma unroll
-    for (int f = DS; f < KF; ++f) push(0.0f, 0.0f);
-}
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4& u, float* x) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+    for (int b = 2; b < DF; ++b) {                                      // column b: pairs (a, a+1), a < 2 floor(b/2)
+        const uint32_t xb = bcast_bf16(X[b >> 1], b & 1), yb = bcast_bf16(Y[b >> 1], b & 1);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        for (int p = 0; p < b / 2; ++p) push(bmul2(X[p], xb), bmul2(Y[p], yb));
     }
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {                                       // x_{b-1} x_b, b = 4k+1 and 4k+3
+        push(bmul2(__byte_perm(X[2 * k], X[2 * k + 1], 0x5410), __byte_perm(X[2 * k], X[2 * k + 1], 0x7632)),
+             bmul2(__byte_perm(Y[2 * k], Y[2 * k + 1], 0x5410), __byte_perm(Y[2 * k], Y[2 * k + 1], 0x7632)));
+    }
+    push(cx, cy);                                                       // constant feature, then zero padding
+#pragma unroll
+    for (int i = 0; i < 3; ++i) push(0u, 0u);
 }
 
 // Everything a CTA needs to know about its share of the work.
@@ -227,19 +252,23 @@ __device__ __forceinline__ unsigned char* smem_generic(uint32_t saddr) {
 }
 
 // Whole CTA, after every role has finished: expand the staged folded state
-// (stage[f][n], n < 64 for S, n = 64 for z) to the 1 + d' + d'^2 rows of S and z.
-// Row r <= d' is feature r; row 1 + d' + a*d' + b is the folded pair (min, max)
-// of (a, b), times 1/sqrt2 off the diagonal (the pair's value is split evenly).
+// (stage[f][n], n < 64 for S, n = 64 for z; f in the kernel's feature order) to
+// the 1 + d' + d'^2 rows of S and z. Row 1 + d' + a*d' + b takes the folded
+// pair (min, max) of (a, b), times 1/sqrt2 off the diagonal (the pair's value
+// is split evenly between (a, b) and (b, a)).
 __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase, int tid, float* S, float* z) {
     constexpr int D = feature_dim(DF);
     const float* stage = reinterpret_cast<const float*>(smem_generic(sbase) + OFF_PK);
     auto source = [](int r, float& coef) {
         coef = 1.0f;
-        if (r <= DF) return r;
+        if (r == 0) return 152;                                  // constant feature
+        if (r <= DF) return r - 1;                               // x_a
         const int p = r - 1 - DF, a = p / DF, b = p % DF;
+        if (a == b) return DF + a;                               // x_a^2 / sqrt2
         const int lo = min(a, b), hi = max(a, b);
-        if (a != b) coef = kSqrtHalf;
-        return 1 + DF + lo * DF - lo * (lo - 1) / 2 + (hi - lo);
+        coef = kSqrtHalf;
+        if ((hi & 1) && lo == hi - 1) return 144 + (hi - 1) / 2; // left-over pair of an odd column
+        return 32 + 2 * (((hi - 1) * (hi - 1)) / 4) + lo;        // column hi, pairs (a, a+1)
     };
     float4* Sd = reinterpret_cast<float4*>(S + w.bh * D * DV);
     for (int idx = tid; idx < D * (DV / 4); idx += kThreads) {
@@ -418,19 +447,11 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
         // phi(K) (MN-major: a 16-byte piece is 8 features of token t; padded
         // tokens contribute nothing) and phi(Q) (TMEM lane t), in one pass.
         const uint32_t pk = sh.sbase + OFF_PK + b * PK_BYTES + cm + (t >> 3) * PK_LBO;
-        float xk[DF], xq[DF];
-        unpack_bf16x8(cur.k[0], xk);
-        unpack_bf16x8(cur.k[1], xk + 8);
-        unpack_bf16x8(cur.q[0], xq);
-        unpack_bf16x8(cur.q[1], xq + 8);
-        uint32_t pkt[16];
-        emit_phi2(xk, valid ? 1.0f : 0.0f, xq, 1.0f, [&](int j, uint4 uk, uint4 uq) {
-            st_shared_v4(pk + j * PK_SBO, uk);
-            pkt[(j & 3) * 4 + 0] = uq.x;
-            pkt[(j & 3) * 4 + 1] = uq.y;
-            pkt[(j & 3) * 4 + 2] = uq.z;
-            pkt[(j & 3) * 4 + 3] = uq.w;
-            if (with_q && (j & 3) == 3) tmem_st16(lane_base + COL_PQ + (j >> 2) * 16, pkt);
+        emit_phi2(cur.k, valid ? 0x3F80u : 0u, cur.q, 0x3F80u, [&](int g, const uint32_t* uk, const uint32_t* uq) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+                st_shared_v4(pk + (4 * g + j) * PK_SBO, make_uint4(uk[4 * j], uk[4 * j + 1], uk[4 * j + 2], uk[4 * j + 3]));
+            if (with_q) tmem_st16(lane_base + COL_PQ + 16 * g, uq);
         });
         fence_proxy_async_smem();
         mbar_arrive(&sh.bars[BAR_IN0 + b]);
