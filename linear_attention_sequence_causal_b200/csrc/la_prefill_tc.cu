@@ -489,16 +489,25 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
             tmem_ld_wait();
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
-                const int blk = 2 * h + p / 4;                  // key block of this piece
-                const bool below = blk < wq, diag = blk == wq;
-                float a8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float x = sv[8 * p + e];
-                    const float a = fmaf(x, fmaf(0.5f, x, 1.0f), 1.0f);
-                    a8[e] = (below || (diag && ((8 * p + e) & 31) <= lane)) ? a : 0.0f;
+                const int blk = 2 * h + p / 4;                  // key block of this piece (warp-uniform)
+                if (blk > wq) {
+                    pc[p] = make_uint4(0, 0, 0, 0);
+                    continue;
                 }
-                pc[p] = pack_bf16x8(a8);
+                uint32_t wd[4];
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) {
+                    const float x0 = sv[8 * p + 2 * q2], x1 = sv[8 * p + 2 * q2 + 1];
+                    wd[q2] = pack_bf16x2(fmaf(x0, fmaf(0.5f, x0, 1.0f), 1.0f), fmaf(x1, fmaf(0.5f, x1, 1.0f), 1.0f));
+                }
+                if (blk == wq) {                                // diagonal block: keep keys j <= i
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) {
+                        const int kk = (8 * p + 2 * q2) & 31;   // key of the pair's low half, within the block
+                        wd[q2] &= (kk <= lane ? 0x0000FFFFu : 0u) | (kk + 1 <= lane ? 0xFFFF0000u : 0u);
+                    }
+                }
+                pc[p] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             }
         }
         if (h == 0) {

@@ -4,26 +4,34 @@
 // tradeoff" (BASED), §4 "Local Exact Attention": exact softmax over the w most
 // recent keys (the query's own position included), O(Nw) work.
 //
-// One CTA computes 128 consecutive queries [i0, i0 + 128) of one head. Every key
-// those queries can see lies in the 192-key span [i0 - 64, i0 + 128), so a whole
-// tile needs exactly one score block and one value block -- no running softmax:
+// A tile is 128 consecutive queries [i0, i0 + 128) of one head. Every key those
+// queries can see lies in the 192-key span [i0 - 64, i0 + 128), so a tile needs
+// exactly one score block and one value block -- no running softmax:
 //   TMA    Q [128 x 64], K and V [192 x 64] (128-byte swizzle; rows before the
 //          sequence start or past its end arrive as zeros)
 //   MMA    S = Q K^T              M=128 N=192 K=64   -> TMEM (192 columns)
 //   CUDA   row i keeps only its band i0+i-w < j <= i0+i; p = exp(scale*(s - max)),
-//          written as bf16 P over the Q/K buffers, l = sum of the rounded p
-//   MMA    O = P V                M=128 N=64 K=192   -> TMEM (64 columns)
-//   CUDA   y = O / l  -> global
+//          written back as bf16 P over the first 96 columns of S (in place)
+//   MMA    O = P V                M=128 N=64 K=192   -> TMEM (A operand P in TMEM)
+//   CUDA   y = O / l, l = the sum of the rounded p -> swizzled tile -> TMA store
 // A warp's 32 query rows touch only 96 of the 192 score columns; it reads just
-// those from TMEM and writes zeros for the rest of its P rows.
+// those and writes zeros for the rest of its P row.
 //
-// Roles: warps 0-3 own query rows (TMEM lanes); warp 4 allocates TMEM and its
-// lane 0 issues the TMA loads, both MMAs and the commits, while lanes 1-31 copy
-// the tile's share of the last w tokens into the ring KV cache (slot t mod w;
-// the first tile also zeroes the slots a prompt shorter than w never fills).
-// Waits are bounded.
+// The kernel is persistent and pipelined: one CTA per SM walks its tiles
+// (tile = CTA + k * grid) with
+//   warp 0      lane 0 issues the TMA loads into a 3-stage ring of {Q, K, V};
+//   warp 1      allocates TMEM; lane 0 issues S of tile n, then O of tile n-1,
+//               so the tensor core works while the softmax of tile n runs;
+//   warps 2-5   softmax + epilogue of even tiles (TMEM buffer 0),
+//   warps 6-9   the same for odd tiles (TMEM buffer 1); the epilogue warps also
+//               copy the tile's share of the last w tokens into the ring KV
+//               cache (slot t mod w) and, on a head's first tile, zero the
+//               slots a prompt shorter than w never fills.
+// Every hand-off is an mbarrier; every wait is bounded.
 #include <cuda.h>
 #include <math.h>
+
+#include <algorithm>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -35,37 +43,264 @@ namespace {
 
 using namespace tc;
 
-constexpr int QT = 128;              // queries per CTA
-constexpr int KW = 192;              // keys per CTA: [i0 - 64, i0 + 128)
+constexpr int QT = 128;              // queries per tile
+constexpr int KW = 192;              // keys per tile: [i0 - 64, i0 + 128)
 constexpr int HD = 64;               // head dim
-constexpr int kThreads = 160;
+constexpr int kStages = 3;           // {Q, K, V} ring depth
+constexpr int kThreads = 320;
 
-// Shared memory (offsets from a 1024-aligned base). P (3 atom columns of
-// 128 rows x 128 B) reuses Q, K and the pad after them once S is computed.
-constexpr uint32_t OFF_Q = 0;                      // 16 KB
-constexpr uint32_t OFF_K = OFF_Q + QT * HD * 2;    // 24 KB
-constexpr uint32_t OFF_P = 0;                      // 48 KB, after S completes
-constexpr uint32_t OFF_V = 3 * QT * 128;           // 24 KB
-constexpr uint32_t OFF_BAR = OFF_V + KW * HD * 2;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 64 + 1024;   // + alignment slack
-static_assert(OFF_K + KW * HD * 2 <= OFF_V, "P region must cover Q and K");
-constexpr uint32_t TX_BYTES = QT * HD * 2 + 2 * KW * HD * 2;
+// Shared memory (offsets from a 1024-aligned base).
+constexpr uint32_t Q_BYTES = QT * HD * 2;          // 16 KB
+constexpr uint32_t KV_BYTES = KW * HD * 2;         // 24 KB each
+constexpr uint32_t STAGE_BYTES = Q_BYTES + 2 * KV_BYTES;
+constexpr uint32_t OFF_STAGE = 0;                  // [kStages] {Q, K, V}
+constexpr uint32_t OFF_YS = kStages * STAGE_BYTES; // [2] y tiles, 128-byte swizzled
+constexpr uint32_t OFF_BAR = OFF_YS + 2 * Q_BYTES;
+constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;   // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+constexpr uint32_t TX_BYTES = STAGE_BYTES;
 
-constexpr uint32_t COL_S = 0;        // 192 columns
-constexpr uint32_t COL_O = 192;      // 64 columns
-constexpr uint32_t TMEM_COLS = 256;
+// TMEM: two buffers of {S / P (192 columns), O (64 columns)}.
+constexpr uint32_t COL_S = 0;
+constexpr uint32_t COL_O = 192;
+constexpr uint32_t BUF_COLS = 256;
+constexpr uint32_t TMEM_COLS = 512;
 
 constexpr uint32_t ID_S = idesc_bf16_f32(128, KW, false, false);
 constexpr uint32_t ID_O = idesc_bf16_f32(128, HD, false, true);
 
-enum { BAR_LOAD, BAR_S, BAR_P, BAR_O, NUM_BARS };
+enum {
+    BAR_FULL0, BAR_FULL1, BAR_FULL2,          // TMA -> MMA: stage s landed
+    BAR_EMPTY0, BAR_EMPTY1, BAR_EMPTY2,       // MMA commit: stage s read (S and O done)
+    BAR_SF0, BAR_SF1,                         // MMA commit: S of buffer b ready
+    BAR_PF0, BAR_PF1,                         // softmax warps -> MMA: P of buffer b written
+    BAR_OF0, BAR_OF1,                         // MMA commit: O of buffer b ready
+    BAR_TE0, BAR_TE1,                         // softmax warps -> MMA: TMEM buffer b read (free)
+    BAR_YR0, BAR_YR1,                         // softmax warps -> store thread: y tile b written
+    BAR_YE0, BAR_YE1,                         // store thread -> softmax warps: the TMA store has read y tile b
+    NUM_BARS
+};
 
-__global__ void __launch_bounds__(kThreads)
+struct Ctx {
+    uint32_t sbase;
+    uint64_t* bars;
+    volatile int* abort_flag;
+    unsigned* status;
+    int N, w, nqb, ntiles;
+};
+
+// 2^x by the hardware approximation (relative error about 2^-22, far below the
+// bf16 rounding P goes through); 2^-inf = +0.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ bool wait_bar(const Ctx& cx, int bar, uint32_t parity) {
+    return mbar_wait(&cx.bars[bar], parity, cx.abort_flag, cx.status);
+}
+
+// ------------------------------------------------------------------ TMA producer (warp 0, lane 0)
+__device__ __forceinline__ void producer(const Ctx& cx, const CUtensorMap* tq, const CUtensorMap* tk,
+                                         const CUtensorMap* tv) {
+    int n = 0;
+    for (int tile = blockIdx.x; tile < cx.ntiles; tile += gridDim.x, ++n) {
+        const int s = n % kStages;
+        if (n >= kStages && !wait_bar(cx, BAR_EMPTY0 + s, ((n / kStages) - 1) & 1)) break;
+        const int bh = tile / cx.nqb, i0 = (tile % cx.nqb) * QT;
+        const uint32_t st = cx.sbase + OFF_STAGE + s * STAGE_BYTES;
+        mbar_expect_tx(&cx.bars[BAR_FULL0 + s], TX_BYTES);
+        tma_load_3d(st, tq, &cx.bars[BAR_FULL0 + s], 0, i0, bh);
+        tma_load_3d(st + Q_BYTES, tk, &cx.bars[BAR_FULL0 + s], 0, i0 - 64, bh);
+        tma_load_3d(st + Q_BYTES + KV_BYTES, tv, &cx.bars[BAR_FULL0 + s], 0, i0 - 64, bh);
+    }
+    // Loads still landing when the CTA ends would write freed shared memory:
+    // wait (bounded) for the last ones.
+    for (int m = max(0, n - kStages); m < n; ++m) {
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(&cx.bars[BAR_FULL0 + m % kStages], (m / kStages) & 1) && global_ns() - t0 < kWaitLimitNs) {}
+    }
+}
+
+// ------------------------------------------------------------------ MMA issuer (warp 1, lane 0)
+__device__ __forceinline__ void mma_issuer(const Ctx& cx, uint32_t tmem, bool skip) {
+    uint64_t* last_bar = nullptr;
+    uint32_t last_parity = 0;
+    auto issue_o = [&](int m) {              // O = P V of local tile m
+        const int s = m % kStages, b = m & 1;
+        const uint32_t v = cx.sbase + OFF_STAGE + s * STAGE_BYTES + Q_BYTES + KV_BYTES;
+        const uint32_t tb = tmem + b * BUF_COLS;
+#pragma unroll
+        for (int j = 0; j < KW / 16; ++j)
+            mma_bf16_ts(tb + COL_O, tb + COL_S + 8 * j, smem_desc_sw128(v + j * 2048, 16, 1024), ID_O, j > 0);
+        mma_commit(&cx.bars[BAR_EMPTY0 + s]);
+        mma_commit(&cx.bars[BAR_OF0 + b]);
+        last_bar = &cx.bars[BAR_OF0 + b];
+        last_parity = (m >> 1) & 1;
+    };
+    int n = 0;
+    bool ok = !skip;                          // testing: issue nothing, every waiter times out
+    for (int tile = blockIdx.x; ok && tile < cx.ntiles; tile += gridDim.x, ++n) {
+        const int s = n % kStages, b = n & 1;
+        if (!wait_bar(cx, BAR_FULL0 + s, (n / kStages) & 1)) { ok = false; break; }
+        if (n >= 2 && !wait_bar(cx, BAR_TE0 + b, ((n >> 1) - 1) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t q = cx.sbase + OFF_STAGE + s * STAGE_BYTES;
+        const uint32_t tb = tmem + b * BUF_COLS;
+#pragma unroll
+        for (int j = 0; j < HD / 16; ++j)
+            mma_bf16(tb + COL_S, smem_desc_sw128(q + 32 * j, 16, 1024), smem_desc_sw128(q + Q_BYTES + 32 * j, 16, 1024),
+                     ID_S, j > 0);
+        mma_commit(&cx.bars[BAR_SF0 + b]);
+        last_bar = &cx.bars[BAR_SF0 + b];
+        last_parity = (n >> 1) & 1;
+        // O of the previous tile, once its softmax has written P.
+        if (n >= 1) {
+            if (!wait_bar(cx, BAR_PF0 + ((n - 1) & 1), ((n - 1) >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            issue_o(n - 1);
+        }
+    }
+    if (ok && n >= 1) {
+        if (wait_bar(cx, BAR_PF0 + ((n - 1) & 1), ((n - 1) >> 1) & 1)) {
+            tc_fence_after();
+            issue_o(n - 1);
+        }
+    }
+    // Never free TMEM under an MMA still in flight.
+    if (*cx.abort_flag && last_bar != nullptr) {
+        const uint64_t t0 = global_ns();
+        while (!mbar_try_wait(last_bar, last_parity) && global_ns() - t0 < kWaitLimitNs) {}
+    }
+}
+
+// ------------------------------------------------------------------ softmax + epilogue (warps 2-9)
+// Warpgroup g takes the tiles of TMEM buffer g; thread = query row i = TMEM lane
+// (quadrant q = warp mod 4). The warp with quadrant 0 has the store thread.
+__device__ __forceinline__ void softmax_wg(const Ctx& cx, uint32_t tmem, int g, int q, int lane,
+                                           const CUtensorMap* ty, const __nv_bfloat16* __restrict__ k,
+                                           const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ k_cache,
+                                           __nv_bfloat16* __restrict__ v_cache, float scale_log2) {
+    const int i = q * 32 + lane;
+    const bool store_thread = q == 0 && lane == 0;
+    const uint32_t lane_base = tmem + g * BUF_COLS + (static_cast<uint32_t>(q * 32) << 16);
+    const uint32_t ys = cx.sbase + OFF_YS + g * Q_BYTES;
+    const int N = cx.N, w = cx.w;
+    int kk = 0;                                  // tiles of this warpgroup so far
+    for (int tile = blockIdx.x + g * gridDim.x; tile < cx.ntiles; tile += 2 * gridDim.x, ++kk) {
+        const int bh = tile / cx.nqb, i0 = (tile % cx.nqb) * QT, kb = i0 - 64, qi = i0 + i;
+        if (!wait_bar(cx, BAR_SF0 + g, kk & 1)) return;
+        tc_fence_after();
+        // Columns [32q, 32q + 96) of S hold every key of this warp's rows.
+        float sc[96];
+#pragma unroll
+        for (int m = 0; m < 6; ++m) tmem_ld16(lane_base + COL_S + 32 * q + 16 * m, sc + 16 * m);
+        tmem_ld_wait();
+        // This row's keys within the loaded window c = 0..95 (span column 32q + c)
+        // form the contiguous range [lo, hi]: the band i - w < j <= i, cut at the
+        // sequence start; a padding row (qi >= N) sees nothing.
+        const int lo = max(lane + 65 - w, -kb - 32 * q);
+        const int hi = qi < N ? lane + 64 : -1;
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < 96; ++c) {
+            sc[c] = (c >= lo && c <= hi) ? sc[c] : -INFINITY;
+            mx = fmaxf(mx, sc[c]);
+        }
+        // p = exp(scale (s - max)) = 2^(s * scale_log2 - max * scale_log2); exp2 of
+        // -inf is 0, so masked keys need no branch.
+        const float off = mx == -INFINITY ? 0.f : -mx * scale_log2;
+        // P row i in bf16 pairs over S: key pair (2m, 2m+1) of the span in column m.
+        // Column groups q..q+2 (16 columns each) hold the band, the rest are zero.
+        float l = 0.f;
+        uint32_t pw[48];
+#pragma unroll
+        for (int m = 0; m < 48; ++m) {
+            const uint32_t u = pack_bf16x2(ex2_approx(fmaf(sc[2 * m], scale_log2, off)),
+                                           ex2_approx(fmaf(sc[2 * m + 1], scale_log2, off)));
+            l += __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);   // the values the MMA will see
+            pw[m] = u;
+        }
+        uint32_t zero[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) zero[e] = 0u;
+#pragma unroll
+        for (int gr = 0; gr < 6; ++gr) {
+            const int rel = gr - q;              // warp-uniform
+            if (rel == 0) tmem_st16(lane_base + COL_S + 16 * gr, pw);
+            else if (rel == 1) tmem_st16(lane_base + COL_S + 16 * gr, pw + 16);
+            else if (rel == 2) tmem_st16(lane_base + COL_S + 16 * gr, pw + 32);
+            else tmem_st16(lane_base + COL_S + 16 * gr, zero);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&cx.bars[BAR_PF0 + g]);
+
+        if (!wait_bar(cx, BAR_OF0 + g, kk & 1)) return;
+        tc_fence_after();
+        float o[HD];
+#pragma unroll
+        for (int m = 0; m < HD / 16; ++m) tmem_ld16(lane_base + COL_O + 16 * m, o + 16 * m);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&cx.bars[BAR_TE0 + g]);
+
+        // y tile: free once the previous TMA store from it has read it.
+        if (kk >= 1) {
+            if (store_thread) {
+                bulk_wait_read_all();
+                mbar_arrive(&cx.bars[BAR_YE0 + g]);
+            }
+            if (!wait_bar(cx, BAR_YE0 + g, (kk - 1) & 1)) return;
+        }
+        const float inv = 1.0f / (l > 0.f ? l : 1.0f);
+#pragma unroll
+        for (int p8 = 0; p8 < HD / 8; ++p8) {
+            float t[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) t[e] = o[8 * p8 + e] * inv;
+            st_shared_v4(ys + i * 128 + ((p8 ^ (i & 7)) << 4), pack_bf16x8(t));
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&cx.bars[BAR_YR0 + g]);
+        if (store_thread) {
+            if (!wait_bar(cx, BAR_YR0 + g, kk & 1)) return;
+            tma_store_3d(ty, ys, 0, i0, bh);
+            bulk_commit();
+        }
+
+        // Ring cache: token u in [max(0, N - w), N) goes to slot u mod w; a head's
+        // first tile also zeroes the slots a prompt shorter than w never fills.
+        if (k_cache != nullptr) {
+            const size_t ring = (size_t)bh * w;
+            if (qi < N && qi >= N - w) {
+                const uint4* ks = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + qi) * HD);
+                const uint4* vs = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + qi) * HD);
+                uint4* kd = reinterpret_cast<uint4*>(k_cache + (ring + qi % w) * HD);
+                uint4* vd = reinterpret_cast<uint4*>(v_cache + (ring + qi % w) * HD);
+#pragma unroll
+                for (int p8 = 0; p8 < HD / 8; ++p8) {
+                    kd[p8] = __ldg(ks + p8);
+                    vd[p8] = __ldg(vs + p8);
+                }
+            }
+            if (i0 == 0 && N + i < w) {
+                uint4* kd = reinterpret_cast<uint4*>(k_cache + (ring + N + i) * HD);
+                uint4* vd = reinterpret_cast<uint4*>(v_cache + (ring + N + i) * HD);
+#pragma unroll
+                for (int p8 = 0; p8 < HD / 8; ++p8) kd[p8] = vd[p8] = make_uint4(0, 0, 0, 0);
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
 swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, const __nv_bfloat16* __restrict__ k,
-                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
+                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap ty,
+                      const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __restrict__ v,
                       __nv_bfloat16* __restrict__ k_cache, __nv_bfloat16* __restrict__ v_cache, int N, int w,
-                      float scale_log2, unsigned* status, unsigned debug) {
+                      int nqb, int ntiles, float scale_log2, unsigned* status, unsigned debug) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -73,162 +308,39 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * NUM_BARS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * NUM_BARS + 4);
+    const Ctx cx{sbase, bars, abort_flag, status, N, w, nqb, ntiles};
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
     const int lane = tid & 31;
-    const int i0 = blockIdx.x * QT;
-    const int bh = blockIdx.y;
-    const int kb = i0 - 64;            // first key of the span
-
     if (tid == 0) {
-        mbar_init(&bars[BAR_LOAD], 1);
-        mbar_init(&bars[BAR_S], 1);
-        mbar_init(&bars[BAR_P], 128);
-        mbar_init(&bars[BAR_O], 1);
+        for (int b = 0; b < NUM_BARS; ++b) {
+            const bool group = (b >= BAR_PF0 && b <= BAR_PF1) || (b >= BAR_TE0 && b <= BAR_TE1) ||
+                               (b >= BAR_YR0 && b <= BAR_YR1);
+            mbar_init(&bars[b], group ? 128 : 1);
+        }
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 4) tmem_alloc(tmem_slot, TMEM_COLS);
+    if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    if (warp < 4) {
-        const int i = tid;                          // query row == TMEM lane
-        const int qi = i0 + i;
-        const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        float l = 1.0f;
-        if (mbar_wait(&bars[BAR_S], 0, abort_flag, status)) {
-            tc_fence_after();
-            // Columns [32*warp, 32*warp + 96) hold every key of this warp's rows.
-            float s[96];
-#pragma unroll
-            for (int m = 0; m < 6; ++m) tmem_ld16(lane_base + COL_S + 32 * warp + 16 * m, s + 16 * m);
-            tmem_ld_wait();
-            const int jl_lo = i + 65 - w;           // band in span coordinates, inclusive
-            const int jl_hi = i + 64;
-            float mx = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 96; ++c) {
-                const int jl = 32 * warp + c;
-                const bool ok = jl >= jl_lo && jl <= jl_hi && kb + jl >= 0 && qi < N;
-                s[c] = ok ? s[c] * scale_log2 : -INFINITY;
-                mx = fmaxf(mx, s[c]);
-            }
-            float sum = 0.f;
-            // P row i: span chunks [4*warp, 4*warp + 12) carry the band, the rest are zero.
-            const uint32_t prow = sbase + OFF_P;
-#pragma unroll
-            for (int c8 = 0; c8 < KW / 8; ++c8) {
-                if (c8 < 4 * warp || c8 >= 4 * warp + 12)
-                    st_shared_v4(prow + (c8 >> 3) * (QT * 128) + sw128_offset(i, c8 & 7), make_uint4(0, 0, 0, 0));
-            }
-#pragma unroll
-            for (int cc = 0; cc < 12; ++cc) {
-                const int c8 = 4 * warp + cc;
-                float p[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const float t = s[8 * cc + e];
-                    p[e] = (t == -INFINITY) ? 0.f : exp2f(t - mx);
-                }
-                const uint4 u = pack_bf16x8(p);
-                // normalise with the bf16 values the MMA will see
-                const uint32_t wds[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    sum += __uint_as_float(wds[e] << 16) + __uint_as_float(wds[e] & 0xFFFF0000u);
-                st_shared_v4(prow + (c8 >> 3) * (QT * 128) + sw128_offset(i, c8 & 7), u);
-            }
-            l = sum > 0.f ? sum : 1.0f;
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bars[BAR_P]);
-            if (mbar_wait(&bars[BAR_O], 0, abort_flag, status)) {
-                tc_fence_after();
-                float o[HD];
-#pragma unroll
-                for (int m = 0; m < HD / 16; ++m) tmem_ld16(lane_base + COL_O + 16 * m, o + 16 * m);
-                tmem_ld_wait();
-                if (qi < N) {
-                    const float inv = 1.0f / l;
-                    uint4* yp = reinterpret_cast<uint4*>(y + ((size_t)bh * N + qi) * HD);
-#pragma unroll
-                    for (int c8 = 0; c8 < HD / 8; ++c8) {
-                        float t[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) t[e] = o[8 * c8 + e] * inv;
-                        yp[c8] = pack_bf16x8(t);
-                    }
-                }
-            }
-        }
-    } else if (lane == 0) {
-        mbar_expect_tx(&bars[BAR_LOAD], TX_BYTES);
-        tma_load_3d(sbase + OFF_Q, &tq, &bars[BAR_LOAD], 0, i0, bh);
-        tma_load_3d(sbase + OFF_K, &tk, &bars[BAR_LOAD], 0, kb, bh);
-        tma_load_3d(sbase + OFF_V, &tv, &bars[BAR_LOAD], 0, kb, bh);
-        bool ok = mbar_wait(&bars[BAR_LOAD], 0, abort_flag, status);
-        int committed = 0;
-        if (debug & DEBUG_SKIP_MMA) ok = false;             // testing: leave every waiter to time out
-        if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < HD / 16; ++j)
-                mma_bf16(tmem + COL_S, smem_desc_sw128(sbase + OFF_Q + 32 * j, 16, 1024),
-                         smem_desc_sw128(sbase + OFF_K + 32 * j, 16, 1024), ID_S, j > 0);
-            mma_commit(&bars[BAR_S]);
-            committed = 1;
-            ok = mbar_wait(&bars[BAR_P], 0, abort_flag, status);
-        }
-        if (ok) {
-            tc_fence_after();
-#pragma unroll
-            for (int j = 0; j < KW / 16; ++j)
-                mma_bf16(tmem + COL_O,
-                         smem_desc_sw128(sbase + OFF_P + (j >> 2) * (QT * 128) + 32 * (j & 3), 16, 1024),
-                         smem_desc_sw128(sbase + OFF_V + j * 2048, 16, 1024), ID_O, j > 0);
-            mma_commit(&bars[BAR_O]);
-            committed = 2;
-        }
-        // Never free TMEM under an MMA still in flight.
-        if (*abort_flag && committed > 0) {
-            const uint64_t t0 = global_ns();
-            uint64_t* last = committed == 2 ? &bars[BAR_O] : &bars[BAR_S];
-            while (!mbar_try_wait(last, 0) && global_ns() - t0 < kWaitLimitNs) {}
-        }
-        // The TMA load may still be landing if its wait gave up: wait (bounded) for it too.
-        if (!ok && committed == 0) {
-            const uint64_t t0 = global_ns();
-            while (!mbar_try_wait(&bars[BAR_LOAD], 0) && global_ns() - t0 < kWaitLimitNs) {}
-        }
-    }
-
-    else if (k_cache != nullptr) {
-        // Ring cache: tokens u in [max(i0, N - w), min(i0 + QT, N)) go to slot u mod w.
-        const int u0 = max(i0, N - w), u1 = min(i0 + QT, N);
-        const size_t head = (size_t)bh * N;
-        const size_t ring = (size_t)bh * w;
-        for (int e = lane - 1; e < (u1 - u0) * 16; e += 31) {
-            const int u = u0 + (e >> 4), c = e & 15;
-            const uint4* src = reinterpret_cast<const uint4*>((c < 8 ? k : v) + (head + u) * HD) + (c & 7);
-            uint4* dst = reinterpret_cast<uint4*>((c < 8 ? k_cache : v_cache) + (ring + u % w) * HD) + (c & 7);
-            *dst = __ldg(src);
-        }
-        if (blockIdx.x == 0) {
-            for (int e = lane - 1; e < max(0, w - N) * 16; e += 31) {
-                const int slot = N + (e >> 4), c = e & 15;
-                uint4* dst = reinterpret_cast<uint4*>((c < 8 ? k_cache : v_cache) + (ring + slot) * HD) + (c & 7);
-                *dst = make_uint4(0, 0, 0, 0);
-            }
-        }
+    if (warp == 0) {
+        if (lane == 0) producer(cx, &tq, &tk, &tv);
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(cx, tmem, (debug & DEBUG_SKIP_MMA) != 0);
+    } else {
+        const int g = (warp - 2) >> 2;
+        softmax_wg(cx, tmem, g, warp & 3, lane, &ty, k, v, k_cache, v_cache, scale_log2);
+        if ((warp & 3) == 0 && lane == 0) bulk_wait_all();   // the y stores have completed
     }
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 1) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
@@ -241,19 +353,25 @@ cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, v
                                   void* v_cache, int B, int H, int N, int w, float scale, unsigned* status,
                                   unsigned debug, cudaStream_t stream) {
     const uint64_t BH = (uint64_t)B * H;
-    CUtensorMap mq, mk, mv;
+    CUtensorMap mq, mk, mv, my;
     if (!make_tmap_bf16_3d(&mq, q, HD, N, BH, HD, QT) || !make_tmap_bf16_3d(&mk, k, HD, N, BH, HD, KW) ||
-        !make_tmap_bf16_3d(&mv, v, HD, N, BH, HD, KW))
+        !make_tmap_bf16_3d(&mv, v, HD, N, BH, HD, KW) || !make_tmap_bf16_3d(&my, y, HD, N, BH, HD, QT))
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(swa_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    const dim3 grid((N + QT - 1) / QT, (unsigned)BH);
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    const int nqb = (N + QT - 1) / QT;
+    const long long ntiles = (long long)nqb * (long long)BH;
+    if (ntiles > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    const int grid = (int)std::min<long long>(ntiles, (long long)sms);
     const float scale_log2 = scale * 1.4426950408889634f;     // exp(x) = exp2(x * log2(e))
     using bf = __nv_bfloat16;
     swa_prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(
-        mq, mk, mv, static_cast<const bf*>(k), static_cast<const bf*>(v), static_cast<bf*>(y),
-        static_cast<bf*>(k_cache), static_cast<bf*>(v_cache), N, w, scale_log2, status, debug);
+        mq, mk, mv, my, static_cast<const bf*>(k), static_cast<const bf*>(v), static_cast<bf*>(k_cache),
+        static_cast<bf*>(v_cache), N, w, nqb, (int)ntiles, scale_log2, status, debug);
     return cudaGetLastError();
 }
 
