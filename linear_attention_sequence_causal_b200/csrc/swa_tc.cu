@@ -20,8 +20,10 @@
 // The kernel is persistent and pipelined: one CTA per SM walks its tiles
 // (tile = CTA + k * grid) with
 //   warp 0      lane 0 issues the TMA loads into a 3-stage ring of {Q, K, V};
-//   warp 1      allocates TMEM; lane 0 issues S of tile n, then O of tile n-1,
-//               so the tensor core works while the softmax of tile n runs;
+//   warp 1      allocates TMEM; lane 0 issues S = Q K^T of each tile;
+//   warp 10     lane 0 issues O = P V of each tile once its softmax is done
+//               (two issuing warps, because one thread keeps only about one
+//               MMA per ~100 cycles in flight);
 //   warps 2-5   softmax + epilogue of even tiles (TMEM buffer 0),
 //   warps 6-9   the same for odd tiles (TMEM buffer 1); the epilogue warps also
 //               copy the tile's share of the last w tokens into the ring KV
@@ -47,7 +49,7 @@ constexpr int QT = 128;              // queries per tile
 constexpr int KW = 192;              // keys per tile: [i0 - 64, i0 + 128)
 constexpr int HD = 64;               // head dim
 constexpr int kStages = 3;           // {Q, K, V} ring depth
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;
 
 // Shared memory (offsets from a 1024-aligned base).
 constexpr uint32_t Q_BYTES = QT * HD * 2;          // 16 KB
@@ -123,28 +125,27 @@ __device__ __forceinline__ void producer(const Ctx& cx, const CUtensorMap* tq, c
     }
 }
 
-// ------------------------------------------------------------------ MMA issuer (warp 1, lane 0)
-__device__ __forceinline__ void mma_issuer(const Ctx& cx, uint32_t tmem, bool skip) {
+// ------------------------------------------------------------------ MMA issuers
+// One thread keeps only about one tcgen05.mma per ~100 cycles in flight, so S
+// and O come from two warps and overlap on the tensor core.
+
+// Never free TMEM under an MMA still in flight: after an abort, wait (bounded)
+// for the issuer's last commit.
+__device__ __forceinline__ void drain(const Ctx& cx, uint64_t* last_bar, uint32_t last_parity) {
+    if (!*cx.abort_flag || last_bar == nullptr) return;
+    const uint64_t t0 = global_ns();
+    while (!mbar_try_wait(last_bar, last_parity) && global_ns() - t0 < kWaitLimitNs) {}
+}
+
+// S = Q K^T of every local tile n (warp 1, lane 0).
+__device__ __forceinline__ void s_issuer(const Ctx& cx, uint32_t tmem) {
     uint64_t* last_bar = nullptr;
     uint32_t last_parity = 0;
-    auto issue_o = [&](int m) {              // O = P V of local tile m
-        const int s = m % kStages, b = m & 1;
-        const uint32_t v = cx.sbase + OFF_STAGE + s * STAGE_BYTES + Q_BYTES + KV_BYTES;
-        const uint32_t tb = tmem + b * BUF_COLS;
-#pragma unroll
-        for (int j = 0; j < KW / 16; ++j)
-            mma_bf16_ts(tb + COL_O, tb + COL_S + 8 * j, smem_desc_sw128(v + j * 2048, 16, 1024), ID_O, j > 0);
-        mma_commit(&cx.bars[BAR_EMPTY0 + s]);
-        mma_commit(&cx.bars[BAR_OF0 + b]);
-        last_bar = &cx.bars[BAR_OF0 + b];
-        last_parity = (m >> 1) & 1;
-    };
     int n = 0;
-    bool ok = !skip;                          // testing: issue nothing, every waiter times out
-    for (int tile = blockIdx.x; ok && tile < cx.ntiles; tile += gridDim.x, ++n) {
+    for (int tile = blockIdx.x; tile < cx.ntiles; tile += gridDim.x, ++n) {
         const int s = n % kStages, b = n & 1;
-        if (!wait_bar(cx, BAR_FULL0 + s, (n / kStages) & 1)) { ok = false; break; }
-        if (n >= 2 && !wait_bar(cx, BAR_TE0 + b, ((n >> 1) - 1) & 1)) { ok = false; break; }
+        if (!wait_bar(cx, BAR_FULL0 + s, (n / kStages) & 1)) break;
+        if (n >= 2 && !wait_bar(cx, BAR_TE0 + b, ((n >> 1) - 1) & 1)) break;   // O of tile n-2 read out
         tc_fence_after();
         const uint32_t q = cx.sbase + OFF_STAGE + s * STAGE_BYTES;
         const uint32_t tb = tmem + b * BUF_COLS;
@@ -155,24 +156,30 @@ __device__ __forceinline__ void mma_issuer(const Ctx& cx, uint32_t tmem, bool sk
         mma_commit(&cx.bars[BAR_SF0 + b]);
         last_bar = &cx.bars[BAR_SF0 + b];
         last_parity = (n >> 1) & 1;
-        // O of the previous tile, once its softmax has written P.
-        if (n >= 1) {
-            if (!wait_bar(cx, BAR_PF0 + ((n - 1) & 1), ((n - 1) >> 1) & 1)) { ok = false; break; }
-            tc_fence_after();
-            issue_o(n - 1);
-        }
     }
-    if (ok && n >= 1) {
-        if (wait_bar(cx, BAR_PF0 + ((n - 1) & 1), ((n - 1) >> 1) & 1)) {
-            tc_fence_after();
-            issue_o(n - 1);
-        }
+    drain(cx, last_bar, last_parity);
+}
+
+// O = P V of every local tile n, once its softmax has written P (warp 10, lane 0).
+__device__ __forceinline__ void o_issuer(const Ctx& cx, uint32_t tmem) {
+    uint64_t* last_bar = nullptr;
+    uint32_t last_parity = 0;
+    int n = 0;
+    for (int tile = blockIdx.x; tile < cx.ntiles; tile += gridDim.x, ++n) {
+        const int s = n % kStages, b = n & 1;
+        if (!wait_bar(cx, BAR_PF0 + b, (n >> 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t v = cx.sbase + OFF_STAGE + s * STAGE_BYTES + Q_BYTES + KV_BYTES;
+        const uint32_t tb = tmem + b * BUF_COLS;
+#pragma unroll
+        for (int j = 0; j < KW / 16; ++j)
+            mma_bf16_ts(tb + COL_O, tb + COL_S + 8 * j, smem_desc_sw128(v + j * 2048, 16, 1024), ID_O, j > 0);
+        mma_commit(&cx.bars[BAR_EMPTY0 + s]);     // S and O of tile n have read the stage
+        mma_commit(&cx.bars[BAR_OF0 + b]);
+        last_bar = &cx.bars[BAR_OF0 + b];
+        last_parity = (n >> 1) & 1;
     }
-    // Never free TMEM under an MMA still in flight.
-    if (*cx.abort_flag && last_bar != nullptr) {
-        const uint64_t t0 = global_ns();
-        while (!mbar_try_wait(last_bar, last_parity) && global_ns() - t0 < kWaitLimitNs) {}
-    }
+    drain(cx, last_bar, last_parity);
 }
 
 // ------------------------------------------------------------------ softmax + epilogue (warps 2-9)
@@ -323,6 +330,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
         mbar_fence_init();
     }
     if (warp == 1) tmem_alloc(tmem_slot, TMEM_COLS);
+    const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;     // testing: issue nothing, every waiter times out
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -331,7 +339,9 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     if (warp == 0) {
         if (lane == 0) producer(cx, &tq, &tk, &tv);
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(cx, tmem, (debug & DEBUG_SKIP_MMA) != 0);
+        if (lane == 0 && !skip_mma) s_issuer(cx, tmem);
+    } else if (warp == 10) {
+        if (lane == 0 && !skip_mma) o_issuer(cx, tmem);
     } else {
         const int g = (warp - 2) >> 2;
         softmax_wg(cx, tmem, g, warp & 3, lane, &ty, k, v, k_cache, v_cache, scale_log2);
