@@ -87,8 +87,8 @@ def load_peaks():
 
 
 KERNEL_SOURCES = {
-    "la_prefill": ["la_prefill_tc.cu", "tcgen05.cuh", "common.cuh"],
-    "swa_prefill": ["swa.cu", "common.cuh"],
+    "la_prefill": ["la_prefill_tc.cu", "tcgen05.cuh", "common.cuh", "tma_host.cu"],
+    "swa_prefill": ["swa_tc.cu", "tcgen05.cuh", "common.cuh", "tma_host.cu"],
     "la_decode": ["la_decode.cu", "common.cuh"],
     "swa_decode": ["swa.cu", "common.cuh"],
 }
@@ -663,6 +663,32 @@ def run_sweep(reps):
                           "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                           "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
         del S, z, kc, vc
+    # large state: d'=32 (D=1057), dv=128, H=8, B=4, N=8192 prefill, then decode at batch 64
+    Bl, Hl, Nl, dfl, dvl = 4, 8, 8192, 32, 128
+    Dl = _feature_dim(dfl)
+    inp = synthetic.la_inputs(Bl, Hl, Nl, dfl, dvl, "bf16", seed=0)
+    q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+    y = torch.empty(Bl, Hl, Nl, dvl, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(Bl, Hl, Dl, dvl, device=dev)
+    z = torch.empty(Bl, Hl, Dl, device=dev)
+    ms = timed(lambda: based.la_prefill(q, k, v, y=y, S=S, z=z), 1)
+    flops, byts = la_prefill_work(Bl, Hl, Nl, dfl, dvl, 32)
+    print(json.dumps({"sweep": "la_prefill_large_state", "us": ms * 1e3, "tokens_per_s": Bl * Nl / (ms / 1e3),
+                      "TFLOP_s": flops / (ms / 1e3) / 1e12,
+                      "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                      "GB_s": byts / (ms / 1e3) / 1e9}), flush=True)
+    del q, k, v, y
+    S = torch.randn(64, Hl, Dl, dvl, device=dev) * 0.01
+    z = torch.rand(64, Hl, Dl, device=dev) + 600.0
+    inp = synthetic.la_inputs(64, Hl, 1, dfl, dvl, "bf16", seed=1)
+    q, k, v = (t[:, :, 0].contiguous().to(dev) for t in (inp.q, inp.k, inp.v))
+    y = torch.empty(64, Hl, dvl, dtype=torch.bfloat16, device=dev)
+    ms = timed(lambda: based.la_decode_step(S, z, q, k, v, y=y), 32)
+    _, byts = la_decode_work(64, Hl, dfl, dvl)
+    print(json.dumps({"sweep": "la_decode_large_state", "batch": 64, "us_per_step": ms * 1e3,
+                      "tokens_per_s": 64 / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                      "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+    del S, z
     # long prefill: B=2, H=16, N=16384
     B, N = 2, 16384
     inp = synthetic.la_inputs(B, H, N, df, dv, "bf16", seed=0)
