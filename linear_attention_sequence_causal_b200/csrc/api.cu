@@ -60,18 +60,23 @@ bool simt_chunk_ok(int d_feat, int chunk) {
     return chunk == 16 || chunk == 32 || (chunk == 64 && d_feat == 16);
 }
 
-enum class LaPath { None, Simt, TensorCore };
+enum class LaPath { None, Simt, TensorCore, Quad };
 
-// Kernel choice for a prefill: the tcgen05 kernel for the bf16 shapes it is
-// built for, the fp32 CUDA-core kernel otherwise.
+// Kernel choice for a prefill. bf16: the chunked tcgen05 kernel where it is
+// built (d' = 16, dv = 64, 128-token chunks), else the tcgen05 quadratic-form
+// kernel (128-token tiles; the state of the other shapes does not fit one SM's
+// tensor memory); explicit chunks of 16, 32 or 64 tokens and every fp32 call
+// take the CUDA-core kernel.
 LaPath choose_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
     const bool bf16 = dtype == BASED_BF16;
     if (*chunk == 0) {
         if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, 128)) { *chunk = 128; return LaPath::TensorCore; }
+        if (bf16 && based::la_prefill_quad_supported(d_feat, d_v)) { *chunk = 128; return LaPath::Quad; }
         *chunk = d_feat == 16 ? 64 : 32;
         return LaPath::Simt;
     }
     if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, *chunk)) return LaPath::TensorCore;
+    if (bf16 && *chunk == 128 && based::la_prefill_quad_supported(d_feat, d_v)) return LaPath::Quad;
     if (simt_chunk_ok(d_feat, *chunk)) return LaPath::Simt;
     return LaPath::None;
 }
@@ -86,6 +91,7 @@ int device_sm_count(int dev) { return num_sms(dev); }
 unsigned current_debug_flags() { return debug_flags(); }
 int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
     switch (choose_la_path(d_feat, d_v, dtype, chunk)) {
+        case LaPath::Quad: return 3;
         case LaPath::TensorCore: return 2;
         case LaPath::Simt: return 1;
         default: return 0;
@@ -142,6 +148,8 @@ based_status_t based_la_prefill(const void* q, const void* k, const void* v, voi
         const size_t need = based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms);
         if (workspace_bytes < need || (need > 0 && !ok_ptr(workspace))) return BASED_ERR_INVALID_ARG;
         e = based::launch_la_prefill_tc(a, sms, stream);
+    } else if (path == LaPath::Quad) {
+        e = based::launch_la_prefill_quad(a, sms, stream);
     } else {
         e = based::launch_la_prefill_simt(a, stream);
     }

@@ -31,6 +31,11 @@ bool la_prefill_tc_supported(int d_feat, int d_v, int chunk);
 size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms);
 cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
 
+// Tensor-core quadratic-form path (bf16, any built d', dv): y from the masked
+// quadratic form, the final state from phi(K)^T [V|1] over all tokens.
+bool la_prefill_quad_supported(int d_feat, int d_v);
+cudaError_t launch_la_prefill_quad(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
                              void* y, int B, int H, int d_feat, int d_v, bool bf16,
                              int num_sms, cudaStream_t stream);

@@ -12,7 +12,7 @@ namespace based {
 unsigned* device_status_word(int dev);
 int device_sm_count(int dev);
 unsigned current_debug_flags();
-int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk);
+int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk);   // 0 none, 1 CUDA cores, 2 chunked tcgen05, 3 quadratic tcgen05
 }  // namespace based
 
 namespace {
@@ -69,7 +69,8 @@ extern "C" based_status_t based_la_prefill_noalloc(const void* q, const void* k,
     if (scratch == nullptr) return BASED_ERR_CUDA;
     based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype == BASED_BF16, chunk,
                            scratch, kScratchBytes, status, based::current_debug_flags()};
-    const cudaError_t e = path == 2 ? based::launch_la_prefill_tc(a, sms, stream)
-                                    : based::launch_la_prefill_simt(a, stream);
+    const cudaError_t e = path == 2   ? based::launch_la_prefill_tc(a, sms, stream)
+                          : path == 3 ? based::launch_la_prefill_quad(a, sms, stream)
+                                      : based::launch_la_prefill_simt(a, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
