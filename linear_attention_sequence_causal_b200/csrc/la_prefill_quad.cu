@@ -12,24 +12,27 @@
 // directly), needs no state during the sweep, and is a dense contraction:
 //   S   = Q_qt K_kt^T                M=128 N=128 K=d'       -> TMEM
 //   A   = 1 + S + S^2/2 (causal mask on the diagonal tile), bf16 over S in TMEM
-//   O  += A V_kt                     M=128 N=dv  K=128      (A operand in TMEM)
-//   l  += row sums of A (the rounded values the MMA sees)
+//   [O|l] += A [V_kt|1]              M=128 N=dv+16 K=128   (A operand in TMEM)
 //   y   = O / l
+// The ones column appended to V gives the denominators l from the same MMA,
+// summed over exactly the bf16 values of A the numerators use.
 // The final state S = phi(K)^T V, z = phi(K)^T 1 is a separate contraction over
 // all tokens (la_state_kernel below).
 //
 // la_quad_kernel is persistent: one CTA per SM takes units (query tile qt, head
 // bh) longest first (qt descending), and for each unit sweeps key tiles
-// kt = 0..qt. Roles (320 threads):
-//   warps 0-3  producers: cp.async of the unit's Q tile and each step's K and V
-//              tiles (thread = token row) into a 4-stage ring, completing on the
-//              stage's mbarrier; rows past the sequence end are zero-filled;
-//   warps 4-7  A: S -> A -> bf16 P in TMEM (thread = query row), row sums; at the
-//              end of a unit, y = O / l to global memory;
-//   warp 8     allocates TMEM; lane 0 issues S of every step (two TMEM buffers);
-//   warp 9     lane 0 issues O += P V of every step.
+// kt = 0..qt. Roles (448 threads):
+//   warps 0-3   producers: cp.async of the unit's Q tile and each step's K and V
+//               tiles (thread = token row) into a 4-stage ring, completing on the
+//               stage's mbarrier; rows past the sequence end are zero-filled;
+//   warps 4-7   A of the even steps: S -> A -> bf16 P in TMEM (thread = query
+//               row); at the end of every unit, y = O / l to global memory;
+//   warps 8-11  A of the odd steps (each group has its own S / P buffer);
+//   warp 12     allocates TMEM; lane 0 issues S of every step;
+//   warp 13     lane 0 issues [O|l] += P [V|1] of every step.
 // Every hand-off is an mbarrier; every wait is bounded.
 #include <algorithm>
+#include <utility>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -42,7 +45,7 @@ using namespace tc;
 
 constexpr int C = 128;               // query and key tile
 constexpr int kStages = 4;
-constexpr int kQuadThreads = 320;
+constexpr int kQuadThreads = 448;
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
@@ -57,21 +60,22 @@ template <int DF, int DV>
 struct QuadLayout {
     // K-major no-swizzle Q and K tiles (8-row x 16-byte core matrices), and the
     // MN-major no-swizzle V tile (core matrix = 8 keys x 8 values).
+    static constexpr int NV = DV + 16;                                     // [V | 1 | 0 ...]
     static constexpr uint32_t QK_BYTES = C * DF * 2;
-    static constexpr uint32_t V_BYTES = C * DV * 2;
+    static constexpr uint32_t V_BYTES = C * NV * 2;
     static constexpr uint32_t QK_LBO = 128, QK_SBO = (DF / 8) * 128;
-    static constexpr uint32_t V_LBO = (DV / 8) * 128, V_SBO = 128;
+    static constexpr uint32_t V_LBO = (NV / 8) * 128, V_SBO = 128;
     static constexpr uint32_t OFF_Q = 0;                                   // [2] by unit parity
     static constexpr uint32_t OFF_K = OFF_Q + 2 * QK_BYTES;                // [kStages]
     static constexpr uint32_t OFF_V = OFF_K + kStages * QK_BYTES;          // [kStages]
     static constexpr uint32_t OFF_BAR = OFF_V + kStages * V_BYTES;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
-    // TMEM: S / P buffers 0 and 1 (128 fp32 columns each), then O (dv columns).
+    // TMEM: S / P buffers 0 and 1 (128 fp32 columns each), then [O | l] (dv + 16 columns).
     static constexpr uint32_t COL_S = 0, COL_O = 2 * C;
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t ID_S = idesc_bf16_f32(128, C, false, false);
-    static constexpr uint32_t ID_O = idesc_bf16_f32(128, DV, false, true);
+    static constexpr uint32_t ID_O = idesc_bf16_f32(128, NV, false, true);
 };
 
 enum {
@@ -147,73 +151,79 @@ __device__ __forceinline__ void quad_producers(const QuadCtx& cx, int t, const _
     asm volatile("cp.async.wait_all;" ::: "memory");
 }
 
-// ------------------------------------------------------------------ A warps (4-7)
-// Thread = query row i of the tile = TMEM lane i (wq = lane quadrant).
+// ------------------------------------------------------------------ A warps (4-11)
+// Group g (warps 4-7: g = 0, warps 8-11: g = 1) forms A for the steps of parity
+// g, in S / P buffer g. Thread = query row i of the tile = TMEM lane i (wq =
+// lane quadrant). Group 0 also writes y = O / l at the end of every unit.
 template <int DF, int DV>
-__device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int wq, int lane,
+__device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int g, int wq, int lane,
                                           __nv_bfloat16* __restrict__ y) {
     using L = QuadLayout<DF, DV>;
     const int i = wq * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t sb = tmem + lane_off + L::COL_S + g * C;
     int step = 0, k_unit = 0;
     for (int u = blockIdx.x; u < cx.nunits; u += gridDim.x, ++k_unit) {
         int qt, bh;
         unit_of(cx, u, qt, bh);
-        float l = 0.f;
         for (int kt = 0; kt <= qt; ++kt, ++step) {
-            const int b = step & 1;
-            const uint32_t sb = tmem + lane_off + L::COL_S + b * C;
-            if (!qwait(cx, QB_SF0 + b, (step >> 1) & 1)) return;
+            if ((step & 1) != g) continue;
+            if (!qwait(cx, QB_SF0 + g, (step >> 1) & 1)) return;
             tc_fence_after();
             const bool diag = kt == qt;          // keys j > i of the diagonal tile are masked
-            // Two halves of 64 keys: half h reads S columns 64h..64h+63 and writes
-            // P columns 32h..32h+31, which overlay S columns already read.
+            // Quarter r reads S columns 32r..32r+31 and writes P columns
+            // 16r..16r+15, which overlay S columns already read.
 #pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                float sv[64];
-#pragma unroll
-                for (int m = 0; m < 4; ++m) tmem_ld16(sb + 64 * h + 16 * m, sv + 16 * m);
+            for (int r = 0; r < 4; ++r) {
+                float sv[32];
+                tmem_ld16(sb + 32 * r, sv);
+                tmem_ld16(sb + 32 * r + 16, sv + 16);
                 tmem_ld_wait();
-                uint32_t pw[32];
+                uint32_t pw[16];
 #pragma unroll
-                for (int m = 0; m < 32; ++m) {
-                    const int j0 = 64 * h + 2 * m;
+                for (int m = 0; m < 16; ++m) {
                     const float x0 = sv[2 * m], x1 = sv[2 * m + 1];
                     uint32_t wd = pack_bf16x2(fmaf(x0, fmaf(0.5f, x0, 1.0f), 1.0f), fmaf(x1, fmaf(0.5f, x1, 1.0f), 1.0f));
-                    if (diag) wd &= (j0 <= i ? 0x0000FFFFu : 0u) | (j0 + 1 <= i ? 0xFFFF0000u : 0u);
-                    l += __uint_as_float(wd << 16) + __uint_as_float(wd & 0xFFFF0000u);
+                    if (diag) {
+                        const int j0 = 32 * r + 2 * m;
+                        wd &= (j0 <= i ? 0x0000FFFFu : 0u) | (j0 + 1 <= i ? 0xFFFF0000u : 0u);
+                    }
                     pw[m] = wd;
                 }
-                tmem_st16(sb + 32 * h, pw);
-                tmem_st16(sb + 32 * h + 16, pw + 16);
+                tmem_st16(sb + 16 * r, pw);
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&cx.bars[QB_PF0 + b]);
+            mbar_arrive(&cx.bars[QB_PF0 + g]);
         }
-        // Epilogue: y = O / l for this unit's rows.
+        if (g != 0) continue;
+        // Epilogue (group 0): y = O / l for this unit's rows.
         if (!qwait(cx, QB_OF, k_unit & 1)) return;
         tc_fence_after();
-        const float inv = 1.0f / l;            // l >= 1/2 for every real row
+        const uint32_t ob = tmem + lane_off + L::COL_O;
+        float lsum[16];
+        tmem_ld16(ob + DV, lsum);
+        tmem_ld_wait();
+        const float inv = 1.0f / lsum[0];      // l >= 1/2 for every real row
         const int tok = qt * C + i;
         uint4* yp = reinterpret_cast<uint4*>(y + ((size_t)bh * cx.N + (tok < cx.N ? tok : 0)) * DV);
 #pragma unroll 1
-        for (int h = 0; h < DV / 64; ++h) {
-            float o[64];
-#pragma unroll
-            for (int m = 0; m < 4; ++m) tmem_ld16(tmem + lane_off + L::COL_O + 64 * h + 16 * m, o + 16 * m);
+        for (int h = 0; h < DV / 32; ++h) {
+            float o[32];
+            tmem_ld16(ob + 32 * h, o);
+            tmem_ld16(ob + 32 * h + 16, o + 16);
             tmem_ld_wait();
-            if (h == DV / 64 - 1) {
+            if (h == DV / 32 - 1) {
                 tc_fence_before();
                 mbar_arrive(&cx.bars[QB_OE]);      // O may be overwritten by the next unit
             }
             if (tok < cx.N) {
 #pragma unroll
-                for (int p8 = 0; p8 < 8; ++p8) {
+                for (int p8 = 0; p8 < 4; ++p8) {
                     float t8[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) t8[e] = o[8 * p8 + e] * inv;
-                    yp[8 * h + p8] = pack_bf16x8(t8);
+                    yp[4 * h + p8] = pack_bf16x8(t8);
                 }
             }
         }
@@ -314,7 +324,18 @@ la_quad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 8) tmem_alloc(tmem_slot, L::TMEM_COLS);
+    if (warp == 12) tmem_alloc(tmem_slot, L::TMEM_COLS);
+    // The ones column of [V | 1] (and the zero pad after it) never changes:
+    // write it once into every stage; cp.async only ever writes the V part.
+    if (tid < C) {
+        const uint32_t cm = (tid & 7) * 16;
+        for (int s = 0; s < kStages; ++s) {
+            const uint32_t vd = smem_u32(smem) + L::OFF_V + s * L::V_BYTES + cm + (tid >> 3) * L::V_LBO;
+            st_shared_v4(vd + (DV / 8) * L::V_SBO, make_uint4(0x3F80u, 0u, 0u, 0u));
+            st_shared_v4(vd + (DV / 8 + 1) * L::V_SBO, make_uint4(0, 0, 0, 0));
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -323,9 +344,9 @@ la_quad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 
     if (warp < 4) {
         quad_producers<DF, DV>(cx, tid, q, k, v);
-    } else if (warp < 8) {
-        quad_rows<DF, DV>(cx, tmem, warp & 3, lane, y);
-    } else if (warp == 8) {
+    } else if (warp < 12) {
+        quad_rows<DF, DV>(cx, tmem, (warp - 4) >> 2, warp & 3, lane, y);
+    } else if (warp == 12) {
         if (lane == 0 && !skip_mma) quad_s_issuer<DF, DV>(cx, tmem);
     } else {
         if (lane == 0 && !skip_mma) quad_o_issuer<DF, DV>(cx, tmem);
@@ -333,7 +354,7 @@ la_quad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 
     tc_fence_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == 12) {
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, L::TMEM_COLS);
@@ -352,6 +373,47 @@ la_quad_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restr
 // carries its 1/sqrt2 already).
 constexpr int kStateThreads = 160;
 
+// Folded feature f of [1, x_a, x_a x_b (a <= b, a-major)] as x[a] * x[b] * coef,
+// x[DF] standing for the constant; coef 0 past the last feature.
+struct FeatPair {
+    int a, b;
+    float coef;
+};
+__host__ __device__ constexpr FeatPair feat_pair(int DF, int f) {
+    if (f == 0) return FeatPair{DF, DF, 1.0f};
+    if (f <= DF) return FeatPair{f - 1, DF, 1.0f};
+    int p = f - 1 - DF, a = 0;
+    while (a < DF && p >= DF - a) { p -= DF - a; ++a; }
+    if (a >= DF) return FeatPair{DF, DF, 0.0f};
+    return FeatPair{a, a + p, p == 0 ? kSqrtHalf : 1.0f};
+}
+
+// phi(k) of one token for the 128 features of tile FT, from x (the token's k in
+// fp32, x[DF] the constant). The feature pairs are evaluated at compile time
+// (template arguments), so x stays in registers.
+template <int DF, int F>
+__device__ __forceinline__ float phi_elem(const float* x) {
+    constexpr FeatPair fp = feat_pair(DF, F);
+    return (x[fp.a] * x[fp.b]) * fp.coef;
+}
+
+template <int DF, int FT, int J, int... E>
+__device__ __forceinline__ uint4 phi_piece(const float* x, std::integer_sequence<int, E...>) {
+    const float f8[8] = {phi_elem<DF, FT * 128 + 8 * J + E>(x)...};
+    return pack_bf16x8(f8);
+}
+
+template <int DF, int FT, int... J>
+__device__ __forceinline__ void state_phi_tile_impl(const float* x, uint32_t row, uint32_t sbo,
+                                                    std::integer_sequence<int, J...>) {
+    ((st_shared_v4(row + J * sbo, phi_piece<DF, FT, J>(x, std::make_integer_sequence<int, 8>{}))), ...);
+}
+
+template <int DF, int FT>
+__device__ __forceinline__ void state_phi_tile(const float* x, uint32_t row, uint32_t sbo) {
+    state_phi_tile_impl<DF, FT>(x, row, sbo, std::make_integer_sequence<int, 16>{});
+}
+
 template <int DF, int DV>
 struct StateLayout {
     static constexpr int DS = sym_feature_dim(DF);
@@ -361,14 +423,13 @@ struct StateLayout {
     static constexpr uint32_t B_BYTES = C * NV * 2;     // [V|1]:    K = token, N = column, MN-major
     static constexpr uint32_t A_LBO = (128 / 8) * 128, A_SBO = 128;
     static constexpr uint32_t B_LBO = (NV / 8) * 128, B_SBO = 128;
-    static constexpr int XS = DF + 1;                   // per-token row: x_0..x_{d'-1}, then the constant
     static constexpr uint32_t OFF_A = 0;                // [2]
     static constexpr uint32_t OFF_B = 2 * A_BYTES;      // [2]
-    static constexpr uint32_t OFF_X = OFF_B + 2 * B_BYTES;
-    static constexpr uint32_t OFF_F = OFF_X + C * (XS + 1) * 4;   // feature table: ia, ib (bytes), coef (float)
+    static constexpr uint32_t OFF_F = OFF_B + 2 * B_BYTES;   // feature table: ia, ib (bytes), coef (float)
     static constexpr uint32_t OFF_BAR = OFF_F + 128 * 8;
     static constexpr uint32_t SMEM_BYTES = OFF_BAR + 64;
     static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+    static_assert(NFT <= 5, "feature tiles dispatched in la_state_kernel");
     static constexpr uint32_t TMEM_COLS = NV <= 128 ? 128 : 256;
     static constexpr uint32_t ID = idesc_bf16_f32(128, NV, true, true);
 };
@@ -384,7 +445,6 @@ la_state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_BAR + 8 * SB_NUM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_BAR + 8 * SB_NUM + 4);
-    float* xs = reinterpret_cast<float*>(smem + L::OFF_X);
     unsigned char* ftab = smem + L::OFF_F;
     const uint32_t sbase = smem_u32(smem);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -425,7 +485,6 @@ la_state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
     if (warp < 4) {
         const int t = tid;
         const uint32_t cm = (t & 7) * 16;
-        float* xrow = xs + t * (L::XS + 1);
         for (int c = 0; c < nchunks; ++c) {
             const int b = c & 1;
             if (c >= 2 && !mbar_wait(&bars[SB_FREE0 + b], ((c >> 1) - 1) & 1, abort_flag, status)) break;
@@ -433,17 +492,18 @@ la_state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
             const bool ok = tok < N;
             const uint4* kp = reinterpret_cast<const uint4*>(k + (bh * N + (ok ? tok : 0)) * DF);
             const uint4* vp = reinterpret_cast<const uint4*>(v + (bh * N + (ok ? tok : 0)) * DV);
+            float x[DF + 1];
 #pragma unroll
             for (int j = 0; j < DF / 8; ++j) {
                 const uint4 u = ok ? __ldg(kp + j) : make_uint4(0, 0, 0, 0);
                 const uint32_t wd[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    xrow[8 * j + 2 * e] = __uint_as_float(wd[e] << 16);
-                    xrow[8 * j + 2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
+                    x[8 * j + 2 * e] = __uint_as_float(wd[e] << 16);
+                    x[8 * j + 2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
                 }
             }
-            xrow[DF] = ok ? 1.0f : 0.0f;
+            x[DF] = ok ? 1.0f : 0.0f;
             // [V | 1]: a 16-byte piece is 8 columns of token t
             const uint32_t vb = sbase + L::OFF_B + b * L::B_BYTES + cm + (t >> 3) * L::B_LBO;
 #pragma unroll
@@ -452,15 +512,12 @@ la_state_kernel(const __nv_bfloat16* __restrict__ k, const __nv_bfloat16* __rest
             st_shared_v4(vb + (DV / 8 + 1) * L::B_SBO, make_uint4(0, 0, 0, 0));
             // phi(K) for the tile's 128 features: a 16-byte piece is 8 features of token t
             const uint32_t ab = sbase + L::OFF_A + b * L::A_BYTES + cm + (t >> 3) * L::A_LBO;
-#pragma unroll 2
-            for (int j = 0; j < 16; ++j) {
-                float f8[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const unsigned char* fe = ftab + 8 * (8 * j + e);
-                    f8[e] = xrow[fe[0]] * xrow[fe[1]] * *reinterpret_cast<const float*>(fe + 4);
-                }
-                st_shared_v4(ab + j * L::A_SBO, pack_bf16x8(f8));
+            switch (blockIdx.x % L::NFT) {
+                case 0: state_phi_tile<DF, 0>(x, ab, L::A_SBO); break;
+                case 1: state_phi_tile<DF, 1>(x, ab, L::A_SBO); break;
+                case 2: state_phi_tile<DF, 2>(x, ab, L::A_SBO); break;
+                case 3: state_phi_tile<DF, 3>(x, ab, L::A_SBO); break;
+                default: state_phi_tile<DF, 4>(x, ab, L::A_SBO); break;
             }
             fence_proxy_async_smem();
             mbar_arrive(&bars[SB_FULL0 + b]);
