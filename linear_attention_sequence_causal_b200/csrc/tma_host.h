@@ -12,4 +12,8 @@ namespace based {
 bool make_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
                        uint32_t box_x, uint32_t box_y);
 
+// The same with the 32-, 64- or 128-byte swizzle (box_x * 2 bytes must not exceed it).
+bool make_tmap_bf16_3d_swizzle(CUtensorMap* map, const void* base, uint64_t x, uint64_t y, uint64_t z,
+                               uint32_t box_x, uint32_t box_y, int swizzle_bytes);
+
 }  // namespace based

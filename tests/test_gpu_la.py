@@ -90,6 +90,30 @@ def test_zero_query_is_cumulative_mean():
     assert_y(to64(y), mean, torch.float32)
 
 
+@pytest.mark.parametrize("d_feat,d_v", [(16, 128), (32, 64), (32, 128)])
+@pytest.mark.parametrize("N", [1, 65, 129, 300])
+def test_quadratic_path_ragged(d_feat, d_v, N):
+    """bf16 shapes whose state exceeds one SM's tensor memory: quadratic-form tiles
+    with a ragged last tile, single-step units, and the separate state contraction."""
+    inp = synthetic.la_inputs(1, 3, N, d_feat, d_v, "bf16", seed=N + d_feat)
+    y, S, z = _run_prefill(inp)
+    _check_full(inp, torch.bfloat16, y, S, z)
+
+
+@pytest.mark.parametrize("d_feat,d_v", [(16, 128), (32, 64)])
+def test_quadratic_path_many_units(d_feat, d_v):
+    """More (query tile, head) units than SMs: every CTA sweeps several units of
+    different lengths, so S buffers, O accumulators and row sums change hands."""
+    B, H, N = 2, 40, 1100
+    inp = synthetic.la_inputs(B, H, N, d_feat, d_v, "bf16", seed=11)
+    y, S, z = _run_prefill(inp)
+    y2, _, _ = _run_prefill(inp, want_state=False)
+    assert torch.equal(y, y2)
+    rng = np.random.default_rng(3)
+    heads = [(0, 0), (0, 17), (1, 39)]
+    _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(N, rng, 24), heads)
+
+
 def test_outputs_stay_in_bounds_and_deterministic():
     inp = synthetic.la_inputs(1, 2, 130, 16, 64, "bf16", seed=8)
     q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
