@@ -8,9 +8,9 @@
 // K-state normalisation (App. D.4), for a chunk c of C = 128 tokens:
 //
 //   s         = Q_c K_c^T                          MMA1  M=128 N=128 K=16
-//   A         = mask(1 + s + s^2/2)                CUDA cores, TMEM -> shared memory (bf16)
+//   A         = mask(1 + s + s^2/2)                CUDA cores, TMEM -> TMEM (bf16, spare columns)
 //   Y         = phi(Q_c) [S | z]_{c-1}             MMA3  M=128 N=80  K=160 (A operand in TMEM)
-//   Y        += A [V_c | 1]                        MMA2  M=128 N=80  K=128
+//   Y        += A [V_c | 1]                        MMA2  M=128 N=80  K=128 (A operand in TMEM)
 //   [S|z]^T  += [V_c | 1]^T phi(K_c)               MMA4  M=128 N=160 K=128, fp32 in TMEM
 //   y_c       = Y[:, :64] / Y[:, 64]               epilogue
 //
@@ -29,13 +29,15 @@
 // Issue structure. One thread can keep only about one tcgen05.mma per ~117
 // cycles in flight (measured on B200 for any N <= 144), while MMAs from two
 // issuing warps into separate accumulators overlap. So two warps issue:
-//   warp 13  the Y chain: MMA3_c, MMA1_{c+1}, MMA2_c (19 instructions);
+//   warp 13  the Y chain: MMA3_c, MMA2_c, MMA1_{c+1} (19 instructions);
 //   warp 12  the state chain: MMA4_c (8 instructions of N = 160; the state is
 //            kept transposed -- TMEM lane = value column, column = feature --
 //            which halves the instruction count of the natural layout).
-// A has its own shared-memory tile, so MMA1_{c+1} can overwrite s as soon as
-// A_c has been formed, and A_{c+1} is computed while MMA2_c still reads A_c
-// (only its stores wait for MMA2_c).
+// A has its own tensor-memory columns, so MMA1_{c+1} can overwrite s as soon
+// as A_c has been formed, and A_{c+1} is computed while MMA2_c still reads A_c
+// (only its stores wait for MMA2_c). Keeping A (and phi(Q)) in tensor memory
+// matters: an MMA of N = 80 with both operands in shared memory is bound by
+// shared-memory bandwidth (6.5 KB per 40 tensor cycles).
 //
 // Other roles (448 threads, one CTA per (b, h, segment)); a warp reaches the
 // TMEM lanes of quadrant (warp mod 4):
@@ -95,9 +97,7 @@ constexpr uint32_t OFF_K = OFF_Q + 2 * QK_BYTES;
 constexpr uint32_t YS_BYTES = C * DV * 2;       // y tile, 128-byte swizzled rows (TMA store source)
 constexpr uint32_t OFF_SB = OFF_K + 2 * QK_BYTES;               // single buffer
 constexpr uint32_t OFF_YS = (OFF_SB + SB_BYTES + 1023) & ~1023u; // [2], 1024-aligned for the swizzle
-constexpr uint32_t A_BYTES = C * C * 2;         // A: M = token i, K = token j, K-major
-constexpr uint32_t OFF_A = OFF_YS + 2 * YS_BYTES;
-constexpr uint32_t OFF_BAR = OFF_A + A_BYTES;
+constexpr uint32_t OFF_BAR = OFF_YS + 2 * YS_BYTES;
 constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 
@@ -106,7 +106,6 @@ constexpr uint32_t PK_LBO = (KF / 8) * 128, PK_SBO = 128;
 constexpr uint32_t VA_LBO = (NV / 8) * 128, VA_SBO = 128;
 constexpr uint32_t QK_LBO = 128, QK_SBO = (DF / 8) * 128;
 constexpr uint32_t SB_LBO = 128, SB_SBO = (KF / 8) * 128;
-constexpr uint32_t A_LBO = 128, A_SBO = (C / 8) * 128;
 // MMA4 reads [V|1]^T as a 128-row A operand: rows 80..127 (never-read output
 // lanes) alias the next 768 bytes, which must lie inside the allocation.
 static_assert(OFF_VA + VA_BYTES + (C / 8 - 1) * VA_LBO + 15 * VA_SBO + 128 <= OFF_Q + 2 * QK_BYTES,
@@ -121,9 +120,16 @@ constexpr uint32_t COL_PQ = 224;   // phi(Q), 160 bf16 = 80 columns
 constexpr uint32_t COL_ST = 320;   // [S|z]^T: lane = value column, 160 fp32 columns = features
 constexpr uint32_t TMEM_COLS = 512;
 static_assert(COL_ST + KF <= TMEM_COLS, "tensor memory");
+// A (bf16, two keys per column) in the columns the regions above leave free:
+// key block kb (32 keys, 16 columns) at col_a(kb).
+__host__ __device__ constexpr uint32_t col_a(int kb) {
+    return kb == 0 ? 480u : kb == 1 ? 496u : kb == 2 ? COL_Y + NV : COL_PQ + KF / 2;
+}
+static_assert(COL_Y + NV + 16 <= COL_PQ && COL_PQ + KF / 2 + 16 <= COL_ST && COL_ST + KF + 32 <= TMEM_COLS,
+              "A columns");
 
 constexpr uint32_t ID_QK = idesc_bf16_f32(128, C, false, false);
-constexpr uint32_t ID_AV = idesc_bf16_f32(128, NV, false, true);   // A K-major (shared memory), [V|1] MN-major
+constexpr uint32_t ID_AV = idesc_bf16_f32(128, NV, false, true);   // A in TMEM, [V|1] MN-major
 constexpr uint32_t ID_INT = idesc_bf16_f32(128, NV, false, false);
 constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 
@@ -137,7 +143,7 @@ enum {
     BAR_PQF,                 // Y-issuer commit: MMA3 done (phi(Q) and the [S|z] bf16 buffer it read are free)
     BAR_S,                   // Y-issuer commit: s ready
     BAR_A,                   // intra warps -> Y issuer: A written to shared memory (s has been read)
-    BAR_AF,                  // Y-issuer commit: MMA2 done (the A tile is free)
+    BAR_AF,                  // Y-issuer commit: MMA2 done (the A columns are free)
     BAR_Y,                   // Y-issuer commit: Y complete
     BAR_YF,                  // epilogue warps -> Y issuer: Y read
     BAR_DS,                  // state-issuer commit: MMA4 done, the TMEM state is the state after chunk c
@@ -466,22 +472,20 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
 // Thread = token i of the chunk = TMEM lane i; WQ = the warp's lane quadrant.
 // Row i of A in bf16, by blocks of 32 keys: blocks below the quadrant's
 // diagonal are unmasked, the diagonal block keeps keys j <= i, blocks above are
-// zero and are neither loaded nor computed. The row goes to the K-major A tile
-// (16-byte pieces of 8 keys); the first store waits for MMA2 of the previous
-// chunk to have read the tile. Arriving on BAR_A also releases s to MMA1 of the
+// zero and are neither loaded nor computed. Block kb goes to the 16 TMEM
+// columns col_a(kb) of lane i; the first store waits for MMA2 of the previous
+// chunk to have read them. Arriving on BAR_A also releases s to MMA1 of the
 // next chunk.
 __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, int lane, int c) {
-    const int t = wq * 32 + lane;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    const uint32_t arow = sh.sbase + OFF_A + (t >> 3) * A_SBO + (t & 7) * 16;
     if (!mbar_wait(&sh.bars[BAR_S], c & 1, sh.abort_flag, sh.status)) return false;
     tc_fence_after();
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
-        uint4 pc[8];
+        uint32_t pw[32];                                         // keys 64h .. 64h+63, two per word
         if (2 * h > wq) {                                        // every key of this batch is in the future
 #pragma unroll
-            for (int p = 0; p < 8; ++p) pc[p] = make_uint4(0, 0, 0, 0);
+            for (int p = 0; p < 32; ++p) pw[p] = 0u;
         } else {
             float sv[64];
 #pragma unroll
@@ -491,7 +495,8 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
             for (int p = 0; p < 8; ++p) {
                 const int blk = 2 * h + p / 4;                  // key block of this piece (warp-uniform)
                 if (blk > wq) {
-                    pc[p] = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int q2 = 0; q2 < 4; ++q2) pw[4 * p + q2] = 0u;
                     continue;
                 }
                 uint32_t wd[4];
@@ -507,17 +512,19 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
                         wd[q2] &= (kk <= lane ? 0x0000FFFFu : 0u) | (kk + 1 <= lane ? 0xFFFF0000u : 0u);
                     }
                 }
-                pc[p] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+#pragma unroll
+                for (int q2 = 0; q2 < 4; ++q2) pw[4 * p + q2] = wd[q2];
             }
         }
         if (h == 0) {
             tc_fence_before();                                  // s has been read
             if (c > 0 && !mbar_wait(&sh.bars[BAR_AF], (c - 1) & 1, sh.abort_flag, sh.status)) return false;
+            tc_fence_after();
         }
-#pragma unroll
-        for (int p = 0; p < 8; ++p) st_shared_v4(arow + (8 * h + p) * A_LBO, pc[p]);
+        tmem_st16(lane_base + col_a(2 * h), pw);
+        tmem_st16(lane_base + col_a(2 * h + 1), pw + 16);
     }
-    fence_proxy_async_smem();
+    tmem_st_wait();
     tc_fence_before();
     mbar_arrive(&sh.bars[BAR_A]);
     return true;
@@ -584,7 +591,6 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
     const uint64_t dk0 = smem_desc(sb + OFF_K, QK_LBO, QK_SBO);
     const uint64_t dva0 = smem_desc(sb + OFF_VA, VA_LBO, VA_SBO);
     const uint64_t dsb0 = smem_desc(sb + OFF_SB, SB_LBO, SB_SBO);
-    const uint64_t da0 = smem_desc(sb + OFF_A, A_LBO, A_SBO);
     uint64_t* bars = sh.bars;
     uint64_t* last_bar = nullptr;
     uint32_t last_parity = 0;
@@ -618,25 +624,25 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
                 mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j, dsb0 + ((j * 2 * SB_LBO) >> 4), ID_INT, j > 0);
         }
         mma_commit(&bars[BAR_PQF]);
-        // A_c formed: s is free for MMA1 of the next chunk, issued ahead of MMA2_c.
+        // MMA2: Y += A [V|1], as soon as A_c is formed.
         if (!wait(BAR_A, c & 1)) break;
         tc_fence_after();
-        if (c + 1 < w.nchunks) {
-            if (!wait(BAR_IN0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
-            tc_fence_after();
-            mma1(c + 1);
-        }
-        // MMA2: Y += A [V|1]
         const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
 #pragma unroll
         for (int j = 0; j < C / 16; ++j)
-            mma_bf16(tmem + COL_Y, da0 + ((j * 2 * A_LBO) >> 4), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
+            mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
                      (did3 || j > 0) ? 1u : 0u);
         mma_commit(&bars[BAR_FREE0 + b]);
         mma_commit(&bars[BAR_AF]);
         mma_commit(&bars[BAR_Y]);
         last_bar = &bars[BAR_Y];
         last_parity = c & 1;
+        // MMA1 of the next chunk (s was freed when A_c was formed).
+        if (c + 1 < w.nchunks) {
+            if (!wait(BAR_IN0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
+            tc_fence_after();
+            mma1(c + 1);
+        }
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
