@@ -51,30 +51,6 @@ constexpr int kStages = 4;
 constexpr int kBufs = 3;            // S / P buffers in TMEM
 constexpr int kQuadThreads = 512;
 
-// a = 1 + s + s^2/2 for two scores at once with Blackwell's packed fp32 FMA.
-__device__ __forceinline__ void taylor_pair(float s0, float s1, float& a0, float& a1) {
-    asm("{\n\t.reg .b64 s, t, h, o;\n\t"
-        "mov.b64 s, {%2, %3};\n\t"
-        "mov.b64 h, 0x3F0000003F000000;\n\t"
-        "mov.b64 o, 0x3F8000003F800000;\n\t"
-        "fma.rn.f32x2 t, s, h, o;\n\t"
-        "fma.rn.f32x2 s, s, t, o;\n\t"
-        "mov.b64 {%0, %1}, s;\n\t}"
-        : "=f"(a0), "=f"(a1)
-        : "f"(s0), "f"(s1));
-}
-
-// (l0, l1) += (a0, a1) with the packed fp32 add.
-__device__ __forceinline__ void add_pair(float& l0, float& l1, float a0, float a1) {
-    asm("{\n\t.reg .b64 l, a;\n\t"
-        "mov.b64 l, {%0, %1};\n\t"
-        "mov.b64 a, {%2, %3};\n\t"
-        "add.rn.f32x2 l, l, a;\n\t"
-        "mov.b64 {%0, %1}, l;\n\t}"
-        : "+f"(l0), "+f"(l1)
-        : "f"(a0), "f"(a1));
-}
-
 template <int DF, int DV>
 struct QuadLayout {
     // Q and K tiles: K-major rows of d' bf16 (32 or 64 bytes) under the swizzle
@@ -107,7 +83,9 @@ enum {
     QB_FULL0, QB_FULL1, QB_FULL2, QB_FULL3,     // TMA: stage s (and the unit's Q) landed
     QB_EMPTY0, QB_EMPTY1, QB_EMPTY2, QB_EMPTY3, // O issuer commit: stage s read
     QB_SF0, QB_SF1, QB_SF2,                     // S issuer commit: S of buffer b ready
-    QB_PF0, QB_PF1, QB_PF2,                     // A group b -> O issuer: P of buffer b written
+    QB_PF0,                                     // [kBufs][2] A group b -> O issuer og: P of buffer b
+                                                // written for a step of O issuer og (step % NO)
+    QB_PF_END = QB_PF0 + 2 * kBufs - 1,
     QB_OB0, QB_OB1, QB_OB2,                     // O issuer commit: P of buffer b consumed
     QB_OF,                                      // every O issuer commits once: a unit's O complete
     QB_OE,                                      // every A thread: O read out, row sums read
@@ -116,6 +94,7 @@ enum {
     QB_NUM
 };
 static_assert(kStages == 4 && kBufs == 3, "barrier table");
+static_assert(8 * QB_NUM + 8 <= 256, "barrier area");
 
 struct QuadCtx {
     uint32_t sbase;
@@ -241,7 +220,7 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
             }
             tmem_st_wait();
             tc_fence_before();
-            mbar_arrive(&cx.bars[QB_PF0 + g]);
+            mbar_arrive(&cx.bars[QB_PF0 + 2 * g + step % L::NO]);
         }
         // Row sums: publish this group's once every group has read the previous
         // unit's (they arrive on OE only after reading them), then pool.
@@ -339,7 +318,11 @@ __device__ __forceinline__ void quad_o_issuer(const QuadCtx& cx, uint32_t tmem, 
         for (int kt = 0; kt <= qt; ++kt, ++step) {
             if (step % L::NO != og) continue;
             const int s = step % kStages, b = step % kBufs;
-            if (!qwait(cx, QB_PF0 + b, (step / kBufs) & 1)) { quad_drain(cx, last, lastp); return; }
+            // One barrier per (buffer, issuer): each is consumed in order by one
+            // thread, so a waiter is never two phases ahead of it (with two
+            // issuers sharing a buffer's barrier, the later one could be, and a
+            // parity wait would then pass on the previous phase).
+            if (!qwait(cx, QB_PF0 + 2 * b + og, (step / (kBufs * L::NO)) & 1)) { quad_drain(cx, last, lastp); return; }
             tc_fence_after();
             const uint64_t dv = smem_desc_sw128(cx.sbase + L::OFF_V + s * L::V_BYTES, L::V_BLOCK, 1024);
             const uint32_t a_tmem = tmem + L::COL_S + b * C;
@@ -378,7 +361,7 @@ la_quad_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     if (tid == 0) {
         for (int b = 0; b < QB_NUM; ++b) {
             uint32_t count = 1;
-            if (b >= QB_PF0 && b <= QB_PF2) count = 128;
+            if (b >= QB_PF0 && b <= QB_PF_END) count = 128;
             if (b == QB_L || b == QB_OE) count = kBufs * 128;
             if (b == QB_OF) count = L::NO;
             mbar_init(&bars[b], count);

@@ -502,8 +502,9 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
                 uint32_t wd[4];
 #pragma unroll
                 for (int q2 = 0; q2 < 4; ++q2) {
-                    const float x0 = sv[8 * p + 2 * q2], x1 = sv[8 * p + 2 * q2 + 1];
-                    wd[q2] = pack_bf16x2(fmaf(x0, fmaf(0.5f, x0, 1.0f), 1.0f), fmaf(x1, fmaf(0.5f, x1, 1.0f), 1.0f));
+                    float a0, a1;
+                    taylor_pair(sv[8 * p + 2 * q2], sv[8 * p + 2 * q2 + 1], a0, a1);
+                    wd[q2] = pack_bf16x2(a0, a1);
                 }
                 if (blk == wq) {                                // diagonal block: keep keys j <= i
 #pragma unroll

@@ -44,28 +44,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // kWaitLimitNs (recording DEV_ERR_TIMEOUT in *status and raising *abort so the
 // other roles stop waiting too), or as soon as another thread raised *abort.
 // Returns false when it gave up.
-static __device__ __noinline__ bool mbar_wait_slow(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                            unsigned* status) {
-    const uint64_t t0 = global_ns();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 31u) == 0) {
-            if (*abort) return false;
-            if (global_ns() - t0 > kWaitLimitNs) {
-                *abort = 1;
-                atomicOr(status, DEV_ERR_TIMEOUT);
-                return false;
-            }
-        }
+//
+// The poll loop is inline (a try_wait may suspend the thread until the phase
+// completes, and wakes it within ~100 cycles); only the periodic check of the
+// abort flag and the clock is out of line. A call to an out-of-line loop costs
+// an instruction-cache miss in a large kernel on every wait that does not
+// succeed at once, which measured several hundred cycles per hand-off.
+// Periodic check of a wait that started at t0 (0: not yet timed): returns the
+// start time, or 0 when the wait must give up.
+static __device__ __noinline__ uint64_t mbar_wait_check(uint64_t t0, volatile int* abort, unsigned* status) {
+    if (*abort) return 0;
+    const uint64_t now = global_ns();
+    if (t0 == 0) return now;
+    if (now - t0 > kWaitLimitNs) {
+        *abort = 1;
+        atomicOr(status, DEV_ERR_TIMEOUT);
+        return 0;
     }
+    return t0;
 }
 
-// The slow path (a spin with time checks) is out of line: the waits are many
-// and the fast path is one instruction, which keeps the kernels' code small.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           unsigned* status) {
-    if (mbar_try_wait(bar, parity)) return true;
-    return mbar_wait_slow(bar, parity, abort, status);
+    uint64_t t0 = 0;
+    for (uint32_t it = 1; !mbar_try_wait(bar, parity); ++it) {
+        if ((it & 63u) == 0) {
+            t0 = mbar_wait_check(t0, abort, status);
+            if (t0 == 0) return false;
+        }
+    }
+    return true;
 }
 
 // ------------------------------------------------------------------ fences
@@ -164,6 +172,31 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// a = 1 + s + s^2/2 for two scores at once with Blackwell's packed fp32 FMA
+// (fma.rn.f32x2): the second-order Taylor weight of BASED's feature map.
+__device__ __forceinline__ void taylor_pair(float s0, float s1, float& a0, float& a1) {
+    asm("{\n\t.reg .b64 s, t, h, o;\n\t"
+        "mov.b64 s, {%2, %3};\n\t"
+        "mov.b64 h, 0x3F0000003F000000;\n\t"
+        "mov.b64 o, 0x3F8000003F800000;\n\t"
+        "fma.rn.f32x2 t, s, h, o;\n\t"
+        "fma.rn.f32x2 s, s, t, o;\n\t"
+        "mov.b64 {%0, %1}, s;\n\t}"
+        : "=f"(a0), "=f"(a1)
+        : "f"(s0), "f"(s1));
+}
+
+// (l0, l1) += (a0, a1) with the packed fp32 add.
+__device__ __forceinline__ void add_pair(float& l0, float& l1, float a0, float a1) {
+    asm("{\n\t.reg .b64 l, a;\n\t"
+        "mov.b64 l, {%0, %1};\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "add.rn.f32x2 l, l, a;\n\t"
+        "mov.b64 {%0, %1}, l;\n\t}"
+        : "+f"(l0), "+f"(l1)
+        : "f"(a0), "f"(a1));
 }
 
 __device__ __forceinline__ uint4 pack_bf16x8(const float* x) {

@@ -114,6 +114,23 @@ def test_quadratic_path_many_units(d_feat, d_v):
     _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(N, rng, 24), heads)
 
 
+def test_quadratic_path_repeated_calls_agree():
+    """Two O issuers (dv = 64) hand P buffers back and forth across many steps:
+    repeated calls must all complete (no expired wait) and agree bit for bit."""
+    B, H, N = 8, 16, 2048
+    inp = synthetic.la_inputs(B, H, N, 32, 64, "bf16", seed=21)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y0, S0, z0 = based.la_prefill(q, k, v)
+    assert based.get_last_error() == 0
+    for _ in range(6):
+        y, S, z = based.la_prefill(q, k, v)
+        assert based.get_last_error() == 0
+        assert torch.equal(y, y0) and torch.equal(S, S0) and torch.equal(z, z0)
+    rng = np.random.default_rng(5)
+    heads = [(0, 0), (7, 15)]
+    _sampled_check(inp, torch.bfloat16, y0, S0, z0, heads, _rows(N, rng, 16), heads)
+
+
 def test_outputs_stay_in_bounds_and_deterministic():
     inp = synthetic.la_inputs(1, 2, 130, 16, 64, "bf16", seed=8)
     q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
