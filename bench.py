@@ -559,6 +559,9 @@ def run_reference(args):
 PROFILE_CASES = {
     # inputs larger than the 126 MB L2 so DRAM counters mean something; a few hundred MB at most
     "la_prefill": "B=32 H=16 N=2048 d'=16 dv=64 bf16 (q,k,v,y 335 MB)",
+    # quadratic-form kernel: K and V tiles are re-read from L2 by design, so a small
+    # case (one eighth of the large-state workload, y only) shows its SM behaviour
+    "la_prefill_large": "B=1 H=8 N=8192 d'=32 dv=128 bf16, y only (q,k,v,y 42 MB)",
     "swa_prefill": "B=16 H=16 N=2048 d=64 w=64 bf16 (q,k,v,y 268 MB)",
     "la_decode": "batch 256, H=16, d'=16, dv=64 (fp32 state 286 MB)",
     "swa_decode": "batch 1024, H=16, d=64, w=64 (ring caches 268 MB)",
@@ -577,6 +580,10 @@ def run_profile(kind, reps):
         inp = synthetic.la_inputs(32, 16, 2048, 16, 64, "bf16", seed=0)
         q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
         fn = lambda: based.la_prefill(q, k, v)
+    elif kind == "la_prefill_large":
+        inp = synthetic.la_inputs(1, 8, 8192, 32, 128, "bf16", seed=0)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        fn = lambda: based.la_prefill(q, k, v, want_state=False)
     elif kind == "swa_prefill":
         inp = synthetic.swa_inputs(16, 16, 2048, 64, "bf16", seed=0)
         q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
