@@ -26,9 +26,10 @@
 //               MMA per ~100 cycles in flight);
 //   warps 2-5   softmax + epilogue of even tiles (TMEM buffer 0),
 //   warps 6-9   the same for odd tiles (TMEM buffer 1); the epilogue warps also
-//               copy the tile's share of the last w tokens into the ring KV
-//               cache (slot t mod w) and, on a head's first tile, zero the
-//               slots a prompt shorter than w never fills.
+//               copy the tile's share of the last w tokens from the shared-
+//               memory stage into the ring KV cache (slot t mod w) and, on a
+//               head's first tile, zero the slots a prompt shorter than w
+//               never fills.
 // Every hand-off is an mbarrier; every wait is bounded.
 #include <cuda.h>
 #include <math.h>
@@ -241,6 +242,27 @@ __device__ __forceinline__ void softmax_wg(const Ctx& cx, uint32_t tmem, int g, 
             else tmem_st16(lane_base + COL_S + 16 * gr, zero);
         }
         tmem_st_wait();
+        // Ring cache: token u in [max(0, N - w), N) goes to slot u mod w. Its K
+        // and V rows are span rows i + 64 of this tile's stage, which stays
+        // ours until O = P V (issued after PF) has completed; the stage data is
+        // read here (its TMA has completed: FULL of this stage, this phase),
+        // not from global memory, which cost the last tile of every head a
+        // dependent round trip.
+        if (k_cache != nullptr && i0 + QT > N - w) {
+            const int n = 2 * kk + g, s = n % kStages;
+            if (!wait_bar(cx, BAR_FULL0 + s, (n / kStages) & 1)) return;
+            if (qi < N && qi >= N - w) {
+                const uint32_t kr = cx.sbase + OFF_STAGE + s * STAGE_BYTES + Q_BYTES + (i + 64) * 128;
+                const uint32_t sw = (uint32_t)((i + 64) & 7);
+                uint4* kd = reinterpret_cast<uint4*>(k_cache + ((size_t)bh * w + qi % w) * HD);
+                uint4* vd = reinterpret_cast<uint4*>(v_cache + ((size_t)bh * w + qi % w) * HD);
+#pragma unroll
+                for (int p8 = 0; p8 < HD / 8; ++p8) {
+                    kd[p8] = ld_shared_v4(kr + ((p8 ^ sw) << 4));
+                    vd[p8] = ld_shared_v4(kr + KV_BYTES + ((p8 ^ sw) << 4));
+                }
+            }
+        }
         tc_fence_before();
         mbar_arrive(&cx.bars[BAR_PF0 + g]);
 
@@ -277,21 +299,10 @@ __device__ __forceinline__ void softmax_wg(const Ctx& cx, uint32_t tmem, int g, 
             bulk_commit();
         }
 
-        // Ring cache: token u in [max(0, N - w), N) goes to slot u mod w; a head's
-        // first tile also zeroes the slots a prompt shorter than w never fills.
+        // Ring cache: a head's first tile zeroes the slots a prompt shorter than
+        // w never fills (the filled slots were written before PF).
         if (k_cache != nullptr) {
             const size_t ring = (size_t)bh * w;
-            if (qi < N && qi >= N - w) {
-                const uint4* ks = reinterpret_cast<const uint4*>(k + ((size_t)bh * N + qi) * HD);
-                const uint4* vs = reinterpret_cast<const uint4*>(v + ((size_t)bh * N + qi) * HD);
-                uint4* kd = reinterpret_cast<uint4*>(k_cache + (ring + qi % w) * HD);
-                uint4* vd = reinterpret_cast<uint4*>(v_cache + (ring + qi % w) * HD);
-#pragma unroll
-                for (int p8 = 0; p8 < HD / 8; ++p8) {
-                    kd[p8] = __ldg(ks + p8);
-                    vd[p8] = __ldg(vs + p8);
-                }
-            }
             if (i0 == 0 && N + i < w) {
                 uint4* kd = reinterpret_cast<uint4*>(k_cache + (ring + N + i) * HD);
                 uint4* vd = reinterpret_cast<uint4*>(v_cache + (ring + N + i) * HD);
