@@ -22,6 +22,16 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(flo
     return __float2bfloat16_rn(x);
 }
 
+// Programmatic dependent launch (a grid launched with
+// cudaLaunchAttributeProgrammaticStreamSerialization may start while the
+// previous grid in the stream drains). grid_dependency_wait() returns once the
+// grids this one depends on have completed and their writes are visible, and is
+// a no-op without such a dependency; nothing produced by an earlier kernel may
+// be read before it. grid_launch_dependents() lets the next such grid be
+// scheduled early.
+__device__ __forceinline__ void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // Global nanosecond timer, used to bound every spin wait.
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;

@@ -76,6 +76,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     const int r_thr = tid / G;
 
     float* Sp = S + (bh * D) * (size_t)DV + 4 * g;
+    grid_dependency_wait();
 
     // First batch of state rows: in flight before anything else.
     float4 buf[kBatch];
@@ -196,13 +197,17 @@ cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = P;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // Programmatic dependent launch: the CTAs are scheduled while the previous
+    // kernel drains and wait (griddepcontrol) before reading anything.
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV>, S, z, static_cast<const T*>(q),
                               static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), P);
 }

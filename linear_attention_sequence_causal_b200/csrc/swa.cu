@@ -239,6 +239,7 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
     const size_t bh = blockIdx.x;
     const int new_slot = (int)(t % w);
 
+    grid_dependency_wait();
     const uint4 knew = __ldg(reinterpret_cast<const uint4*>(k + bh * kHead) + c);
     const uint4 vnew = __ldg(reinterpret_cast<const uint4*>(v + bh * kHead) + c);
     const uint4 qu = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
@@ -264,6 +265,7 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
         reinterpret_cast<uint4*>(kc + (bh * w + new_slot) * kHead)[c] = knew;
         reinterpret_cast<uint4*>(vc + (bh * w + new_slot) * kHead)[c] = vnew;
     }
+    grid_launch_dependents();           // the next step may be scheduled; it waits for this one to finish
     float qv[8];
     {
         const uint32_t wd[4] = {qu.x, qu.y, qu.z, qu.w};
@@ -350,10 +352,23 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                               bool bf16, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
     if (bf16) {
-        swa_decode_bf16_kernel<<<B * H, 128, 0, stream>>>(
-            static_cast<__nv_bfloat16*>(k_cache), static_cast<__nv_bfloat16*>(v_cache), (long long)t,
-            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
-            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w, scale);
+        // Programmatic dependent launch: a step's CTAs are scheduled while the
+        // previous kernel drains and wait (griddepcontrol) before reading.
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(B * H));
+        cfg.blockDim = dim3(128);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, swa_decode_bf16_kernel, static_cast<__nv_bfloat16*>(k_cache),
+                                           static_cast<__nv_bfloat16*>(v_cache), (long long)t,
+                                           static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+                                           static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w,
+                                           scale);
+        if (e != cudaSuccess) return e;
     } else {
         swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(
             static_cast<float*>(k_cache), static_cast<float*>(v_cache), (long long)t,
