@@ -731,6 +731,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
+    grid_dependency_wait();                              // inputs and workspace may come from the previous kernel
     const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;   // testing: issue nothing, every waiter times out
 
     if (warp < 4) {
@@ -813,14 +814,12 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
     CUtensorMap ty;
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {
-        la_prefill_tc_kernel<<<BH * (nseg - 1), kThreads, SMEM_BYTES, stream>>>(
-            ty, q, k, v, y, a.S, a.z, a.N, nseg, seg_chunks, 1, ws, a.status, a.debug);
-        e = cudaGetLastError();
+        e = launch_pdl(la_prefill_tc_kernel, dim3(BH * (nseg - 1)), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v,
+                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, ws, a.status, a.debug);
         if (e != cudaSuccess) return e;
     }
-    la_prefill_tc_kernel<<<BH * nseg, kThreads, SMEM_BYTES, stream>>>(ty, q, k, v, y, a.S, a.z, a.N, nseg, seg_chunks,
-                                                                    0, ws, a.status, a.debug);
-    return cudaGetLastError();
+    return launch_pdl(la_prefill_tc_kernel, dim3(BH * nseg), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v, y, a.S,
+                      a.z, a.N, nseg, seg_chunks, 0, ws, a.status, a.debug);
 }
 
 }  // namespace based

@@ -346,6 +346,7 @@ swa_prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    grid_dependency_wait();                                  // inputs may come from the previous kernel
 
     if (warp == 0) {
         if (lane == 0) producer(cx, &tq, &tk, &tv);
@@ -390,10 +391,9 @@ cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, v
     const int grid = (int)std::min<long long>(ntiles, (long long)sms);
     const float scale_log2 = scale * 1.4426950408889634f;     // exp(x) = exp2(x * log2(e))
     using bf = __nv_bfloat16;
-    swa_prefill_tc_kernel<<<grid, kThreads, SMEM_BYTES, stream>>>(
-        mq, mk, mv, my, static_cast<const bf*>(k), static_cast<const bf*>(v), static_cast<bf*>(k_cache),
-        static_cast<bf*>(v_cache), N, w, nqb, (int)ntiles, scale_log2, status, debug);
-    return cudaGetLastError();
+    return launch_pdl(swa_prefill_tc_kernel, dim3(grid), dim3(kThreads), SMEM_BYTES, stream, mq, mk, mv, my,
+                      static_cast<const bf*>(k), static_cast<const bf*>(v), static_cast<bf*>(k_cache),
+                      static_cast<bf*>(v_cache), N, w, nqb, (int)ntiles, scale_log2, status, debug);
 }
 
 }  // namespace based
