@@ -46,6 +46,11 @@ from .taylor_la import (  # noqa: F401
     la_recurrent,
     la_chunked,
     la_taylor_terms,
+    packed_dim,
+    packed_pairs,
+    feature_map_packed,
+    la_state_packed,
+    la_recurrent_packed,
 )
 from .swa import (  # noqa: F401
     swa,

@@ -210,3 +210,68 @@ def la_taylor_terms(q, k, v):
     terms = tuple(w @ v for w in (w0, w1, w2))
     dens = tuple(w.sum(axis=-1) for w in (w0, w1, w2))
     return terms, dens
+
+
+# ---------------------------------------------------------------- symmetric (packed) state
+#
+# The order-2 block of phi is the outer product x (x) x, which is symmetric:
+# entries (a, b) and (b, a) are equal. Folding each pair gives an equivalent
+# feature map of width 1 + d' + d'(d'+1)/2 (153 at d' = 16, 561 at d' = 32):
+#     phi_s(x) = [1, x, (x_a x_b * c_ab)_{a <= b, a-major}],  c_aa = 1/sqrt(2), c_ab = 1,
+# for which phi_s(q).phi_s(k) = 1 + q.k + sum_a q_a^2 k_a^2 / 2 + sum_{a<b} q_a q_b k_a k_b
+#                             = 1 + q.k + (q.k)^2/2 = phi(q).phi(k).
+# This is a derivation from BASED §4's feature map, not a form the pages print.
+# The packed state S_s = sum_j phi_s(k_j) v_j^T, z_s = sum_j phi_s(k_j) carries
+# the same information in about half the rows.
+
+
+def packed_dim(d_feat: int) -> int:
+    """Width 1 + d' + d'(d'+1)/2 of the symmetric (packed) feature map."""
+    return 1 + d_feat + d_feat * (d_feat + 1) // 2
+
+
+def packed_pairs(d_feat: int):
+    """The (a, b) pairs of the packed order-2 features, a <= b, a-major."""
+    return [(a, b) for a in range(d_feat) for b in range(a, d_feat)]
+
+
+def feature_map_packed(x: np.ndarray) -> np.ndarray:
+    """phi_s(x) = [1, x, x_a x_b (a <= b, a-major; x_a^2 / sqrt(2) on the diagonal)], float64."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    cols = []
+    for a, b in packed_pairs(d):
+        p = x[..., a] * x[..., b]
+        cols.append(p * _SQRT_HALF if a == b else p)
+    second = np.stack(cols, axis=-1)
+    ones = np.ones(x.shape[:-1] + (1,), dtype=np.float64)
+    return np.concatenate([ones, x, second], axis=-1)
+
+
+def la_state_packed(k, v):
+    """Packed S_s = sum_j phi_s(k_j) v_j^T and z_s = sum_j phi_s(k_j), phi_s built explicitly."""
+    fk = feature_map_packed(k)
+    v = np.asarray(v, dtype=np.float64)
+    return np.swapaxes(fk, -1, -2) @ v, fk.sum(axis=-2)
+
+
+def la_recurrent_packed(q, k, v, S0=None, z0=None):
+    """The recurrent form of la_recurrent with the packed feature map and state."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    *lead, n, d_feat = q.shape
+    dv = v.shape[-1]
+    Ds = packed_dim(d_feat)
+    S = np.zeros(tuple(lead) + (Ds, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    z = np.zeros(tuple(lead) + (Ds,)) if z0 is None else np.array(z0, dtype=np.float64)
+    y = np.empty(tuple(lead) + (n, dv), dtype=np.float64)
+    fq = feature_map_packed(q)
+    fk = feature_map_packed(k)
+    for t in range(n):
+        S += fk[..., t, :, None] * v[..., t, None, :]
+        z += fk[..., t, :]
+        num = np.einsum("...f,...fe->...e", fq[..., t, :], S)
+        den = np.einsum("...f,...f->...", fq[..., t, :], z)
+        y[..., t, :] = num / den[..., None]
+    return y, S, z

@@ -193,6 +193,67 @@ def test_la_converges_to_softmax_at_third_order():
     assert 6.5 < r1 < 9.5 and 7.0 < r2 < 9.0, (r1, r2)
 
 
+# ---------------------------------------------------------------- packed (symmetric) state
+
+def test_packed_width_and_pair_order():
+    assert oracle.packed_dim(16) == 153 and oracle.packed_dim(32) == 561
+    assert oracle.packed_pairs(3) == [(0, 0), (0, 1), (0, 2), (1, 1), (1, 2), (2, 2)]
+    assert len(oracle.packed_pairs(32)) == 32 * 33 // 2
+
+
+def test_packed_feature_map_hand_example():
+    # d' = 2, x = (3, -2): [1, x0, x1, x0^2/sqrt2, x0 x1, x1^2/sqrt2], written out by hand.
+    r = math.sqrt(0.5)
+    want = [1.0, 3.0, -2.0, 9.0 * r, -6.0, 4.0 * r]
+    got = oracle.feature_map_packed(np.array([3.0, -2.0]))
+    assert np.allclose(got, want, rtol=0, atol=1e-15)
+
+
+@pytest.mark.parametrize("d", [1, 2, 16, 32])
+def test_packed_product_is_taylor_polynomial(d):
+    q = RNG.standard_normal((40, d))
+    k = RNG.standard_normal((40, d))
+    s = np.sum(q * k, axis=-1)
+    got = np.sum(oracle.feature_map_packed(q) * oracle.feature_map_packed(k), axis=-1)
+    assert np.allclose(got, 1.0 + s + 0.5 * s * s, rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("d,dv", [(16, 64), (32, 8)])
+def test_packed_state_folds_the_full_state(d, dv):
+    # Independent constructions: the full state from phi, the packed one from
+    # phi_s. Entry (a, b), a < b, of the packed state is the two mirrored full
+    # entries (each x_a x_b / sqrt2) added and scaled by 1/sqrt2.
+    _, k, v = _qkv(1, 2, 37, d, dv, seed=5)
+    S, z = oracle.la_state(k, v)
+    Ss, zs = oracle.la_state_packed(k, v)
+    assert np.allclose(Ss[..., : 1 + d, :], S[..., : 1 + d, :], rtol=1e-12, atol=1e-12)
+    assert np.allclose(zs[..., : 1 + d], z[..., : 1 + d], rtol=1e-12, atol=1e-12)
+    r = math.sqrt(0.5)
+    for idx, (a, b) in enumerate(oracle.packed_pairs(d)):
+        f_ab, f_ba = 1 + d + a * d + b, 1 + d + b * d + a
+        want_S = S[..., f_ab, :] if a == b else (S[..., f_ab, :] + S[..., f_ba, :]) * r
+        want_z = z[..., f_ab] if a == b else (z[..., f_ab] + z[..., f_ba]) * r
+        assert np.allclose(Ss[..., 1 + d + idx, :], want_S, rtol=1e-12, atol=1e-12)
+        assert np.allclose(zs[..., 1 + d + idx], want_z, rtol=1e-12, atol=1e-12)
+
+
+def test_packed_recurrent_matches_quadratic_form():
+    q, k, v = _qkv(2, 2, 50, 16, 8, seed=9)
+    y, Ss, zs = oracle.la_recurrent_packed(q, k, v)
+    assert np.allclose(y, oracle.la_quadratic(q, k, v), rtol=1e-10, atol=1e-12)
+    Ss_ref, zs_ref = oracle.la_state_packed(k, v)
+    assert np.allclose(Ss, Ss_ref, rtol=1e-12, atol=1e-12)
+    assert np.allclose(zs, zs_ref, rtol=1e-12, atol=1e-12)
+    assert np.all(zs[..., 0] == 50.0)
+
+
+def test_packed_decode_continues_packed_prefill():
+    q, k, v = _qkv(1, 3, 40, 32, 4, seed=11)
+    S0, z0 = oracle.la_state_packed(k[..., :25, :], v[..., :25, :])
+    y, _, _ = oracle.la_recurrent_packed(q[..., 25:, :], k[..., 25:, :], v[..., 25:, :], S0, z0)
+    assert np.allclose(y, oracle.la_quadratic(q, k, v)[..., 25:, :], rtol=1e-10, atol=1e-12)
+
+
 # ---------------------------------------------------------------- sliding window
 
 def test_swa_hand_example(golden_dir):
@@ -314,3 +375,26 @@ def test_mutant_window_off_by_one_caught(golden_dir):
     # a window of w+1 keys (reading "preceding w keys" as excluding self)
     y = oracle.swa(a("q"), a("k"), a("v"), g["w"] + 1, g["scale"])
     assert not np.allclose(y[0, 0, :, 0], g["y"])
+
+
+def _mut_phi_packed(x, diag_scale, off_scale):
+    """A copy of the packed feature map with the pair coefficients replaced."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    cols = [x[..., a] * x[..., b] * (diag_scale if a == b else off_scale) for a, b in oracle.packed_pairs(d)]
+    return np.concatenate([np.ones(x.shape[:-1] + (1,)), x, np.stack(cols, axis=-1)], axis=-1)
+
+
+@pytest.mark.parametrize("diag_scale,off_scale", [
+    (1.0, 1.0),                  # 1/sqrt2 dropped on the diagonal
+    (math.sqrt(0.5), math.sqrt(0.5)),   # off-diagonal pairs scaled as in the unfolded map
+])
+def test_mutant_packed_coefficients_caught(diag_scale, off_scale):
+    q = RNG.standard_normal((10, 16))
+    k = RNG.standard_normal((10, 16))
+    s = np.einsum("nd,nd->n", q, k)
+    lhs = np.einsum("nf,nf->n", _mut_phi_packed(q, diag_scale, off_scale), _mut_phi_packed(k, diag_scale, off_scale))
+    assert not np.allclose(lhs, 1 + s + s * s / 2)
+    r = math.sqrt(0.5)
+    assert not np.allclose(_mut_phi_packed(np.array([3.0, -2.0]), diag_scale, off_scale),
+                           [1.0, 3.0, -2.0, 9.0 * r, -6.0, 4.0 * r])
