@@ -166,6 +166,45 @@ BASED_API based_status_t based_la_decode_step(float* S, float* z,
                                     based_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * Symmetric (packed) state layout -- an extension of this library, not a form
+ * the pages print. The order-2 block of phi is the symmetric outer product
+ * x (x) x, so the state needs only one row per unordered pair (a, b):
+ *     phi_s(x) = [1, x, x_a x_b for a <= b (a-major), times 1/sqrt2 when a == b],
+ * D_s = 1 + d_feat + d_feat (d_feat + 1) / 2 rows (153 at d_feat 16, 561 at 32),
+ * with phi_s(q).phi_s(k) = phi(q).phi(k) = 1 + q.k + (q.k)^2/2 (derived from
+ * BASED §4 "Taylor Linear Attention"). Row order: 0 the constant, 1..d_feat
+ * the x_a, then 1 + d_feat + p for the p-th pair (a, b) in the order
+ * (0,0), (0,1), .., (0,d_feat-1), (1,1), .., (d_feat-1,d_feat-1). In terms of
+ * the full layout, packed row (a, b) equals full row (a, a) when a == b and
+ * (full (a, b) + full (b, a)) / sqrt2 when a < b. Decode reads and writes
+ * ~44 % fewer state bytes per token in this layout.
+ */
+
+/*
+ * based_la_prefill_packed -- based_la_prefill, writing the final state in the
+ * symmetric layout: S [B, H, D_s, d_v] and z [B, H, D_s] (float). Arguments,
+ * workspace (based_la_prefill_workspace gives its size), results for y, and
+ * errors are those of based_la_prefill.
+ */
+BASED_API based_status_t based_la_prefill_packed(const void* q, const void* k, const void* v, void* y,
+                                                 float* S, float* z,
+                                                 int B, int H, int N, int d_feat, int d_v,
+                                                 based_dtype_t dtype, int chunk,
+                                                 void* workspace, size_t workspace_bytes,
+                                                 cudaStream_t stream);
+
+/*
+ * based_la_decode_step_packed -- based_la_decode_step on a state in the
+ * symmetric layout: S [B, H, D_s, d_v] and z [B, H, D_s], read and written in
+ * place. Arguments, results and errors are otherwise those of
+ * based_la_decode_step.
+ */
+BASED_API based_status_t based_la_decode_step_packed(float* S, float* z,
+                                                     const void* q, const void* k, const void* v, void* y,
+                                                     int B, int H, int d_feat, int d_v,
+                                                     based_dtype_t dtype, cudaStream_t stream);
+
+/*
  * based_swa_prefill -- causal sliding-window softmax attention over N tokens:
  *     y_i = sum_j softmax_j(scale * q_i.k_j) v_j  over  i - w < j <= i
  * (w keys including the query's own position). BASED §4 "Local Exact

@@ -9,6 +9,7 @@ from .binding import (  # noqa: F401
     BasedError,
     SYMBOLS,
     feature_dim,
+    packed_dim,
     get_last_error,
     la_decode_step,
     la_prefill,

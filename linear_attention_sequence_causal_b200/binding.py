@@ -27,6 +27,8 @@ SYMBOLS = (
     "based_la_prefill_workspace",
     "based_la_prefill_noalloc",
     "based_la_decode_step",
+    "based_la_prefill_packed",
+    "based_la_decode_step_packed",
     "based_swa_prefill",
     "based_swa_decode",
     "based_get_last_error",
@@ -54,6 +56,10 @@ def _declare(lib):
     lib.based_la_prefill_workspace.restype = sz
     lib.based_la_decode_step.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.based_la_decode_step.restype = i
+    lib.based_la_prefill_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, vp, sz, vp]
+    lib.based_la_prefill_packed.restype = i
+    lib.based_la_decode_step_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.based_la_decode_step_packed.restype = i
     lib.based_swa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.based_swa_prefill.restype = i
     lib.based_swa_decode.argtypes = [vp, vp, ctypes.c_int64, vp, vp, vp, vp, i, i, i, i, f, i, vp]
@@ -125,20 +131,26 @@ def feature_dim(d_feat: int) -> int:
     return 1 + d_feat + d_feat * d_feat
 
 
+def packed_dim(d_feat: int) -> int:
+    """Rows of the symmetric (packed) state: 1 + d' + d'(d'+1)/2."""
+    return 1 + d_feat + d_feat * (d_feat + 1) // 2
+
+
 def la_prefill_workspace(B, H, N, d_feat, d_v, dtype=torch.bfloat16, chunk=0) -> int:
     return int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, _DTYPES[dtype], chunk))
 
 
 def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None, z=None,
-               workspace=None) -> Tuple[torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
+               workspace=None, packed: bool = False) -> Tuple[torch.Tensor, Optional[torch.Tensor], Optional[torch.Tensor]]:
     """Causal Taylor linear attention over [B,H,N,*] inputs; returns (y, S, z).
 
-    S [B,H,D,dv] and z [B,H,D] (float32) hold the final state when want_state.
+    S [B,H,D,dv] and z [B,H,D] (float32) hold the final state when want_state;
+    D = 1 + d' + d'^2, or 1 + d' + d'(d'+1)/2 with packed (symmetric layout).
     """
     dt = _dtype_code(q, k, v)
     B, H, N, d_feat = q.shape
     d_v = v.shape[-1]
-    D = feature_dim(d_feat)
+    D = packed_dim(d_feat) if packed else feature_dim(d_feat)
     dev = q.device
     with torch.cuda.device(dev):
         if y is None:
@@ -151,10 +163,12 @@ def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None,
         ws_bytes = int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, dt, chunk))
         if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-        st = lib().based_la_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z),
-                                    B, H, N, d_feat, d_v, dt, chunk,
-                                    _ptr(workspace) if ws_bytes else None, ws_bytes, _stream(dev))
-    _check(st, "based_la_prefill")
+        if S is not None and (tuple(S.shape) != (B, H, D, d_v) or tuple(z.shape) != (B, H, D)):
+            raise BasedError(ERR_INVALID_ARG, f"S, z must be [{B},{H},{D},{d_v}] and [{B},{H},{D}]")
+        fn = lib().based_la_prefill_packed if packed else lib().based_la_prefill
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z), B, H, N, d_feat, d_v, dt, chunk,
+                _ptr(workspace) if ws_bytes else None, ws_bytes, _stream(dev))
+    _check(st, "based_la_prefill_packed" if packed else "based_la_prefill")
     return y, S, z
 
 
@@ -180,18 +194,25 @@ def la_prefill_noalloc(q, k, v, chunk: int = 0, want_state: bool = True, y=None,
     return y, S, z
 
 
-def la_decode_step(S, z, q, k, v, y=None) -> torch.Tensor:
-    """One recurrent step, S and z updated in place; q, k [B,H,d'], v [B,H,dv]."""
+def la_decode_step(S, z, q, k, v, y=None, packed: bool = False) -> torch.Tensor:
+    """One recurrent step, S and z updated in place; q, k [B,H,d'], v [B,H,dv].
+
+    packed: S, z are in the symmetric layout (1 + d' + d'(d'+1)/2 rows)."""
     dt = _dtype_code(q, k, v)
     B, H, d_feat = q.shape
     d_v = v.shape[-1]
+    D = packed_dim(d_feat) if packed else feature_dim(d_feat)
+    if tuple(S.shape) != (B, H, D, d_v) or tuple(z.shape) != (B, H, D):
+        raise BasedError(ERR_INVALID_ARG, f"S, z must be [{B},{H},{D},{d_v}] and [{B},{H},{D}]")
+    if S.dtype != torch.float32 or z.dtype != torch.float32 or not (S.is_contiguous() and z.is_contiguous()):
+        raise BasedError(ERR_INVALID_ARG, "S and z must be contiguous float32")
     dev = q.device
     with torch.cuda.device(dev):
         if y is None:
             y = torch.empty((B, H, d_v), dtype=q.dtype, device=dev)
-        st = lib().based_la_decode_step(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(y),
-                                        B, H, d_feat, d_v, dt, _stream(dev))
-    _check(st, "based_la_decode_step")
+        fn = lib().based_la_decode_step_packed if packed else lib().based_la_decode_step
+        st = fn(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(y), B, H, d_feat, d_v, dt, _stream(dev))
+    _check(st, "based_la_decode_step_packed" if packed else "based_la_decode_step")
     return y
 
 

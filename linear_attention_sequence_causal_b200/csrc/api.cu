@@ -124,10 +124,13 @@ size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int d_v, base
     return based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, num_sms(dev));
 }
 
-based_status_t based_la_prefill(const void* q, const void* k, const void* v, void* y, float* S,
-                                float* z, int B, int H, int N, int d_feat, int d_v,
-                                based_dtype_t dtype, int chunk, void* workspace,
-                                size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+based_status_t la_prefill_impl(const void* q, const void* k, const void* v, void* y, float* S, float* z, int B,
+                               int H, int N, int d_feat, int d_v, based_dtype_t dtype, int chunk, void* workspace,
+                               size_t workspace_bytes, bool packed, cudaStream_t stream) {
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
     if ((S == nullptr) != (z == nullptr)) return BASED_ERR_INVALID_ARG;
     if (S != nullptr && (!aligned16(S) || !aligned16(z))) return BASED_ERR_INVALID_ARG;
@@ -142,7 +145,7 @@ based_status_t based_la_prefill(const void* q, const void* k, const void* v, voi
     if (path == LaPath::None) return BASED_ERR_UNSUPPORTED;
 
     based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype == BASED_BF16, chunk,
-                           workspace, workspace_bytes, status, debug_flags()};
+                           workspace, workspace_bytes, status, debug_flags(), packed};
     cudaError_t e;
     if (path == LaPath::TensorCore) {
         const size_t need = based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms);
@@ -156,9 +159,8 @@ based_status_t based_la_prefill(const void* q, const void* k, const void* v, voi
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
-based_status_t based_la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
-                                    void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
-                                    cudaStream_t stream) {
+based_status_t la_decode_impl(float* S, float* z, const void* q, const void* k, const void* v, void* y, int B,
+                              int H, int d_feat, int d_v, based_dtype_t dtype, bool packed, cudaStream_t stream) {
     if (!ok_ptr(S) || !ok_ptr(z) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y))
         return BASED_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
@@ -167,9 +169,41 @@ based_status_t based_la_decode_step(float* S, float* z, const void* q, const voi
     if (!current_device(&dev)) return BASED_ERR_CUDA;
     const int sms = num_sms(dev);
     if (sms <= 0) return BASED_ERR_CUDA;
-    const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, B, H, d_feat, d_v,
-                                                  dtype == BASED_BF16, sms, stream);
+    const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, B, H, d_feat, d_v, dtype == BASED_BF16,
+                                                  packed, sms, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+based_status_t based_la_prefill(const void* q, const void* k, const void* v, void* y, float* S,
+                                float* z, int B, int H, int N, int d_feat, int d_v,
+                                based_dtype_t dtype, int chunk, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream) {
+    return la_prefill_impl(q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype, chunk, workspace, workspace_bytes,
+                           false, stream);
+}
+
+based_status_t based_la_prefill_packed(const void* q, const void* k, const void* v, void* y, float* S,
+                                       float* z, int B, int H, int N, int d_feat, int d_v,
+                                       based_dtype_t dtype, int chunk, void* workspace,
+                                       size_t workspace_bytes, cudaStream_t stream) {
+    return la_prefill_impl(q, k, v, y, S, z, B, H, N, d_feat, d_v, dtype, chunk, workspace, workspace_bytes,
+                           true, stream);
+}
+
+based_status_t based_la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
+                                    void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
+                                    cudaStream_t stream) {
+    return la_decode_impl(S, z, q, k, v, y, B, H, d_feat, d_v, dtype, false, stream);
+}
+
+based_status_t based_la_decode_step_packed(float* S, float* z, const void* q, const void* k, const void* v,
+                                           void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
+                                           cudaStream_t stream) {
+    return la_decode_impl(S, z, q, k, v, y, B, H, d_feat, d_v, dtype, true, stream);
 }
 
 based_status_t based_swa_prefill(const void* q, const void* k, const void* v, void* y, void* k_cache,

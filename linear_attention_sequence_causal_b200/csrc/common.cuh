@@ -53,6 +53,18 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
+// Symmetric (packed) feature order: 0 is the constant, 1..d' are x_a, and
+// 1 + d' + p for the p-th pair (a, b), a <= b, a-major, is x_a x_b (times
+// 1/sqrt2 when a == b). packed_pair(p) returns (a, b) of pair p.
+__host__ __device__ inline void packed_pair(int p, int d_feat, int& a, int& b) {
+    a = 0;
+    while (p >= d_feat - a) {
+        p -= d_feat - a;
+        ++a;
+    }
+    b = a + p;
+}
+
 // Global nanosecond timer, used to bound every spin wait.
 __device__ __forceinline__ uint64_t global_ns() {
     uint64_t t;

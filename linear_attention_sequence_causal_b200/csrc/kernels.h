@@ -17,6 +17,7 @@ struct LaPrefillArgs {
     void* workspace; size_t ws_bytes;
     unsigned* status;                // device status word
     unsigned debug;                  // DEBUG_* bits (testing only)
+    bool packed = false;             // final state in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
 };
 
 // Testing aid: with this bit the tensor-core kernels issue no MMA, so their
@@ -36,8 +37,9 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
 bool la_prefill_quad_supported(int d_feat, int d_v);
 cudaError_t launch_la_prefill_quad(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
 
+// `packed`: S and z hold the symmetric layout (1 + d' + d'(d'+1)/2 rows).
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
-                             void* y, int B, int H, int d_feat, int d_v, bool bf16,
+                             void* y, int B, int H, int d_feat, int d_v, bool bf16, bool packed,
                              int num_sms, cudaStream_t stream);
 
 cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y,

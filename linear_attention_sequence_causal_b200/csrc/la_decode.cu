@@ -7,6 +7,9 @@
 //
 // The step is bound by HBM: each (b, h) reads and writes its fp32 state once
 // (D x dv + D floats, 70 KB at d' = 16, dv = 64) while doing ~0.5 flop per byte.
+// The same kernel serves the symmetric layout (1 + d' + d'(d'+1)/2 rows: 39 KB
+// at d' = 16), whose rows (a, b), a <= b, hold x_a x_b unscaled off the
+// diagonal; each CTA tabulates the pairs of its rows once.
 //
 // Work split: a head's D feature rows are cut into P contiguous row ranges,
 // one CTA each, and the P CTAs of a head form one thread-block cluster
@@ -44,6 +47,16 @@ __device__ __forceinline__ float phi_entry(const float* x, int f) {
     return (x[p / DF] * x[p % DF]) * kSqrtHalf;
 }
 
+// Feature f of the symmetric layout; `pair` = (a << 8) | b of its pair (a <= b).
+template <int DF>
+__device__ __forceinline__ float phi_entry_packed(const float* x, int f, unsigned pair) {
+    if (f == 0) return 1.0f;
+    if (f <= DF) return x[f - 1];
+    const int a = pair >> 8, b = pair & 0xFF;
+    const float p = x[a] * x[b];
+    return a == b ? p * kSqrtHalf : p;
+}
+
 __device__ __forceinline__ void fma4(float4& acc, float s, const float4& x) {
     acc.x = fmaf(s, x.x, acc.x);
     acc.y = fmaf(s, x.y, acc.y);
@@ -51,11 +64,11 @@ __device__ __forceinline__ void fma4(float4& acc, float s, const float4& x) {
     acc.w = fmaf(s, x.w, acc.w);
 }
 
-template <typename T, int DF, int DV>
+template <typename T, int DF, int DV, bool PACKED>
 __global__ void __launch_bounds__(kThreads)
 la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restrict__ q,
                  const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y, int P) {
-    constexpr int D = feature_dim(DF);
+    constexpr int D = PACKED ? sym_feature_dim(DF) : feature_dim(DF);
     constexpr int G = DV / 4;              // float4 column groups per row
     constexpr int RPS = kThreads / G;      // rows per sweep of the CTA
     constexpr int NW = kThreads / 32;
@@ -66,6 +79,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     __shared__ float4 s_red[NW][G];
     __shared__ float s_dred[NW];
     __shared__ float s_out[DV + 1];        // this CTA's partial numerator and denominator
+    __shared__ unsigned short s_pair[PACKED ? 2 * kThreads : 1];   // pair (a, b) of this CTA's rows
 
     const int tid = threadIdx.x;
     const int rank = (int)(blockIdx.x % (unsigned)P);
@@ -100,7 +114,18 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
         s_x[1][tid] = to_f32(k[bh * DF + tid]);
     }
     if (tid < DV) s_v[tid] = to_f32(v[bh * DV + tid]);
+    if constexpr (PACKED) {
+        for (int j = tid; j < f1 - f0; j += kThreads) {
+            int a = 0, b = 0;
+            if (f0 + j > DF) packed_pair(f0 + j - 1 - DF, DF, a, b);
+            s_pair[j] = (unsigned short)((a << 8) | b);
+        }
+    }
     __syncthreads();
+    auto phi = [&](const float* x, int f) {
+        if constexpr (PACKED) return phi_entry_packed<DF>(x, f, s_pair[f - f0]);
+        else return phi_entry<DF>(x, f);
+    };
 
     // Denominator part over this CTA's rows; z updated in place.
     float dpart = 0.f;
@@ -108,9 +133,9 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     for (int i = 0; i < 2; ++i) {
         const int f = f0 + tid + i * kThreads;
         if (f < f1) {
-            const float zn = zr[i] + phi_entry<DF>(s_x[1], f);
+            const float zn = zr[i] + phi(s_x[1], f);
             zbh[f] = zn;
-            dpart = fmaf(phi_entry<DF>(s_x[0], f), zn, dpart);
+            dpart = fmaf(phi(s_x[0], f), zn, dpart);
         }
     }
 
@@ -122,9 +147,9 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
             const int f = base + u * RPS;
             if (f < f1) {
                 float4 s = buf[u];
-                fma4(s, phi_entry<DF>(s_x[1], f), vv);
+                fma4(s, phi(s_x[1], f), vv);
                 *reinterpret_cast<float4*>(Sp + (size_t)f * DV) = s;
-                fma4(acc, phi_entry<DF>(s_x[0], f), s);
+                fma4(acc, phi(s_x[0], f), s);
             }
         }
         const int next = base + kBatch * RPS;
@@ -188,10 +213,10 @@ int ranks_per_head(int BH, int D, int num_sms) {
     return P;
 }
 
-template <typename T, int DF, int DV>
+template <typename T, int DF, int DV, bool PACKED>
 cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const void* v, void* y,
                          int BH, int num_sms, cudaStream_t stream) {
-    const int P = ranks_per_head(BH, feature_dim(DF), num_sms);
+    const int P = ranks_per_head(BH, PACKED ? sym_feature_dim(DF) : feature_dim(DF), num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)BH * P);
     cfg.blockDim = dim3(kThreads);
@@ -208,28 +233,31 @@ cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV>, S, z, static_cast<const T*>(q),
+    return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV, PACKED>, S, z, static_cast<const T*>(q),
                               static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), P);
 }
 
-template <typename T>
+template <typename T, bool PACKED>
 cudaError_t dispatch(float* S, float* z, const void* q, const void* k, const void* v, void* y,
                      int BH, int d_feat, int d_v, int num_sms, cudaStream_t stream) {
-    if (d_feat == 16 && d_v == 64) return launch_typed<T, 16, 64>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 16 && d_v == 128) return launch_typed<T, 16, 128>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 64) return launch_typed<T, 32, 64>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 128) return launch_typed<T, 32, 128>(S, z, q, k, v, y, BH, num_sms, stream);
+    if (d_feat == 16 && d_v == 64) return launch_typed<T, 16, 64, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
+    if (d_feat == 16 && d_v == 128) return launch_typed<T, 16, 128, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
+    if (d_feat == 32 && d_v == 64) return launch_typed<T, 32, 64, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
+    if (d_feat == 32 && d_v == 128) return launch_typed<T, 32, 128, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
-                             void* y, int B, int H, int d_feat, int d_v, bool bf16, int num_sms,
+                             void* y, int B, int H, int d_feat, int d_v, bool bf16, bool packed, int num_sms,
                              cudaStream_t stream) {
     const int BH = B * H;
-    return bf16 ? dispatch<__nv_bfloat16>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream)
-                : dispatch<float>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream);
+    if (packed)
+        return bf16 ? dispatch<__nv_bfloat16, true>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream)
+                    : dispatch<float, true>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream);
+    return bf16 ? dispatch<__nv_bfloat16, false>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream)
+                : dispatch<float, false>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream);
 }
 
 }  // namespace based

@@ -487,7 +487,7 @@ enum { SB_FULL0, SB_FULL1, SB_PHI0, SB_PHI1, SB_FREE0, SB_FREE1, SB_DONE, SB_NUM
 template <int DF, int DV>
 __global__ void __launch_bounds__(kStateThreads, 2)
 la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                float* __restrict__ S, float* __restrict__ z, int N, unsigned* status, unsigned debug) {
+                float* __restrict__ S, float* __restrict__ z, int N, int packed, unsigned* status, unsigned debug) {
     using L = StateLayout<DF, DV>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -615,17 +615,17 @@ la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
         }
     }
 
-    // Epilogue: thread = feature f0 + tid (TMEM lane), rows of the full layout.
+    // Epilogue: thread = feature f0 + tid (TMEM lane), rows of the full or the symmetric layout.
     if (warp < 4 && mbar_wait(&bars[SB_DONE], 0, abort_flag, status)) {
         tc_fence_after();
         const int f = f0 + tid;
         const int ia = ftab[8 * tid], ib = ftab[8 * tid + 1];
-        constexpr int D = feature_dim(DF);
+        // Full layout: the constant, the d' linear rows, and each folded pair in
+        // rows (a, b) and (b, a). Symmetric layout: the folded row itself.
+        const int D = packed ? L::DS : feature_dim(DF);
         int r0 = 0, r1 = -1;
         float coef = 1.0f;
-        if (f == 0) {
-            r0 = 0;
-        } else if (f <= DF) {
+        if (packed || f <= DF) {
             r0 = f;
         } else {
             r0 = 1 + DF + ia * DF + ib;
@@ -691,7 +691,8 @@ cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t 
     auto sk = la_state_kernel<DF, DV>;
     e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    sk<<<BH * SL::NFT, kStateThreads, SL::SMEM_BYTES, stream>>>(sk_map, sv_map, a.S, a.z, a.N, a.status, a.debug);
+    sk<<<BH * SL::NFT, kStateThreads, SL::SMEM_BYTES, stream>>>(sk_map, sv_map, a.S, a.z, a.N, a.packed ? 1 : 0,
+                                                                 a.status, a.debug);
     return cudaGetLastError();
 }
 

@@ -21,7 +21,8 @@
 // i.e. 1 + d' + d'(d'+1)/2 distinct features instead of 1 + d' + d'^2. The final
 // state is written out in the full layout: S[1+d'+a*d'+b] = S[1+d'+b*d'+a] is
 // the folded entry scaled by 1/sqrt2 when a != b, and the folded entry itself
-// when a == b.
+// when a == b -- or, for the packed entry points, as it is (the fold is the
+// symmetric layout).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -65,7 +66,7 @@ struct SimtSmem {
 template <typename T, int DF, int DV, int C>
 __global__ void __launch_bounds__(kThreads)
 la_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                       T* __restrict__ y, float* __restrict__ S, float* __restrict__ z, int N) {
+                       T* __restrict__ y, float* __restrict__ S, float* __restrict__ z, int N, int packed) {
     using L = SimtSmem<DF, C>;
     constexpr int DS = L::DS;
     constexpr int D = feature_dim(DF);
@@ -161,7 +162,18 @@ la_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         __syncthreads();
     }
 
-    if (S != nullptr) {
+    if (S != nullptr && packed) {
+        // The symmetric layout is the kernel's own: row f of S and z as accumulated.
+        float* Sb = S + bh * (size_t)DS * DV;
+        for (int e = tid; e < DS * kCW; e += kThreads) {
+            const int ff = e / kCW, cc = e % kCW;
+            Sb[(size_t)ff * DV + c0 + cc] = sS[ff * kCW + cc];
+        }
+        if (blockIdx.x == 0) {
+            float* zb = z + bh * (size_t)DS;
+            for (int ff = tid; ff < DS; ff += kThreads) zb[ff] = sz[ff];
+        }
+    } else if (S != nullptr) {
         float* Sb = S + bh * (size_t)D * DV;
         for (int e = tid; e < D * kCW; e += kThreads) {
             const int ff = e / kCW, cc = e % kCW;
@@ -204,7 +216,7 @@ cudaError_t launch_c(const LaPrefillArgs& a, cudaStream_t stream) {
     const dim3 grid(DV / kCW, a.B * a.H);
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(a.q), static_cast<const T*>(a.k),
                                           static_cast<const T*>(a.v), static_cast<T*>(a.y), a.S, a.z,
-                                          a.N);
+                                          a.N, a.packed ? 1 : 0);
     return cudaGetLastError();
 }
 

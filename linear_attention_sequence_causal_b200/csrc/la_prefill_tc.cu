@@ -229,6 +229,7 @@ struct Work {
     bool totals;             // totals pass: state chain only, result to the workspace
     bool has_init;           // main pass, segment > 0: starts from the workspace prefix sum
     bool final_state;        // main pass, last segment: writes S and z
+    bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this segment's total
     const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1
 };
@@ -261,39 +262,49 @@ __device__ __forceinline__ unsigned char* smem_generic(uint32_t saddr) {
 // (stage[f][n], n < 64 for S, n = 64 for z; f in the kernel's feature order) to
 // the 1 + d' + d'^2 rows of S and z. Row 1 + d' + a*d' + b takes the folded
 // pair (min, max) of (a, b), times 1/sqrt2 off the diagonal (the pair's value
-// is split evenly between (a, b) and (b, a)).
+// is split evenly between (a, b) and (b, a)). In the symmetric layout each
+// folded pair is one row, unscaled.
 __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase, int tid, float* S, float* z) {
-    constexpr int D = feature_dim(DF);
     const float* stage = reinterpret_cast<const float*>(smem_generic(sbase) + OFF_PK);
-    auto source = [](int r, float& coef) {
+    // Kernel feature of folded pair (lo, hi), lo < hi.
+    auto pair_source = [](int lo, int hi) {
+        if ((hi & 1) && lo == hi - 1) return 144 + (hi - 1) / 2;  // left-over pair of an odd column
+        return 32 + 2 * (((hi - 1) * (hi - 1)) / 4) + lo;         // column hi, pairs (a, a+1)
+    };
+    // Full layout: row r of the 1 + d' + d'^2 rows, with its scale.
+    auto source = [&](int r, float& coef) {
         coef = 1.0f;
         if (r == 0) return 152;                                  // constant feature
         if (r <= DF) return r - 1;                               // x_a
         const int p = r - 1 - DF, a = p / DF, b = p % DF;
         if (a == b) return DF + a;                               // x_a^2 / sqrt2
-        const int lo = min(a, b), hi = max(a, b);
         coef = kSqrtHalf;
-        if ((hi & 1) && lo == hi - 1) return 144 + (hi - 1) / 2; // left-over pair of an odd column
-        return 32 + 2 * (((hi - 1) * (hi - 1)) / 4) + lo;        // column hi, pairs (a, a+1)
+        return pair_source(min(a, b), max(a, b));
     };
+    // Symmetric layout: row r of the 1 + d' + d'(d'+1)/2 rows (a <= b, a-major),
+    // which holds the kernel's folded feature unscaled.
+    auto source_packed = [&](int r) {
+        if (r == 0) return 152;
+        if (r <= DF) return r - 1;
+        int a, b;
+        packed_pair(r - 1 - DF, DF, a, b);
+        return a == b ? DF + a : pair_source(a, b);
+    };
+    const int D = w.packed ? DS : feature_dim(DF);
     float4* Sd = reinterpret_cast<float4*>(S + w.bh * D * DV);
     for (int idx = tid; idx < D * (DV / 4); idx += kThreads) {
         const int r = idx / (DV / 4), g = idx % (DV / 4);
-        float coef;
-        const int f = source(r, coef);
+        float coef = 1.0f;
+        const int f = w.packed ? source_packed(r) : source(r, coef);
         const float4 x = *reinterpret_cast<const float4*>(stage + f * kStageStride + 4 * g);
         Sd[idx] = make_float4(x.x * coef, x.y * coef, x.z * coef, x.w * coef);
     }
     for (int r = tid; r < D; r += kThreads) {
-        float coef;
-        const int f = source(r, coef);
+        float coef = 1.0f;
+        const int f = w.packed ? source_packed(r) : source(r, coef);
         z[w.bh * D + r] = stage[f * kStageStride + DV] * coef;
     }
 }
-
-// ------------------------------------------------------------------ state warps (4-6)
-// Thread = TMEM lane n = value column n (n < 64), the ones column (n = 64) or
-// padding (65..95). Whole-warp calls.
 
 // Segment start state: row n = sum of the totals of segments 0..seg-1, placed in
 // the TMEM accumulator (fp32) and in the [S|z] buffer (bf16) for MMA3 of chunk 0.
@@ -688,7 +699,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
                      float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_chunks, int mode,
-                     float* __restrict__ ws, unsigned* status, unsigned debug) {
+                     int packed, float* __restrict__ ws, unsigned* status, unsigned debug) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * NUM_BARS);
@@ -710,6 +721,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     w.nchunks = (w.t_end - w.t_begin + C - 1) / C;
     w.has_init = !w.totals && w.seg > 0;
     w.final_state = !w.totals && w.seg == nseg - 1;
+    w.packed = packed != 0;
     w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) + w.seg) * kTotalFloats : nullptr;
     w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
 
@@ -815,11 +827,11 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {
         e = launch_pdl(la_prefill_tc_kernel, dim3(BH * (nseg - 1)), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v,
-                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, ws, a.status, a.debug);
+                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, a.packed ? 1 : 0, ws, a.status, a.debug);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(la_prefill_tc_kernel, dim3(BH * nseg), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v, y, a.S,
-                      a.z, a.N, nseg, seg_chunks, 0, ws, a.status, a.debug);
+                      a.z, a.N, nseg, seg_chunks, 0, a.packed ? 1 : 0, ws, a.status, a.debug);
 }
 
 }  // namespace based

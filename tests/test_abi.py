@@ -59,8 +59,9 @@ FAKE = ctypes.c_void_p(1 << 20)        # aligned, never dereferenced: validation
 MISALIGNED = ctypes.c_void_p((1 << 20) + 8)
 
 
-def test_la_prefill_rejects_bad_arguments(lib):
-    f = lib.based_la_prefill
+@pytest.mark.parametrize("entry", ["based_la_prefill", "based_la_prefill_packed"])
+def test_la_prefill_rejects_bad_arguments(lib, entry):
+    f = getattr(lib, entry)
     ok = dict(B=1, H=1, N=16, df=16, dv=64, dt=1, chunk=0)
 
     def call(q=FAKE, S=FAKE, z=FAKE, **kw):
@@ -83,6 +84,10 @@ def test_decode_and_swa_reject_bad_arguments(lib):
     assert lib.based_la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 64, 1, None) \
         == binding.ERR_INVALID_ARG
     assert lib.based_la_decode_step(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 24, 64, 1, None) \
+        == binding.ERR_UNSUPPORTED
+    assert lib.based_la_decode_step_packed(FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 64, 1, None) \
+        == binding.ERR_INVALID_ARG
+    assert lib.based_la_decode_step_packed(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 16, 96, 1, None) \
         == binding.ERR_UNSUPPORTED
     sp = lib.based_swa_prefill
     assert sp(FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 8, 64, 0, 0.125, 1, None) == binding.ERR_INVALID_ARG
