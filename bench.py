@@ -62,8 +62,9 @@ def swa_prefill_work(B, H, N, d, w):
     return flops, byts
 
 
-def la_decode_work(B, H, d_feat, d_v):
-    D = _feature_dim(d_feat)
+def la_decode_work(B, H, d_feat, d_v, packed=False):
+    """Per step: read and write the fp32 state once (D rows, or D_s in the symmetric layout)."""
+    D = (1 + d_feat + d_feat * (d_feat + 1) // 2) if packed else _feature_dim(d_feat)
     flops = B * H * (4 * D * d_v + 4 * D + d_feat * d_feat)
     byts = B * H * (2 * (D * d_v + D) * 4 + (2 * d_feat + 2 * d_v) * 2)
     return flops, byts
@@ -685,6 +686,15 @@ def run_sweep(reps):
         print(json.dumps({"sweep": "la_decode", "batch": batch, "us_per_step": ms * 1e3,
                           "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                           "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+        Dp = based.packed_dim(df)
+        Sp = torch.randn(batch, H, Dp, dv, device=dev) * 0.01
+        zp = torch.rand(batch, H, Dp, device=dev) + 600.0
+        ms = timed(lambda: based.la_decode_step(Sp, zp, q, k, v, y=y, packed=True), 32)
+        _, byts = la_decode_work(batch, H, df, dv, packed=True)
+        print(json.dumps({"sweep": "la_decode_packed", "batch": batch, "us_per_step": ms * 1e3,
+                          "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                          "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+        del Sp, zp
         kc = torch.randn(batch, H, 64, 64, device=dev).bfloat16()
         vc = torch.randn(batch, H, 64, 64, device=dev).bfloat16()
         sq = torch.randn(batch, H, 64, device=dev).bfloat16()
@@ -718,6 +728,15 @@ def run_sweep(reps):
     ms = timed(lambda: based.la_decode_step(S, z, q, k, v, y=y), 32)
     _, byts = la_decode_work(64, Hl, dfl, dvl)
     print(json.dumps({"sweep": "la_decode_large_state", "batch": 64, "us_per_step": ms * 1e3,
+                      "tokens_per_s": 64 / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                      "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+    del S, z
+    Dpl = based.packed_dim(dfl)
+    S = torch.randn(64, Hl, Dpl, dvl, device=dev) * 0.01
+    z = torch.rand(64, Hl, Dpl, device=dev) + 600.0
+    ms = timed(lambda: based.la_decode_step(S, z, q, k, v, y=y, packed=True), 32)
+    _, byts = la_decode_work(64, Hl, dfl, dvl, packed=True)
+    print(json.dumps({"sweep": "la_decode_large_state_packed", "batch": 64, "us_per_step": ms * 1e3,
                       "tokens_per_s": 64 / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                       "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
     del S, z
