@@ -51,6 +51,7 @@ from .taylor_la import (  # noqa: F401
     feature_map_packed,
     la_state_packed,
     la_recurrent_packed,
+    la_backward,
 )
 from .swa import (  # noqa: F401
     swa,

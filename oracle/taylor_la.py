@@ -275,3 +275,39 @@ def la_recurrent_packed(q, k, v, S0=None, z0=None):
         den = np.einsum("...f,...f->...", fq[..., t, :], z)
         y[..., t, :] = num / den[..., None]
     return y, S, z
+
+
+# ---------------------------------------------------------------- backward (training)
+#
+# Gradients of the causal Taylor linear attention of la_quadratic (the pages'
+# prefill "during training", BASED §5 "Execution stages"). With s_ij = q_i.k_j,
+# a_ij = 1 + s_ij + s_ij^2/2 (j <= i), den_i = sum_j a_ij, y_i = sum_j a_ij v_j / den_i
+# and an upstream gradient dy:
+#     g_i   = dy_i / den_i,          c_i = g_i . y_i,
+#     da_ij = g_i . v_j - c_i        (the quotient rule: num_i / den_i),
+#     ds_ij = da_ij (1 + s_ij)       (d a / d s = 1 + s),
+#     dq_i  = sum_{j<=i} ds_ij k_j,  dk_j = sum_{i>=j} ds_ij q_i,
+#     dv_j  = sum_{i>=j} a_ij g_i.
+
+
+def la_backward(q, k, v, dy):
+    """(dq, dk, dv) of la_quadratic for the upstream gradient dy, float64."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    n = q.shape[-2]
+    mask = np.tril(np.ones((n, n), dtype=bool))
+    s = q @ np.swapaxes(k, -1, -2)
+    a = np.where(mask, 1.0 + s + 0.5 * s * s, 0.0)
+    den = a.sum(axis=-1)
+    _check_den(den, np.arange(1, n + 1, dtype=np.float64))
+    y = (a @ v) / den[..., None]
+    g = dy / den[..., None]
+    c = np.sum(g * y, axis=-1)
+    da = np.where(mask, g @ np.swapaxes(v, -1, -2) - c[..., None], 0.0)
+    ds = da * (1.0 + s)
+    dq = ds @ k
+    dk = np.swapaxes(ds, -1, -2) @ q
+    dv = np.swapaxes(a, -1, -2) @ g
+    return dq, dk, dv

@@ -398,3 +398,52 @@ def test_mutant_packed_coefficients_caught(diag_scale, off_scale):
     r = math.sqrt(0.5)
     assert not np.allclose(_mut_phi_packed(np.array([3.0, -2.0]), diag_scale, off_scale),
                            [1.0, 3.0, -2.0, 9.0 * r, -6.0, 4.0 * r])
+
+
+# ---------------------------------------------------------------- backward (training)
+
+def _torch_forward(q, k, v):
+    """The masked quadratic form written directly in torch float64 (for autograd)."""
+    n = q.shape[-2]
+    s = q @ k.transpose(-1, -2)
+    a = torch.tril(1.0 + s + 0.5 * s * s)
+    return (a @ v) / a.sum(dim=-1, keepdim=True)
+
+
+@pytest.mark.parametrize("d,dv,N", [(16, 8, 40), (32, 16, 23), (2, 3, 7)])
+def test_backward_matches_autograd(d, dv, N):
+    q, k, v = _qkv(2, 2, N, d, dv, seed=N)
+    dy = np.random.default_rng(N + 1).standard_normal((2, 2, N, dv))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    _torch_forward(tq, tk, tv).backward(torch.tensor(dy))
+    dq, dk, dvv = oracle.la_backward(q, k, v, dy)
+    for got, want in ((dq, tq.grad), (dk, tk.grad), (dvv, tv.grad)):
+        assert np.allclose(got, want.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_matches_finite_differences():
+    q, k, v = _qkv(1, 1, 6, 3, 2, seed=3)
+    dy = np.random.default_rng(4).standard_normal((1, 1, 6, 2))
+    loss = lambda q_, k_, v_: float(np.sum(oracle.la_quadratic(q_, k_, v_) * dy))
+    dq, dk, dvv = oracle.la_backward(q, k, v, dy)
+    h = 1e-6
+    for x, grad, which in ((q, dq, 0), (k, dk, 1), (v, dvv, 2)):
+        for idx in np.ndindex(x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            args_p[which], args_m[which] = xp, xm
+            fd = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            assert abs(fd - grad[idx]) <= 1e-6 * max(1.0, abs(fd)), (which, idx, fd, grad[idx])
+
+
+def test_backward_of_first_token_only_touches_itself():
+    # y_0 = v_0 (one causal key): dy on token 0 alone gives dv_0 = dy_0 and no q, k gradient.
+    q, k, v = _qkv(1, 1, 5, 4, 3, seed=8)
+    dy = np.zeros((1, 1, 5, 3))
+    dy[..., 0, :] = [1.0, -2.0, 0.5]
+    dq, dk, dvv = oracle.la_backward(q, k, v, dy)
+    assert np.allclose(dq, 0) and np.allclose(dk, 0)
+    assert np.allclose(dvv[..., 0, :], dy[..., 0, :]) and np.allclose(dvv[..., 1:, :], 0)
