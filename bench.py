@@ -56,6 +56,15 @@ def la_prefill_work(B, H, N, d_feat, d_v, chunk):
     return flops, byts
 
 
+def la_backward_work(B, H, N, d_feat, d_v):
+    """Gradients of the causal quadratic form: per query-key pair of the causal triangle
+    the products s = q.k, g.v, ds k, ds q and a g (2(3d' + 2dv) flops); bytes: q, k, v,
+    y, dy read and dq, dk, dv written once (bf16)."""
+    flops = B * H * N * (N + 1) * (3 * d_feat + 2 * d_v)
+    byts = B * H * N * (4 * d_feat + 4 * d_v) * 2
+    return flops, byts
+
+
 def swa_prefill_work(B, H, N, d, w):
     flops = B * H * N * 4 * w * d
     byts = B * H * N * 4 * d * 2 + B * H * 2 * w * d * 2      # q, k, v, y + ring cache
@@ -591,6 +600,7 @@ PROFILE_CASES = {
     "swa_prefill": "B=16 H=16 N=2048 d=64 w=64 bf16 (q,k,v,y 268 MB)",
     "la_decode": "batch 256, H=16, d'=16, dv=64 (fp32 state 286 MB)",
     "swa_decode": "batch 1024, H=16, d=64, w=64 (ring caches 268 MB)",
+    "la_backward": "B=8 H=16 N=2048 d'=16 dv=64 bf16 (q,k,v,y,dy,dq,dk,dv 168 MB)",
 }
 
 
@@ -614,6 +624,12 @@ def run_profile(kind, reps):
         inp = synthetic.swa_inputs(16, 16, 2048, 64, "bf16", seed=0)
         q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
         fn = lambda: based.swa_prefill(q, k, v, w=64)
+    elif kind == "la_backward":
+        inp = synthetic.la_inputs(8, 16, 2048, 16, 64, "bf16", seed=0)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        dy = synthetic.upstream_grad((8, 16, 2048, 64), "bf16", seed=1)[0].to(dev)
+        y, _, _ = based.la_prefill(q, k, v, want_state=False)
+        fn = lambda: based.la_backward(q, k, v, y, dy)
     elif kind == "la_decode":
         S = torch.randn(256, 16, 273, 64, device=dev)
         z = torch.rand(256, 16, 273, device=dev) + 300.0
@@ -740,6 +756,22 @@ def run_sweep(reps):
                       "tokens_per_s": 64 / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                       "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
     del S, z
+    # backward (training) pass at the 360M shape and the large-state shape
+    for (Bb, Hb, Nb, dfb, dvb) in ((8, 16, 2048, 16, 64), (4, 8, 8192, 32, 128)):
+        inp = synthetic.la_inputs(Bb, Hb, Nb, dfb, dvb, "bf16", seed=2)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        dy = synthetic.upstream_grad((Bb, Hb, Nb, dvb), "bf16", seed=3)[0].to(dev)
+        y, _, _ = based.la_prefill(q, k, v, want_state=False)
+        grads = tuple(torch.empty_like(t) for t in (q, k, v))
+        ws = torch.empty(based.la_backward_workspace(Bb, Hb, Nb, dfb, dvb), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: based.la_backward(q, k, v, y, dy, *grads, workspace=ws), 1)
+        flops, byts = la_backward_work(Bb, Hb, Nb, dfb, dvb)
+        print(json.dumps({"sweep": "la_backward", "shape": f"B={Bb} H={Hb} N={Nb} d'={dfb} dv={dvb}",
+                          "us": ms * 1e3, "tokens_per_s": Bb * Nb / (ms / 1e3),
+                          "TFLOP_s": flops / (ms / 1e3) / 1e12,
+                          "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+                          "GB_s": byts / (ms / 1e3) / 1e9}), flush=True)
+        del q, k, v, dy, y, grads, ws
     # long prefill: B=2, H=16, N=16384
     B, N = 2, 16384
     inp = synthetic.la_inputs(B, H, N, df, dv, "bf16", seed=0)

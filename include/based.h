@@ -205,6 +205,41 @@ BASED_API based_status_t based_la_decode_step_packed(float* S, float* z,
                                                      based_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * based_la_backward -- gradients of the causal Taylor linear attention of
+ * based_la_prefill (the training form of the prefill stage, BASED §5
+ * "Execution stages"). With s_ij = q_i.k_j, a_ij = 1 + s_ij + s_ij^2/2,
+ * den_i = sum_{j<=i} a_ij and the forward's output y, for an upstream
+ * gradient dy:
+ *     g_i = dy_i / den_i,   c_i = g_i . y_i,
+ *     ds_ij = (g_i . v_j - c_i)(1 + s_ij)   for j <= i (0 otherwise),
+ *     dq_i = sum_j ds_ij k_j,   dk_j = sum_i ds_ij q_i,   dv_j = sum_i a_ij g_i.
+ * These are the derivatives of y_i = sum_{j<=i} a_ij v_j / den_i, the exact
+ * quadratic form of the feature map of §4 "Taylor Linear Attention".
+ *
+ *   q, k      [B, H, N, d_feat] bf16      (the prefill's inputs)
+ *   v         [B, H, N, d_v] bf16
+ *   y         [B, H, N, d_v] bf16         (the prefill's output for q, k, v)
+ *   dy        [B, H, N, d_v] bf16         upstream gradient
+ *   dq, dk    [B, H, N, d_feat] bf16      written
+ *   dv        [B, H, N, d_v] bf16         written
+ *   workspace >= based_la_backward_workspace(...) bytes of device memory,
+ *             256-byte aligned; caller-owned, scratch for the call (g as bf16
+ *             and c as fp32 per token, rows padded to a multiple of 128).
+ * All pointers are device memory, 16-byte aligned, contiguous row-major, owned
+ * by the caller; outputs must not alias inputs. Built for bf16 with
+ * d_feat in {16, 32} and d_v in {64, 128}; fp32 and other sizes return
+ * BASED_ERR_UNSUPPORTED. Three kernels are queued on `stream` (asynchronous);
+ * BASED_ERR_TIMEOUT from based_get_last_error means a bounded wait expired and
+ * the outputs are undefined.
+ */
+BASED_API size_t based_la_backward_workspace(int B, int H, int N, int d_feat, int d_v, based_dtype_t dtype);
+BASED_API based_status_t based_la_backward(const void* q, const void* k, const void* v, const void* y,
+                                           const void* dy, void* dq, void* dk, void* dv,
+                                           int B, int H, int N, int d_feat, int d_v,
+                                           based_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                           cudaStream_t stream);
+
+/*
  * based_swa_prefill -- causal sliding-window softmax attention over N tokens:
  *     y_i = sum_j softmax_j(scale * q_i.k_j) v_j  over  i - w < j <= i
  * (w keys including the query's own position). BASED §4 "Local Exact

@@ -11,6 +11,8 @@ from .binding import (  # noqa: F401
     feature_dim,
     packed_dim,
     get_last_error,
+    la_backward,
+    la_backward_workspace,
     la_decode_step,
     la_prefill,
     la_prefill_noalloc,

@@ -29,6 +29,8 @@ SYMBOLS = (
     "based_la_decode_step",
     "based_la_prefill_packed",
     "based_la_decode_step_packed",
+    "based_la_backward_workspace",
+    "based_la_backward",
     "based_swa_prefill",
     "based_swa_decode",
     "based_get_last_error",
@@ -60,6 +62,10 @@ def _declare(lib):
     lib.based_la_prefill_packed.restype = i
     lib.based_la_decode_step_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.based_la_decode_step_packed.restype = i
+    lib.based_la_backward_workspace.argtypes = [i, i, i, i, i, i]
+    lib.based_la_backward_workspace.restype = sz
+    lib.based_la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+    lib.based_la_backward.restype = i
     lib.based_swa_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, f, i, vp]
     lib.based_swa_prefill.restype = i
     lib.based_swa_decode.argtypes = [vp, vp, ctypes.c_int64, vp, vp, vp, vp, i, i, i, i, f, i, vp]
@@ -192,6 +198,37 @@ def la_prefill_noalloc(q, k, v, chunk: int = 0, want_state: bool = True, y=None,
                                             B, H, N, d_feat, d_v, dt, chunk, _stream(dev))
     _check(st, "based_la_prefill_noalloc")
     return y, S, z
+
+
+def la_backward_workspace(B, H, N, d_feat, d_v, dtype=torch.bfloat16) -> int:
+    return int(lib().based_la_backward_workspace(B, H, N, d_feat, d_v, _DTYPES[dtype]))
+
+
+def la_backward(q, k, v, y, dy, dq=None, dk=None, dv=None, workspace=None):
+    """Gradients (dq, dk, dv) of the causal Taylor linear attention for the
+    upstream gradient dy; y is the forward output for q, k, v. bf16 [B,H,N,*]."""
+    dt = _dtype_code(q, k, v, y, dy)
+    B, H, N, d_feat = q.shape
+    d_v = v.shape[-1]
+    if tuple(k.shape) != (B, H, N, d_feat) or tuple(v.shape[:3]) != (B, H, N) or \
+            tuple(y.shape) != (B, H, N, d_v) or tuple(dy.shape) != (B, H, N, d_v):
+        raise BasedError(ERR_INVALID_ARG, "q, k [B,H,N,d'] and v, y, dy [B,H,N,dv] expected")
+    dev = q.device
+    with torch.cuda.device(dev):
+        dq = torch.empty_like(q) if dq is None else dq
+        dk = torch.empty_like(k) if dk is None else dk
+        dv = torch.empty_like(v) if dv is None else dv
+        for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+            if t.shape != ref.shape or t.dtype != ref.dtype or not t.is_contiguous() or t.device != dev:
+                raise BasedError(ERR_INVALID_ARG, f"{name} must match its input's shape, dtype and device")
+        ws_bytes = int(lib().based_la_backward_workspace(B, H, N, d_feat, d_v, dt))
+        if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = lib().based_la_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(dy), _ptr(dq), _ptr(dk), _ptr(dv),
+                                     B, H, N, d_feat, d_v, dt, _ptr(workspace) if ws_bytes else None,
+                                     ws_bytes, _stream(dev))
+    _check(st, "based_la_backward")
+    return dq, dk, dv
 
 
 def la_decode_step(S, z, q, k, v, y=None, packed: bool = False) -> torch.Tensor:

@@ -206,6 +206,34 @@ based_status_t based_la_decode_step_packed(float* S, float* z, const void* q, co
     return la_decode_impl(S, z, q, k, v, y, B, H, d_feat, d_v, dtype, true, stream);
 }
 
+size_t based_la_backward_workspace(int B, int H, int N, int d_feat, int d_v, based_dtype_t dtype) {
+    if (B <= 0 || H <= 0 || N <= 0 || dtype != BASED_BF16 || !based::la_backward_supported(d_feat, d_v)) return 0;
+    return based::la_backward_workspace(B, H, N, d_v);
+}
+
+based_status_t based_la_backward(const void* q, const void* k, const void* v, const void* y, const void* dy,
+                                 void* dq, void* dk, void* dv, int B, int H, int N, int d_feat, int d_v,
+                                 based_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                 cudaStream_t stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y) || !ok_ptr(dy)) return BASED_ERR_INVALID_ARG;
+    if (!ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv)) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (dtype != BASED_BF16 || !based::la_backward_supported(d_feat, d_v)) return BASED_ERR_UNSUPPORTED;
+    const long long tiles = (long long)B * H * ((N + 127) / 128);
+    if (tiles > (1LL << 24)) return BASED_ERR_UNSUPPORTED;
+    const size_t need = based::la_backward_workspace(B, H, N, d_v);
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
+        return BASED_ERR_INVALID_ARG;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const int sms = num_sms(dev);
+    unsigned* status = status_word(dev);
+    if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
+    based::LaBackwardArgs a{q, k, v, y, dy, dq, dk, dv, B, H, N, d_feat, d_v, workspace, status, debug_flags()};
+    const cudaError_t e = based::launch_la_backward(a, sms, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
 based_status_t based_swa_prefill(const void* q, const void* k, const void* v, void* y, void* k_cache,
                                  void* v_cache, int B, int H, int N, int d, int w, float scale,
                                  based_dtype_t dtype, cudaStream_t stream) {

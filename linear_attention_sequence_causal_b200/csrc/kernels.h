@@ -37,6 +37,21 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
 bool la_prefill_quad_supported(int d_feat, int d_v);
 cudaError_t launch_la_prefill_quad(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
 
+// Backward (training) pass of the causal Taylor linear attention, bf16 tensor
+// cores: dq, dk, dv from q, k, v, the forward's y and the upstream dy.
+struct LaBackwardArgs {
+    const void* q; const void* k; const void* v; const void* y; const void* dy;
+    void* dq; void* dk; void* dv;
+    int B, H, N, d_feat, d_v;
+    void* workspace;                 // >= la_backward_workspace(B, H, N, d_v) bytes, 256-byte aligned
+    unsigned* status;
+    unsigned debug;
+};
+bool la_backward_supported(int d_feat, int d_v);
+size_t la_backward_workspace(int B, int H, int N, int d_v);
+size_t la_backward_g_bytes(const LaBackwardArgs& a);
+cudaError_t launch_la_backward(const LaBackwardArgs& a, int num_sms, cudaStream_t stream);
+
 // `packed`: S and z hold the symmetric layout (1 + d' + d'(d'+1)/2 rows).
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
                              void* y, int B, int H, int d_feat, int d_v, bool bf16, bool packed,

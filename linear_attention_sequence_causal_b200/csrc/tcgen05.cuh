@@ -266,6 +266,14 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
                  : "memory");
 }
 
+// 1-D bulk copy global -> shared, completing `bar`'s transaction count. Both
+// addresses 16-byte aligned, `bytes` a multiple of 16.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // 3-D tiled TMA load into shared memory, completing `bar`'s transaction count.
 // Coordinates: x innermost (elements), then y, z; y may be negative or past the
 // end (the box is zero-filled there); x must keep 16-byte alignment.

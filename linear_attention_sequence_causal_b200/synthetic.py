@@ -73,3 +73,9 @@ WORKLOADS = {
 }
 SWA_WINDOW = 64
 SWA_HEAD_DIM = 64
+
+
+def upstream_grad(shape, dtype: str = "bf16", seed: int = 0):
+    """An upstream gradient dy ~ N(0, 1) of `shape`: (tensor of the dtype, float64 copy)."""
+    rng = np.random.default_rng(seed)
+    return _round(rng.standard_normal(shape, dtype=np.float32), dtype)

@@ -101,6 +101,36 @@ def test_decode_and_swa_reject_bad_arguments(lib):
     assert sd(FAKE, FAKE, 0, FAKE, FAKE, FAKE, FAKE, 1, 1, 64, 80, 0.125, 1, None) == binding.ERR_UNSUPPORTED
 
 
+def test_la_backward_rejects_bad_arguments(lib):
+    f = lib.based_la_backward
+    ok = dict(B=1, H=1, N=16, df=16, dv=64, dt=1, ws=FAKE, nbytes=1 << 20)
+
+    def call(q=FAKE, dq=FAKE, **kw):
+        a = dict(ok, **kw)
+        return f(q, FAKE, FAKE, FAKE, FAKE, dq, FAKE, FAKE, a["B"], a["H"], a["N"], a["df"], a["dv"],
+                 a["dt"], a["ws"], a["nbytes"], None)
+
+    assert call(q=None) == binding.ERR_INVALID_ARG
+    assert call(dq=MISALIGNED) == binding.ERR_INVALID_ARG
+    assert call(N=0) == binding.ERR_INVALID_ARG
+    assert call(dt=7) == binding.ERR_INVALID_ARG
+    assert call(dt=0) == binding.ERR_UNSUPPORTED             # fp32: bf16 tensor cores only
+    assert call(df=8) == binding.ERR_UNSUPPORTED
+    assert call(dv=96) == binding.ERR_UNSUPPORTED
+    assert call(ws=None) == binding.ERR_INVALID_ARG
+    assert call(ws=MISALIGNED) == binding.ERR_INVALID_ARG    # 256-byte alignment
+    assert call(nbytes=16) == binding.ERR_INVALID_ARG        # smaller than the query
+
+
+def test_la_backward_workspace_query(lib):
+    # g (bf16) and c (fp32) per token, rows padded to a multiple of 128.
+    assert lib.based_la_backward_workspace(2, 3, 300, 16, 64, 1) == 2 * 3 * 384 * (64 * 2 + 4)
+    assert lib.based_la_backward_workspace(1, 1, 128, 32, 128, 1) == 128 * (128 * 2 + 4)
+    assert lib.based_la_backward_workspace(1, 1, 128, 32, 128, 0) == 0
+    assert lib.based_la_backward_workspace(1, 1, 0, 32, 128, 1) == 0
+    assert lib.based_la_backward_workspace(1, 1, 8, 24, 128, 1) == 0
+
+
 def test_workspace_query_rejects_bad_arguments(lib):
     assert lib.based_la_prefill_workspace(0, 1, 1, 16, 64, 1, 0) == 0
     assert lib.based_la_prefill_workspace(1, 1, 1, 8, 64, 1, 0) == 0
