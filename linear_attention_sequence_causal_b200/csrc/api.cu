@@ -208,7 +208,7 @@ based_status_t based_la_decode_step_packed(float* S, float* z, const void* q, co
 
 size_t based_la_backward_workspace(int B, int H, int N, int d_feat, int d_v, based_dtype_t dtype) {
     if (B <= 0 || H <= 0 || N <= 0 || dtype != BASED_BF16 || !based::la_backward_supported(d_feat, d_v)) return 0;
-    return based::la_backward_workspace(B, H, N, d_v);
+    return based::la_backward_workspace(B, H, N, d_feat, d_v);
 }
 
 based_status_t based_la_backward(const void* q, const void* k, const void* v, const void* y, const void* dy,
@@ -221,7 +221,7 @@ based_status_t based_la_backward(const void* q, const void* k, const void* v, co
     if (dtype != BASED_BF16 || !based::la_backward_supported(d_feat, d_v)) return BASED_ERR_UNSUPPORTED;
     const long long tiles = (long long)B * H * ((N + 127) / 128);
     if (tiles > (1LL << 24)) return BASED_ERR_UNSUPPORTED;
-    const size_t need = based::la_backward_workspace(B, H, N, d_v);
+    const size_t need = based::la_backward_workspace(B, H, N, d_feat, d_v);
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || workspace_bytes < need)
         return BASED_ERR_INVALID_ARG;
     int dev;

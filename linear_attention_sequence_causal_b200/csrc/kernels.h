@@ -43,12 +43,12 @@ struct LaBackwardArgs {
     const void* q; const void* k; const void* v; const void* y; const void* dy;
     void* dq; void* dk; void* dv;
     int B, H, N, d_feat, d_v;
-    void* workspace;                 // >= la_backward_workspace(B, H, N, d_v) bytes, 256-byte aligned
+    void* workspace;                 // >= la_backward_workspace(B, H, N, d_feat, d_v) bytes, 256-byte aligned
     unsigned* status;
     unsigned debug;
 };
 bool la_backward_supported(int d_feat, int d_v);
-size_t la_backward_workspace(int B, int H, int N, int d_v);
+size_t la_backward_workspace(int B, int H, int N, int d_feat, int d_v);
 size_t la_backward_g_bytes(const LaBackwardArgs& a);
 cudaError_t launch_la_backward(const LaBackwardArgs& a, int num_sms, cudaStream_t stream);
 

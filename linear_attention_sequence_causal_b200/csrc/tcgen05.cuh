@@ -188,6 +188,21 @@ __device__ __forceinline__ void taylor_pair(float s0, float s1, float& a0, float
         : "f"(s0), "f"(s1));
 }
 
+// (d0, d1) = (x - c)(1 + s) for two columns at once, as t = x - c, d = t s + t
+// (sub.rn.f32x2 and fma.rn.f32x2): the score gradient of the Taylor weight.
+__device__ __forceinline__ void dscore_pair(float x0, float x1, float c0, float c1, float s0, float s1, float& d0,
+                                            float& d1) {
+    asm("{\n\t.reg .b64 x, c, s, t;\n\t"
+        "mov.b64 x, {%2, %3};\n\t"
+        "mov.b64 c, {%4, %5};\n\t"
+        "mov.b64 s, {%6, %7};\n\t"
+        "sub.rn.f32x2 t, x, c;\n\t"
+        "fma.rn.f32x2 t, t, s, t;\n\t"
+        "mov.b64 {%0, %1}, t;\n\t}"
+        : "=f"(d0), "=f"(d1)
+        : "f"(x0), "f"(x1), "f"(c0), "f"(c1), "f"(s0), "f"(s1));
+}
+
 // (l0, l1) += (a0, a1) with the packed fp32 add.
 __device__ __forceinline__ void add_pair(float& l0, float& l1, float a0, float a1) {
     asm("{\n\t.reg .b64 l, a;\n\t"
