@@ -266,6 +266,12 @@ BASED_API based_status_t based_swa_prefill(const void* q, const void* k, const v
  *   k_cache, v_cache [B, H, w, d] dtype, read and written in place
  *   q, k, v, y       [B, H, d]    dtype
  *   t >= 0;  d 64;  1 <= w <= 64
+ *
+ * Ordering: the bf16 kernel is launched as a programmatic dependent of the
+ * previous work in `stream` and reads the ring slots other than t mod w and
+ * (t-1) mod w before that work has finished. The kernel immediately before it
+ * in the stream must therefore not write those slots of this cache; decode
+ * steps on one cache issued in order (t after t-1, or t repeated) satisfy this.
  */
 BASED_API based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t,
                                 const void* q, const void* k, const void* v, void* y,

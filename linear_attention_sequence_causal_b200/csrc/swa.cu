@@ -239,25 +239,39 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
     const size_t bh = blockIdx.x;
     const int new_slot = (int)(t % w);
 
-    grid_dependency_wait();
-    const uint4 knew = __ldg(reinterpret_cast<const uint4*>(k + bh * kHead) + c);
-    const uint4 vnew = __ldg(reinterpret_cast<const uint4*>(v + bh * kHead) + c);
-    const uint4 qu = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
+    // Slots that neither this step (t) nor the previous one (t - 1) writes are
+    // loaded before the wait for the previous kernel in the stream: only that
+    // kernel can still be running, and consecutive decode steps on one cache
+    // write slot (t - 1) mod w at most. The rest is loaded after the wait.
+    const int prev_slot = (int)((t + w - 1) % w);
     uint4 kr[4], vr[4];
-    bool valid[4];
+    bool valid[4], late[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const int slot = 16 * p + 4 * warp + (lane >> 3);
         // newest token held by the slot: u = t - ((t - slot) mod w); empty while u < 0
         valid[p] = slot < w && t - ((((t - slot) % w) + w) % w) >= 0;
+        late[p] = slot == new_slot || slot == prev_slot;
         kr[p] = vr[p] = make_uint4(0, 0, 0, 0);
-        if (valid[p]) {
+        if (valid[p] && !late[p]) {
+            kr[p] = __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
+            vr[p] = __ldg(reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead) + c);
+        }
+    }
+    grid_dependency_wait();
+    const uint4 knew = __ldg(reinterpret_cast<const uint4*>(k + bh * kHead) + c);
+    const uint4 vnew = __ldg(reinterpret_cast<const uint4*>(v + bh * kHead) + c);
+    const uint4 qu = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        if (valid[p] && late[p]) {
             if (slot == new_slot) {
                 kr[p] = knew;
                 vr[p] = vnew;
             } else {
-                kr[p] = __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
-                vr[p] = __ldg(reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead) + c);
+                kr[p] = reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead)[c];
+                vr[p] = reinterpret_cast<const uint4*>(vc + (bh * w + slot) * kHead)[c];
             }
         }
     }

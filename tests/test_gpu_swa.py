@@ -95,6 +95,31 @@ def test_decode_continues_prefill(dtype, batch, prompt, steps, w):
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
 
+@pytest.mark.parametrize("w,prompt", [(64, 100), (16, 0), (64, 0)])
+def test_decode_steps_back_to_back(w, prompt):
+    """Consecutive decode kernels with nothing between them on the stream: each
+    step's early reads of the ring overlap the previous step's kernel."""
+    batch, H, steps = 4, 16, 150
+    inp = synthetic.swa_inputs(batch, H, prompt + steps, 64, "bf16", seed=w + prompt)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    if prompt > 0:
+        _, kc, vc = based.swa_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                                      v[:, :, :prompt].contiguous(), w=w, scale=SCALE)
+    else:
+        kc = torch.zeros((batch, H, w, 64), dtype=q.dtype, device=DEV)
+        vc = torch.zeros_like(kc)
+    qd, kd, vd = (x[:, :, prompt:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
+    ys = torch.empty((steps, batch, H, 64), dtype=q.dtype, device=DEV)
+    torch.cuda.synchronize()
+    for t in range(steps):
+        based.swa_decode(kc, vc, prompt + t, qd[t], kd[t], vd[t], w=w, scale=SCALE, y=ys[t])
+    assert based.get_last_error() == 0
+    ref = oracle.swa(inp.q64, inp.k64, inp.v64, w, SCALE)
+    assert_y(to64(ys).transpose(1, 2, 0, 3), ref[..., prompt:, :], torch.bfloat16, "decode y")
+    rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, w)
+    assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
+
+
 def test_unsupported_head_dim():
     x = torch.zeros(1, 1, 8, 128, device=DEV)
     with pytest.raises(based.BasedError) as e:
