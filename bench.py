@@ -720,6 +720,13 @@ def run_sweep(reps):
         print(json.dumps({"sweep": "swa_decode", "batch": batch, "us_per_step": ms * 1e3,
                           "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                           "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+        # one BASED decode step: the linear-attention and sliding-window layers on the same batch
+        ms = timed(lambda: (based.la_decode_step(S, z, q, k, v, y=y),
+                            based.swa_decode(kc, vc, 1000, sq, sq, sq, w=64, scale=0.125, y=ys)), 32)
+        byts = la_decode_work(batch, H, df, dv)[1] + swa_decode_work(batch, H, 64, 64)[1]
+        print(json.dumps({"sweep": "based_decode_step", "batch": batch, "us_per_step": ms * 1e3,
+                          "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                          "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
         del S, z, kc, vc
     # large state: d'=32 (D=1057), dv=128, H=8, B=4, N=8192 prefill, then decode at batch 64
     Bl, Hl, Nl, dfl, dvl = 4, 8, 8192, 32, 128
