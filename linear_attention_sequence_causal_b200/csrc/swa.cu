@@ -230,27 +230,28 @@ cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void
 __global__ void __launch_bounds__(128)
 swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                       const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, float scale) {
+                       const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, int new_slot,
+                       float scale) {
     __shared__ float s_sc[kMaxW];
     __shared__ float s_part[4][kHead];
     const int tid = threadIdx.x;
     const int warp = tid >> 5, lane = tid & 31;
     const int c = lane & 7;
     const size_t bh = blockIdx.x;
-    const int new_slot = (int)(t % w);
 
     // Slots that neither this step (t) nor the previous one (t - 1) writes are
     // loaded before the wait for the previous kernel in the stream: only that
     // kernel can still be running, and consecutive decode steps on one cache
     // write slot (t - 1) mod w at most. The rest is loaded after the wait.
-    const int prev_slot = (int)((t + w - 1) % w);
+    const int prev_slot = new_slot == 0 ? w - 1 : new_slot - 1;
     uint4 kr[4], vr[4];
     bool valid[4], late[4];
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
         const int slot = 16 * p + 4 * warp + (lane >> 3);
-        // newest token held by the slot: u = t - ((t - slot) mod w); empty while u < 0
-        valid[p] = slot < w && t - ((((t - slot) % w) + w) % w) >= 0;
+        // newest token held by the slot: u = t - ((t - slot) mod w), empty while u < 0,
+        // that is: every slot once t >= w, else the slots <= t.
+        valid[p] = slot < w && (t >= w || slot <= t);
         late[p] = slot == new_slot || slot == prev_slot;
         kr[p] = vr[p] = make_uint4(0, 0, 0, 0);
         if (valid[p] && !late[p]) {
@@ -381,7 +382,7 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                                            static_cast<__nv_bfloat16*>(v_cache), (long long)t,
                                            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w,
-                                           scale);
+                                           (int)(t % w), scale);   // the new token's slot
         if (e != cudaSuccess) return e;
     } else {
         swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(

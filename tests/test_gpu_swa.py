@@ -120,6 +120,34 @@ def test_decode_steps_back_to_back(w, prompt):
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
 
+@pytest.mark.parametrize("w,prompt", [(64, 100), (16, 0), (40, 7)])
+def test_decode_large_batch(w, prompt):
+    """2048 heads (batch 128 x 16), more than one wave of CTAs; early steps
+    (prompt 0) and windows that do not divide the step count."""
+    batch, H, steps = 128, 16, 70
+    inp = synthetic.swa_inputs(batch, H, prompt + steps, 64, "bf16", seed=3 * w + prompt)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    if prompt > 0:
+        _, kc, vc = based.swa_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                                      v[:, :, :prompt].contiguous(), w=w, scale=SCALE)
+    else:
+        kc = torch.zeros((batch, H, w, 64), dtype=q.dtype, device=DEV)
+        vc = torch.zeros_like(kc)
+    qd, kd, vd = (x[:, :, prompt:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
+    ys = torch.empty((steps, batch, H, 64), dtype=q.dtype, device=DEV)
+    for t in range(steps):
+        based.swa_decode(kc, vc, prompt + t, qd[t], kd[t], vd[t], w=w, scale=SCALE, y=ys[t])
+    assert based.get_last_error() == 0
+    heads = [(0, 0), (batch - 1, H - 1), (batch // 2, 5), (77, 11)]
+    bs = [b for b, _ in heads]
+    hs = [h for _, h in heads]
+    ref = oracle.swa(inp.q64[bs, hs], inp.k64[bs, hs], inp.v64[bs, hs], w, SCALE)
+    got = to64(ys).transpose(1, 2, 0, 3)[bs, hs]
+    assert_y(got, ref[..., prompt:, :], torch.bfloat16, "decode y")
+    rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, w)
+    assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
+
+
 def test_unsupported_head_dim():
     x = torch.zeros(1, 1, 8, 128, device=DEV)
     with pytest.raises(based.BasedError) as e:
