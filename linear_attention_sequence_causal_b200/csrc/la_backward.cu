@@ -52,7 +52,7 @@ struct BwdLayout {
     static constexpr uint32_t V_BLOCK = C * 128;              // 64 columns x 128 rows, 128-byte swizzle
     static constexpr uint32_t V_BYTES = C * DV * 2;           // dv-wide tile
     static constexpr bool HAS_C = MODE == MODE_DKV;           // c of the stage's query tile
-    static constexpr int STAGES = 2;                          // ring stages of the other side's tiles
+    static constexpr int STAGES = 4;                          // ring stages of the other side's tiles
     static constexpr int NPI = MODE == MODE_DQ ? 1 : 2;       // product issuers
     static constexpr uint32_t STAGE_BYTES = QK_BYTES + V_BYTES + (HAS_C ? 1024 : 0);
     static constexpr uint32_t OFF_A1 = 0;                     // own d'-wide tile
@@ -88,9 +88,9 @@ struct BwdLayout {
 };
 
 enum {
-    BB_FULL0 = 0,             // [2] TMA: ring stage s landed
-    BB_EMPTY0 = 2,            // [2] MMA commits: ring stage s read (S / X and the products)
-    BB_OWNFULL = 4,           // TMA: the unit's own tiles landed
+    BB_FULL0 = 0,             // [4] TMA: ring stage s landed
+    BB_EMPTY0 = 4,            // [4] MMA commits: ring stage s read (S / X and the products)
+    BB_OWNFULL = 8,           // TMA: the unit's own tiles landed
     BB_OWNFREE,               // MMA commit: the unit's own tiles no longer read
     BB_SF,                    // MMA commit: S and X of the step ready
     BB_SXFREE,                // row warps: S and X of the step read into registers
@@ -427,26 +427,9 @@ __device__ __forceinline__ void bwd_rows(const BwdCtx& cx, uint32_t tmem, int wq
 #pragma unroll
             for (int g2 = 0; g2 < kRowGroups; ++g2) den += lsum[g2 * 128 + r];
             const float inv = 1.0f / den;                    // den >= (row + 1) / 2
-            // dq_i = dQ'_i / den_i: 16-column slices of the accumulator by group.
-            if (!bwait(cx, BB_ACCF, k_unit & 1)) return;
-            tc_fence_after();
-#pragma unroll
-            for (int i = cg; i < DF / 16; i += kRowGroups) {
-                float acc[16];
-                tmem_ld16(tl + L::COL_ACC2 + 16 * i, acc);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 16; ++e) acc[e] *= inv;
-                if (real) {
-                    uint4* op = reinterpret_cast<uint4*>(dq + ((size_t)bh * cx.N + row) * DF + 16 * i);
-                    op[0] = pack_bf16x8(acc);
-                    op[1] = pack_bf16x8(acc + 8);
-                }
-            }
-            tc_fence_before();
-            mbar_arrive(&cx.bars[BB_ACCE]);                  // the accumulator may be reused
             // g = dy / den (bf16, the operand of DKV's products) and c = g . y over this
-            // group's dv / groups columns; group 0 adds the partial c. Rows past the end are 0.
+            // group's dv / groups columns; group 0 adds the partial c. Rows past the end
+            // are 0. This needs den only, so it runs while the last products complete.
             constexpr int CPG = DV / kRowGroups;             // columns per group: 16 or 32
             uint4* gp = reinterpret_cast<uint4*>(G + ((size_t)bh * cx.Npad + row) * DV + cg * CPG);
             float c = 0.f;
@@ -480,6 +463,24 @@ __device__ __forceinline__ void bwd_rows(const BwdCtx& cx, uint32_t tmem, int wq
             }
             csum[cg * 128 + r] = c;
             mbar_arrive(&cx.bars[BB_CSUM]);
+            // dq_i = dQ'_i / den_i: 16-column slices of the accumulator by group.
+            if (!bwait(cx, BB_ACCF, k_unit & 1)) return;
+            tc_fence_after();
+#pragma unroll
+            for (int i = cg; i < DF / 16; i += kRowGroups) {
+                float acc[16];
+                tmem_ld16(tl + L::COL_ACC2 + 16 * i, acc);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 16; ++e) acc[e] *= inv;
+                if (real) {
+                    uint4* op = reinterpret_cast<uint4*>(dq + ((size_t)bh * cx.N + row) * DF + 16 * i);
+                    op[0] = pack_bf16x8(acc);
+                    op[1] = pack_bf16x8(acc + 8);
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&cx.bars[BB_ACCE]);                  // the accumulator may be reused
             if (cg == 0) {
                 if (!bwait(cx, BB_CSUM, k_unit & 1)) return;
                 float ct = 0.f;
