@@ -52,6 +52,13 @@ from .taylor_la import (  # noqa: F401
     la_state_packed,
     la_recurrent_packed,
     la_backward,
+    DECAY_CHUNK,
+    decay_chunks,
+    decay_per_step,
+    decay_weights,
+    la_quadratic_decay,
+    la_recurrent_decay,
+    la_state_decay,
 )
 from .swa import (  # noqa: F401
     swa,

@@ -311,3 +311,112 @@ def la_backward(q, k, v, dy):
     dk = np.swapaxes(ds, -1, -2) @ q
     dv = np.swapaxes(a, -1, -2) @ g
     return dq, dk, dv
+
+
+# ---------------------------------------------------------------------------
+# Coarse input-dependent decay.
+#
+# BASED App. C "Extended Architecture Details" (Decay) and App. D.4 "BASED
+# Quality Ablations" (Input-dependent decay) describe a coarser input-dependent
+# decay of the state that avoids a parallel scan, and print no formula. Reading taken (one scalar per chunk of DECAY_CHUNK tokens, applied to
+# the state where a chunk begins; the chunk's own tokens are not decayed among
+# themselves):
+#     S_c = gamma_c S_{c-1} + sum_{t in chunk c} phi(k_t) v_t^T,   z likewise;
+# token i of chunk c reads gamma_c S_{c-1} + (its chunk's keys j <= i). Pairwise,
+# key j contributes to query i >= j with the weight
+#     w_ij = prod_{c = chunk(j)+1 .. chunk(i)} gamma_c   (1 inside one chunk),
+# in the numerator and the denominator alike. gamma is [..., n_chunks], caller
+# supplied (the projection that makes it input-dependent is outside this path).
+
+DECAY_CHUNK = 128
+
+
+def decay_chunks(n: int) -> int:
+    """Number of decay chunks covering n tokens."""
+    return (n + DECAY_CHUNK - 1) // DECAY_CHUNK
+
+
+def decay_weights(gamma, n: int) -> np.ndarray:
+    """w [..., n, n]: w_ij = product of gamma over the chunks after chunk(j) up to
+    chunk(i), for j <= i; 0 above the diagonal. Built with explicit loops over
+    the chunk pairs."""
+    gamma = np.asarray(gamma, dtype=np.float64)
+    nc = decay_chunks(n)
+    assert gamma.shape[-1] == nc, (gamma.shape, nc)
+    lead = gamma.shape[:-1]
+    pair = np.ones(lead + (nc, nc), dtype=np.float64)    # pair[ci, cj]
+    for ci in range(nc):
+        for cj in range(ci):
+            w = np.ones(lead, dtype=np.float64)
+            for c in range(cj + 1, ci + 1):
+                w = w * gamma[..., c]
+            pair[..., ci, cj] = w
+    chunk = np.arange(n) // DECAY_CHUNK
+    w = pair[..., chunk[:, None], chunk[None, :]]
+    return np.where(np.tril(np.ones((n, n), dtype=bool)), w, 0.0)
+
+
+def la_quadratic_decay(q, k, v, gamma) -> np.ndarray:
+    """y_i = sum_{j<=i} w_ij a_ij v_j / sum_{j<=i} w_ij a_ij with a_ij = 1 + s + s^2/2."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    n = q.shape[-2]
+    s = q @ np.swapaxes(k, -1, -2)
+    a = (1.0 + s + 0.5 * s * s) * decay_weights(gamma, n)
+    return (a @ v) / a.sum(axis=-1)[..., None]
+
+
+def la_state_decay(k, v, gamma):
+    """Final S, z: sum_j u_j phi(k_j) v_j^T and sum_j u_j phi(k_j), with u_j the
+    product of gamma over the chunks after chunk(j)."""
+    fk = feature_map(k)
+    v = np.asarray(v, dtype=np.float64)
+    gamma = np.asarray(gamma, dtype=np.float64)
+    n = fk.shape[-2]
+    nc = decay_chunks(n)
+    u = np.ones(gamma.shape[:-1] + (n,), dtype=np.float64)
+    for j in range(n):
+        for c in range(j // DECAY_CHUNK + 1, nc):
+            u[..., j] = u[..., j] * gamma[..., c]
+    fku = fk * u[..., None]
+    return np.swapaxes(fku, -1, -2) @ v, fku.sum(axis=-2)
+
+
+def la_recurrent_decay(q, k, v, gamma_step, S0=None, z0=None):
+    """Token by token with a decay per step: S <- gamma_t S, z <- gamma_t z, then
+    S += phi(k_t) v_t^T, z += phi(k_t), y_t = phi(q_t) S / phi(q_t) z.
+
+    gamma_step is [..., n] (1 except where a chunk begins); this is the decode
+    step's form. Returns (y, S, z)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    g = np.asarray(gamma_step, dtype=np.float64)
+    *lead, n, d_feat = q.shape
+    dv = v.shape[-1]
+    D = feature_dim(d_feat)
+    S = np.zeros(tuple(lead) + (D, dv)) if S0 is None else np.array(S0, dtype=np.float64)
+    z = np.zeros(tuple(lead) + (D,)) if z0 is None else np.array(z0, dtype=np.float64)
+    y = np.empty(tuple(lead) + (n, dv), dtype=np.float64)
+    fq = feature_map(q)
+    fk = feature_map(k)
+    for t in range(n):
+        S = S * g[..., t, None, None] + fk[..., t, :, None] * v[..., t, None, :]
+        z = z * g[..., t, None] + fk[..., t, :]
+        num = np.einsum("...f,...fe->...e", fq[..., t, :], S)
+        den = np.einsum("...f,...f->...", fq[..., t, :], z)
+        y[..., t, :] = num / den[..., None]
+    return y, S, z
+
+
+def decay_per_step(gamma, n: int, t0: int = 0) -> np.ndarray:
+    """gamma_step [..., n] for tokens t0 .. t0+n-1: gamma_c on the first token of
+    chunk c (c >= 1), 1 elsewhere. gamma holds one value per chunk from chunk 0."""
+    gamma = np.asarray(gamma, dtype=np.float64)
+    out = np.ones(gamma.shape[:-1] + (n,), dtype=np.float64)
+    for t in range(n):
+        tok = t0 + t
+        if tok > 0 and tok % DECAY_CHUNK == 0:
+            out[..., t] = gamma[..., tok // DECAY_CHUNK]
+    return out

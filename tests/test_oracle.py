@@ -447,3 +447,89 @@ def test_backward_of_first_token_only_touches_itself():
     dq, dk, dvv = oracle.la_backward(q, k, v, dy)
     assert np.allclose(dq, 0) and np.allclose(dk, 0)
     assert np.allclose(dvv[..., 0, :], dy[..., 0, :]) and np.allclose(dvv[..., 1:, :], 0)
+
+
+# ---------------------------------------------------------------- coarse decay (reading: one gamma per 128-token chunk)
+
+def _decay_case(B, H, N, d, dv, seed):
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((B, H, N, d)) * d ** -0.25
+    k = rng.standard_normal((B, H, N, d)) * d ** -0.25
+    v = rng.standard_normal((B, H, N, dv))
+    gamma = rng.uniform(0.5, 1.0, (B, H, oracle.decay_chunks(N)))
+    return q, k, v, gamma
+
+
+def test_decay_closed_form_with_constant_scores():
+    """q = 0 makes every a_ij = 1, so y_i is the w-weighted mean of v_j: for query i in
+    chunk 1, keys of chunk 0 weigh gamma_1 and keys of chunk 1 weigh 1."""
+    N, dv = 300, 3
+    rng = np.random.default_rng(7)
+    q = np.zeros((1, N, 4))
+    k = rng.standard_normal((1, N, 4))
+    v = rng.standard_normal((1, N, dv))
+    g = np.array([[0.9, 0.5, 0.25]])
+    y = oracle.la_quadratic_decay(q, k, v, g)[0]
+    for i in (0, 127, 128, 200, 255):
+        if i < 128:
+            ref = v[0, : i + 1].mean(axis=0)
+        else:
+            ref = (0.5 * v[0, :128].sum(axis=0) + v[0, 128 : i + 1].sum(axis=0)) / (0.5 * 128 + (i - 127))
+        assert np.allclose(y[i], ref, rtol=1e-13, atol=1e-13)
+    # chunk 2: chunk 0 weighs gamma_1 gamma_2, chunk 1 weighs gamma_2
+    i = 299
+    num = 0.5 * 0.25 * v[0, :128].sum(axis=0) + 0.25 * v[0, 128:256].sum(axis=0) + v[0, 256:300].sum(axis=0)
+    den = 0.5 * 0.25 * 128 + 0.25 * 128 + 44
+    assert np.allclose(y[i], num / den, rtol=1e-13, atol=1e-13)
+
+
+def test_decay_of_one_is_the_undecayed_attention():
+    q, k, v, g = _decay_case(1, 2, 260, 8, 5, 1)
+    y = oracle.la_quadratic_decay(q, k, v, np.ones_like(g))
+    assert np.allclose(y, oracle.la_quadratic(q, k, v), rtol=1e-12, atol=1e-12)
+    S, z = oracle.la_state_decay(k, v, np.ones_like(g))
+    S0, z0 = oracle.la_state(k, v)
+    assert np.allclose(S, S0, rtol=1e-12) and np.allclose(z, z0, rtol=1e-12)
+
+
+def test_decay_quadratic_matches_recurrence_and_state():
+    """Two independent formulations: pairwise weights against the per-step state
+    recurrence (decay where a chunk begins), outputs and final state."""
+    q, k, v, g = _decay_case(2, 1, 290, 4, 3, 2)
+    y_quad = oracle.la_quadratic_decay(q, k, v, g)
+    y_rec, S, z = oracle.la_recurrent_decay(q, k, v, oracle.decay_per_step(g, 290))
+    assert np.allclose(y_quad, y_rec, rtol=1e-10, atol=1e-12)
+    S2, z2 = oracle.la_state_decay(k, v, g)
+    assert np.allclose(S, S2, rtol=1e-10, atol=1e-10) and np.allclose(z, z2, rtol=1e-10)
+
+
+def test_decay_recurrence_continues_across_a_split():
+    """Prefill state of the first 256 tokens, then steps from t0 = 256: the first of
+    them begins chunk 2 and takes gamma_2."""
+    q, k, v, g = _decay_case(1, 1, 300, 4, 3, 3)
+    S0, z0 = oracle.la_state_decay(k[..., :256, :], v[..., :256, :], g[..., :2])
+    y2, S2, z2 = oracle.la_recurrent_decay(q[..., 256:, :], k[..., 256:, :], v[..., 256:, :],
+                                           oracle.decay_per_step(g, 44, t0=256), S0, z0)
+    y_all = oracle.la_quadratic_decay(q, k, v, g)
+    assert np.allclose(y2, y_all[..., 256:, :], rtol=1e-10, atol=1e-12)
+    S, z = oracle.la_state_decay(k, v, g)
+    assert np.allclose(S2, S, rtol=1e-10, atol=1e-10)
+
+
+@pytest.mark.parametrize("mutant", ["own_chunk_decayed", "no_decay_in_den"])
+def test_decay_mutants_caught(mutant):
+    """A plausible slip -- decaying a chunk's own keys, or leaving the denominator
+    undecayed -- breaks the closed form."""
+    N = 300
+    rng = np.random.default_rng(8)
+    q = np.zeros((1, N, 4))
+    k = rng.standard_normal((1, N, 4))
+    v = rng.standard_normal((1, N, 2))
+    g = np.array([[0.9, 0.5, 0.25]])
+    w = oracle.decay_weights(g, N)[0]
+    if mutant == "own_chunk_decayed":
+        w = w * g[0, np.arange(N) // 128][None, :]          # the key's own chunk decayed too
+        y = (w @ v[0]) / w.sum(axis=-1)[:, None]
+    else:
+        y = (w @ v[0]) / np.tril(np.ones((N, N))).sum(axis=-1)[:, None]
+    assert not np.allclose(y, oracle.la_quadratic_decay(q, k, v, g)[0], rtol=1e-6, atol=1e-6)
