@@ -763,6 +763,23 @@ def run_sweep(reps):
                       "tokens_per_s": 64 / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
                       "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
     del S, z
+    # coarse decay (one gamma per 128-token tile): the quadratic-form path at the 360M and large shapes
+    for (Bd, Hd, Nd, dfd, dvd, cd) in ((8, 16, 2048, 16, 64, 128), (4, 8, 8192, 32, 128, 32)):
+        inp = synthetic.la_inputs(Bd, Hd, Nd, dfd, dvd, "bf16", seed=4)
+        q, k, v = (t.to(dev) for t in (inp.q, inp.k, inp.v))
+        gam = torch.full((Bd, Hd, (Nd + 127) // 128), 0.95, dtype=torch.float32, device=dev)
+        yd = torch.empty(Bd, Hd, Nd, dvd, dtype=torch.bfloat16, device=dev)
+        Dd = _feature_dim(dfd)
+        Sd = torch.empty(Bd, Hd, Dd, dvd, device=dev)
+        zd = torch.empty(Bd, Hd, Dd, device=dev)
+        wsd = torch.empty(based.lib().based_la_prefill_decay_workspace(Bd, Hd, Nd), dtype=torch.uint8, device=dev)
+        ms = timed(lambda: based.la_prefill_decay(q, k, v, gam, y=yd, S=Sd, z=zd, workspace=wsd), 1)
+        flops, byts = la_prefill_work(Bd, Hd, Nd, dfd, dvd, cd)
+        print(json.dumps({"sweep": "la_prefill_decay", "shape": f"B={Bd} H={Hd} N={Nd} d'={dfd} dv={dvd}",
+                          "us": ms * 1e3, "tokens_per_s": Bd * Nd / (ms / 1e3),
+                          "TFLOP_s": flops / (ms / 1e3) / 1e12,
+                          "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"]}), flush=True)
+        del q, k, v, gam, yd, Sd, zd, wsd
     # backward (training) pass at the 360M shape and the large-state shape
     for (Bb, Hb, Nb, dfb, dvb) in ((8, 16, 2048, 16, 64), (4, 8, 8192, 32, 128)):
         inp = synthetic.la_inputs(Bb, Hb, Nb, dfb, dvb, "bf16", seed=2)

@@ -205,6 +205,43 @@ BASED_API based_status_t based_la_decode_step_packed(float* S, float* z,
                                                      based_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * Coarse input-dependent decay (BASED App. C "Extended Architecture Details",
+ * Decay; App. D.4 "BASED Quality Ablations"). The pages print no formula; the
+ * reading implemented: one scalar gamma per 128-token tile scales the state
+ * where the tile begins, S_c = gamma_c S_{c-1} + sum_{t in tile c} phi(k_t) v_t^T
+ * (z likewise), and a tile's own keys are not decayed among themselves. Key j
+ * reaches query i >= j with the weight prod_{c = tile(j)+1 .. tile(i)} gamma_c,
+ * in the numerator and the denominator alike. gamma values lie in (0, 1].
+ *
+ * based_la_prefill_decay -- based_la_prefill with decay: gamma [B, H,
+ * ceil(N/128)] fp32 (device), one value per tile (tile 0's is unused). The
+ * quadratic-form tensor-core path: bf16 only, d_feat in {16, 32}, d_v in {64,
+ * 128}; other dtypes or sizes return BASED_ERR_UNSUPPORTED. S and z (optional
+ * together, full 1 + d' + d'^2 layout) receive the decayed final state.
+ * workspace >= based_la_prefill_decay_workspace(B, H, N) bytes of device memory,
+ * 16-byte aligned (per-tile log2 prefix sums of gamma).
+ */
+BASED_API size_t based_la_prefill_decay_workspace(int B, int H, int N);
+BASED_API based_status_t based_la_prefill_decay(const void* q, const void* k, const void* v, void* y,
+                                                float* S, float* z, const float* gamma,
+                                                int B, int H, int N, int d_feat, int d_v,
+                                                based_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                                cudaStream_t stream);
+
+/*
+ * based_la_decode_step_decay -- based_la_decode_step (packed = 0) or
+ * based_la_decode_step_packed (packed = 1) with the state first scaled by
+ * gamma [B, H] fp32 (device): S <- gamma S, z <- gamma z, then the token's
+ * update and output. Pass the tile's gamma on the first token of a 128-token
+ * tile and 1 otherwise to continue a decayed prefill. Errors as the undecayed
+ * step; gamma NULL returns BASED_ERR_INVALID_ARG.
+ */
+BASED_API based_status_t based_la_decode_step_decay(float* S, float* z, const void* q, const void* k,
+                                                    const void* v, void* y, const float* gamma,
+                                                    int B, int H, int d_feat, int d_v,
+                                                    based_dtype_t dtype, int packed, cudaStream_t stream);
+
+/*
  * based_la_backward -- gradients of the causal Taylor linear attention of
  * based_la_prefill (the training form of the prefill stage, BASED §5
  * "Execution stages"). With s_ij = q_i.k_j, a_ij = 1 + s_ij + s_ij^2/2,

@@ -14,7 +14,9 @@ from .binding import (  # noqa: F401
     la_backward,
     la_backward_workspace,
     la_decode_step,
+    la_decode_step_decay,
     la_prefill,
+    la_prefill_decay,
     la_prefill_noalloc,
     la_prefill_workspace,
     lib,

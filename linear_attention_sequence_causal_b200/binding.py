@@ -29,6 +29,9 @@ SYMBOLS = (
     "based_la_decode_step",
     "based_la_prefill_packed",
     "based_la_decode_step_packed",
+    "based_la_prefill_decay_workspace",
+    "based_la_prefill_decay",
+    "based_la_decode_step_decay",
     "based_la_backward_workspace",
     "based_la_backward",
     "based_swa_prefill",
@@ -62,6 +65,12 @@ def _declare(lib):
     lib.based_la_prefill_packed.restype = i
     lib.based_la_decode_step_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.based_la_decode_step_packed.restype = i
+    lib.based_la_prefill_decay_workspace.argtypes = [i, i, i]
+    lib.based_la_prefill_decay_workspace.restype = sz
+    lib.based_la_prefill_decay.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
+    lib.based_la_prefill_decay.restype = i
+    lib.based_la_decode_step_decay.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp]
+    lib.based_la_decode_step_decay.restype = i
     lib.based_la_backward_workspace.argtypes = [i, i, i, i, i, i]
     lib.based_la_backward_workspace.restype = sz
     lib.based_la_backward.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
@@ -198,6 +207,55 @@ def la_prefill_noalloc(q, k, v, chunk: int = 0, want_state: bool = True, y=None,
                                             B, H, N, d_feat, d_v, dt, chunk, _stream(dev))
     _check(st, "based_la_prefill_noalloc")
     return y, S, z
+
+
+DECAY_TILE = 128
+
+
+def la_prefill_decay(q, k, v, gamma, want_state: bool = True, y=None, S=None, z=None, workspace=None):
+    """Causal Taylor linear attention with coarse decay: gamma [B,H,ceil(N/128)] float32,
+    one value per 128-token tile (bf16 q, k, v). Returns (y, S, z)."""
+    dt = _dtype_code(q, k, v)
+    B, H, N, d_feat = q.shape
+    d_v = v.shape[-1]
+    D = feature_dim(d_feat)
+    nt = (N + DECAY_TILE - 1) // DECAY_TILE
+    if tuple(gamma.shape) != (B, H, nt) or gamma.dtype != torch.float32 or not gamma.is_contiguous() \
+            or gamma.device != q.device:
+        raise BasedError(ERR_INVALID_ARG, f"gamma must be a contiguous float32 [{B},{H},{nt}] on q's device")
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty((B, H, N, d_v), dtype=q.dtype, device=dev)
+        if want_state:
+            S = torch.empty((B, H, D, d_v), dtype=torch.float32, device=dev) if S is None else S
+            z = torch.empty((B, H, D), dtype=torch.float32, device=dev) if z is None else z
+        else:
+            S = z = None
+        ws_bytes = int(lib().based_la_prefill_decay_workspace(B, H, N))
+        if workspace is None or workspace.numel() < ws_bytes:
+            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        st = lib().based_la_prefill_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z), _ptr(gamma),
+                                          B, H, N, d_feat, d_v, dt, _ptr(workspace), ws_bytes, _stream(dev))
+    _check(st, "based_la_prefill_decay")
+    return y, S, z
+
+
+def la_decode_step_decay(S, z, q, k, v, gamma, y=None, packed: bool = False) -> torch.Tensor:
+    """One recurrent step after scaling the state by gamma [B,H] float32 (S, z in place)."""
+    dt = _dtype_code(q, k, v)
+    B, H, d_feat = q.shape
+    d_v = v.shape[-1]
+    if tuple(gamma.shape) != (B, H) or gamma.dtype != torch.float32 or not gamma.is_contiguous():
+        raise BasedError(ERR_INVALID_ARG, f"gamma must be a contiguous float32 [{B},{H}]")
+    dev = q.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty((B, H, d_v), dtype=q.dtype, device=dev)
+        st = lib().based_la_decode_step_decay(_ptr(S), _ptr(z), _ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(gamma),
+                                              B, H, d_feat, d_v, dt, 1 if packed else 0, _stream(dev))
+    _check(st, "based_la_decode_step_decay")
+    return y
 
 
 def la_backward_workspace(B, H, N, d_feat, d_v, dtype=torch.bfloat16) -> int:

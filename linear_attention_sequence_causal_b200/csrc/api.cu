@@ -159,17 +159,19 @@ based_status_t la_prefill_impl(const void* q, const void* k, const void* v, void
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
-based_status_t la_decode_impl(float* S, float* z, const void* q, const void* k, const void* v, void* y, int B,
-                              int H, int d_feat, int d_v, based_dtype_t dtype, bool packed, cudaStream_t stream) {
+based_status_t la_decode_impl(float* S, float* z, const void* q, const void* k, const void* v, void* y,
+                              const float* gamma, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
+                              bool packed, cudaStream_t stream) {
     if (!ok_ptr(S) || !ok_ptr(z) || !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y))
         return BASED_ERR_INVALID_ARG;
+    if (gamma != nullptr && (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0) return BASED_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
     if (!la_dims_built(d_feat, d_v) || (long long)B * H > (1LL << 30)) return BASED_ERR_UNSUPPORTED;
     int dev;
     if (!current_device(&dev)) return BASED_ERR_CUDA;
     const int sms = num_sms(dev);
     if (sms <= 0) return BASED_ERR_CUDA;
-    const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, B, H, d_feat, d_v, dtype == BASED_BF16,
+    const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, gamma, B, H, d_feat, d_v, dtype == BASED_BF16,
                                                   packed, sms, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
@@ -194,16 +196,53 @@ based_status_t based_la_prefill_packed(const void* q, const void* k, const void*
                            true, stream);
 }
 
+size_t based_la_prefill_decay_workspace(int B, int H, int N) {
+    if (B <= 0 || H <= 0 || N <= 0) return 0;
+    return (size_t)B * H * ((N + 127) / 128) * sizeof(float);
+}
+
+based_status_t based_la_prefill_decay(const void* q, const void* k, const void* v, void* y, float* S, float* z,
+                                      const float* gamma, int B, int H, int N, int d_feat, int d_v,
+                                      based_dtype_t dtype, void* workspace, size_t workspace_bytes,
+                                      cudaStream_t stream) {
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
+    if ((S == nullptr) != (z == nullptr)) return BASED_ERR_INVALID_ARG;
+    if (S != nullptr && (!aligned16(S) || !aligned16(z))) return BASED_ERR_INVALID_ARG;
+    if (gamma == nullptr || (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || H <= 0 || N <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (dtype != BASED_BF16 || !based::la_prefill_quad_supported(d_feat, d_v) || (long long)B * H > 65535)
+        return BASED_ERR_UNSUPPORTED;
+    const size_t need = based_la_prefill_decay_workspace(B, H, N);
+    if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need) return BASED_ERR_INVALID_ARG;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const int sms = num_sms(dev);
+    unsigned* status = status_word(dev);
+    if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
+    based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, true, 128, nullptr, 0, status, debug_flags(), false};
+    a.gamma = gamma;
+    a.dlog = static_cast<float*>(workspace);
+    const cudaError_t e = based::launch_la_prefill_quad(a, sms, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
 based_status_t based_la_decode_step(float* S, float* z, const void* q, const void* k, const void* v,
                                     void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
                                     cudaStream_t stream) {
-    return la_decode_impl(S, z, q, k, v, y, B, H, d_feat, d_v, dtype, false, stream);
+    return la_decode_impl(S, z, q, k, v, y, nullptr, B, H, d_feat, d_v, dtype, false, stream);
 }
 
 based_status_t based_la_decode_step_packed(float* S, float* z, const void* q, const void* k, const void* v,
                                            void* y, int B, int H, int d_feat, int d_v, based_dtype_t dtype,
                                            cudaStream_t stream) {
-    return la_decode_impl(S, z, q, k, v, y, B, H, d_feat, d_v, dtype, true, stream);
+    return la_decode_impl(S, z, q, k, v, y, nullptr, B, H, d_feat, d_v, dtype, true, stream);
+}
+
+based_status_t based_la_decode_step_decay(float* S, float* z, const void* q, const void* k, const void* v,
+                                          void* y, const float* gamma, int B, int H, int d_feat, int d_v,
+                                          based_dtype_t dtype, int packed, cudaStream_t stream) {
+    if (gamma == nullptr) return BASED_ERR_INVALID_ARG;
+    return la_decode_impl(S, z, q, k, v, y, gamma, B, H, d_feat, d_v, dtype, packed != 0, stream);
 }
 
 size_t based_la_backward_workspace(int B, int H, int N, int d_feat, int d_v, based_dtype_t dtype) {

@@ -18,6 +18,8 @@ struct LaPrefillArgs {
     unsigned* status;                // device status word
     unsigned debug;                  // DEBUG_* bits (testing only)
     bool packed = false;             // final state in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
+    const float* gamma = nullptr;    // coarse decay: [B*H][ceil(N/128)] per 128-token tile (quadratic path)
+    float* dlog = nullptr;           // with gamma: [B*H][ceil(N/128)] fp32 scratch for its log2 prefix
 };
 
 // Testing aid: with this bit the tensor-core kernels issue no MMA, so their
@@ -53,9 +55,10 @@ size_t la_backward_g_bytes(const LaBackwardArgs& a);
 cudaError_t launch_la_backward(const LaBackwardArgs& a, int num_sms, cudaStream_t stream);
 
 // `packed`: S and z hold the symmetric layout (1 + d' + d'(d'+1)/2 rows).
+// gamma: [B, H] fp32 decay applied to S, z before the token (nullptr: none).
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
-                             void* y, int B, int H, int d_feat, int d_v, bool bf16, bool packed,
-                             int num_sms, cudaStream_t stream);
+                             void* y, const float* gamma, int B, int H, int d_feat, int d_v, bool bf16,
+                             bool packed, int num_sms, cudaStream_t stream);
 
 cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y,
                                void* k_cache, void* v_cache, int B, int H, int N, int d, int w,

@@ -67,7 +67,8 @@ __device__ __forceinline__ void fma4(float4& acc, float s, const float4& x) {
 template <typename T, int DF, int DV, bool PACKED>
 __global__ void __launch_bounds__(kThreads)
 la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restrict__ q,
-                 const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y, int P) {
+                 const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y,
+                 const float* __restrict__ gamma, int P) {
     constexpr int D = PACKED ? sym_feature_dim(DF) : feature_dim(DF);
     constexpr int G = DV / 4;              // float4 column groups per row
     constexpr int RPS = kThreads / G;      // rows per sweep of the CTA
@@ -99,6 +100,9 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
         const int f = f0 + r_thr + u * RPS;
         if (f < f1) buf[u] = *reinterpret_cast<const float4*>(Sp + (size_t)f * DV);
     }
+
+    // Decay of the state before this token (1 without decay): S <- gamma S, z <- gamma z.
+    const float gdec = gamma != nullptr ? gamma[bh] : 1.0f;
 
     // This thread's z rows (at most two: a CTA holds at most 2 * kThreads rows).
     float* zbh = z + bh * D;
@@ -133,7 +137,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     for (int i = 0; i < 2; ++i) {
         const int f = f0 + tid + i * kThreads;
         if (f < f1) {
-            const float zn = zr[i] + phi(s_x[1], f);
+            const float zn = fmaf(gdec, zr[i], phi(s_x[1], f));
             zbh[f] = zn;
             dpart = fmaf(phi(s_x[0], f), zn, dpart);
         }
@@ -146,7 +150,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
         for (int u = 0; u < kBatch; ++u) {
             const int f = base + u * RPS;
             if (f < f1) {
-                float4 s = buf[u];
+                float4 s = make_float4(gdec * buf[u].x, gdec * buf[u].y, gdec * buf[u].z, gdec * buf[u].w);
                 fma4(s, phi(s_x[1], f), vv);
                 *reinterpret_cast<float4*>(Sp + (size_t)f * DV) = s;
                 fma4(acc, phi(s_x[0], f), s);
@@ -215,7 +219,7 @@ int ranks_per_head(int BH, int D, int num_sms) {
 
 template <typename T, int DF, int DV, bool PACKED>
 cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const void* v, void* y,
-                         int BH, int num_sms, cudaStream_t stream) {
+                         const float* gamma, int BH, int num_sms, cudaStream_t stream) {
     const int P = ranks_per_head(BH, PACKED ? sym_feature_dim(DF) : feature_dim(DF), num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)BH * P);
@@ -234,30 +238,30 @@ cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV, PACKED>, S, z, static_cast<const T*>(q),
-                              static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), P);
+                              static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), gamma, P);
 }
 
 template <typename T, bool PACKED>
 cudaError_t dispatch(float* S, float* z, const void* q, const void* k, const void* v, void* y,
-                     int BH, int d_feat, int d_v, int num_sms, cudaStream_t stream) {
-    if (d_feat == 16 && d_v == 64) return launch_typed<T, 16, 64, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 16 && d_v == 128) return launch_typed<T, 16, 128, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 64) return launch_typed<T, 32, 64, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 128) return launch_typed<T, 32, 128, PACKED>(S, z, q, k, v, y, BH, num_sms, stream);
+                     const float* gamma, int BH, int d_feat, int d_v, int num_sms, cudaStream_t stream) {
+    if (d_feat == 16 && d_v == 64) return launch_typed<T, 16, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
+    if (d_feat == 16 && d_v == 128) return launch_typed<T, 16, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
+    if (d_feat == 32 && d_v == 64) return launch_typed<T, 32, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
+    if (d_feat == 32 && d_v == 128) return launch_typed<T, 32, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
     return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
-                             void* y, int B, int H, int d_feat, int d_v, bool bf16, bool packed, int num_sms,
-                             cudaStream_t stream) {
+                             void* y, const float* gamma, int B, int H, int d_feat, int d_v, bool bf16, bool packed,
+                             int num_sms, cudaStream_t stream) {
     const int BH = B * H;
     if (packed)
-        return bf16 ? dispatch<__nv_bfloat16, true>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream)
-                    : dispatch<float, true>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream);
-    return bf16 ? dispatch<__nv_bfloat16, false>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream)
-                : dispatch<float, false>(S, z, q, k, v, y, BH, d_feat, d_v, num_sms, stream);
+        return bf16 ? dispatch<__nv_bfloat16, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream)
+                    : dispatch<float, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream);
+    return bf16 ? dispatch<__nv_bfloat16, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream)
+                : dispatch<float, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream);
 }
 
 }  // namespace based

@@ -103,6 +103,7 @@ struct QuadCtx {
     volatile int* abort_flag;
     unsigned* status;
     int N, BH, nqt, nunits;
+    const float* dlog;                          // decay: [BH][nqt] log2 prefix of gamma, or nullptr
 };
 
 __device__ __forceinline__ bool qwait(const QuadCtx& cx, int bar, uint32_t parity) {
@@ -159,13 +160,19 @@ __device__ __forceinline__ void quad_producer(const QuadCtx& cx, const CUtensorM
 }
 
 // A of one slice (16 keys, from column j_base) of row i: P = bf16(1 + S + S^2/2),
-// masked past i on the diagonal tile, with the row sum accumulated in fp32.
-__device__ __forceinline__ void quad_slice(const float* sv, uint32_t* pw, int j_base, int i, bool diag, float& l0,
-                                           float& l1) {
+// times the decay weight w of the tile pair (DECAY), masked past i on the
+// diagonal tile, with the row sum accumulated in fp32.
+template <bool DECAY>
+__device__ __forceinline__ void quad_slice(const float* sv, uint32_t* pw, int j_base, int i, bool diag, float w,
+                                           float& l0, float& l1) {
 #pragma unroll
     for (int m = 0; m < 8; ++m) {
         float a0, a1;
         taylor_pair(sv[2 * m], sv[2 * m + 1], a0, a1);
+        if constexpr (DECAY) {
+            a0 *= w;                             // the tile pair's decay weight
+            a1 *= w;
+        }
         if (diag) {
             const int j0 = j_base + 2 * m;
             a0 = j0 <= i ? a0 : 0.0f;
@@ -200,6 +207,10 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
             if (!qwait(cx, QB_SF0 + g, (step / kBufs) & 1)) return;
             tc_fence_after();
             const bool diag = kt == qt;          // keys j > i of the diagonal tile are masked
+            // Coarse decay: key tile kt reaches query tile qt scaled by the product
+            // of gamma over tiles kt+1..qt = 2^(L[qt] - L[kt]).
+            const bool decay = cx.dlog != nullptr;
+            const float w = decay ? exp2f(cx.dlog[(size_t)bh * cx.nqt + qt] - cx.dlog[(size_t)bh * cx.nqt + kt]) : 1.0f;
             // Slice c reads S columns 16c..16c+15 and writes P columns 8c..8c+7,
             // which overlay S columns already read; the next slice's load is in
             // flight while a slice is computed.
@@ -210,11 +221,13 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
 #pragma unroll 1
             for (int c2 = 0; c2 < 4; ++c2) {
                 tmem_ld16(sb + 32 * c2 + 16, s1);
-                quad_slice(s0, pw, 32 * c2, i, diag, l0, l1);
+                if (decay) quad_slice<true>(s0, pw, 32 * c2, i, diag, w, l0, l1);
+                else quad_slice<false>(s0, pw, 32 * c2, i, diag, w, l0, l1);
                 tmem_st8(sb + 16 * c2, pw);
                 tmem_ld_wait();
                 if (c2 < 3) tmem_ld16(sb + 32 * c2 + 32, s0);
-                quad_slice(s1, pw, 32 * c2 + 16, i, diag, l0, l1);
+                if (decay) quad_slice<true>(s1, pw, 32 * c2 + 16, i, diag, w, l0, l1);
+                else quad_slice<false>(s1, pw, 32 * c2 + 16, i, diag, w, l0, l1);
                 tmem_st8(sb + 16 * c2 + 8, pw);
                 if (c2 < 3) tmem_ld_wait();
             }
@@ -346,7 +359,7 @@ template <int DF, int DV>
 __global__ void __launch_bounds__(kQuadThreads, 1)
 la_quad_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ y, int N, int BH, int nqt,
-               unsigned* status, unsigned debug) {
+               const float* __restrict__ dlog, unsigned* status, unsigned debug) {
     using L = QuadLayout<DF, DV>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -356,7 +369,7 @@ la_quad_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::OFF_BAR + 8 * QB_NUM);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::OFF_BAR + 8 * QB_NUM + 4);
     const QuadCtx cx{sbase, bars, reinterpret_cast<float*>(smem + L::OFF_L), abort_flag, status, N, BH, nqt,
-                     nqt * BH};
+                     nqt * BH, dlog};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int b = 0; b < QB_NUM; ++b) {
@@ -435,26 +448,26 @@ __device__ __forceinline__ float phi_elem(const float* x) {
 }
 
 template <int DF, int F0, int... E>
-__device__ __forceinline__ uint4 phi_piece(const float* x, std::integer_sequence<int, E...>) {
-    const float f8[8] = {phi_elem<DF, F0 + E>(x)...};
+__device__ __forceinline__ uint4 phi_piece(const float* x, float u, std::integer_sequence<int, E...>) {
+    const float f8[8] = {(phi_elem<DF, F0 + E>(x) * u)...};
     return pack_bf16x8(f8);
 }
 
 template <int DF, int F0, int... J>
-__device__ __forceinline__ void state_phi_half_impl(const float* x, uint32_t row, uint32_t sbo,
+__device__ __forceinline__ void state_phi_half_impl(const float* x, float u, uint32_t row, uint32_t sbo,
                                                     std::integer_sequence<int, J...>) {
-    ((st_shared_v4(row + J * sbo, phi_piece<DF, F0 + 8 * J>(x, std::make_integer_sequence<int, 8>{}))), ...);
+    ((st_shared_v4(row + J * sbo, phi_piece<DF, F0 + 8 * J>(x, u, std::make_integer_sequence<int, 8>{}))), ...);
 }
 
 // Features [64 H, 64 H + 64) for the selector sel == H (H < HMAX).
 template <int DF, int H, int HMAX>
-__device__ __forceinline__ void state_phi_half(int sel, const float* x, uint32_t row, uint32_t sbo) {
+__device__ __forceinline__ void state_phi_half(int sel, const float* x, float u, uint32_t row, uint32_t sbo) {
     if constexpr (H < HMAX) {
         if (sel == H) {
-            state_phi_half_impl<DF, 64 * H>(x, row, sbo, std::make_integer_sequence<int, 8>{});
+            state_phi_half_impl<DF, 64 * H>(x, u, row, sbo, std::make_integer_sequence<int, 8>{});
             return;
         }
-        state_phi_half<DF, H + 1, HMAX>(sel, x, row, sbo);
+        state_phi_half<DF, H + 1, HMAX>(sel, x, u, row, sbo);
     }
 }
 
@@ -487,7 +500,8 @@ enum { SB_FULL0, SB_FULL1, SB_PHI0, SB_PHI1, SB_FREE0, SB_FREE1, SB_DONE, SB_NUM
 template <int DF, int DV>
 __global__ void __launch_bounds__(kStateThreads, 2)
 la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                float* __restrict__ S, float* __restrict__ z, int N, int packed, unsigned* status, unsigned debug) {
+                float* __restrict__ S, float* __restrict__ z, int N, int packed, const float* __restrict__ dlog,
+                unsigned* status, unsigned debug) {
     using L = StateLayout<DF, DV>;
     extern __shared__ unsigned char smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -502,6 +516,7 @@ la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
     const int ft = blockIdx.x % L::NFT;
     const int f0 = ft * 128;
     const int nchunks = (N + CS - 1) / CS;
+    const int nqt = (N + 127) / 128;                      // 128-token decay tiles
 
     if (tid < 128) {
         // Feature f0 + tid of the folded order [1, x_a, x_a x_b (a <= b, a-major)]
@@ -564,7 +579,12 @@ la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
                 }
             }
             x[DF] = c * CS + t < N ? 1.0f : 0.0f;
-            state_phi_half<DF, 0, 2 * L::NFT>(2 * ft + fh, x, arow + b * L::A_BYTES, L::A_SBO);
+            // Coarse decay: token t's contribution to the final state is scaled by the
+            // product of gamma over the 128-token tiles after its own.
+            const int tok = c * CS + t;
+            const float u = dlog != nullptr ? exp2f(dlog[(size_t)bh * nqt + nqt - 1] - dlog[(size_t)bh * nqt + tok / 128])
+                                            : 1.0f;
+            state_phi_half<DF, 0, 2 * L::NFT>(2 * ft + fh, x, u, arow + b * L::A_BYTES, L::A_SBO);
             fence_proxy_async_smem();
             mbar_arrive(&bars[SB_PHI0 + b]);
         }
@@ -662,6 +682,19 @@ la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
     }
 }
 
+// Coarse decay: L[bh][c] = sum over tiles c' <= c of log2 gamma[bh][c'], so that
+// the product of gamma over tiles a+1..b is 2^(L[b] - L[a]).
+__global__ void decay_log2_prefix_kernel(const float* __restrict__ gamma, float* __restrict__ dlog, int BH,
+                                         int nqt) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    float acc = 0.0f;
+    for (int c = 0; c < nqt; ++c) {
+        acc += log2f(gamma[(size_t)bh * nqt + c]);
+        dlog[(size_t)bh * nqt + c] = acc;
+    }
+}
+
 template <int DF, int DV>
 cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
     using bf = __nv_bfloat16;
@@ -679,8 +712,14 @@ cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t 
     cudaError_t e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QL::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<long long>(nunits, num_sms);
-    qk<<<grid, kQuadThreads, QL::SMEM_BYTES, stream>>>(mq, mk, mv, static_cast<bf*>(a.y), a.N, BH, nqt, a.status,
-                                                       a.debug);
+    const float* dlog = nullptr;
+    if (a.gamma != nullptr) {
+        if (a.dlog == nullptr) return cudaErrorInvalidValue;
+        decay_log2_prefix_kernel<<<(BH + 127) / 128, 128, 0, stream>>>(a.gamma, a.dlog, BH, nqt);
+        dlog = a.dlog;
+    }
+    qk<<<grid, kQuadThreads, QL::SMEM_BYTES, stream>>>(mq, mk, mv, static_cast<bf*>(a.y), a.N, BH, nqt, dlog,
+                                                       a.status, a.debug);
     e = cudaGetLastError();
     if (e != cudaSuccess || a.S == nullptr) return e;
     using SL = StateLayout<DF, DV>;
@@ -692,7 +731,7 @@ cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t 
     e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     sk<<<BH * SL::NFT, kStateThreads, SL::SMEM_BYTES, stream>>>(sk_map, sv_map, a.S, a.z, a.N, a.packed ? 1 : 0,
-                                                                 a.status, a.debug);
+                                                                 dlog, a.status, a.debug);
     return cudaGetLastError();
 }
 

@@ -122,6 +122,30 @@ def test_la_backward_rejects_bad_arguments(lib):
     assert call(nbytes=16) == binding.ERR_INVALID_ARG        # smaller than the query
 
 
+def test_decay_entries_reject_bad_arguments(lib):
+    pd = lib.based_la_prefill_decay
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 16, 64, 1, FAKE, 1 << 20, None)
+
+    def call(**kw):
+        a = list(ok)
+        names = ["q", "k", "v", "y", "S", "z", "gamma", "B", "H", "N", "df", "dv", "dt", "ws", "nbytes", "st"]
+        for key, val in kw.items():
+            a[names.index(key)] = val
+        return pd(*a)
+
+    assert call(gamma=None) == binding.ERR_INVALID_ARG
+    assert call(S=None) == binding.ERR_INVALID_ARG            # S without z
+    assert call(ws=None) == binding.ERR_INVALID_ARG
+    assert call(nbytes=8) == binding.ERR_INVALID_ARG          # smaller than the query (3 tiles x 4 bytes)
+    assert call(dt=0) == binding.ERR_UNSUPPORTED              # fp32: bf16 tensor cores only
+    assert call(df=24) == binding.ERR_UNSUPPORTED
+    assert lib.based_la_prefill_decay_workspace(2, 3, 300) == 2 * 3 * 3 * 4
+    assert lib.based_la_prefill_decay_workspace(1, 1, 0) == 0
+    dd = lib.based_la_decode_step_decay
+    assert dd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 64, 1, 0, None) == binding.ERR_INVALID_ARG
+    assert dd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 24, 64, 1, 0, None) == binding.ERR_UNSUPPORTED
+
+
 def test_la_backward_workspace_query(lib):
     # g (bf16) and c (fp32) per token, rows padded to a multiple of 128.
     assert lib.based_la_backward_workspace(2, 3, 300, 16, 64, 1) == 2 * 3 * 384 * (64 * 2 + 4)
