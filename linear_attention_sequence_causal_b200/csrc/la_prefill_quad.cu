@@ -189,7 +189,7 @@ __device__ __forceinline__ void quad_slice(const float* sv, uint32_t* pw, int j_
 // groups pool their row sums through shared memory and write y = O / l, group g
 // for the 32-column blocks h = g, g + kBufs, ... Thread = query row i = TMEM
 // lane (wq = lane quadrant).
-template <int DF, int DV>
+template <int DF, int DV, bool DECAY>
 __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int g, int wq, int lane,
                                           __nv_bfloat16* __restrict__ y) {
     using L = QuadLayout<DF, DV>;
@@ -209,8 +209,7 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
             const bool diag = kt == qt;          // keys j > i of the diagonal tile are masked
             // Coarse decay: key tile kt reaches query tile qt scaled by the product
             // of gamma over tiles kt+1..qt = 2^(L[qt] - L[kt]).
-            const bool decay = cx.dlog != nullptr;
-            const float w = decay ? exp2f(cx.dlog[(size_t)bh * cx.nqt + qt] - cx.dlog[(size_t)bh * cx.nqt + kt]) : 1.0f;
+            const float w = DECAY ? exp2f(cx.dlog[(size_t)bh * cx.nqt + qt] - cx.dlog[(size_t)bh * cx.nqt + kt]) : 1.0f;
             // Slice c reads S columns 16c..16c+15 and writes P columns 8c..8c+7,
             // which overlay S columns already read; the next slice's load is in
             // flight while a slice is computed.
@@ -221,13 +220,11 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
 #pragma unroll 1
             for (int c2 = 0; c2 < 4; ++c2) {
                 tmem_ld16(sb + 32 * c2 + 16, s1);
-                if (decay) quad_slice<true>(s0, pw, 32 * c2, i, diag, w, l0, l1);
-                else quad_slice<false>(s0, pw, 32 * c2, i, diag, w, l0, l1);
+                quad_slice<DECAY>(s0, pw, 32 * c2, i, diag, w, l0, l1);
                 tmem_st8(sb + 16 * c2, pw);
                 tmem_ld_wait();
                 if (c2 < 3) tmem_ld16(sb + 32 * c2 + 32, s0);
-                if (decay) quad_slice<true>(s1, pw, 32 * c2 + 16, i, diag, w, l0, l1);
-                else quad_slice<false>(s1, pw, 32 * c2 + 16, i, diag, w, l0, l1);
+                quad_slice<DECAY>(s1, pw, 32 * c2 + 16, i, diag, w, l0, l1);
                 tmem_st8(sb + 16 * c2 + 8, pw);
                 if (c2 < 3) tmem_ld_wait();
             }
@@ -355,7 +352,7 @@ __device__ __forceinline__ void quad_o_issuer(const QuadCtx& cx, uint32_t tmem, 
     quad_drain(cx, last, lastp);
 }
 
-template <int DF, int DV>
+template <int DF, int DV, bool DECAY>
 __global__ void __launch_bounds__(kQuadThreads, 1)
 la_quad_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                const __grid_constant__ CUtensorMap tv, __nv_bfloat16* __restrict__ y, int N, int BH, int nqt,
@@ -396,7 +393,7 @@ la_quad_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ C
     } else if (warp < 4) {
         if (lane == 0 && !skip_mma && warp - 2 < L::NO) quad_o_issuer<DF, DV>(cx, tmem, warp - 2);
     } else {
-        quad_rows<DF, DV>(cx, tmem, (warp - 4) >> 2, warp & 3, lane, y);
+        quad_rows<DF, DV, DECAY>(cx, tmem, (warp - 4) >> 2, warp & 3, lane, y);
     }
 
     tc_fence_before();
@@ -497,7 +494,7 @@ struct StateLayout {
 
 enum { SB_FULL0, SB_FULL1, SB_PHI0, SB_PHI1, SB_FREE0, SB_FREE1, SB_DONE, SB_NUM };
 
-template <int DF, int DV>
+template <int DF, int DV, bool DECAY>
 __global__ void __launch_bounds__(kStateThreads, 2)
 la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                 float* __restrict__ S, float* __restrict__ z, int N, int packed, const float* __restrict__ dlog,
@@ -582,8 +579,7 @@ la_state_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__ 
             // Coarse decay: token t's contribution to the final state is scaled by the
             // product of gamma over the 128-token tiles after its own.
             const int tok = c * CS + t;
-            const float u = dlog != nullptr ? exp2f(dlog[(size_t)bh * nqt + nqt - 1] - dlog[(size_t)bh * nqt + tok / 128])
-                                            : 1.0f;
+            const float u = DECAY ? exp2f(dlog[(size_t)bh * nqt + nqt - 1] - dlog[(size_t)bh * nqt + tok / 128]) : 1.0f;
             state_phi_half<DF, 0, 2 * L::NFT>(2 * ft + fh, x, u, arow + b * L::A_BYTES, L::A_SBO);
             fence_proxy_async_smem();
             mbar_arrive(&bars[SB_PHI0 + b]);
@@ -708,7 +704,7 @@ cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t 
         !make_tmap_bf16_3d_swizzle(&mk, a.k, DF, a.N, BH, DF, C, QL::QK_SWIZZLE) ||
         !make_tmap_bf16_3d_swizzle(&mv, a.v, DV, a.N, BH, 64, C, 128))
         return cudaErrorInvalidValue;
-    auto qk = la_quad_kernel<DF, DV>;
+    auto qk = a.gamma != nullptr ? la_quad_kernel<DF, DV, true> : la_quad_kernel<DF, DV, false>;
     cudaError_t e = cudaFuncSetAttribute(qk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)QL::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int grid = (int)std::min<long long>(nunits, num_sms);
@@ -727,7 +723,7 @@ cudaError_t launch_quad_typed(const LaPrefillArgs& a, int num_sms, cudaStream_t 
     if (!make_tmap_bf16_3d_swizzle(&sk_map, a.k, DF, a.N, BH, DF, CS, SL::K_SWIZZLE) ||
         !make_tmap_bf16_3d_swizzle(&sv_map, a.v, DV, a.N, BH, 64, CS, 128))
         return cudaErrorInvalidValue;
-    auto sk = la_state_kernel<DF, DV>;
+    auto sk = a.gamma != nullptr ? la_state_kernel<DF, DV, true> : la_state_kernel<DF, DV, false>;
     e = cudaFuncSetAttribute(sk, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SL::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     sk<<<BH * SL::NFT, kStateThreads, SL::SMEM_BYTES, stream>>>(sk_map, sv_map, a.S, a.z, a.N, a.packed ? 1 : 0,
