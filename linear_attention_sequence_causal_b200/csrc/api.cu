@@ -222,7 +222,9 @@ based_status_t based_la_prefill_decay(const void* q, const void* k, const void* 
     based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, true, 128, nullptr, 0, status, debug_flags(), false};
     a.gamma = gamma;
     a.dlog = static_cast<float*>(workspace);
-    const cudaError_t e = based::launch_la_prefill_quad(a, sms, stream);
+    // The chunked kernel where it is built (d' = 16, dv = 64), else the quadratic form.
+    const cudaError_t e = based::la_prefill_tc_supported(d_feat, d_v, 128) ? based::launch_la_prefill_tc(a, sms, stream)
+                                                                           : based::launch_la_prefill_quad(a, sms, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 

@@ -232,6 +232,7 @@ struct Work {
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this segment's total
     const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1
+    const float* gamma;      // coarse decay: this sequence's gamma per 128-token chunk, or nullptr (one segment)
 };
 
 struct Shared {
@@ -358,6 +359,7 @@ __device__ __forceinline__ void store_total(const Work& w, int n, uint32_t taddr
 // After MMA4 of chunk c: read the fp32 state row (two batches of 80 columns),
 // release it to MMA4 of chunk c+1, publish it as bf16 row n of the [S|z] buffer
 // for MMA3 of chunk c+1 -- or, after the last chunk, stage the final state.
+template <bool DECAY>
 __device__ __forceinline__ bool state_step(const Work& w, int c, int n, uint32_t taddr, const Shared& sh,
                                            float* S, float* z) {
     if (!mbar_wait(&sh.bars[BAR_DS], c & 1, sh.abort_flag, sh.status)) return false;
@@ -368,12 +370,25 @@ __device__ __forceinline__ bool state_step(const Work& w, int c, int n, uint32_t
     // for SBR phase c-1 before issuing MMA3_c, keeps SBR at most one phase ahead
     // of its waiter: a barrier two phases ahead would look unfinished to it.
     if (!last && !mbar_wait(&sh.bars[BAR_PQF], c & 1, sh.abort_flag, sh.status)) return false;
+    // Coarse decay: chunk c+1 reads gamma_{c+1} S_c, and its state update adds to
+    // gamma_{c+1} S_c, so the state is scaled in tensor memory before MMA4_{c+1}
+    // (which waits for DSF) and published scaled.
+    const bool decay = DECAY && !last;
+    const float g = decay ? w.gamma[c + 1] : 1.0f;
     float r[80];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
         for (int m = 0; m < 5; ++m) tmem_ld16(taddr + 80 * half + 16 * m, r + 16 * m);
         tmem_ld_wait();
+        if (decay) {                                     // compiled only into the DECAY kernel
+#pragma unroll
+            for (int i = 0; i < 80; ++i) r[i] *= g;
+#pragma unroll
+            for (int m = 0; m < 5; ++m)
+                tmem_st16(taddr + 80 * half + 16 * m, reinterpret_cast<const uint32_t*>(r + 16 * m));
+            if (half == 1) tmem_st_wait();
+        }
         if (half == 1 && !last) {
             tc_fence_before();
             mbar_arrive(&sh.bars[BAR_DSF]);
@@ -694,12 +709,14 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
 }
 
 // mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2.
+template <bool DECAY>
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
                      float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_chunks, int mode,
-                     int packed, float* __restrict__ ws, unsigned* status, unsigned debug) {
+                     int packed, float* __restrict__ ws, const float* __restrict__ gamma, unsigned* status,
+                     unsigned debug) {
     extern __shared__ __align__(1024) unsigned char smem[];
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
     uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * NUM_BARS);
@@ -724,6 +741,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     w.packed = packed != 0;
     w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) + w.seg) * kTotalFloats : nullptr;
     w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
+    w.gamma = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
 
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) {
@@ -759,7 +777,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
             if (state && w.has_init) init_state(w, n, taddr, sh);
             bool ok = intra(sh, tmem, wq, lane, 0);
             for (int c = 0; ok && c < w.nchunks; ++c) {
-                if (state) ok = state_step(w, c, n, taddr, sh, S, z);
+                if (state) ok = state_step<DECAY>(w, c, n, taddr, sh, S, z);
                 if (ok && c + 1 < w.nchunks) ok = intra(sh, tmem, wq, lane, c + 1);
             }
         }
@@ -811,12 +829,16 @@ size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chu
 
 cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
     if (!la_prefill_tc_supported(a.d_feat, a.d_v, a.chunk) || !a.bf16) return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(la_prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_BYTES);
+    auto kern = a.gamma != nullptr ? la_prefill_tc_kernel<true> : la_prefill_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
     if (e != cudaSuccess) return e;
     const int BH = a.B * a.H;
     int nseg, seg_chunks;
     plan_segments(BH, a.N, num_sms, &nseg, &seg_chunks);
+    if (a.gamma != nullptr) {                            // coarse decay: one segment per sequence
+        nseg = 1;
+        seg_chunks = (a.N + C - 1) / C;
+    }
     using bf = __nv_bfloat16;
     auto q = static_cast<const bf*>(a.q);
     auto k = static_cast<const bf*>(a.k);
@@ -826,12 +848,12 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
     CUtensorMap ty;
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {
-        e = launch_pdl(la_prefill_tc_kernel, dim3(BH * (nseg - 1)), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v,
-                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, a.packed ? 1 : 0, ws, a.status, a.debug);
+        e = launch_pdl(kern, dim3(BH * (nseg - 1)), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v,
+                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(la_prefill_tc_kernel, dim3(BH * nseg), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v, y, a.S,
-                      a.z, a.N, nseg, seg_chunks, 0, a.packed ? 1 : 0, ws, a.status, a.debug);
+    return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v, y, a.S,
+                      a.z, a.N, nseg, seg_chunks, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
 }
 
 }  // namespace based
