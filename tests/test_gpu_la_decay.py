@@ -98,10 +98,13 @@ def test_decode_decay_packed_from_empty_state():
     assert_y(to64(torch.stack(ys, dim=2)), ref, torch.bfloat16, "decode y")
 
 
-def test_prefill_decay_long_sampled_heads():
-    """4096 tokens (32 tiles), d'=32, dv=128, gamma near 1 as a trained decay would be."""
+@pytest.mark.parametrize("d_feat,d_v", [(16, 64), (32, 128)])
+def test_prefill_decay_long_sampled_heads(d_feat, d_v):
+    """4096 tokens (32 tiles), gamma near 1 as a trained decay would be: the chunked
+    kernel (d'=16, dv=64) rescales its state 31 times, the quadratic form weighs
+    tile pairs up to 31 tiles apart."""
     B, H, N = 1, 4, 4096
-    inp = synthetic.la_inputs(B, H, N, 32, 128, "bf16", seed=11)
+    inp = synthetic.la_inputs(B, H, N, d_feat, d_v, "bf16", seed=11)
     g, g64 = _gamma(B, H, N, seed=12, lo=0.9)
     q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
     y, S, z = based.la_prefill_decay(q, k, v, g.to(DEV))
