@@ -47,3 +47,21 @@ def test_stalled_swa_prefill_reports_timeout(monkeypatch):
     y, _, _ = based.swa_prefill(q, k, v, w=64)
     assert based.get_last_error() == 0
     assert_y(to64(y), oracle.swa(inp.q64, inp.k64, inp.v64, 64, 1 / math.sqrt(64)), torch.bfloat16)
+
+
+def test_stalled_la_backward_reports_timeout(monkeypatch):
+    import torch
+    inp = synthetic.la_inputs(1, 2, 300, 16, 64, "bf16", seed=5)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    dy, dy64 = synthetic.upstream_grad((1, 2, 300, 64), "bf16", seed=6)
+    dy = dy.to(DEV)
+    y, _, _ = based.la_prefill(q, k, v, want_state=False)
+    monkeypatch.setenv("BASED_DEBUG_SKIP_MMA", "1")
+    based.la_backward(q, k, v, y, dy)                 # both launches succeed; their waits expire
+    assert based.get_last_error() == TIMEOUT
+    monkeypatch.delenv("BASED_DEBUG_SKIP_MMA")
+    dq, dk, dv = based.la_backward(q, k, v, y, dy)
+    assert based.get_last_error() == 0
+    ref = oracle.la_backward(inp.q64, inp.k64, inp.v64, dy64)
+    for got, r in zip((dq, dk, dv), ref):
+        assert float(np.abs(to64(got) - r).max() / np.abs(r).max()) < 2e-2
