@@ -772,7 +772,8 @@ def run_sweep(reps):
         Dd = _feature_dim(dfd)
         Sd = torch.empty(Bd, Hd, Dd, dvd, device=dev)
         zd = torch.empty(Bd, Hd, Dd, device=dev)
-        wsd = torch.empty(based.lib().based_la_prefill_decay_workspace(Bd, Hd, Nd), dtype=torch.uint8, device=dev)
+        wsd = torch.empty(max(16, based.lib().based_la_prefill_decay_workspace(Bd, Hd, Nd, dfd, dvd)),
+                          dtype=torch.uint8, device=dev)
         ms = timed(lambda: based.la_prefill_decay(q, k, v, gam, y=yd, S=Sd, z=zd, workspace=wsd), 1)
         flops, byts = la_prefill_work(Bd, Hd, Nd, dfd, dvd, cd)
         print(json.dumps({"sweep": "la_prefill_decay", "shape": f"B={Bd} H={Hd} N={Nd} d'={dfd} dv={dvd}",

@@ -219,10 +219,12 @@ BASED_API based_status_t based_la_decode_step_packed(float* S, float* z,
  * d_feat 16 / d_v 64, the quadratic form otherwise); other dtypes or sizes
  * return BASED_ERR_UNSUPPORTED. S and z (optional
  * together, full 1 + d' + d'^2 layout) receive the decayed final state.
- * workspace >= based_la_prefill_decay_workspace(B, H, N) bytes of device memory,
- * 16-byte aligned (per-tile log2 prefix sums of gamma).
+ * workspace >= based_la_prefill_decay_workspace(B, H, N, d_feat, d_v) bytes of
+ * device memory, 16-byte aligned (segment totals of the chunked kernel, or the
+ * per-tile log2 prefix sums of gamma; the chunked kernel's size depends on the
+ * current device's SM count, and may be 0).
  */
-BASED_API size_t based_la_prefill_decay_workspace(int B, int H, int N);
+BASED_API size_t based_la_prefill_decay_workspace(int B, int H, int N, int d_feat, int d_v);
 BASED_API based_status_t based_la_prefill_decay(const void* q, const void* k, const void* v, void* y,
                                                 float* S, float* z, const float* gamma,
                                                 int B, int H, int N, int d_feat, int d_v,

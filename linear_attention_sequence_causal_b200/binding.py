@@ -65,7 +65,7 @@ def _declare(lib):
     lib.based_la_prefill_packed.restype = i
     lib.based_la_decode_step_packed.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
     lib.based_la_decode_step_packed.restype = i
-    lib.based_la_prefill_decay_workspace.argtypes = [i, i, i]
+    lib.based_la_prefill_decay_workspace.argtypes = [i, i, i, i, i]
     lib.based_la_prefill_decay_workspace.restype = sz
     lib.based_la_prefill_decay.argtypes = [vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, vp, sz, vp]
     lib.based_la_prefill_decay.restype = i
@@ -232,11 +232,12 @@ def la_prefill_decay(q, k, v, gamma, want_state: bool = True, y=None, S=None, z=
             z = torch.empty((B, H, D), dtype=torch.float32, device=dev) if z is None else z
         else:
             S = z = None
-        ws_bytes = int(lib().based_la_prefill_decay_workspace(B, H, N))
+        ws_bytes = int(lib().based_la_prefill_decay_workspace(B, H, N, d_feat, d_v))
         if workspace is None or workspace.numel() < ws_bytes:
-            workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+            workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=dev)
         st = lib().based_la_prefill_decay(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z), _ptr(gamma),
-                                          B, H, N, d_feat, d_v, dt, _ptr(workspace), ws_bytes, _stream(dev))
+                                          B, H, N, d_feat, d_v, dt, _ptr(workspace), workspace.numel(),
+                                          _stream(dev))
     _check(st, "based_la_prefill_decay")
     return y, S, z
 

@@ -196,9 +196,15 @@ based_status_t based_la_prefill_packed(const void* q, const void* k, const void*
                            true, stream);
 }
 
-size_t based_la_prefill_decay_workspace(int B, int H, int N) {
-    if (B <= 0 || H <= 0 || N <= 0) return 0;
-    return (size_t)B * H * ((N + 127) / 128) * sizeof(float);
+size_t based_la_prefill_decay_workspace(int B, int H, int N, int d_feat, int d_v) {
+    if (B <= 0 || H <= 0 || N <= 0 || !based::la_prefill_quad_supported(d_feat, d_v)) return 0;
+    if (based::la_prefill_tc_supported(d_feat, d_v, 128)) {
+        // The chunked kernel: segment totals, sized for this device's SMs.
+        int dev;
+        if (!current_device(&dev)) return 0;
+        return based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, 128, num_sms(dev));
+    }
+    return (size_t)B * H * ((N + 127) / 128) * sizeof(float);   // the quadratic form: log2 prefix of gamma
 }
 
 based_status_t based_la_prefill_decay(const void* q, const void* k, const void* v, void* y, float* S, float* z,
@@ -212,19 +218,26 @@ based_status_t based_la_prefill_decay(const void* q, const void* k, const void* 
     if (B <= 0 || H <= 0 || N <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
     if (dtype != BASED_BF16 || !based::la_prefill_quad_supported(d_feat, d_v) || (long long)B * H > 65535)
         return BASED_ERR_UNSUPPORTED;
-    const size_t need = based_la_prefill_decay_workspace(B, H, N);
-    if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need) return BASED_ERR_INVALID_ARG;
+    const bool chunked = based::la_prefill_tc_supported(d_feat, d_v, 128);
+    if (!chunked) {
+        const size_t need = (size_t)B * H * ((N + 127) / 128) * sizeof(float);
+        if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < need) return BASED_ERR_INVALID_ARG;
+    }
     int dev;
     if (!current_device(&dev)) return BASED_ERR_CUDA;
     const int sms = num_sms(dev);
     unsigned* status = status_word(dev);
     if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
-    based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, true, 128, nullptr, 0, status, debug_flags(), false};
+    if (chunked) {
+        const size_t need = based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, 128, sms);
+        if (workspace_bytes < need || (need > 0 && !ok_ptr(workspace))) return BASED_ERR_INVALID_ARG;
+    }
+    based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, true, 128, workspace, workspace_bytes,
+                           status, debug_flags(), false};
     a.gamma = gamma;
-    a.dlog = static_cast<float*>(workspace);
+    a.dlog = chunked ? nullptr : static_cast<float*>(workspace);
     // The chunked kernel where it is built (d' = 16, dv = 64), else the quadratic form.
-    const cudaError_t e = based::la_prefill_tc_supported(d_feat, d_v, 128) ? based::launch_la_prefill_tc(a, sms, stream)
-                                                                           : based::launch_la_prefill_quad(a, sms, stream);
+    const cudaError_t e = chunked ? based::launch_la_prefill_tc(a, sms, stream) : based::launch_la_prefill_quad(a, sms, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 

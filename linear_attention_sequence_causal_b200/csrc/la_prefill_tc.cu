@@ -232,7 +232,10 @@ struct Work {
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this segment's total
     const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1
-    const float* gamma;      // coarse decay: this sequence's gamma per 128-token chunk, or nullptr (one segment)
+    const float* gamma;      // coarse decay: gamma of this segment's chunks (index = local chunk), or nullptr
+    const float* gamma_head; // coarse decay: gamma of the sequence's chunks (index = global chunk)
+    int c0;                  // global index of this segment's first chunk
+    int seg_chunks;          // chunks per segment
 };
 
 struct Shared {
@@ -309,6 +312,10 @@ __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase,
 
 // Segment start state: row n = sum of the totals of segments 0..seg-1, placed in
 // the TMEM accumulator (fp32) and in the [S|z] buffer (bf16) for MMA3 of chunk 0.
+// With coarse decay (DECAY), the total of segment s' (its own state, started from
+// zero) counts with the product of gamma over the chunks from segment s'+1 up to
+// and including this segment's first chunk, whose gamma scales the state it enters.
+template <bool DECAY>
 __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr, const Shared& sh) {
     const bool real = n < NV;
 #pragma unroll 1
@@ -317,13 +324,19 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = 0.f;
         if (real) {
-            for (int s = 0; s < w.seg; ++s) {
+            float ws = DECAY ? w.gamma_head[w.c0] : 1.0f;   // weight of segment s, nearest first
+            for (int s = w.seg - 1; s >= 0; --s) {
                 const float4* src = reinterpret_cast<const float4*>(w.ws_in + s * kTotalFloats + (size_t)n * KF + 16 * m);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float4 t = __ldg(src + j);
-                    r[4 * j] += t.x; r[4 * j + 1] += t.y; r[4 * j + 2] += t.z; r[4 * j + 3] += t.w;
+                    r[4 * j] = fmaf(ws, t.x, r[4 * j]);
+                    r[4 * j + 1] = fmaf(ws, t.y, r[4 * j + 1]);
+                    r[4 * j + 2] = fmaf(ws, t.z, r[4 * j + 2]);
+                    r[4 * j + 3] = fmaf(ws, t.w, r[4 * j + 3]);
                 }
+                if constexpr (DECAY)
+                    for (int c = s * w.seg_chunks; c < (s + 1) * w.seg_chunks; ++c) ws *= w.gamma_head[c];
             }
         }
         uint32_t u[16];
@@ -338,10 +351,40 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
     mbar_arrive(&sh.bars[BAR_INIT]);
 }
 
+// Totals pass with coarse decay: after MMA4 of every chunk but the last, scale the
+// state by the next chunk's gamma in tensor memory and release it (DSF) to the
+// next MMA4; the total is then the segment's own decayed state.
+__device__ __forceinline__ bool totals_decay_steps(const Work& w, int n, uint32_t taddr, const Shared& sh) {
+    for (int c = 0; c + 1 < w.nchunks; ++c) {
+        if (!mbar_wait(&sh.bars[BAR_DS], c & 1, sh.abort_flag, sh.status)) return false;
+        tc_fence_after();
+        const float g = w.gamma[c + 1];
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            float r[80];
+#pragma unroll
+            for (int m = 0; m < 5; ++m) tmem_ld16(taddr + 80 * half + 16 * m, r + 16 * m);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 80; ++i) r[i] *= g;
+#pragma unroll
+            for (int m = 0; m < 5; ++m)
+                tmem_st16(taddr + 80 * half + 16 * m, reinterpret_cast<const uint32_t*>(r + 16 * m));
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&sh.bars[BAR_DSF]);
+    }
+    return true;
+}
+
 // Totals pass: once the last MMA4 has landed, copy row n of the accumulated
 // [S|z]^T (fp32) to this segment's slot in the workspace.
 __device__ __forceinline__ void store_total(const Work& w, int n, uint32_t taddr, const Shared& sh) {
-    if (!mbar_wait(&sh.bars[BAR_DS], 0, sh.abort_flag, sh.status)) return;
+    // Without decay the last MMA4 is the only DS commit (phase 0); with decay every
+    // chunk commits, and the last is phase (nchunks - 1) mod 2.
+    const uint32_t parity = w.gamma != nullptr ? (uint32_t)((w.nchunks - 1) & 1) : 0u;
+    if (!mbar_wait(&sh.bars[BAR_DS], parity, sh.abort_flag, sh.status)) return;
     tc_fence_after();
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -687,7 +730,8 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     for (int c = 0; ok && c < w.nchunks; ++c) {
         const int b = c & 1;
         if (!wait(BAR_IN0 + b, (c >> 1) & 1)) break;
-        if (c > 0 && !w.totals && !wait(BAR_DSF, (c - 1) & 1)) break;
+        const bool per_chunk = !w.totals || w.gamma != nullptr;   // the state warps step every chunk
+        if (c > 0 && per_chunk && !wait(BAR_DSF, (c - 1) & 1)) break;
         tc_fence_after();
         const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
         const uint64_t dpk = dpk0 + ((b * PK_BYTES) >> 4);
@@ -698,11 +742,11 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
         mma_commit(&bars[BAR_FREE0 + b]);
         last_bar = &bars[BAR_FREE0 + b];
         last_parity = (c >> 1) & 1;
-        // Totals pass: the state is read once, after the last chunk (phase 0).
-        if (!w.totals || c + 1 == w.nchunks) {
+        // Undecayed totals pass: the state is read once, after the last chunk (phase 0).
+        if (per_chunk || c + 1 == w.nchunks) {
             mma_commit(&bars[BAR_DS]);
             last_bar = &bars[BAR_DS];
-            last_parity = w.totals ? 0u : (uint32_t)(c & 1);
+            last_parity = per_chunk ? (uint32_t)(c & 1) : 0u;
         }
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
@@ -741,7 +785,10 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     w.packed = packed != 0;
     w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) + w.seg) * kTotalFloats : nullptr;
     w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
-    w.gamma = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
+    w.c0 = w.t_begin / C;
+    w.seg_chunks = seg_chunks;
+    w.gamma_head = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
+    w.gamma = gamma != nullptr ? w.gamma_head + w.c0 : nullptr;
 
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) {
@@ -772,9 +819,9 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
         const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + COL_ST;
         const bool state = wq < 3;
         if (w.totals) {
-            if (state) store_total(w, n, taddr, sh);
+            if (state && (w.gamma == nullptr || totals_decay_steps(w, n, taddr, sh))) store_total(w, n, taddr, sh);
         } else {
-            if (state && w.has_init) init_state(w, n, taddr, sh);
+            if (state && w.has_init) init_state<DECAY>(w, n, taddr, sh);
             bool ok = intra(sh, tmem, wq, lane, 0);
             for (int c = 0; ok && c < w.nchunks; ++c) {
                 if (state) ok = state_step<DECAY>(w, c, n, taddr, sh, S, z);
@@ -835,16 +882,14 @@ cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream
     const int BH = a.B * a.H;
     int nseg, seg_chunks;
     plan_segments(BH, a.N, num_sms, &nseg, &seg_chunks);
-    if (a.gamma != nullptr) {                            // coarse decay: one segment per sequence
-        nseg = 1;
-        seg_chunks = (a.N + C - 1) / C;
-    }
     using bf = __nv_bfloat16;
     auto q = static_cast<const bf*>(a.q);
     auto k = static_cast<const bf*>(a.k);
     auto v = static_cast<const bf*>(a.v);
     auto y = static_cast<bf*>(a.y);
     float* ws = static_cast<float*>(a.workspace);
+    if (nseg > 1 && (ws == nullptr || a.ws_bytes < la_prefill_tc_workspace(a.B, a.H, a.N, a.d_feat, a.d_v, C, num_sms)))
+        return cudaErrorInvalidValue;                    // the segment totals need their workspace
     CUtensorMap ty;
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {

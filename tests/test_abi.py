@@ -124,7 +124,8 @@ def test_la_backward_rejects_bad_arguments(lib):
 
 def test_decay_entries_reject_bad_arguments(lib):
     pd = lib.based_la_prefill_decay
-    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 16, 64, 1, FAKE, 1 << 20, None)
+    # d'=32, dv=128: the quadratic-form path, whose workspace need is known without a device
+    ok = (FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 300, 32, 128, 1, FAKE, 1 << 20, None)
 
     def call(**kw):
         a = list(ok)
@@ -139,8 +140,9 @@ def test_decay_entries_reject_bad_arguments(lib):
     assert call(nbytes=8) == binding.ERR_INVALID_ARG          # smaller than the query (3 tiles x 4 bytes)
     assert call(dt=0) == binding.ERR_UNSUPPORTED              # fp32: bf16 tensor cores only
     assert call(df=24) == binding.ERR_UNSUPPORTED
-    assert lib.based_la_prefill_decay_workspace(2, 3, 300) == 2 * 3 * 3 * 4
-    assert lib.based_la_prefill_decay_workspace(1, 1, 0) == 0
+    assert lib.based_la_prefill_decay_workspace(2, 3, 300, 32, 128) == 2 * 3 * 3 * 4
+    assert lib.based_la_prefill_decay_workspace(1, 1, 0, 32, 128) == 0
+    assert lib.based_la_prefill_decay_workspace(1, 1, 64, 24, 128) == 0
     dd = lib.based_la_decode_step_decay
     assert dd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 1, 16, 64, 1, 0, None) == binding.ERR_INVALID_ARG
     assert dd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 24, 64, 1, 0, None) == binding.ERR_UNSUPPORTED
