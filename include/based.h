@@ -214,10 +214,10 @@ BASED_API based_status_t based_la_decode_step_packed(float* S, float* z,
  * in the numerator and the denominator alike. gamma values lie in (0, 1].
  *
  * based_la_prefill_decay -- based_la_prefill with decay: gamma [B, H,
- * ceil(N/128)] fp32 (device), one value per tile (tile 0's is unused). bf16
- * only, d_feat in {16, 32}, d_v in {64, 128} (the chunked tensor-core kernel at
- * d_feat 16 / d_v 64, the quadratic form otherwise); other dtypes or sizes
- * return BASED_ERR_UNSUPPORTED. S and z (optional
+ * ceil(N/128)] fp32 (device), one value per tile (tile 0's is unused).
+ * d_feat in {16, 32}, d_v in {64, 128}, else BASED_ERR_UNSUPPORTED. bf16 runs
+ * on the tensor cores (the chunked kernel at d_feat 16 / d_v 64, the quadratic
+ * form otherwise), fp32 on the CUDA cores (no workspace). S and z (optional
  * together, full 1 + d' + d'^2 layout) receive the decayed final state.
  * workspace >= based_la_prefill_decay_workspace(B, H, N, d_feat, d_v) bytes of
  * device memory, 16-byte aligned (segment totals of the chunked kernel, or the

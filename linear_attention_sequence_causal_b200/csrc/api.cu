@@ -197,6 +197,7 @@ based_status_t based_la_prefill_packed(const void* q, const void* k, const void*
 }
 
 size_t based_la_prefill_decay_workspace(int B, int H, int N, int d_feat, int d_v) {
+    // (The bf16 paths; an fp32 call runs on the CUDA cores and needs none.)
     if (B <= 0 || H <= 0 || N <= 0 || !based::la_prefill_quad_supported(d_feat, d_v)) return 0;
     if (based::la_prefill_tc_supported(d_feat, d_v, 128)) {
         // The chunked kernel: segment totals, sized for this device's SMs.
@@ -216,8 +217,19 @@ based_status_t based_la_prefill_decay(const void* q, const void* k, const void* 
     if (S != nullptr && (!aligned16(S) || !aligned16(z))) return BASED_ERR_INVALID_ARG;
     if (gamma == nullptr || (reinterpret_cast<uintptr_t>(gamma) & 3u) != 0) return BASED_ERR_INVALID_ARG;
     if (B <= 0 || H <= 0 || N <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
-    if (dtype != BASED_BF16 || !based::la_prefill_quad_supported(d_feat, d_v) || (long long)B * H > 65535)
-        return BASED_ERR_UNSUPPORTED;
+    if (!la_dims_built(d_feat, d_v) || (long long)B * H > 65535) return BASED_ERR_UNSUPPORTED;
+    if (dtype == BASED_F32) {
+        // fp32: the CUDA-core kernel, default chunk (64 tokens at d' = 16, 32 at d' = 32).
+        int dev;
+        if (!current_device(&dev)) return BASED_ERR_CUDA;
+        unsigned* status = status_word(dev);
+        if (status == nullptr) return BASED_ERR_CUDA;
+        based::LaPrefillArgs a{q, k, v, y, S, z, B, H, N, d_feat, d_v, false, d_feat == 16 ? 64 : 32,
+                               nullptr, 0, status, debug_flags(), false};
+        a.gamma = gamma;
+        const cudaError_t e = based::launch_la_prefill_simt(a, stream);
+        return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+    }
     const bool chunked = based::la_prefill_tc_supported(d_feat, d_v, 128);
     if (!chunked) {
         const size_t need = (size_t)B * H * ((N + 127) / 128) * sizeof(float);

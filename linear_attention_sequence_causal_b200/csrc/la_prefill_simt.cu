@@ -9,6 +9,8 @@
 //     A   = (1 + Q_c K_c^T + (Q_c K_c^T)^2 / 2) masked to j <= i
 //     y_c = (A V_c + phi(Q_c) S) / (rowsum A + phi(Q_c) z)
 //     S  += phi(K_c)^T V_c,   z += colsum phi(K_c)
+// (with coarse decay, S and z are first scaled by gamma where a 128-token tile
+// begins).
 //
 // This is the fp32 path (fp32 inputs, and any (d', dv) without a tensor-core
 // kernel). Each CTA owns one (b, h) and a 16-column slice of dv, keeps its slice
@@ -66,7 +68,8 @@ struct SimtSmem {
 template <typename T, int DF, int DV, int C>
 __global__ void __launch_bounds__(kThreads)
 la_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                       T* __restrict__ y, float* __restrict__ S, float* __restrict__ z, int N, int packed) {
+                       T* __restrict__ y, float* __restrict__ S, float* __restrict__ z, int N, int packed,
+                       const float* __restrict__ gamma) {
     using L = SimtSmem<DF, C>;
     constexpr int DS = L::DS;
     constexpr int D = feature_dim(DF);
@@ -101,8 +104,16 @@ la_prefill_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     const T* vb = v + bh * (size_t)N * DV;
     T* yb = y + bh * (size_t)N * DV;
 
+    // Coarse decay: gamma of each 128-token tile scales the state where the tile
+    // begins (a chunk of C <= 128 tokens never spans two tiles).
+    const float* gh = gamma != nullptr ? gamma + bh * (size_t)((N + 127) / 128) : nullptr;
     for (int t0 = 0; t0 < N; t0 += C) {
         const int nv = min(C, N - t0);
+        if (gh != nullptr && t0 > 0 && t0 % 128 == 0) {
+            const float g = gh[t0 / 128];
+            for (int e = tid; e < DS * kCW; e += kThreads) sS[e] *= g;
+            for (int e = tid; e < DS; e += kThreads) sz[e] *= g;
+        }
         for (int e = tid; e < C * DF; e += kThreads) {
             const int t = e / DF;
             const bool ok = t < nv;
@@ -216,7 +227,7 @@ cudaError_t launch_c(const LaPrefillArgs& a, cudaStream_t stream) {
     const dim3 grid(DV / kCW, a.B * a.H);
     kern<<<grid, kThreads, smem, stream>>>(static_cast<const T*>(a.q), static_cast<const T*>(a.k),
                                           static_cast<const T*>(a.v), static_cast<T*>(a.y), a.S, a.z,
-                                          a.N, a.packed ? 1 : 0);
+                                          a.N, a.packed ? 1 : 0, a.gamma);
     return cudaGetLastError();
 }
 

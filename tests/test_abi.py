@@ -138,8 +138,8 @@ def test_decay_entries_reject_bad_arguments(lib):
     assert call(S=None) == binding.ERR_INVALID_ARG            # S without z
     assert call(ws=None) == binding.ERR_INVALID_ARG
     assert call(nbytes=8) == binding.ERR_INVALID_ARG          # smaller than the query (3 tiles x 4 bytes)
-    assert call(dt=0) == binding.ERR_UNSUPPORTED              # fp32: bf16 tensor cores only
     assert call(df=24) == binding.ERR_UNSUPPORTED
+    assert call(dt=7) == binding.ERR_INVALID_ARG
     assert lib.based_la_prefill_decay_workspace(2, 3, 300, 32, 128) == 2 * 3 * 3 * 4
     assert lib.based_la_prefill_decay_workspace(1, 1, 0, 32, 128) == 0
     assert lib.based_la_prefill_decay_workspace(1, 1, 64, 24, 128) == 0

@@ -114,3 +114,18 @@ def test_prefill_decay_long_sampled_heads(d_feat, d_v):
         assert_y(to64(y[0, h]), ref, torch.bfloat16, f"y head {h}")
         rS, rz = oracle.la_state_decay(inp.k64[0, h], inp.v64[0, h], g64[0, h])
         assert_state(to64(S[0, h]), rS, torch.bfloat16, f"S head {h}")
+
+
+@pytest.mark.parametrize("d_feat,d_v", [(16, 64), (32, 128)])
+def test_prefill_decay_fp32_cuda_cores(d_feat, d_v):
+    """fp32 inputs: the CUDA-core kernel scales its state at every 128-token tile."""
+    B, H, N = 1, 2, 400
+    inp = synthetic.la_inputs(B, H, N, d_feat, d_v, "f32", seed=d_feat)
+    g, g64 = _gamma(B, H, N, seed=13)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y, S, z = based.la_prefill_decay(q, k, v, g.to(DEV))
+    assert based.get_last_error() == 0
+    assert_y(to64(y), oracle.la_quadratic_decay(inp.q64, inp.k64, inp.v64, g64), torch.float32)
+    rS, rz = oracle.la_state_decay(inp.k64, inp.v64, g64)
+    assert_state(to64(S), rS, torch.float32, "S")
+    assert_state(to64(z), rz, torch.float32, "z")
