@@ -79,3 +79,35 @@ def upstream_grad(shape, dtype: str = "bf16", seed: int = 0):
     """An upstream gradient dy ~ N(0, 1) of `shape`: (tensor of the dtype, float64 copy)."""
     rng = np.random.default_rng(seed)
     return _round(rng.standard_normal(shape, dtype=np.float32), dtype)
+
+
+@dataclass
+class ConvInputs:
+    """Inputs of the short gated convolution: the two projected streams and the filter.
+
+    u_gate, u_conv [B, N, d] torch CPU tensors of the compute dtype (plus float64
+    copies of the rounded values); h [d, K] and bias [d] float32 (plus float64 copies).
+    """
+
+    u_gate: torch.Tensor
+    u_conv: torch.Tensor
+    h: torch.Tensor
+    bias: torch.Tensor
+    gate64: np.ndarray
+    conv64: np.ndarray
+    h64: np.ndarray
+    bias64: np.ndarray
+
+
+def conv_inputs(B, N, d, taps, dtype="bf16", seed=0) -> ConvInputs:
+    """u_gate, u_conv ~ N(0, 1); filter taps ~ N(0, 1/K); bias ~ N(0, 0.1^2)."""
+    rng = np.random.default_rng(seed)
+    g = rng.standard_normal((B, N, d), dtype=np.float32)
+    x = rng.standard_normal((B, N, d), dtype=np.float32)
+    h = rng.standard_normal((d, taps), dtype=np.float32) * np.float32(taps ** -0.5)
+    b = rng.standard_normal((d,), dtype=np.float32) * np.float32(0.1)
+    tg, g64 = _round(g, dtype)
+    tx, x64 = _round(x, dtype)
+    th, h64 = _round(h, "f32")
+    tb, b64 = _round(b, "f32")
+    return ConvInputs(tg, tx, th, tb, g64, x64, h64, b64)

@@ -27,7 +27,9 @@ the recall-throughput tradeoff", BASED, arXiv 2402.18668v2, unless noted):
   (causally masked, quadratic) and an off-diagonal (cumulative state) part --
   App. B "Forward / Generation Prefill" (Algorithm 1);
 * the chunkwise form (intra-chunk + inter-chunk terms) -- "Gated Slot
-  Attention", App. A.1 "Hardware-Efficient Training".
+  Attention", App. A.1 "Hardware-Efficient Training";
+* the short gated convolution (BaseConv) mixer -- §4 "The BASED Architecture"
+  (Additional mixers) and App. C "Extended Architecture Details" (Convolution).
 
 Parity pins (see tests/test_oracle.py): closed forms, hand-derived golden
 values, equivalence of independent formulations, textbook special cases, a
@@ -65,5 +67,12 @@ from .swa import (  # noqa: F401
     swa_rows,
     swa_ring_after_prefill,
     swa_decode_step,
+)
+from .baseconv import (  # noqa: F401
+    silu,
+    short_conv,
+    baseconv,
+    baseconv_state,
+    baseconv_decode_step,
 )
 from . import brute  # noqa: F401
