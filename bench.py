@@ -85,6 +85,21 @@ def swa_decode_work(B, H, d, w):
     return flops, byts
 
 
+def baseconv_prefill_work(B, N, d, K):
+    """u_gate and u_conv read and y written once (bf16), the state rows written once; per
+    element K FMAs, the gate product and SiLU (counted as 4: negate, exp, add, divide)."""
+    flops = B * N * d * (2 * K + 5)
+    byts = B * N * d * 3 * 2 + B * (K - 1) * d * 2 + d * (K + 1) * 4
+    return flops, byts
+
+
+def baseconv_decode_work(B, d, K):
+    """Per step: the K-1 state rows read and written, u_gate and u_conv read, y written (bf16)."""
+    flops = B * d * (2 * K + 5)
+    byts = B * d * (2 * (K - 1) + 3) * 2 + d * (K + 1) * 4
+    return flops, byts
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -601,6 +616,8 @@ PROFILE_CASES = {
     "la_decode": "batch 256, H=16, d'=16, dv=64 (fp32 state 286 MB)",
     "swa_decode": "batch 1024, H=16, d=64, w=64 (ring caches 268 MB)",
     "la_backward": "B=8 H=16 N=2048 d'=16 dv=64 bf16 (q,k,v,y,dy,dq,dk,dv 168 MB)",
+    # below L2 size, but ncu flushes the caches before every pass, so DRAM counters still count
+    "baseconv": "B=8 N=2048 d=1024 K=4 bf16 (u_gate,u_conv,y 100 MB)",
 }
 
 
@@ -630,6 +647,10 @@ def run_profile(kind, reps):
         dy = synthetic.upstream_grad((8, 16, 2048, 64), "bf16", seed=1)[0].to(dev)
         y, _, _ = based.la_prefill(q, k, v, want_state=False)
         fn = lambda: based.la_backward(q, k, v, y, dy)
+    elif kind == "baseconv":
+        c = synthetic.conv_inputs(8, 2048, 1024, 4, "bf16", seed=0)
+        g, x, h, bias = (t.to(dev) for t in (c.u_gate, c.u_conv, c.h, c.bias))
+        fn = lambda: based.baseconv_prefill(g, x, h, bias)
     elif kind == "la_decode":
         S = torch.randn(256, 16, 273, 64, device=dev)
         z = torch.rand(256, 16, 273, device=dev) + 300.0
@@ -657,9 +678,10 @@ def run_profile(kind, reps):
     print(json.dumps({"profile": kind, "case": PROFILE_CASES[kind], "ms": ts}))
 
 
-def run_sweep(reps):
-    """Extra lines beside the headline: the decode batch sweep (a CUDA graph of 32
-    steps per replay) and the long-prefill workload, each against its roofline."""
+def run_sweep(reps, only=None):
+    """Extra lines beside the headline: the short gated convolution, the decode batch
+    sweep (a CUDA graph of 32 steps per replay) and the long-prefill workload, each
+    against its roofline. only="baseconv" stops after the convolution lines."""
     import torch
 
     import linear_attention_sequence_causal_b200 as based
@@ -689,6 +711,40 @@ def run_sweep(reps):
         b.record(stream)
         torch.cuda.synchronize(dev)
         return a.elapsed_time(b) / (reps * n_inner)
+
+    # short gated convolution (BaseConv) at the 360M model width d=1024, K=4. The graph
+    # runs three input sets in turn, so each launch reads inputs evicted from the
+    # 126 MB L2 by the two launches before it (3 x 100 MB).
+    Bc, Nc, dc, Kc = 8, 2048, 1024, 4
+    cs = [synthetic.conv_inputs(Bc, Nc, dc, Kc, "bf16", seed=s) for s in range(3)]
+    hc, bc = cs[0].h.to(dev), cs[0].bias.to(dev)
+    bufs = [(c.u_gate.to(dev), c.u_conv.to(dev), torch.empty(Bc, Nc, dc, dtype=torch.bfloat16, device=dev),
+             torch.empty(Bc, Kc - 1, dc, dtype=torch.bfloat16, device=dev)) for c in cs]
+    del cs
+
+    def conv_sets():
+        for g, x, y, st in bufs:
+            based.baseconv_prefill(g, x, hc, bc, state=st, y=y)
+
+    ms = timed(conv_sets, 1) / len(bufs)
+    flops, byts = baseconv_prefill_work(Bc, Nc, dc, Kc)
+    print(json.dumps({"sweep": "baseconv_prefill", "shape": f"B={Bc} N={Nc} d={dc} K={Kc}", "us": ms * 1e3,
+                      "tokens_per_s": Bc * Nc / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                      "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                      "l2": "3 input sets rotated"}), flush=True)
+    del bufs
+    for batch in (64, 128, 256):
+        c = synthetic.conv_inputs(batch, Kc, dc, Kc, "bf16", seed=batch)
+        g, x = c.u_gate[:, 0].contiguous().to(dev), c.u_conv[:, 0].contiguous().to(dev)
+        st = c.u_conv[:, 1:].contiguous().to(dev)
+        y = torch.empty_like(g)
+        ms = timed(lambda: based.baseconv_decode(st, g, x, hc, bc, y=y), 32)
+        _, byts = baseconv_decode_work(batch, dc, Kc)
+        print(json.dumps({"sweep": "baseconv_decode", "batch": batch, "us_per_step": ms * 1e3,
+                          "tokens_per_s": batch / (ms / 1e3), "GB_s": byts / (ms / 1e3) / 1e9,
+                          "hbm_frac": byts / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}), flush=True)
+    if only == "baseconv":
+        return
 
     H, df, dv, D = 16, 16, 64, _feature_dim(16)
     for batch in (1, 16, 64, 128, 256):
@@ -830,13 +886,14 @@ def main(argv=None):
     p.add_argument("--preroll-s", type=float, default=1.0, help="loaded seconds before the timed region")
     p.add_argument("--profile", choices=sorted(PROFILE_CASES), help="run one kernel on its ncu capture case")
     p.add_argument("--profile-reps", type=int, default=3)
-    p.add_argument("--sweep", action="store_true", help="decode batch sweep and long-prefill lines")
+    p.add_argument("--sweep", nargs="?", const="all", choices=("all", "baseconv"),
+                   help="decode batch sweep and long-prefill lines (baseconv: the convolution lines only)")
     args = p.parse_args(argv)
     if args.profile:
         run_profile(args.profile, args.profile_reps)
         return
     if args.sweep:
-        run_sweep(max(3, min(args.steps, 20)))
+        run_sweep(max(3, min(args.steps, 20)), only=args.sweep)
         return
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

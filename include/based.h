@@ -319,6 +319,47 @@ BASED_API based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t 
                                 based_dtype_t dtype, cudaStream_t stream);
 
 /*
+ * based_baseconv_prefill -- the sequence-mixing core of a short gated
+ * convolution (BaseConv) layer over N tokens. BASED §4 "The BASED Architecture"
+ * (Additional mixers) and App. C "Extended Architecture Details" (Convolution):
+ * a short convolution with a SiLU, combined with the projected input by an
+ * elementwise product. The layer's input and output projections are per-token
+ * affine maps that the caller applies; this call takes the two projected
+ * streams u_gate and u_conv and computes, per sequence, channel and token t,
+ *     c_t = bias + sum_{j=0}^{K-1} h[:, j] * u_conv[t - (K-1) + j]
+ *           (causal and depthwise; u_conv is zero before token 0, so tap
+ *            K-1 meets token t itself)
+ *     y_t = u_gate[t] * SiLU(c_t),   SiLU(x) = x / (1 + exp(-x)).
+ *
+ *   u_gate, u_conv, y  [B, N, d] dtype, channels innermost; 16-byte aligned.
+ *                      y must not overlap u_conv or state.
+ *   h      [d, K] fp32 filter taps, 16-byte aligned, read only.
+ *   bias   [d] fp32, 16-byte aligned, or NULL for none.
+ *   state  [B, K-1, d] dtype, or NULL: written with u_conv of tokens
+ *          N-K+1 .. N-1, oldest first, zeros for positions before token 0
+ *          (the input of based_baseconv_decode). Unused when K = 1.
+ *   B, N >= 1;  d a multiple of 4;  1 <= K <= 8 (else BASED_ERR_UNSUPPORTED).
+ * Arithmetic in fp32; y rounded to the dtype. No workspace, no waits.
+ */
+BASED_API based_status_t based_baseconv_prefill(const void* u_gate, const void* u_conv, const float* h,
+                                      const float* bias, void* y, void* state,
+                                      int B, int N, int d, int K,
+                                      based_dtype_t dtype, cudaStream_t stream);
+
+/*
+ * based_baseconv_decode -- one generated token per sequence through the same
+ * filter: c = bias + sum_{j<K-1} h[:, j] * state[j] + h[:, K-1] * u_conv,
+ * y = u_gate * SiLU(c); then the state drops its oldest row and appends u_conv.
+ *
+ *   state          [B, K-1, d] dtype, read and written in place (may be NULL when K = 1)
+ *   u_gate, u_conv, y  [B, d] dtype
+ *   h, bias, d, K  as for based_baseconv_prefill
+ */
+BASED_API based_status_t based_baseconv_decode(void* state, const void* u_gate, const void* u_conv,
+                                     const float* h, const float* bias, void* y,
+                                     int B, int d, int K, based_dtype_t dtype, cudaStream_t stream);
+
+/*
  * based_get_last_error -- synchronises `stream`, then reports and clears the
  * device status word of the current device: BASED_ERR_TIMEOUT if a bounded
  * wait in a kernel expired since the last call, BASED_ERR_CUDA if the stream

@@ -1,4 +1,5 @@
-"""BASED hot path on B200: causal Taylor linear attention + sliding-window attention.
+"""BASED hot path on B200: causal Taylor linear attention + sliding-window attention,
+plus the short gated convolution (BaseConv) mixer.
 
 The computation lives in libbased.so (hand-written sm_100a CUDA kernels behind
 the C ABI of include/based.h); this package is its ctypes binding. Importing it
@@ -23,6 +24,8 @@ from .binding import (  # noqa: F401
     library_path,
     status_string,
     swa_decode,
+    baseconv_prefill,
+    baseconv_decode,
     swa_prefill,
 )
 

@@ -36,6 +36,8 @@ SYMBOLS = (
     "based_la_backward",
     "based_swa_prefill",
     "based_swa_decode",
+    "based_baseconv_prefill",
+    "based_baseconv_decode",
     "based_get_last_error",
     "based_status_string",
     "based_version",
@@ -79,6 +81,10 @@ def _declare(lib):
     lib.based_swa_prefill.restype = i
     lib.based_swa_decode.argtypes = [vp, vp, ctypes.c_int64, vp, vp, vp, vp, i, i, i, i, f, i, vp]
     lib.based_swa_decode.restype = i
+    lib.based_baseconv_prefill.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, vp]
+    lib.based_baseconv_prefill.restype = i
+    lib.based_baseconv_decode.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, vp]
+    lib.based_baseconv_decode.restype = i
     lib.based_get_last_error.argtypes = [vp]
     lib.based_get_last_error.restype = i
     lib.based_status_string.argtypes = [i]
@@ -346,6 +352,66 @@ def swa_decode(k_cache, v_cache, t: int, q, k, v, w: int = 64, scale: Optional[f
         st = lib().based_swa_decode(_ptr(k_cache), _ptr(v_cache), int(t), _ptr(q), _ptr(k), _ptr(v),
                                     _ptr(y), B, H, d, w, scale, dt, _stream(dev))
     _check(st, "based_swa_decode")
+    return y
+
+
+def _conv_filter(h, bias, d: int):
+    if h.dtype != torch.float32 or not h.is_cuda or not h.is_contiguous() or h.dim() != 2 or h.shape[0] != d:
+        raise BasedError(ERR_INVALID_ARG, "h must be a contiguous CUDA float32 tensor [d, K]")
+    if bias is not None and (bias.dtype != torch.float32 or not bias.is_cuda or not bias.is_contiguous()
+                             or tuple(bias.shape) != (d,)):
+        raise BasedError(ERR_INVALID_ARG, "bias must be a contiguous CUDA float32 tensor [d]")
+    return int(h.shape[1])
+
+
+def baseconv_prefill(u_gate, u_conv, h, bias=None, state=True, y=None):
+    """Short gated convolution over [B, N, d] streams: y = u_gate * SiLU(bias + causal h * u_conv).
+
+    h [d, K] float32 (tap K-1 meets the current token); bias [d] float32 or None.
+    Returns (y, state): state [B, K-1, d] holds u_conv of the last K-1 tokens
+    (zeros before token 0); `state` may be False (not written) or a tensor to write.
+    """
+    dt = _dtype_code(u_gate, u_conv)
+    B, N, d = u_gate.shape
+    if tuple(u_conv.shape) != (B, N, d):
+        raise BasedError(ERR_INVALID_ARG, "u_gate and u_conv must have one shape [B, N, d]")
+    K = _conv_filter(h, bias, d)
+    dev = u_gate.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(u_gate)
+        if isinstance(state, torch.Tensor):
+            _dtype_code(state, u_gate)
+            if tuple(state.shape) != (B, max(K - 1, 0), d):
+                raise BasedError(ERR_INVALID_ARG, "state must be [B, K-1, d]")
+            st_t = state
+        else:
+            st_t = torch.empty((B, max(K - 1, 0), d), dtype=u_gate.dtype, device=dev) if state else None
+        st = lib().based_baseconv_prefill(_ptr(u_gate), _ptr(u_conv), _ptr(h), _ptr(bias), _ptr(y),
+                                          _ptr(st_t) if (st_t is not None and K > 1) else None,
+                                          B, N, d, K, dt, _stream(dev))
+    _check(st, "based_baseconv_prefill")
+    return y, st_t
+
+
+def baseconv_decode(state, u_gate, u_conv, h, bias=None, y=None) -> torch.Tensor:
+    """One token per sequence through the filter; state [B, K-1, d] is updated in place."""
+    dt = _dtype_code(u_gate, u_conv)
+    B, d = u_gate.shape
+    K = _conv_filter(h, bias, d)
+    if K > 1:
+        if state is None:
+            raise BasedError(ERR_INVALID_ARG, "a filter of K > 1 taps needs its state [B, K-1, d]")
+        _dtype_code(state, u_gate)
+        if tuple(state.shape) != (B, K - 1, d):
+            raise BasedError(ERR_INVALID_ARG, "state must be [B, K-1, d]")
+    dev = u_gate.device
+    with torch.cuda.device(dev):
+        if y is None:
+            y = torch.empty_like(u_gate)
+        st = lib().based_baseconv_decode(_ptr(state) if K > 1 else None, _ptr(u_gate), _ptr(u_conv), _ptr(h),
+                                         _ptr(bias), _ptr(y), B, d, K, dt, _stream(dev))
+    _check(st, "based_baseconv_decode")
     return y
 
 

@@ -331,6 +331,38 @@ based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t, const v
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
+based_status_t based_baseconv_prefill(const void* u_gate, const void* u_conv, const float* h,
+                                      const float* bias, void* y, void* state, int B, int N, int d, int K,
+                                      based_dtype_t dtype, cudaStream_t stream) {
+    if (!ok_ptr(u_gate) || !ok_ptr(u_conv) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
+    if (!ok_ptr(h) || (bias != nullptr && !aligned16(bias))) return BASED_ERR_INVALID_ARG;
+    if (state != nullptr && !aligned16(state)) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || N <= 0 || d <= 0 || K <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (d % 4 != 0 || K > based::kMaxConvTaps || (long long)B * (d / 4) > (1LL << 30))
+        return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const int sms = num_sms(dev);
+    if (sms <= 0) return BASED_ERR_CUDA;
+    const cudaError_t e = based::launch_baseconv_prefill(u_gate, u_conv, h, bias, y, state, B, N, d, K,
+                                                         dtype == BASED_BF16, sms, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
+based_status_t based_baseconv_decode(void* state, const void* u_gate, const void* u_conv, const float* h,
+                                     const float* bias, void* y, int B, int d, int K, based_dtype_t dtype,
+                                     cudaStream_t stream) {
+    if (!ok_ptr(u_gate) || !ok_ptr(u_conv) || !ok_ptr(y)) return BASED_ERR_INVALID_ARG;
+    if (!ok_ptr(h) || (bias != nullptr && !aligned16(bias))) return BASED_ERR_INVALID_ARG;
+    if (K > 1 && !ok_ptr(state)) return BASED_ERR_INVALID_ARG;
+    if (B <= 0 || d <= 0 || K <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
+    if (d % 4 != 0 || K > based::kMaxConvTaps || (long long)B * (d / 4) > (1LL << 30))
+        return BASED_ERR_UNSUPPORTED;
+    const cudaError_t e = based::launch_baseconv_decode(state, u_gate, u_conv, h, bias, y, B, d, K,
+                                                        dtype == BASED_BF16, stream);
+    return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
+}
+
 based_status_t based_get_last_error(cudaStream_t stream) {
     if (cudaStreamSynchronize(stream) != cudaSuccess) return BASED_ERR_CUDA;
     int dev;

@@ -1,0 +1,326 @@
+// Short gated convolution (BaseConv) mixing core: causal depthwise K-tap filter,
+// SiLU on the filtered branch, Hadamard gate.
+//
+// BASED ("Simple linear attention language models balance the recall-throughput
+// tradeoff") §4 "The BASED Architecture" (Additional mixers) and App. C
+// "Extended Architecture Details" (Convolution): a short convolution and a SiLU
+// combined with the projected input by an elementwise product. For the two
+// projected streams u_gate, u_conv [B, N, d] (channels innermost):
+//     c_t = bias + sum_{j<K} h[:, j] * u_conv[t - (K-1) + j]   (zero before token 0)
+//     y_t = u_gate[t] * SiLU(c_t)
+// The work is a few FMAs per element against 3 element transfers, so both
+// kernels are bound by HBM: the design goal is to move each element once, in
+// 16-byte coalesced pieces, with enough loads in flight to cover DRAM latency.
+//
+// Prefill: one thread owns 4 consecutive channels of one sequence over a run of
+// `seg` tokens, `seg` chosen so that the grid fills the resident thread slots
+// once. It keeps the last K-1 values of u_conv in registers (a sliding
+// window), so every u_conv element is read once plus a K-1 token halo per run
+// (served by L2: the neighbouring run read it from DRAM). Consecutive threads
+// own consecutive channel groups, so a warp reads 256 contiguous bytes of a
+// bf16 token row per stream. Tokens are processed 4 at a time with all 8 loads
+// issued before the arithmetic. The run that ends the sequence writes the
+// generation state (the last K-1 values of u_conv, oldest first).
+//
+// Decode: one thread per (sequence, 4 channels): read the K-1 state rows and
+// the new token, write y and the shifted state in place. No thread reads what
+// another writes.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "kernels.h"
+
+namespace based {
+namespace {
+
+constexpr int kVec = 4;        // channels per thread: 8 bytes of bf16, 16 of fp32
+constexpr int kUnroll = 4;     // tokens whose loads are issued together
+constexpr int kThreads = 128;        // prefill block
+constexpr int kDecodeThreads = 64;   // decode block: small batches still spread over many SMs
+
+template <bool BF16>
+__device__ __forceinline__ void unpack(uint2 r, float (&x)[kVec]) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+}
+
+// Read-only inputs: through the non-coherent path.
+template <bool BF16>
+__device__ __forceinline__ void load4(const void* base, size_t off, float (&x)[kVec]) {
+    if constexpr (BF16) {
+        unpack<BF16>(__ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + off)), x);
+    } else {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + off));
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    }
+}
+
+// Plain load, for the decode state that the same kernel rewrites.
+template <bool BF16>
+__device__ __forceinline__ void load4_rw(const void* base, size_t off, float (&x)[kVec]) {
+    if constexpr (BF16) {
+        unpack<BF16>(*reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + off), x);
+    } else {
+        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void store4(void* base, size_t off, const float (&x)[kVec]) {
+    if constexpr (BF16) {
+        uint2 r;
+        *reinterpret_cast<__nv_bfloat162*>(&r.x) = __floats2bfloat162_rn(x[0], x[1]);
+        *reinterpret_cast<__nv_bfloat162*>(&r.y) = __floats2bfloat162_rn(x[2], x[3]);
+        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + off) = r;
+    } else {
+        *reinterpret_cast<float4*>(static_cast<float*>(base) + off) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+}
+
+// x * sigmoid(x). For x < -87, exp(-x) exceeds 2^126 and the fast divide returns 0,
+// the limit of the function there.
+__device__ __forceinline__ float silu(float c) { return __fdividef(c, 1.0f + __expf(-c)); }
+
+// The K taps of 4 consecutive channels are 4K consecutive floats of h [d, K],
+// 16-byte aligned because the first channel is a multiple of 4: K float4 loads.
+template <int K>
+__device__ __forceinline__ void load_filter(const float* __restrict__ h, const float* __restrict__ bias,
+                                            int c0, float (&hr)[K][kVec], float (&br)[kVec]) {
+    const float4* hp = reinterpret_cast<const float4*>(h + (size_t)c0 * K);
+    float flat[kVec * K];
+#pragma unroll
+    for (int i = 0; i < K; ++i) {
+        const float4 f = __ldg(hp + i);
+        flat[4 * i] = f.x; flat[4 * i + 1] = f.y; flat[4 * i + 2] = f.z; flat[4 * i + 3] = f.w;
+    }
+#pragma unroll
+    for (int e = 0; e < kVec; ++e)
+#pragma unroll
+        for (int j = 0; j < K; ++j) hr[j][e] = flat[e * K + j];
+    if (bias != nullptr) {
+        const float4 b = __ldg(reinterpret_cast<const float4*>(bias + c0));
+        br[0] = b.x; br[1] = b.y; br[2] = b.z; br[3] = b.w;
+    } else {
+#pragma unroll
+        for (int e = 0; e < kVec; ++e) br[e] = 0.0f;
+    }
+}
+
+// Resident blocks per SM asked of the compiler: the most that keeps the filter,
+// the window and 4 tokens of loads in registers without spilling (24 warps per
+// SM at K = 3 or 4).
+constexpr int prefill_min_blocks(int K, bool bf16) {
+    return K <= 2 ? 8 : K <= 3 ? 6 : K == 4 ? (bf16 ? 6 : 5) : K <= 6 ? 4 : 3;
+}
+
+template <int K, bool BF16>
+__global__ void __launch_bounds__(kThreads, prefill_min_blocks(K, BF16))
+baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ conv,
+                        const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
+                        void* __restrict__ state, int N, int d, int seg, int nseg, int groups, int items) {
+    const int item = blockIdx.x * kThreads + threadIdx.x;
+    if (item >= items) return;
+    const int cg = item % groups;
+    const int rest = item / groups;
+    const int s = rest % nseg;
+    const int b = rest / nseg;
+    const int c0 = cg * kVec;
+    const int t0 = s * seg;
+    const int t1 = min(N, t0 + seg);
+    const size_t row0 = (size_t)b * N;
+
+    float hr[K][kVec], br[kVec];
+    load_filter<K>(h, bias, c0, hr, br);
+
+    // win[j] holds u_conv of token t - (K-1) + j for the token t about to be processed.
+    float win[K > 1 ? K - 1 : 1][kVec];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) {
+        const int t = t0 - (K - 1) + j;
+        if (t >= 0) {
+            load4<BF16>(conv, (row0 + t) * d + c0, win[j]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < kVec; ++e) win[j][e] = 0.0f;
+        }
+    }
+
+    for (int t = t0; t < t1; t += kUnroll) {
+        float g[kUnroll][kVec], x[kUnroll][kVec];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (t + u < t1) {
+                const size_t off = (row0 + t + u) * d + c0;
+                load4<BF16>(gate, off, g[u]);
+                load4<BF16>(conv, off, x[u]);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            if (t + u < t1) {
+                float out[kVec];
+#pragma unroll
+                for (int e = 0; e < kVec; ++e) {
+                    float c = br[e];
+#pragma unroll
+                    for (int j = 0; j < K - 1; ++j) c = fmaf(hr[j][e], win[j][e], c);
+                    c = fmaf(hr[K - 1][e], x[u][e], c);
+                    out[e] = g[u][e] * silu(c);
+                }
+                store4<BF16>(y, (row0 + t + u) * d + c0, out);
+#pragma unroll
+                for (int j = 0; j + 1 < K - 1; ++j)
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) win[j][e] = win[j + 1][e];
+                if constexpr (K > 1) {
+#pragma unroll
+                    for (int e = 0; e < kVec; ++e) win[K - 2][e] = x[u][e];
+                }
+            }
+        }
+    }
+
+    // The window now holds tokens N-K+1 .. N-1 (zeros before token 0).
+    if (state != nullptr && t1 == N) {
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) store4<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, win[j]);
+    }
+}
+
+template <int K, bool BF16>
+__global__ void __launch_bounds__(kDecodeThreads)
+baseconv_decode_kernel(void* __restrict__ state, const void* __restrict__ gate, const void* __restrict__ conv,
+                       const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
+                       int d, int groups, int items) {
+    const int item = blockIdx.x * kDecodeThreads + threadIdx.x;
+    if (item >= items) return;
+    const int cg = item % groups;
+    const int b = item / groups;
+    const int c0 = cg * kVec;
+
+    float hr[K][kVec], br[kVec];
+    load_filter<K>(h, bias, c0, hr, br);
+
+    float st[K > 1 ? K - 1 : 1][kVec];
+#pragma unroll
+    for (int j = 0; j < K - 1; ++j) load4_rw<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j]);
+    float g[kVec], x[kVec];
+    load4<BF16>(gate, (size_t)b * d + c0, g);
+    load4<BF16>(conv, (size_t)b * d + c0, x);
+
+    float out[kVec];
+#pragma unroll
+    for (int e = 0; e < kVec; ++e) {
+        float c = br[e];
+#pragma unroll
+        for (int j = 0; j < K - 1; ++j) c = fmaf(hr[j][e], st[j][e], c);
+        c = fmaf(hr[K - 1][e], x[e], c);
+        out[e] = g[e] * silu(c);
+    }
+    store4<BF16>(y, (size_t)b * d + c0, out);
+    if constexpr (K > 1) {
+#pragma unroll
+        for (int j = 0; j + 1 < K - 1; ++j) store4<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j + 1]);
+        store4<BF16>(state, ((size_t)b * (K - 1) + (K - 2)) * d + c0, x);
+    }
+}
+
+// Token run per thread: split each (sequence, channel group) column into as
+// many runs as the resident thread slots allow, so that the grid is one wave
+// of equal runs (no tail) with the fewest halo re-reads.
+int prefill_segment(int B, int N, int groups, long long slots) {
+    const long long columns = (long long)B * groups;
+    const long long runs = std::max(1LL, std::min<long long>(N, slots / columns));
+    return (int)((N + runs - 1) / runs);
+}
+
+template <int K, bool BF16>
+cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
+                      void* y, void* state, int B, int N, int d, int num_sms) {
+    static int occupancy = 0;   // resident blocks per SM; a property of the compiled kernel
+    if (occupancy == 0) {
+        int o = 0;
+        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+            &o, baseconv_prefill_kernel<K, BF16>, kThreads, 0);
+        if (e != cudaSuccess) return e;
+        occupancy = std::max(1, o);
+    }
+    const int groups = d / kVec;
+    const int seg = prefill_segment(B, N, groups, (long long)num_sms * occupancy * kThreads);
+    const int nseg = (N + seg - 1) / seg;
+    const long long items = (long long)B * nseg * groups;
+    if (items > 0x7fffffffLL - kThreads) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)((items + kThreads - 1) / kThreads));
+    baseconv_prefill_kernel<K, BF16><<<grid, kThreads, 0, st>>>(gate, conv, h, bias, y, state, N, d, seg, nseg,
+                                                                 groups, (int)items);
+    return cudaGetLastError();
+}
+
+template <int K, bool BF16>
+cudaError_t decode_k(cudaStream_t st, void* state, const void* gate, const void* conv, const float* h,
+                     const float* bias, void* y, int B, int d) {
+    const int groups = d / kVec;
+    const long long items = (long long)B * groups;
+    if (items > 0x7fffffffLL - kDecodeThreads) return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)((items + kDecodeThreads - 1) / kDecodeThreads));
+    baseconv_decode_kernel<K, BF16><<<grid, kDecodeThreads, 0, st>>>(state, gate, conv, h, bias, y, d, groups,
+                                                                      (int)items);
+    return cudaGetLastError();
+}
+
+template <bool BF16>
+cudaError_t prefill_any(int K, cudaStream_t st, const void* gate, const void* conv, const float* h,
+                        const float* bias, void* y, void* state, int B, int N, int d, int num_sms) {
+    switch (K) {
+        case 1: return prefill_k<1, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 2: return prefill_k<2, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 3: return prefill_k<3, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 4: return prefill_k<4, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 5: return prefill_k<5, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 6: return prefill_k<6, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 7: return prefill_k<7, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 8: return prefill_k<8, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+template <bool BF16>
+cudaError_t decode_any(int K, cudaStream_t st, void* state, const void* gate, const void* conv, const float* h,
+                       const float* bias, void* y, int B, int d) {
+    switch (K) {
+        case 1: return decode_k<1, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 2: return decode_k<2, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 3: return decode_k<3, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 4: return decode_k<4, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 5: return decode_k<5, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 6: return decode_k<6, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 7: return decode_k<7, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 8: return decode_k<8, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const float* h, const float* bias,
+                                    void* y, void* state, int B, int N, int d, int K, bool bf16, int num_sms,
+                                    cudaStream_t stream) {
+    if (B <= 0 || N <= 0 || d <= 0 || d % kVec != 0 || K < 1 || K > kMaxConvTaps || num_sms <= 0)
+        return cudaErrorInvalidValue;
+    return bf16 ? prefill_any<true>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms)
+                : prefill_any<false>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms);
+}
+
+cudaError_t launch_baseconv_decode(void* state, const void* gate, const void* conv, const float* h,
+                                   const float* bias, void* y, int B, int d, int K, bool bf16,
+                                   cudaStream_t stream) {
+    if (B <= 0 || d <= 0 || d % kVec != 0 || K < 1 || K > kMaxConvTaps) return cudaErrorInvalidValue;
+    return bf16 ? decode_any<true>(K, stream, state, gate, conv, h, bias, y, B, d)
+                : decode_any<false>(K, stream, state, gate, conv, h, bias, y, B, d);
+}
+
+}  // namespace based

@@ -74,4 +74,13 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                               const void* k, const void* v, void* y, int B, int H, int d, int w,
                               float scale, bool bf16, cudaStream_t stream);
 
+// Short gated convolution: filter taps K in [1, kMaxConvTaps], d a multiple of 4.
+constexpr int kMaxConvTaps = 8;
+cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const float* h, const float* bias,
+                                    void* y, void* state, int B, int N, int d, int K, bool bf16, int num_sms,
+                                    cudaStream_t stream);
+cudaError_t launch_baseconv_decode(void* state, const void* gate, const void* conv, const float* h,
+                                   const float* bias, void* y, int B, int d, int K, bool bf16,
+                                   cudaStream_t stream);
+
 }  // namespace based

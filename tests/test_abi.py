@@ -148,6 +148,40 @@ def test_decay_entries_reject_bad_arguments(lib):
     assert dd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 24, 64, 1, 0, None) == binding.ERR_UNSUPPORTED
 
 
+def test_baseconv_entries_reject_bad_arguments(lib):
+    pf = lib.based_baseconv_prefill
+    names = ["g", "x", "h", "bias", "y", "state", "B", "N", "d", "K", "dt", "st"]
+    ok = [FAKE, FAKE, FAKE, None, FAKE, FAKE, 2, 100, 64, 4, 1, None]
+
+    def call(f, okv, nm, **kw):
+        a = list(okv)
+        for key, val in kw.items():
+            a[nm.index(key)] = val
+        return f(*a)
+
+    p = lambda **kw: call(pf, ok, names, **kw)
+    assert p(g=None) == binding.ERR_INVALID_ARG
+    assert p(x=MISALIGNED) == binding.ERR_INVALID_ARG
+    assert p(h=None) == binding.ERR_INVALID_ARG
+    assert p(h=ctypes.c_void_p((1 << 20) + 4)) == binding.ERR_INVALID_ARG     # taps read 16 bytes at a time
+    assert p(bias=ctypes.c_void_p((1 << 20) + 4)) == binding.ERR_INVALID_ARG
+    assert p(state=MISALIGNED) == binding.ERR_INVALID_ARG
+    assert p(N=0) == binding.ERR_INVALID_ARG
+    assert p(K=0) == binding.ERR_INVALID_ARG
+    assert p(dt=5) == binding.ERR_INVALID_ARG
+    assert p(d=62) == binding.ERR_UNSUPPORTED                               # channels in groups of 4
+    assert p(K=9) == binding.ERR_UNSUPPORTED
+    dn = ["state", "g", "x", "h", "bias", "y", "B", "d", "K", "dt", "st"]
+    dok = [FAKE, FAKE, FAKE, FAKE, None, FAKE, 2, 64, 4, 0, None]
+    q = lambda **kw: call(lib.based_baseconv_decode, dok, dn, **kw)
+    assert q(state=None) == binding.ERR_INVALID_ARG                         # K > 1 needs a state
+    assert q(y=MISALIGNED) == binding.ERR_INVALID_ARG
+    assert q(B=0) == binding.ERR_INVALID_ARG
+    assert q(d=10) == binding.ERR_UNSUPPORTED
+    assert q(K=9) == binding.ERR_UNSUPPORTED
+    assert q(K=1, d=10, state=None) == binding.ERR_UNSUPPORTED               # K = 1 needs no state
+
+
 def test_la_backward_workspace_query(lib):
     # g (bf16) and c (fp32) per token, rows padded to a multiple of 128.
     assert lib.based_la_backward_workspace(2, 3, 300, 16, 64, 1) == 2 * 3 * 384 * (64 * 2 + 4)
