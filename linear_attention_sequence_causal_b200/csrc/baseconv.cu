@@ -18,9 +18,11 @@
 // window), so every u_conv element is read once plus a K-1 token halo per run
 // (served by L2: the neighbouring run read it from DRAM). Consecutive threads
 // own consecutive channel groups, so a warp reads 256 contiguous bytes of a
-// bf16 token row per stream. Tokens are processed 4 at a time with all 8 loads
-// issued before the arithmetic. The run that ends the sequence writes the
-// generation state (the last K-1 values of u_conv, oldest first).
+// bf16 token row per stream. The streams reach shared memory by cp.async in
+// stages of 4 tokens, 3 stages in flight while the thread computes one, so
+// DRAM latency is covered without holding the data in registers. The run that
+// ends the sequence writes the generation state (the last K-1 values of
+// u_conv, oldest first).
 //
 // Decode: one thread per (sequence, 4 channels): read the K-1 state rows and
 // the new token, write y and the shifted state in place. No thread reads what
@@ -81,6 +83,35 @@ __device__ __forceinline__ void store4(void* base, size_t off, const float (&x)[
     }
 }
 
+// One thread's kVec channels of one token: 8 bytes of bf16, 16 of fp32.
+template <bool BF16> struct ChunkT { using type = uint2; };
+template <> struct ChunkT<false> { using type = uint4; };
+template <bool BF16> using Chunk = typename ChunkT<BF16>::type;
+// Ring depth: 4 stages of bf16 (32 KB per block), 2 of fp32 (32 KB per block).
+template <bool BF16> constexpr int kStages = BF16 ? 4 : 2;
+
+template <bool BF16>
+__device__ __forceinline__ void copy_async(Chunk<BF16>* dst, const void* base, size_t off) {
+    const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+    if constexpr (BF16) {
+        const void* src = static_cast<const __nv_bfloat16*>(base) + off;
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(src) : "memory");
+    } else {
+        const void* src = static_cast<const float*>(base) + off;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(src) : "memory");
+    }
+}
+
+template <bool BF16>
+__device__ __forceinline__ void unpack_chunk(const Chunk<BF16>& r, float (&x)[kVec]) {
+    if constexpr (BF16) {
+        unpack<BF16>(r, x);
+    } else {
+        x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
+        x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
+    }
+}
+
 // x * sigmoid(x). For x < -87, exp(-x) exceeds 2^126 and the fast divide returns 0,
 // the limit of the function there.
 __device__ __forceinline__ float silu(float c) { return __fdividef(c, 1.0f + __expf(-c)); }
@@ -133,6 +164,31 @@ baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ 
     const int t1 = min(N, t0 + seg);
     const size_t row0 = (size_t)b * N;
 
+    // Async-copy ring: stage q holds tokens t0 + q*kUnroll .. +kUnroll-1 of both
+    // streams in slot q % kStages. Each thread copies and later reads only its
+    // own entries (column threadIdx.x), so the only wait is cp.async.wait_group
+    // on its own copies; kStages-1 stages stay in flight while one is computed.
+    __shared__ Chunk<BF16> ring[kStages<BF16>][kUnroll][2][kThreads];
+    const int tid = threadIdx.x;
+    const int nstage = (t1 - t0 + kUnroll - 1) / kUnroll;
+    auto issue = [&](int q) {
+        if (q < nstage) {
+            const int slot = q % kStages<BF16>;
+#pragma unroll
+            for (int u = 0; u < kUnroll; ++u) {
+                const int t = t0 + q * kUnroll + u;
+                if (t < t1) {
+                    const size_t off = (row0 + t) * d + c0;
+                    copy_async<BF16>(&ring[slot][u][0][tid], gate, off);
+                    copy_async<BF16>(&ring[slot][u][1][tid], conv, off);
+                }
+            }
+        }
+        asm volatile("cp.async.commit_group;\n" ::: "memory");
+    };
+#pragma unroll
+    for (int q = 0; q < kStages<BF16> - 1; ++q) issue(q);
+
     float hr[K][kVec], br[kVec];
     load_filter<K>(h, bias, c0, hr, br);
 
@@ -149,36 +205,33 @@ baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ 
         }
     }
 
-    for (int t = t0; t < t1; t += kUnroll) {
-        float g[kUnroll][kVec], x[kUnroll][kVec];
+    for (int q = 0; q < nstage; ++q) {
+        issue(q + kStages<BF16> - 1);
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(kStages<BF16> - 1) : "memory");
+        const int slot = q % kStages<BF16>;
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
-                const size_t off = (row0 + t + u) * d + c0;
-                load4<BF16>(gate, off, g[u]);
-                load4<BF16>(conv, off, x[u]);
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kUnroll; ++u) {
-            if (t + u < t1) {
-                float out[kVec];
+            const int t = t0 + q * kUnroll + u;
+            if (t < t1) {
+                float g[kVec], x[kVec], out[kVec];
+                unpack_chunk<BF16>(ring[slot][u][0][tid], g);
+                unpack_chunk<BF16>(ring[slot][u][1][tid], x);
 #pragma unroll
                 for (int e = 0; e < kVec; ++e) {
                     float c = br[e];
 #pragma unroll
                     for (int j = 0; j < K - 1; ++j) c = fmaf(hr[j][e], win[j][e], c);
-                    c = fmaf(hr[K - 1][e], x[u][e], c);
-                    out[e] = g[u][e] * silu(c);
+                    c = fmaf(hr[K - 1][e], x[e], c);
+                    out[e] = g[e] * silu(c);
                 }
-                store4<BF16>(y, (row0 + t + u) * d + c0, out);
+                store4<BF16>(y, (row0 + t) * d + c0, out);
 #pragma unroll
                 for (int j = 0; j + 1 < K - 1; ++j)
 #pragma unroll
                     for (int e = 0; e < kVec; ++e) win[j][e] = win[j + 1][e];
                 if constexpr (K > 1) {
 #pragma unroll
-                    for (int e = 0; e < kVec; ++e) win[K - 2][e] = x[u][e];
+                    for (int e = 0; e < kVec; ++e) win[K - 2][e] = x[e];
                 }
             }
         }
@@ -243,9 +296,13 @@ cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const
                       void* y, void* state, int B, int N, int d, int num_sms) {
     static int occupancy = 0;   // resident blocks per SM; a property of the compiled kernel
     if (occupancy == 0) {
+        // the ring lives in shared memory: prefer the largest shared-memory carveout
+        cudaError_t e = cudaFuncSetAttribute(baseconv_prefill_kernel<K, BF16>,
+                                             cudaFuncAttributePreferredSharedMemoryCarveout,
+                                             cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
         int o = 0;
-        const cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
-            &o, baseconv_prefill_kernel<K, BF16>, kThreads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, baseconv_prefill_kernel<K, BF16>, kThreads, 0);
         if (e != cudaSuccess) return e;
         occupancy = std::max(1, o);
     }
