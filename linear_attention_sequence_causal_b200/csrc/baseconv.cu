@@ -12,17 +12,18 @@
 // kernels are bound by HBM: the design goal is to move each element once, in
 // 16-byte coalesced pieces, with enough loads in flight to cover DRAM latency.
 //
-// Prefill: one thread owns 4 consecutive channels of one sequence over a run of
-// `seg` tokens, `seg` chosen so that the grid fills the resident thread slots
-// once. It keeps the last K-1 values of u_conv in registers (a sliding
-// window), so every u_conv element is read once plus a K-1 token halo per run
-// (served by L2: the neighbouring run read it from DRAM). Consecutive threads
-// own consecutive channel groups, so a warp reads 256 contiguous bytes of a
-// bf16 token row per stream. The streams reach shared memory by cp.async in
-// stages of 4 tokens, 3 stages in flight while the thread computes one, so
-// DRAM latency is covered without holding the data in registers. The run that
-// ends the sequence writes the generation state (the last K-1 values of
-// u_conv, oldest first).
+// Prefill: one thread owns V consecutive channels (8 of bf16 when d allows,
+// else 4) of one sequence over a run of `seg` tokens, `seg` chosen so that the
+// grid fills the resident thread slots once. It keeps the last K-1 values of
+// u_conv in registers (a sliding window), so every u_conv element is read once
+// plus a K-1 token halo per run (served by L2: the neighbouring run read it
+// from DRAM). Consecutive threads own consecutive channel groups, so a warp
+// reads 512 contiguous bytes of a token row per stream (256 with 4 bf16
+// channels). The streams reach shared memory by cp.async in stages of 4
+// tokens, 2 or 3 stages in flight while the thread computes one, so DRAM
+// latency is covered without holding the data in registers. The run that ends
+// the sequence writes the generation state (the last K-1 values of u_conv,
+// oldest first).
 //
 // Decode: one thread per (sequence, 4 channels): read the K-1 state rows and
 // the new token, write y and the shifted state in place. No thread reads what
@@ -37,201 +38,217 @@
 namespace based {
 namespace {
 
-constexpr int kVec = 4;        // channels per thread: 8 bytes of bf16, 16 of fp32
-constexpr int kUnroll = 4;     // tokens whose loads are issued together
+constexpr int kUnroll = 4;           // tokens per ring stage
 constexpr int kThreads = 128;        // prefill block
 constexpr int kDecodeThreads = 64;   // decode block: small batches still spread over many SMs
 
-template <bool BF16>
-__device__ __forceinline__ void unpack(uint2 r, float (&x)[kVec]) {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-    x[0] = a.x; x[1] = a.y; x[2] = b.x; x[3] = b.y;
+// V channels of one token of the dtype: 8 bytes (bf16, V = 4) or 16 bytes
+// (bf16, V = 8; fp32, V = 4), moved as one vector.
+template <bool BF16, int V> struct Piece;
+template <> struct Piece<true, 4> { using raw = uint2; };
+template <> struct Piece<true, 8> { using raw = uint4; };
+template <> struct Piece<false, 4> { using raw = uint4; };
+template <bool BF16, int V> using Raw = typename Piece<BF16, V>::raw;
+
+template <bool BF16, int V>
+__device__ __forceinline__ const Raw<BF16, V>* at(const void* base, size_t off) {
+    if constexpr (BF16) return reinterpret_cast<const Raw<BF16, V>*>(static_cast<const __nv_bfloat16*>(base) + off);
+    else return reinterpret_cast<const Raw<BF16, V>*>(static_cast<const float*>(base) + off);
+}
+
+template <bool BF16, int V>
+__device__ __forceinline__ Raw<BF16, V>* at(void* base, size_t off) {
+    if constexpr (BF16) return reinterpret_cast<Raw<BF16, V>*>(static_cast<__nv_bfloat16*>(base) + off);
+    else return reinterpret_cast<Raw<BF16, V>*>(static_cast<float*>(base) + off);
+}
+
+template <bool BF16, int V>
+__device__ __forceinline__ void to_float(const Raw<BF16, V>& r, float (&x)[V]) {
+    if constexpr (BF16) {
+        const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&r);
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) {
+            const float2 f = __bfloat1622float2(p[i]);
+            x[2 * i] = f.x;
+            x[2 * i + 1] = f.y;
+        }
+    } else {
+        const float* p = reinterpret_cast<const float*>(&r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) x[i] = p[i];
+    }
+}
+
+template <bool BF16, int V>
+__device__ __forceinline__ Raw<BF16, V> from_float(const float (&x)[V]) {
+    Raw<BF16, V> r;
+    if constexpr (BF16) {
+        __nv_bfloat162* p = reinterpret_cast<__nv_bfloat162*>(&r);
+#pragma unroll
+        for (int i = 0; i < V / 2; ++i) p[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    } else {
+        float* p = reinterpret_cast<float*>(&r);
+#pragma unroll
+        for (int i = 0; i < V; ++i) p[i] = x[i];
+    }
+    return r;
 }
 
 // Read-only inputs: through the non-coherent path.
-template <bool BF16>
-__device__ __forceinline__ void load4(const void* base, size_t off, float (&x)[kVec]) {
-    if constexpr (BF16) {
-        unpack<BF16>(__ldg(reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + off)), x);
-    } else {
-        const float4 a = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + off));
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    }
+template <bool BF16, int V>
+__device__ __forceinline__ void load_ro(const void* base, size_t off, float (&x)[V]) {
+    to_float<BF16, V>(__ldg(at<BF16, V>(base, off)), x);
 }
 
 // Plain load, for the decode state that the same kernel rewrites.
-template <bool BF16>
-__device__ __forceinline__ void load4_rw(const void* base, size_t off, float (&x)[kVec]) {
-    if constexpr (BF16) {
-        unpack<BF16>(*reinterpret_cast<const uint2*>(static_cast<const __nv_bfloat16*>(base) + off), x);
-    } else {
-        const float4 a = *reinterpret_cast<const float4*>(static_cast<const float*>(base) + off);
-        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
-    }
+template <bool BF16, int V>
+__device__ __forceinline__ void load_rw(const void* base, size_t off, float (&x)[V]) {
+    to_float<BF16, V>(*at<BF16, V>(base, off), x);
 }
 
-template <bool BF16>
-__device__ __forceinline__ void store4(void* base, size_t off, const float (&x)[kVec]) {
-    if constexpr (BF16) {
-        uint2 r;
-        *reinterpret_cast<__nv_bfloat162*>(&r.x) = __floats2bfloat162_rn(x[0], x[1]);
-        *reinterpret_cast<__nv_bfloat162*>(&r.y) = __floats2bfloat162_rn(x[2], x[3]);
-        *reinterpret_cast<uint2*>(static_cast<__nv_bfloat16*>(base) + off) = r;
-    } else {
-        *reinterpret_cast<float4*>(static_cast<float*>(base) + off) = make_float4(x[0], x[1], x[2], x[3]);
-    }
+template <bool BF16, int V>
+__device__ __forceinline__ void store(void* base, size_t off, const float (&x)[V]) {
+    *at<BF16, V>(base, off) = from_float<BF16, V>(x);
 }
 
-// One thread's kVec channels of one token: 8 bytes of bf16, 16 of fp32.
-template <bool BF16> struct ChunkT { using type = uint2; };
-template <> struct ChunkT<false> { using type = uint4; };
-template <bool BF16> using Chunk = typename ChunkT<BF16>::type;
-// Ring depth: 4 stages of bf16 (32 KB per block), 2 of fp32 (32 KB per block).
-template <bool BF16> constexpr int kStages = BF16 ? 4 : 2;
-
-template <bool BF16>
-__device__ __forceinline__ void copy_async(Chunk<BF16>* dst, const void* base, size_t off) {
+template <bool BF16, int V>
+__device__ __forceinline__ void copy_async(Raw<BF16, V>* dst, const void* base, size_t off) {
     const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
-    if constexpr (BF16) {
-        const void* src = static_cast<const __nv_bfloat16*>(base) + off;
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(src) : "memory");
-    } else {
-        const void* src = static_cast<const float*>(base) + off;
+    const void* src = at<BF16, V>(base, off);
+    if constexpr (sizeof(Raw<BF16, V>) == 16)
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(src) : "memory");
-    }
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(s), "l"(src) : "memory");
 }
 
-template <bool BF16>
-__device__ __forceinline__ void unpack_chunk(const Chunk<BF16>& r, float (&x)[kVec]) {
-    if constexpr (BF16) {
-        unpack<BF16>(r, x);
-    } else {
-        x[0] = __uint_as_float(r.x); x[1] = __uint_as_float(r.y);
-        x[2] = __uint_as_float(r.z); x[3] = __uint_as_float(r.w);
-    }
-}
+// Ring depth: 4 stages of 8-byte pieces (32 KB per block), 3 of 16-byte pieces (48 KB).
+template <bool BF16, int V> constexpr int kStages = sizeof(Raw<BF16, V>) == 16 ? 3 : 4;
 
 // x * sigmoid(x). For x < -87, exp(-x) exceeds 2^126 and the fast divide returns 0,
 // the limit of the function there.
 __device__ __forceinline__ float silu(float c) { return __fdividef(c, 1.0f + __expf(-c)); }
 
-// The K taps of 4 consecutive channels are 4K consecutive floats of h [d, K],
-// 16-byte aligned because the first channel is a multiple of 4: K float4 loads.
-template <int K>
+// The K taps of V consecutive channels are VK consecutive floats of h [d, K],
+// 16-byte aligned because the first channel is a multiple of V (4 or 8).
+template <int K, int V>
 __device__ __forceinline__ void load_filter(const float* __restrict__ h, const float* __restrict__ bias,
-                                            int c0, float (&hr)[K][kVec], float (&br)[kVec]) {
+                                            int c0, float (&hr)[K][V], float (&br)[V]) {
     const float4* hp = reinterpret_cast<const float4*>(h + (size_t)c0 * K);
-    float flat[kVec * K];
+    float flat[V * K];
 #pragma unroll
-    for (int i = 0; i < K; ++i) {
+    for (int i = 0; i < V * K / 4; ++i) {
         const float4 f = __ldg(hp + i);
         flat[4 * i] = f.x; flat[4 * i + 1] = f.y; flat[4 * i + 2] = f.z; flat[4 * i + 3] = f.w;
     }
 #pragma unroll
-    for (int e = 0; e < kVec; ++e)
+    for (int e = 0; e < V; ++e)
 #pragma unroll
         for (int j = 0; j < K; ++j) hr[j][e] = flat[e * K + j];
     if (bias != nullptr) {
-        const float4 b = __ldg(reinterpret_cast<const float4*>(bias + c0));
-        br[0] = b.x; br[1] = b.y; br[2] = b.z; br[3] = b.w;
+#pragma unroll
+        for (int i = 0; i < V / 4; ++i) {
+            const float4 b = __ldg(reinterpret_cast<const float4*>(bias + c0) + i);
+            br[4 * i] = b.x; br[4 * i + 1] = b.y; br[4 * i + 2] = b.z; br[4 * i + 3] = b.w;
+        }
     } else {
 #pragma unroll
-        for (int e = 0; e < kVec; ++e) br[e] = 0.0f;
+        for (int e = 0; e < V; ++e) br[e] = 0.0f;
     }
 }
 
-// Resident blocks per SM asked of the compiler: the most that keeps the filter,
-// the window and 4 tokens of loads in registers without spilling (24 warps per
-// SM at K = 3 or 4).
-constexpr int prefill_min_blocks(int K, bool bf16) {
-    return K <= 2 ? 8 : K <= 3 ? 6 : K == 4 ? (bf16 ? 6 : 5) : K <= 6 ? 4 : 3;
+// Resident blocks per SM asked of the compiler: the most that keeps the filter
+// and the window in registers without spilling and that the ring's shared
+// memory allows (6 blocks of 4-channel threads at K = 3 or 4; 4 blocks of
+// 8-channel threads, whose 48 KB rings allow no more).
+constexpr int prefill_min_blocks(int K, bool bf16, int V) {
+    return V == 8 ? 4 : K <= 2 ? 8 : K <= 3 ? 6 : K == 4 ? (bf16 ? 6 : 5) : K <= 6 ? 4 : 3;
 }
 
-template <int K, bool BF16>
-__global__ void __launch_bounds__(kThreads, prefill_min_blocks(K, BF16))
+template <int K, bool BF16, int V>
+__global__ void __launch_bounds__(kThreads, prefill_min_blocks(K, BF16, V))
 baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ conv,
                         const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
                         void* __restrict__ state, int N, int d, int seg, int nseg, int groups, int items) {
+    constexpr int S = kStages<BF16, V>;
     const int item = blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
     const int cg = item % groups;
     const int rest = item / groups;
     const int s = rest % nseg;
     const int b = rest / nseg;
-    const int c0 = cg * kVec;
+    const int c0 = cg * V;
     const int t0 = s * seg;
     const int t1 = min(N, t0 + seg);
     const size_t row0 = (size_t)b * N;
 
     // Async-copy ring: stage q holds tokens t0 + q*kUnroll .. +kUnroll-1 of both
-    // streams in slot q % kStages. Each thread copies and later reads only its
-    // own entries (column threadIdx.x), so the only wait is cp.async.wait_group
-    // on its own copies; kStages-1 stages stay in flight while one is computed.
-    __shared__ Chunk<BF16> ring[kStages<BF16>][kUnroll][2][kThreads];
+    // streams in slot q % S. Each thread copies and later reads only its own
+    // entries (column threadIdx.x), so the only wait is cp.async.wait_group on
+    // its own copies; S-1 stages stay in flight while one is computed.
+    __shared__ Raw<BF16, V> ring[S][kUnroll][2][kThreads];
     const int tid = threadIdx.x;
     const int nstage = (t1 - t0 + kUnroll - 1) / kUnroll;
     auto issue = [&](int q) {
         if (q < nstage) {
-            const int slot = q % kStages<BF16>;
+            const int slot = q % S;
 #pragma unroll
             for (int u = 0; u < kUnroll; ++u) {
                 const int t = t0 + q * kUnroll + u;
                 if (t < t1) {
                     const size_t off = (row0 + t) * d + c0;
-                    copy_async<BF16>(&ring[slot][u][0][tid], gate, off);
-                    copy_async<BF16>(&ring[slot][u][1][tid], conv, off);
+                    copy_async<BF16, V>(&ring[slot][u][0][tid], gate, off);
+                    copy_async<BF16, V>(&ring[slot][u][1][tid], conv, off);
                 }
             }
         }
         asm volatile("cp.async.commit_group;\n" ::: "memory");
     };
 #pragma unroll
-    for (int q = 0; q < kStages<BF16> - 1; ++q) issue(q);
+    for (int q = 0; q < S - 1; ++q) issue(q);
 
-    float hr[K][kVec], br[kVec];
-    load_filter<K>(h, bias, c0, hr, br);
+    float hr[K][V], br[V];
+    load_filter<K, V>(h, bias, c0, hr, br);
 
     // win[j] holds u_conv of token t - (K-1) + j for the token t about to be processed.
-    float win[K > 1 ? K - 1 : 1][kVec];
+    float win[K > 1 ? K - 1 : 1][V];
 #pragma unroll
     for (int j = 0; j < K - 1; ++j) {
         const int t = t0 - (K - 1) + j;
         if (t >= 0) {
-            load4<BF16>(conv, (row0 + t) * d + c0, win[j]);
+            load_ro<BF16, V>(conv, (row0 + t) * d + c0, win[j]);
         } else {
 #pragma unroll
-            for (int e = 0; e < kVec; ++e) win[j][e] = 0.0f;
+            for (int e = 0; e < V; ++e) win[j][e] = 0.0f;
         }
     }
 
     for (int q = 0; q < nstage; ++q) {
-        issue(q + kStages<BF16> - 1);
-        asm volatile("cp.async.wait_group %0;\n" ::"n"(kStages<BF16> - 1) : "memory");
-        const int slot = q % kStages<BF16>;
+        issue(q + S - 1);
+        asm volatile("cp.async.wait_group %0;\n" ::"n"(S - 1) : "memory");
+        const int slot = q % S;
 #pragma unroll
         for (int u = 0; u < kUnroll; ++u) {
             const int t = t0 + q * kUnroll + u;
             if (t < t1) {
-                float g[kVec], x[kVec], out[kVec];
-                unpack_chunk<BF16>(ring[slot][u][0][tid], g);
-                unpack_chunk<BF16>(ring[slot][u][1][tid], x);
+                float g[V], x[V], out[V];
+                to_float<BF16, V>(ring[slot][u][0][tid], g);
+                to_float<BF16, V>(ring[slot][u][1][tid], x);
 #pragma unroll
-                for (int e = 0; e < kVec; ++e) {
+                for (int e = 0; e < V; ++e) {
                     float c = br[e];
 #pragma unroll
                     for (int j = 0; j < K - 1; ++j) c = fmaf(hr[j][e], win[j][e], c);
                     c = fmaf(hr[K - 1][e], x[e], c);
                     out[e] = g[e] * silu(c);
                 }
-                store4<BF16>(y, (row0 + t) * d + c0, out);
+                store<BF16, V>(y, (row0 + t) * d + c0, out);
 #pragma unroll
                 for (int j = 0; j + 1 < K - 1; ++j)
 #pragma unroll
-                    for (int e = 0; e < kVec; ++e) win[j][e] = win[j + 1][e];
+                    for (int e = 0; e < V; ++e) win[j][e] = win[j + 1][e];
                 if constexpr (K > 1) {
 #pragma unroll
-                    for (int e = 0; e < kVec; ++e) win[K - 2][e] = x[e];
+                    for (int e = 0; e < V; ++e) win[K - 2][e] = x[e];
                 }
             }
         }
@@ -240,45 +257,48 @@ baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ 
     // The window now holds tokens N-K+1 .. N-1 (zeros before token 0).
     if (state != nullptr && t1 == N) {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) store4<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, win[j]);
+        for (int j = 0; j < K - 1; ++j) store<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, win[j]);
     }
 }
+
+constexpr int kDecodeVec = 4;   // channels per decode thread
 
 template <int K, bool BF16>
 __global__ void __launch_bounds__(kDecodeThreads)
 baseconv_decode_kernel(void* __restrict__ state, const void* __restrict__ gate, const void* __restrict__ conv,
                        const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
                        int d, int groups, int items) {
+    constexpr int V = kDecodeVec;
     const int item = blockIdx.x * kDecodeThreads + threadIdx.x;
     if (item >= items) return;
     const int cg = item % groups;
     const int b = item / groups;
-    const int c0 = cg * kVec;
+    const int c0 = cg * V;
 
-    float hr[K][kVec], br[kVec];
-    load_filter<K>(h, bias, c0, hr, br);
+    float hr[K][V], br[V];
+    load_filter<K, V>(h, bias, c0, hr, br);
 
-    float st[K > 1 ? K - 1 : 1][kVec];
+    float st[K > 1 ? K - 1 : 1][V];
 #pragma unroll
-    for (int j = 0; j < K - 1; ++j) load4_rw<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j]);
-    float g[kVec], x[kVec];
-    load4<BF16>(gate, (size_t)b * d + c0, g);
-    load4<BF16>(conv, (size_t)b * d + c0, x);
+    for (int j = 0; j < K - 1; ++j) load_rw<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j]);
+    float g[V], x[V];
+    load_ro<BF16, V>(gate, (size_t)b * d + c0, g);
+    load_ro<BF16, V>(conv, (size_t)b * d + c0, x);
 
-    float out[kVec];
+    float out[V];
 #pragma unroll
-    for (int e = 0; e < kVec; ++e) {
+    for (int e = 0; e < V; ++e) {
         float c = br[e];
 #pragma unroll
         for (int j = 0; j < K - 1; ++j) c = fmaf(hr[j][e], st[j][e], c);
         c = fmaf(hr[K - 1][e], x[e], c);
         out[e] = g[e] * silu(c);
     }
-    store4<BF16>(y, (size_t)b * d + c0, out);
+    store<BF16, V>(y, (size_t)b * d + c0, out);
     if constexpr (K > 1) {
 #pragma unroll
-        for (int j = 0; j + 1 < K - 1; ++j) store4<BF16>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j + 1]);
-        store4<BF16>(state, ((size_t)b * (K - 1) + (K - 2)) * d + c0, x);
+        for (int j = 0; j + 1 < K - 1; ++j) store<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j + 1]);
+        store<BF16, V>(state, ((size_t)b * (K - 1) + (K - 2)) * d + c0, x);
     }
 }
 
@@ -291,36 +311,36 @@ int prefill_segment(int B, int N, int groups, long long slots) {
     return (int)((N + runs - 1) / runs);
 }
 
-template <int K, bool BF16>
+template <int K, bool BF16, int V>
 cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
                       void* y, void* state, int B, int N, int d, int num_sms) {
     static int occupancy = 0;   // resident blocks per SM; a property of the compiled kernel
     if (occupancy == 0) {
         // the ring lives in shared memory: prefer the largest shared-memory carveout
-        cudaError_t e = cudaFuncSetAttribute(baseconv_prefill_kernel<K, BF16>,
+        cudaError_t e = cudaFuncSetAttribute(baseconv_prefill_kernel<K, BF16, V>,
                                              cudaFuncAttributePreferredSharedMemoryCarveout,
                                              cudaSharedmemCarveoutMaxShared);
         if (e != cudaSuccess) return e;
         int o = 0;
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, baseconv_prefill_kernel<K, BF16>, kThreads, 0);
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, baseconv_prefill_kernel<K, BF16, V>, kThreads, 0);
         if (e != cudaSuccess) return e;
         occupancy = std::max(1, o);
     }
-    const int groups = d / kVec;
+    const int groups = d / V;
     const int seg = prefill_segment(B, N, groups, (long long)num_sms * occupancy * kThreads);
     const int nseg = (N + seg - 1) / seg;
     const long long items = (long long)B * nseg * groups;
     if (items > 0x7fffffffLL - kThreads) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((items + kThreads - 1) / kThreads));
-    baseconv_prefill_kernel<K, BF16><<<grid, kThreads, 0, st>>>(gate, conv, h, bias, y, state, N, d, seg, nseg,
-                                                                 groups, (int)items);
+    baseconv_prefill_kernel<K, BF16, V><<<grid, kThreads, 0, st>>>(gate, conv, h, bias, y, state, N, d, seg,
+                                                                    nseg, groups, (int)items);
     return cudaGetLastError();
 }
 
 template <int K, bool BF16>
 cudaError_t decode_k(cudaStream_t st, void* state, const void* gate, const void* conv, const float* h,
                      const float* bias, void* y, int B, int d) {
-    const int groups = d / kVec;
+    const int groups = d / kDecodeVec;
     const long long items = (long long)B * groups;
     if (items > 0x7fffffffLL - kDecodeThreads) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((items + kDecodeThreads - 1) / kDecodeThreads));
@@ -329,18 +349,30 @@ cudaError_t decode_k(cudaStream_t st, void* state, const void* gate, const void*
     return cudaGetLastError();
 }
 
+// 16-byte pieces (8 bf16 channels) when the channel count allows and the filter
+// is short enough for 8 channels of taps and window to stay in registers, else
+// 4 channels.
+template <int K, bool BF16>
+cudaError_t prefill_v(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
+                      void* y, void* state, int B, int N, int d, int num_sms) {
+    if constexpr (BF16 && K <= 5) {
+        if (d % 8 == 0) return prefill_k<K, true, 8>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+    }
+    return prefill_k<K, BF16, 4>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+}
+
 template <bool BF16>
 cudaError_t prefill_any(int K, cudaStream_t st, const void* gate, const void* conv, const float* h,
                         const float* bias, void* y, void* state, int B, int N, int d, int num_sms) {
     switch (K) {
-        case 1: return prefill_k<1, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 2: return prefill_k<2, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 3: return prefill_k<3, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 4: return prefill_k<4, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 5: return prefill_k<5, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 6: return prefill_k<6, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 7: return prefill_k<7, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 8: return prefill_k<8, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 1: return prefill_v<1, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 2: return prefill_v<2, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 3: return prefill_v<3, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 4: return prefill_v<4, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 5: return prefill_v<5, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 6: return prefill_v<6, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 7: return prefill_v<7, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 8: return prefill_v<8, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -366,7 +398,7 @@ cudaError_t decode_any(int K, cudaStream_t st, void* state, const void* gate, co
 cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const float* h, const float* bias,
                                     void* y, void* state, int B, int N, int d, int K, bool bf16, int num_sms,
                                     cudaStream_t stream) {
-    if (B <= 0 || N <= 0 || d <= 0 || d % kVec != 0 || K < 1 || K > kMaxConvTaps || num_sms <= 0)
+    if (B <= 0 || N <= 0 || d <= 0 || d % 4 != 0 || K < 1 || K > kMaxConvTaps || num_sms <= 0)
         return cudaErrorInvalidValue;
     return bf16 ? prefill_any<true>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms)
                 : prefill_any<false>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms);
@@ -375,7 +407,7 @@ cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const fl
 cudaError_t launch_baseconv_decode(void* state, const void* gate, const void* conv, const float* h,
                                    const float* bias, void* y, int B, int d, int K, bool bf16,
                                    cudaStream_t stream) {
-    if (B <= 0 || d <= 0 || d % kVec != 0 || K < 1 || K > kMaxConvTaps) return cudaErrorInvalidValue;
+    if (B <= 0 || d <= 0 || d % kDecodeVec != 0 || K < 1 || K > kMaxConvTaps) return cudaErrorInvalidValue;
     return bf16 ? decode_any<true>(K, stream, state, gate, conv, h, bias, y, B, d)
                 : decode_any<false>(K, stream, state, gate, conv, h, bias, y, B, d);
 }
