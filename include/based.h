@@ -1,6 +1,7 @@
 /*
  * based.h -- C ABI of the B200 (sm_100a) BASED hot path: causal Taylor linear
- * attention and sliding-window softmax attention, prefill and decode.
+ * attention and sliding-window softmax attention, prefill and decode, plus the
+ * short gated convolution (BaseConv) mixer.
  *
  * The method is that of "Simple linear attention language models balance the
  * recall-throughput tradeoff" (BASED, arXiv 2402.18668v2):
@@ -13,7 +14,9 @@
  *     so that phi(q).phi(k) = 1 + q.k + (q.k)^2/2;
  *   - outputs normalised by the "K-state" z (App. D.4 "State size");
  *   - exact softmax attention inside a small sliding window with a w-sized KV
- *     cache (§4 "Local Exact Attention").
+ *     cache (§4 "Local Exact Attention");
+ *   - short gated convolutions beside the window layers (§4, Additional
+ *     mixers; App. C "Extended Architecture Details", Convolution).
  *
  * Conventions shared by every call
  * --------------------------------
@@ -21,8 +24,9 @@
  *   and live in device memory of the current CUDA device. Every pointer must
  *   be 16-byte aligned. The library never allocates memory and keeps no
  *   pointer after a call returns; the caller owns every buffer.
- * - dtype selects the element type of q, k, v, y and the SWA caches:
- *   BASED_F32 (float) or BASED_BF16 (__nv_bfloat16). S and z are always float.
+ * - dtype selects the element type of q, k, v, y, the SWA caches and the
+ *   convolution's streams and state: BASED_F32 (float) or BASED_BF16
+ *   (__nv_bfloat16). S, z and the convolution's taps and bias are always float.
  *   Arithmetic is fp32 (fp32 accumulation of bf16 tensor-core products on the
  *   bf16 prefill path).
  * - Work is enqueued on `stream` (0 = legacy default stream); every call is
