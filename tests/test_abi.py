@@ -201,3 +201,8 @@ def test_python_binding_requires_cuda_tensors():
     x = torch.zeros(1, 1, 4, 16)
     with pytest.raises(based.BasedError):
         based.la_prefill(x, x, torch.zeros(1, 1, 4, 64))
+    u = torch.zeros(1, 4, 8)
+    with pytest.raises(based.BasedError):
+        based.baseconv_prefill(u, u, torch.zeros(8, 4))
+    with pytest.raises(based.BasedError):
+        based.baseconv_decode(torch.zeros(1, 3, 8), u[:, 0], u[:, 0], torch.zeros(8, 4))
