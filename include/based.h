@@ -316,6 +316,12 @@ BASED_API based_status_t based_swa_prefill(const void* q, const void* k, const v
  * (t-1) mod w before that work has finished. The kernel immediately before it
  * in the stream must therefore not write those slots of this cache; decode
  * steps on one cache issued in order (t after t-1, or t repeated) satisfy this.
+ * The library records every ring that based_swa_prefill writes (the 256 most
+ * recent), and the first decode on such a ring reads every slot only after
+ * the previous work has finished, so prefill then decode back to back on one
+ * stream is safe. A ring written by anything else (a copy, a caller's kernel)
+ * needs another kernel, or a stream synchronisation, between that write and
+ * the first decode.
  */
 BASED_API based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t,
                                 const void* q, const void* k, const void* v, void* y,

@@ -157,6 +157,18 @@ def packed_dim(d_feat: int) -> int:
     return 1 + d_feat + d_feat * (d_feat + 1) // 2
 
 
+def _check_state_shape(S, z, B, H, D, d_v):
+    """S [B,H,D,dv] and z [B,H,D] float32, contiguous (either may be None: not given):
+    the kernels write exactly that much."""
+    for name, t, shape in (("S", S, (B, H, D, d_v)), ("z", z, (B, H, D))):
+        if t is None:
+            continue
+        if tuple(t.shape) != shape:
+            raise BasedError(ERR_INVALID_ARG, f"S, z must be [{B},{H},{D},{d_v}] and [{B},{H},{D}]")
+        if t.dtype != torch.float32 or not t.is_contiguous():
+            raise BasedError(ERR_INVALID_ARG, f"{name} must be contiguous float32")
+
+
 def la_prefill_workspace(B, H, N, d_feat, d_v, dtype=torch.bfloat16, chunk=0) -> int:
     return int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, _DTYPES[dtype], chunk))
 
@@ -181,11 +193,10 @@ def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None,
             z = torch.empty((B, H, D), dtype=torch.float32, device=dev) if z is None else z
         else:
             S = z = None
+        _check_state_shape(S, z, B, H, D, d_v)
         ws_bytes = int(lib().based_la_prefill_workspace(B, H, N, d_feat, d_v, dt, chunk))
         if ws_bytes and (workspace is None or workspace.numel() < ws_bytes):
             workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-        if S is not None and (tuple(S.shape) != (B, H, D, d_v) or tuple(z.shape) != (B, H, D)):
-            raise BasedError(ERR_INVALID_ARG, f"S, z must be [{B},{H},{D},{d_v}] and [{B},{H},{D}]")
         fn = lib().based_la_prefill_packed if packed else lib().based_la_prefill
         st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(y), _ptr(S), _ptr(z), B, H, N, d_feat, d_v, dt, chunk,
                 _ptr(workspace) if ws_bytes else None, ws_bytes, _stream(dev))
@@ -196,10 +207,12 @@ def la_prefill(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None,
 def la_prefill_noalloc(q, k, v, chunk: int = 0, want_state: bool = True, y=None, S=None, z=None):
     """la_prefill without a workspace: the library's fixed device scratch is used
     instead (for callers that must not allocate; calls must not overlap on the GPU)."""
-    dt = _dtype_code(q, k, v)
     B, H, N, d_feat = q.shape
     d_v = v.shape[-1]
     D = feature_dim(d_feat)
+    if want_state:
+        _check_state_shape(S, z, B, H, D, d_v)     # caller-supplied S, z (None: allocated below)
+    dt = _dtype_code(q, k, v)
     dev = q.device
     with torch.cuda.device(dev):
         if y is None:

@@ -3,6 +3,9 @@
 #include <atomic>
 #include <cstdint>
 #include <cstdlib>
+#include <mutex>
+
+#include <cuda.h>
 
 #include "../../include/based.h"
 #include "common.cuh"
@@ -14,21 +17,74 @@ namespace {
 __device__ unsigned g_based_status;
 
 constexpr int kMaxDevices = 64;
-std::atomic<unsigned*> g_status_ptr[kMaxDevices];
 std::atomic<int> g_num_sms[kMaxDevices];
 
 bool current_device(int* dev) { return cudaGetDevice(dev) == cudaSuccess && *dev >= 0 && *dev < kMaxDevices; }
 
-unsigned* status_word(int dev) {
-    unsigned* p = g_status_ptr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_based_status) != cudaSuccess) return nullptr;
-        p = static_cast<unsigned*>(addr);
-        g_status_ptr[dev].store(p, std::memory_order_release);
-    }
-    return p;
+// Unique id of the calling thread's current CUDA context (0 if unknown), from
+// the driver through cudaGetDriverEntryPoint (the library does not link libcuda).
+unsigned long long current_context_id() {
+    using GetCurrent = CUresult (*)(CUcontext*);
+    using GetId = CUresult (*)(CUcontext, unsigned long long*);
+    static GetCurrent get_current = nullptr;
+    static GetId get_id = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_current = reinterpret_cast<GetCurrent>(p);
+        if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            get_id = reinterpret_cast<GetId>(p);
+    });
+    CUcontext ctx = nullptr;
+    unsigned long long id = 0;
+    if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr ||
+        get_id(ctx, &id) != CUDA_SUCCESS)
+        return 0;
+    return id;
 }
+
+// Device addresses of the library's __device__ symbols, per device and per
+// context: cudaDeviceReset destroys the primary context with the module in it,
+// and the next call runs in a new context where the symbol has a new address.
+// A lookup is redone whenever the current context's id differs from the one
+// the address was taken in.
+struct SymbolSlot {
+    const void* symbol;
+    int dev;
+    unsigned long long ctx;
+    void* addr;
+};
+constexpr int kSymbolSlots = 4 * kMaxDevices;
+std::mutex g_symbol_mu;
+SymbolSlot g_symbols[kSymbolSlots];
+int g_symbols_n = 0;
+
+void* symbol_address(const void* symbol, int dev) {
+    const unsigned long long ctx = current_context_id();
+    std::lock_guard<std::mutex> lock(g_symbol_mu);
+    int slot = -1;
+    for (int i = 0; i < g_symbols_n; ++i) {
+        if (g_symbols[i].symbol == symbol && g_symbols[i].dev == dev) {
+            if (ctx != 0 && g_symbols[i].ctx == ctx) return g_symbols[i].addr;
+            slot = i;
+            break;
+        }
+    }
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, symbol) != cudaSuccess || addr == nullptr) return nullptr;
+    if (slot < 0) {
+        if (g_symbols_n == kSymbolSlots) return addr;           // table full: no caching
+        slot = g_symbols_n++;
+    }
+    g_symbols[slot] = SymbolSlot{symbol, dev, ctx, addr};
+    return addr;
+}
+
+unsigned* status_word(int dev) { return static_cast<unsigned*>(symbol_address(&g_based_status, dev)); }
 
 int num_sms(int dev) {
     int n = g_num_sms[dev].load(std::memory_order_relaxed);
@@ -46,6 +102,42 @@ int num_sms(int dev) {
 unsigned debug_flags() {
     const char* e = std::getenv("BASED_DEBUG_SKIP_MMA");
     return (e != nullptr && e[0] == '1') ? based::DEBUG_SKIP_MMA : 0u;
+}
+
+// Ring caches written whole by based_swa_prefill and not decoded from since.
+// The first based_swa_decode on such a ring loads every slot after its
+// dependency wait, because the prefill may be the kernel just before it in the
+// stream and it writes every slot. Later steps read the slots that the step
+// before them cannot write before the wait. The table keeps the most recent
+// kFreshRings rings; a ring pushed out by that many later prefills of other
+// rings is decoded as if no prefill had written it.
+constexpr int kFreshRings = 256;
+struct FreshRing { const void* cache; int dev; };
+std::mutex g_fresh_mu;
+FreshRing g_fresh[kFreshRings];
+int g_fresh_n = 0;
+
+void mark_ring_fresh(const void* cache, int dev) {
+    std::lock_guard<std::mutex> lock(g_fresh_mu);
+    for (int i = 0; i < g_fresh_n; ++i)
+        if (g_fresh[i].cache == cache && g_fresh[i].dev == dev) return;
+    if (g_fresh_n == kFreshRings) --g_fresh_n;                  // forget the oldest
+    for (int i = g_fresh_n; i > 0; --i) g_fresh[i] = g_fresh[i - 1];
+    g_fresh[0] = FreshRing{cache, dev};
+    ++g_fresh_n;
+}
+
+// True (and the entry removed) when `cache` was written by a prefill since its last decode.
+bool take_ring_fresh(const void* cache, int dev) {
+    std::lock_guard<std::mutex> lock(g_fresh_mu);
+    for (int i = 0; i < g_fresh_n; ++i) {
+        if (g_fresh[i].cache == cache && g_fresh[i].dev == dev) {
+            for (int j = i; j + 1 < g_fresh_n; ++j) g_fresh[j] = g_fresh[j + 1];
+            --g_fresh_n;
+            return true;
+        }
+    }
+    return false;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -87,6 +179,7 @@ namespace based {
 
 // Lookups shared with the allocation-free prefill entry point (noalloc.cu).
 unsigned* device_status_word(int dev) { return status_word(dev); }
+void* device_symbol_address(const void* symbol, int dev) { return symbol_address(symbol, dev); }
 int device_sm_count(int dev) { return num_sms(dev); }
 unsigned current_debug_flags() { return debug_flags(); }
 int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
@@ -315,6 +408,7 @@ based_status_t based_swa_prefill(const void* q, const void* k, const void* v, vo
     if (status == nullptr) return BASED_ERR_CUDA;
     const cudaError_t e = based::launch_swa_prefill(q, k, v, y, k_cache, v_cache, B, H, N, d, w, scale,
                                                     dtype == BASED_BF16, status, debug_flags(), stream);
+    if (e == cudaSuccess && k_cache != nullptr) mark_ring_fresh(k_cache, dev);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
@@ -326,8 +420,11 @@ based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t, const v
     if (t < 0 || B <= 0 || H <= 0 || w <= 0 || d <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
     if (!(scale == scale) || scale - scale != 0.0f) return BASED_ERR_INVALID_ARG;
     if (d != 64 || w > 64 || (long long)B * H > (1LL << 30)) return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    const bool preload = !take_ring_fresh(k_cache, dev);
     const cudaError_t e = based::launch_swa_decode(k_cache, v_cache, t, q, k, v, y, B, H, d, w, scale,
-                                                   dtype == BASED_BF16, stream);
+                                                   dtype == BASED_BF16, preload, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 

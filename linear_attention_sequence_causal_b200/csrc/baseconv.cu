@@ -32,6 +32,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "kernels.h"
 
@@ -314,7 +315,13 @@ int prefill_segment(int B, int N, int groups, long long slots) {
 template <int K, bool BF16, int V>
 cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
                       void* y, void* state, int B, int N, int d, int num_sms) {
-    static int occupancy = 0;   // resident blocks per SM; a property of the compiled kernel
+    // Resident blocks per SM, a property of the compiled kernel on a device:
+    // looked up once per device (the carveout attribute is set per device too).
+    constexpr int kDevices = 64;
+    static std::atomic<int> occ[kDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevices) return cudaErrorInvalidDevice;
+    int occupancy = occ[dev].load(std::memory_order_relaxed);
     if (occupancy == 0) {
         // the ring lives in shared memory: prefer the largest shared-memory carveout
         cudaError_t e = cudaFuncSetAttribute(baseconv_prefill_kernel<K, BF16, V>,
@@ -325,6 +332,7 @@ cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, baseconv_prefill_kernel<K, BF16, V>, kThreads, 0);
         if (e != cudaSuccess) return e;
         occupancy = std::max(1, o);
+        occ[dev].store(occupancy, std::memory_order_relaxed);   // same value from every racing thread
     }
     const int groups = d / V;
     const int seg = prefill_segment(B, N, groups, (long long)num_sms * occupancy * kThreads);

@@ -70,9 +70,12 @@ cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, v
                                   void* v_cache, int B, int H, int N, int w, float scale, unsigned* status,
                                   unsigned debug, cudaStream_t stream);
 
+// preload: the bf16 kernel may read the ring slots other than t mod w and
+// (t-1) mod w before its dependency wait (see based_swa_decode in based.h);
+// false when the kernel before it may have written any slot of this ring.
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q,
                               const void* k, const void* v, void* y, int B, int H, int d, int w,
-                              float scale, bool bf16, cudaStream_t stream);
+                              float scale, bool bf16, bool preload, cudaStream_t stream);
 
 // Short gated convolution: filter taps K in [1, kMaxConvTaps], d a multiple of 4.
 constexpr int kMaxConvTaps = 8;

@@ -2,14 +2,13 @@
 // not allocate device memory themselves (see include/based.h). The segment
 // totals that based_la_prefill keeps in a caller-provided workspace live here
 // in a fixed array that is part of the library's device image.
-#include <atomic>
-
 #include "../../include/based.h"
 #include "common.cuh"
 #include "kernels.h"
 
 namespace based {
 unsigned* device_status_word(int dev);
+void* device_symbol_address(const void* symbol, int dev);   // per device and CUDA context
 int device_sm_count(int dev);
 unsigned current_debug_flags();
 int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk);   // 0 none, 1 CUDA cores, 2 chunked tcgen05, 3 quadratic tcgen05
@@ -24,21 +23,12 @@ constexpr size_t kScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::atomic<void*> g_scratch_ptr[kMaxDevices];
 
 // Device address of g_prefill_scratch on device `dev` (which must be current).
 // The symbol's name in host code is only a stand-in; its device address is
-// looked up once per device, on the first call there.
-void* scratch_address(int dev) {
-    void* p = g_scratch_ptr[dev].load(std::memory_order_acquire);
-    if (p == nullptr) {
-        void* addr = nullptr;
-        if (cudaGetSymbolAddress(&addr, g_prefill_scratch) != cudaSuccess || addr == nullptr) return nullptr;
-        g_scratch_ptr[dev].store(addr, std::memory_order_release);
-        p = addr;
-    }
-    return p;
-}
+// looked up on the first call in each CUDA context of the device (again after
+// a cudaDeviceReset, which gives the device a new context and module).
+void* scratch_address(int dev) { return based::device_symbol_address(&g_prefill_scratch, dev); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }

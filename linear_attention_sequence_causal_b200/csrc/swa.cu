@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(128)
 swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, int new_slot,
-                       float scale) {
+                       float scale, int preload) {
     __shared__ float s_sc[kMaxW];
     __shared__ float s_part[4][kHead];
     const int tid = threadIdx.x;
@@ -243,6 +243,8 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
     // loaded before the wait for the previous kernel in the stream: only that
     // kernel can still be running, and consecutive decode steps on one cache
     // write slot (t - 1) mod w at most. The rest is loaded after the wait.
+    // Without `preload` (the ring was just written whole, by a prefill) every
+    // slot is loaded after the wait.
     const int prev_slot = new_slot == 0 ? w - 1 : new_slot - 1;
     uint4 kr[4], vr[4];
     bool valid[4], late[4];
@@ -252,7 +254,7 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
         // newest token held by the slot: u = t - ((t - slot) mod w), empty while u < 0,
         // that is: every slot once t >= w, else the slots <= t.
         valid[p] = slot < w && (t >= w || slot <= t);
-        late[p] = slot == new_slot || slot == prev_slot;
+        late[p] = !preload || slot == new_slot || slot == prev_slot;
         kr[p] = vr[p] = make_uint4(0, 0, 0, 0);
         if (valid[p] && !late[p]) {
             kr[p] = __ldg(reinterpret_cast<const uint4*>(kc + (bh * w + slot) * kHead) + c);
@@ -364,7 +366,7 @@ cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void
 
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
                               const void* v, void* y, int B, int H, int d, int w, float scale,
-                              bool bf16, cudaStream_t stream) {
+                              bool bf16, bool preload, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
     if (bf16) {
         // Programmatic dependent launch: a step's CTAs are scheduled while the
@@ -382,7 +384,7 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                                            static_cast<__nv_bfloat16*>(v_cache), (long long)t,
                                            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w,
-                                           (int)(t % w), scale);   // the new token's slot
+                                           (int)(t % w), scale, preload ? 1 : 0);   // the new token's slot
         if (e != cudaSuccess) return e;
     } else {
         swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(

@@ -206,3 +206,19 @@ def test_python_binding_requires_cuda_tensors():
         based.baseconv_prefill(u, u, torch.zeros(8, 4))
     with pytest.raises(based.BasedError):
         based.baseconv_decode(torch.zeros(1, 3, 8), u[:, 0], u[:, 0], torch.zeros(8, 4))
+
+
+def test_noalloc_binding_rejects_wrong_state_shapes():
+    """The kernels write exactly [B,H,D,dv] and [B,H,D] floats: a caller's S or z
+    of another shape is refused before any tensor reaches the library."""
+    import torch
+    q = torch.zeros(1, 2, 8, 16)
+    v = torch.zeros(1, 2, 8, 64)
+    D = 1 + 16 + 16 * 16
+    good_S, good_z = torch.zeros(1, 2, D, 64), torch.zeros(1, 2, D)
+    for S, z in ((torch.zeros(1, 2, D - 1, 64), good_z), (good_S, torch.zeros(1, 2, D + 1)),
+                 (torch.zeros(1, 1, D, 64), good_z), (good_S.double(), good_z)):
+        with pytest.raises(based.BasedError) as e:
+            based.la_prefill_noalloc(q, q, v, S=S, z=z)
+        assert e.value.status == binding.ERR_INVALID_ARG
+        assert "S, z must be" in str(e.value) or "contiguous float32" in str(e.value)

@@ -120,6 +120,34 @@ def test_decode_steps_back_to_back(w, prompt):
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
 
+@pytest.mark.parametrize("w", [64, 16])
+def test_prefill_then_decode_back_to_back(w):
+    """based_swa_prefill immediately followed by based_swa_decode on the same
+    stream, every buffer allocated beforehand, so no other kernel runs between
+    them. The ring holds stale values (a large constant) before each prefill:
+    a decode that read any slot before the prefill had finished would attend
+    to them."""
+    batch, H, prompt = 64, 16, 2048
+    inp = synthetic.swa_inputs(batch, H, prompt + 2, 64, "bf16", seed=31 + w)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    qp, kp, vp = (x[:, :, :prompt].contiguous() for x in (q, k, v))
+    qd, kd, vd = (x[:, :, prompt].contiguous() for x in (q, k, v))
+    yp = torch.empty_like(qp)
+    kc = torch.empty((batch, H, w, 64), dtype=q.dtype, device=DEV)
+    vc = torch.empty_like(kc)
+    yd = torch.empty_like(qd)
+    ref = oracle.swa(inp.q64[..., :prompt + 1, :], inp.k64[..., :prompt + 1, :], inp.v64[..., :prompt + 1, :],
+                     w, SCALE)[..., prompt, :]
+    for _ in range(3):
+        kc.fill_(30.0)
+        vc.fill_(-30.0)
+        torch.cuda.synchronize()
+        based.swa_prefill(qp, kp, vp, w=w, scale=SCALE, y=yp, k_cache=kc, v_cache=vc)
+        based.swa_decode(kc, vc, prompt, qd, kd, vd, w=w, scale=SCALE, y=yd)
+        assert based.get_last_error() == 0
+        assert_y(to64(yd), ref, torch.bfloat16, "first decode after prefill")
+
+
 @pytest.mark.parametrize("w,prompt", [(64, 100), (16, 0), (40, 7)])
 def test_decode_large_batch(w, prompt):
     """2048 heads (batch 128 x 16), more than one wave of CTAs; early steps
