@@ -87,16 +87,17 @@ typedef enum {
  *   z       [B, H, D]          float, written
  *           S and z may both be NULL (final state not wanted), not just one.
  *   d_feat  16 or 32;  d_v  64 or 128;  N >= 1;  B, H >= 1
- *   chunk   tokens per on-diagonal tile: 0 (library's choice) or one of the
- *           values built for the call: 16, 32 (and 64 at d_feat 16) run on the
- *           CUDA cores in fp32 arithmetic, for both dtypes; 128 (BASED_BF16
- *           only) runs on the tensor cores -- the chunked form with the state
- *           in tensor memory at d_feat 16, d_v 64, and the quadratic masked form
- *           in 128-token tiles (final state from a separate contraction) for the
- *           other shapes, whose state does not fit one SM's tensor memory.
- *           0 picks 128 for bf16 and the largest CUDA-core chunk for fp32.
- *           Other values return BASED_ERR_UNSUPPORTED. The result does not
- *           depend on the chunk beyond rounding.
+ *   chunk   tokens per chunk (on-diagonal tile): 0 (library's choice) or one
+ *           of the values built for the call. BASED_BF16 at d_feat 16, d_v 64:
+ *           64, 128 or 256 on the tensor cores, the chunked form with the state
+ *           in tensor memory. BASED_BF16, other shapes (whose state does not
+ *           fit one SM's tensor memory): 128, the quadratic masked form in
+ *           128-token tiles with the final state from a separate contraction.
+ *           Both dtypes: 16, 32 (and 64 at d_feat 16 for BASED_F32) on the
+ *           CUDA cores in fp32 arithmetic. 0 picks 128 for bf16 and the largest
+ *           CUDA-core chunk for fp32. Other values return
+ *           BASED_ERR_UNSUPPORTED. The result does not depend on the chunk
+ *           beyond rounding.
  *   workspace, workspace_bytes
  *           device scratch of at least based_la_prefill_workspace(...) bytes
  *           (NULL allowed when that size is 0). Used to split long sequences

@@ -155,10 +155,10 @@ bool simt_chunk_ok(int d_feat, int chunk) {
 enum class LaPath { None, Simt, TensorCore, Quad };
 
 // Kernel choice for a prefill. bf16: the chunked tcgen05 kernel where it is
-// built (d' = 16, dv = 64, 128-token chunks), else the tcgen05 quadratic-form
-// kernel (128-token tiles; the state of the other shapes does not fit one SM's
-// tensor memory); explicit chunks of 16, 32 or 64 tokens and every fp32 call
-// take the CUDA-core kernel.
+// built (d' = 16, dv = 64; chunks of 64, 128 or 256 tokens, 128 by default),
+// else the tcgen05 quadratic-form kernel (128-token tiles; the state of the
+// other shapes does not fit one SM's tensor memory); other explicit chunks
+// (16, 32, and 64 for those shapes) and every fp32 call take the CUDA-core kernel.
 LaPath choose_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
     const bool bf16 = dtype == BASED_BF16;
     if (*chunk == 0) {

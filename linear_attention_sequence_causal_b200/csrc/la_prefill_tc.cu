@@ -4,15 +4,31 @@
 // tradeoff" (BASED), App. B "Forward / Generation Prefill": the feature map and
 // the causal dot product are computed together, tile by tile; a tile's output is
 // a quadratic on-diagonal part under a local causal mask plus a linear
-// off-diagonal part read from the cumulative state of earlier tiles. With the
-// K-state normalisation (App. D.4), for a chunk c of C = 128 tokens:
+// off-diagonal part read from the cumulative state of earlier chunks. With the
+// K-state normalisation (App. D.4), for a tile t of 128 tokens (the M of every
+// MMA below) inside a chunk of CL tokens:
 //
-//   s         = Q_c K_c^T                          MMA1  M=128 N=128 K=16
+//   s         = Q_t K_j^T                          MMA1  M=128 N=128 K=16
 //   A         = mask(1 + s + s^2/2)                CUDA cores, TMEM -> TMEM (bf16, spare columns)
-//   Y         = phi(Q_c) [S | z]_{c-1}             MMA3  M=128 N=80  K=160 (A operand in TMEM)
-//   Y        += A [V_c | 1]                        MMA2  M=128 N=80  K=128 (A operand in TMEM)
-//   [S|z]^T  += [V_c | 1]^T phi(K_c)               MMA4  M=128 N=160 K=128, fp32 in TMEM
-//   y_c       = Y[:, :64] / Y[:, 64]               epilogue
+//   Y         = phi(Q_t) [S | z]_{chunk start}     MMA3  M=128 N=80  K=160 (A operand in TMEM)
+//   Y        += A [V_j | 1]                        MMA2  M=128 N=80  K=128 (A operand in TMEM)
+//   [S|z]^T  += [V_t | 1]^T phi(K_t)               MMA4  M=128 N=160 K=128, fp32 in TMEM
+//   y_t       = Y[:, :64] / Y[:, 64]               epilogue
+//
+// The chunk length CL decides which pairs (query, key) go through the
+// quadratic form (same chunk) and which through the state (earlier chunks):
+//   CL = 128  one chunk per tile: j = t, causal mask; the state after each tile
+//             is read out and published for the next tile's MMA3.
+//   CL = 256  two tiles per chunk: an odd tile adds the full (unmasked) block
+//             j = t-1 of its chunk, and its MMA3 reads the same state as the
+//             even tile before it; the state is read out after odd tiles only.
+//   CL = 64   two chunks per tile: the mask keeps each query's own chunk only
+//             (block diagonal); MMA3 runs twice, for rows 0-63 with the state
+//             before the tile and for rows 64-127 with the state after its
+//             first 64 tokens (phi(Q) has the other half's rows zeroed for each
+//             pass), and MMA4 is split at token 64 so that state is read out
+//             in between.
+// All three give the same sum up to rounding.
 //
 // The ones column appended to V makes every product carry its own
 // denominator: A [V | 1] gives the row sums of A, phi(Q)[S | z] gives phi(q).z,
@@ -23,32 +39,33 @@
 // memory. The order-2 block is folded by symmetry,
 // (q.k)^2/2 = sum_a (q_a^2/sqrt2)(k_a^2/sqrt2) + sum_{a<b} (q_a q_b)(k_a k_b),
 // giving 1 + 16 + 136 = 153 features (padded to 160) instead of 273, in an
-// order that suits packed bf16x2 multiplies (see phi_word); the final state is
+// order that suits packed bf16x2 multiplies (see emit_phi2); the final state is
 // expanded back to the 273-row layout on the way out.
 //
 // Issue structure. One thread can keep only about one tcgen05.mma per ~117
 // cycles in flight (measured on B200 for any N <= 144), while MMAs from two
 // issuing warps into separate accumulators overlap. So two warps issue:
-//   warp 13  the Y chain: MMA3_c, MMA2_c, MMA1_{c+1} (19 instructions);
-//   warp 12  the state chain: MMA4_c (8 instructions of N = 160; the state is
-//            kept transposed -- TMEM lane = value column, column = feature --
-//            which halves the instruction count of the natural layout).
-// A has its own tensor-memory columns, so MMA1_{c+1} can overwrite s as soon
-// as A_c has been formed, and A_{c+1} is computed while MMA2_c still reads A_c
-// (only its stores wait for MMA2_c). Keeping A (and phi(Q)) in tensor memory
-// matters: an MMA of N = 80 with both operands in shared memory is bound by
-// shared-memory bandwidth (6.5 KB per 40 tensor cycles).
+//   warp 13  the Y chain: MMA3, MMA2 of every block of the tile, MMA1 of the
+//            next block;
+//   warp 12  the state chain: MMA4 (8 instructions of N = 160 per tile; the
+//            state is kept transposed -- TMEM lane = value column, column =
+//            feature -- which halves the instruction count of the natural layout).
+// A has its own tensor-memory columns, so MMA1 of the next block can overwrite
+// s as soon as A has been formed, and the next A is computed while MMA2 still
+// reads the previous one (only its stores wait for MMA2). Keeping A (and
+// phi(Q)) in tensor memory matters: an MMA of N = 80 with both operands in
+// shared memory is bound by shared-memory bandwidth (6.5 KB per 40 tensor cycles).
 //
 // Other roles (448 threads, one CTA per (b, h, segment)); a warp reaches the
 // TMEM lanes of quadrant (warp mod 4):
-//   warps 0-3   producers: thread t loads token t of chunk c+1 (prefetched in
-//               registers a chunk ahead) and writes Q, K, [V|1] and phi(K) into
+//   warps 0-3   producers: thread t loads token t of tile c+1 (prefetched in
+//               registers a tile ahead) and writes Q, K, [V|1] and phi(K) into
 //               the free half of the double-buffered shared-memory tiles, then
-//               phi(Q) into TMEM once MMA3_c has consumed the previous one.
+//               phi(Q) into TMEM once MMA3 has consumed the previous one.
 //   warps 4-7   intra + state: turn s into A (TMEM lane = token); warps 4-6
-//               also read the fp32 state after MMA4_c (lane = value column,
-//               0..79) and publish it as the bf16 B operand of MMA3_{c+1}, and
-//               stage the final state or write a segment total.
+//               also read the fp32 state after MMA4 (lane = value column,
+//               0..79) and publish it as the bf16 B operand of the next MMA3,
+//               and stage the final state or write a segment total.
 //   warps 8-11  epilogue: turn Y into y (TMEM lane = token) in a 128-byte
 //               swizzled shared-memory tile that one thread stores with TMA.
 // Every hand-off is an mbarrier; every wait is bounded.
@@ -77,7 +94,7 @@ using namespace tc;
 
 constexpr int DF = 16;           // feature dim d'
 constexpr int DV = 64;           // value dim
-constexpr int C = 128;           // tokens per chunk
+constexpr int C = 128;           // tokens per tile (the M of every MMA)
 constexpr int DS = 153;          // distinct (symmetric) features
 constexpr int KF = 160;          // DS padded to the MMA K step
 constexpr int NV = 80;           // [V | 1] padded to the MMA N step
@@ -85,7 +102,7 @@ constexpr int kThreads = 448;
 constexpr int kStateLanes = 96;  // warps 4-6 read state lanes 0..95 (0..79 hold data)
 
 // ------------------------------------------------------------------ shared memory
-// [b] tiles are double-buffered by chunk parity.
+// [b] tiles are double-buffered by tile parity.
 constexpr uint32_t PK_BYTES = C * KF * 2;       // phi(K): K = token, N = feature, MN-major
 constexpr uint32_t VA_BYTES = C * NV * 2;       // [V|1]:  K = token, N = column, MN-major
 constexpr uint32_t QK_BYTES = C * DF * 2;       // Q, K:   M/N = token, K = d', K-major
@@ -95,11 +112,15 @@ constexpr uint32_t OFF_VA = OFF_PK + 2 * PK_BYTES;
 constexpr uint32_t OFF_Q = OFF_VA + 2 * VA_BYTES;
 constexpr uint32_t OFF_K = OFF_Q + 2 * QK_BYTES;
 constexpr uint32_t YS_BYTES = C * DV * 2;       // y tile, 128-byte swizzled rows (TMA store source)
-constexpr uint32_t OFF_SB = OFF_K + 2 * QK_BYTES;               // single buffer
-constexpr uint32_t OFF_YS = (OFF_SB + SB_BYTES + 1023) & ~1023u; // [2], 1024-aligned for the swizzle
-constexpr uint32_t OFF_BAR = OFF_YS + 2 * YS_BYTES;
-constexpr uint32_t SMEM_BYTES = OFF_BAR + 256;
-static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+constexpr uint32_t OFF_SB = OFF_K + 2 * QK_BYTES;               // [S|z] of the state before the tile
+constexpr uint32_t OFF_SB1 = OFF_SB + SB_BYTES;                 // CL = 64: the state after its first chunk
+// The rest depends on whether the second [S|z] buffer is used (CL = 64).
+__host__ __device__ constexpr uint32_t off_ys(int cl) {       // [2], 1024-aligned for the swizzle
+    return ((cl == 64 ? OFF_SB1 + SB_BYTES : OFF_SB + SB_BYTES) + 1023) & ~1023u;
+}
+__host__ __device__ constexpr uint32_t off_bar(int cl) { return off_ys(cl) + 2 * YS_BYTES; }
+__host__ __device__ constexpr uint32_t smem_bytes(int cl) { return off_bar(cl) + 256; }
+static_assert(smem_bytes(64) <= 227 * 1024 && smem_bytes(128) <= 227 * 1024, "shared memory");
 
 // Core-matrix strides (bytes): LBO along K, SBO along M/N.
 constexpr uint32_t PK_LBO = (KF / 8) * 128, PK_SBO = 128;
@@ -137,22 +158,48 @@ constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 constexpr size_t kTotalFloats = (size_t)KF * NV;
 
 enum {
-    BAR_IN0, BAR_IN1,        // producers -> issuers: Q, K, [V|1], phi(K) of a chunk are in buffer b
+    BAR_IN0, BAR_IN1,        // producers -> issuers: Q, K, [V|1], phi(K) of a tile are in buffer b
     BAR_FREE0, BAR_FREE1,    // both issuers' commits: every MMA reading buffer b has completed
-    BAR_PQIN,                // producers -> Y issuer: phi(Q) is in TMEM
-    BAR_PQF,                 // Y-issuer commit: MMA3 done (phi(Q) and the [S|z] bf16 buffer it read are free)
-    BAR_S,                   // Y-issuer commit: s ready
-    BAR_A,                   // intra warps -> Y issuer: A written to shared memory (s has been read)
-    BAR_AF,                  // Y-issuer commit: MMA2 done (the A columns are free)
-    BAR_Y,                   // Y-issuer commit: Y complete
+    BAR_PQIN,                // producers -> Y issuer: phi(Q) (one MMA3 pass's rows) is in TMEM
+    BAR_PQF,                 // Y-issuer commit: MMA3 (CL = 64: of rows 0-63) done; phi(Q) and the [S|z] buffer it read are free
+    BAR_PQF_HI,              // CL = 64: the same for the MMA3 of rows 64-127
+    BAR_S,                   // Y-issuer commit: s of a block ready
+    BAR_A,                   // intra warps -> Y issuer: A of a block written (s has been read)
+    BAR_AF,                  // Y-issuer commit: MMA2 of a block done (the A columns are free)
+    BAR_Y,                   // Y-issuer commit: Y of a tile complete
     BAR_YF,                  // epilogue warps -> Y issuer: Y read
-    BAR_DS,                  // state-issuer commit: MMA4 done, the TMEM state is the state after chunk c
+    BAR_DS,                  // state-issuer commit: MMA4 done, the TMEM state is the state to read out
     BAR_DSF,                 // state warps -> state issuer: fp32 state read
-    BAR_SBR,                 // state warps -> Y issuer: [S|z] bf16 written
+    BAR_SBR,                 // state warps -> Y issuer: [S|z] bf16 written (buffer OFF_SB)
+    BAR_SBR1,                // CL = 64: the same for buffer OFF_SB1
     BAR_INIT,                // state warps -> issuers: start state of the segment is in TMEM and the [S|z] buffer
     BAR_YSR0, BAR_YSR1,      // epilogue warps -> store thread: y tile b written
     BAR_YSF0, BAR_YSF1,      // store thread -> epilogue warps: the TMA store has read y tile b
     NUM_BARS
+};
+static_assert(8 * NUM_BARS + 8 <= 256, "barrier area");
+
+// ------------------------------------------------------------------ chunk plan
+// Tiles per chunk (CL >= 128) and chunks per tile (CL < 128); the MMA tile is
+// always 128 tokens. A tile's position in its chunk, its intra blocks and its
+// state read-outs follow from CL and the tile's index c in the segment
+// (segments start on chunk boundaries).
+template <int CL>
+struct Plan {
+    static_assert(CL == 64 || CL == 128 || CL == 256, "chunk length");
+    static constexpr int kTilesPerChunk = CL > C ? CL / C : 1;
+    static constexpr int kSteps = CL < C ? 2 : 1;       // MMA4 steps (and read-outs) per tile
+    // Intra blocks of tile c: key tiles c - blocks(c) + 1 .. c.
+    __device__ static int blocks(int c) { return CL == 256 ? 1 + (c & 1) : 1; }
+    // Blocks of tiles 0..c-1.
+    __device__ static int blocks_before(int c) { return CL == 256 ? c + (c >> 1) : c; }
+    // Whether the state is read out after tile c (of ntiles): after every tile
+    // but the first of a pair at CL = 256, and always after the last.
+    __device__ static bool reads_after(int c, int ntiles) {
+        return CL != 256 || (c & 1) || c + 1 == ntiles;
+    }
+    // Read-outs before tile c's.
+    __device__ static int readouts_before(int c) { return CL == 256 ? (c >> 1) : kSteps * c; }
 };
 
 // ------------------------------------------------------------------ feature map
@@ -225,17 +272,17 @@ struct Work {
     size_t bh;               // (b, h)
     int seg, nseg;           // segment index, segments per sequence
     int t_begin, t_end;      // tokens [t_begin, t_end) of the sequence
-    int nchunks;
+    int ntiles;              // 128-token tiles of the segment
     bool totals;             // totals pass: state chain only, result to the workspace
     bool has_init;           // main pass, segment > 0: starts from the workspace prefix sum
     bool final_state;        // main pass, last segment: writes S and z
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this segment's total
     const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1
-    const float* gamma;      // coarse decay: gamma of this segment's chunks (index = local chunk), or nullptr
-    const float* gamma_head; // coarse decay: gamma of the sequence's chunks (index = global chunk)
-    int c0;                  // global index of this segment's first chunk
-    int seg_chunks;          // chunks per segment
+    const float* gamma;      // coarse decay: gamma of this segment's tiles (index = local tile), or nullptr
+    const float* gamma_head; // coarse decay: gamma of the sequence's tiles (index = global tile)
+    int c0;                  // global index of this segment's first tile
+    int seg_tiles;           // tiles per segment
 };
 
 struct Shared {
@@ -246,9 +293,9 @@ struct Shared {
 };
 
 // 16 bf16 values (one 16-column TMEM load) as two K-major 16-byte pieces of
-// row n of the [S|z] buffer, features 16m..16m+15.
-__device__ __forceinline__ void store_sb16(uint32_t sbase, int n, int m, const float* r) {
-    const uint32_t row = sbase + OFF_SB + (n >> 3) * SB_SBO + (n & 7) * 16;
+// row n of an [S|z] buffer (at byte offset `off`), features 16m..16m+15.
+__device__ __forceinline__ void store_sb16(uint32_t sbase, uint32_t off, int n, int m, const float* r) {
+    const uint32_t row = sbase + off + (n >> 3) * SB_SBO + (n & 7) * 16;
     st_shared_v4(row + (2 * m) * SB_LBO, pack_bf16x8(r));
     st_shared_v4(row + (2 * m + 1) * SB_LBO, pack_bf16x8(r + 8));
 }
@@ -311,10 +358,10 @@ __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase,
 }
 
 // Segment start state: row n = sum of the totals of segments 0..seg-1, placed in
-// the TMEM accumulator (fp32) and in the [S|z] buffer (bf16) for MMA3 of chunk 0.
+// the TMEM accumulator (fp32) and in the [S|z] buffer (bf16) for the first MMA3.
 // With coarse decay (DECAY), the total of segment s' (its own state, started from
-// zero) counts with the product of gamma over the chunks from segment s'+1 up to
-// and including this segment's first chunk, whose gamma scales the state it enters.
+// zero) counts with the product of gamma over the tiles from segment s'+1 up to
+// and including this segment's first tile, whose gamma scales the state it enters.
 template <bool DECAY>
 __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr, const Shared& sh) {
     const bool real = n < NV;
@@ -336,14 +383,14 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
                     r[4 * j + 3] = fmaf(ws, t.w, r[4 * j + 3]);
                 }
                 if constexpr (DECAY)
-                    for (int c = s * w.seg_chunks; c < (s + 1) * w.seg_chunks; ++c) ws *= w.gamma_head[c];
+                    for (int c = s * w.seg_tiles; c < (s + 1) * w.seg_tiles; ++c) ws *= w.gamma_head[c];
             }
         }
         uint32_t u[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(r[i]);
         tmem_st16(taddr + 16 * m, u);
-        if (real) store_sb16(sh.sbase, n, m, r);
+        if (real) store_sb16(sh.sbase, OFF_SB, n, m, r);
     }
     tmem_st_wait();
     fence_proxy_async_smem();
@@ -351,11 +398,11 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
     mbar_arrive(&sh.bars[BAR_INIT]);
 }
 
-// Totals pass with coarse decay: after MMA4 of every chunk but the last, scale the
-// state by the next chunk's gamma in tensor memory and release it (DSF) to the
+// Totals pass with coarse decay: after MMA4 of every tile but the last, scale the
+// state by the next tile's gamma in tensor memory and release it (DSF) to the
 // next MMA4; the total is then the segment's own decayed state.
 __device__ __forceinline__ bool totals_decay_steps(const Work& w, int n, uint32_t taddr, const Shared& sh) {
-    for (int c = 0; c + 1 < w.nchunks; ++c) {
+    for (int c = 0; c + 1 < w.ntiles; ++c) {
         if (!mbar_wait(&sh.bars[BAR_DS], c & 1, sh.abort_flag, sh.status)) return false;
         tc_fence_after();
         const float g = w.gamma[c + 1];
@@ -382,8 +429,8 @@ __device__ __forceinline__ bool totals_decay_steps(const Work& w, int n, uint32_
 // [S|z]^T (fp32) to this segment's slot in the workspace.
 __device__ __forceinline__ void store_total(const Work& w, int n, uint32_t taddr, const Shared& sh) {
     // Without decay the last MMA4 is the only DS commit (phase 0); with decay every
-    // chunk commits, and the last is phase (nchunks - 1) mod 2.
-    const uint32_t parity = w.gamma != nullptr ? (uint32_t)((w.nchunks - 1) & 1) : 0u;
+    // tile commits, and the last is phase (ntiles - 1) mod 2.
+    const uint32_t parity = w.gamma != nullptr ? (uint32_t)((w.ntiles - 1) & 1) : 0u;
     if (!mbar_wait(&sh.bars[BAR_DS], parity, sh.abort_flag, sh.status)) return;
     tc_fence_after();
 #pragma unroll
@@ -399,37 +446,38 @@ __device__ __forceinline__ void store_total(const Work& w, int n, uint32_t taddr
     }
 }
 
-// After MMA4 of chunk c: read the fp32 state row (two batches of 80 columns),
-// release it to MMA4 of chunk c+1, publish it as bf16 row n of the [S|z] buffer
-// for MMA3 of chunk c+1 -- or, after the last chunk, stage the final state.
+// One read-out of the state (read-out number r): read the fp32 state row (two
+// batches of 80 columns), release it to the next MMA4, and publish it as bf16
+// row n of the [S|z] buffer at `sb_off` for the next MMA3 that reads it -- or,
+// after the last tile, stage the final state. The buffer is overwritten only
+// once the MMA3 that last read it has completed (barrier `free_bar`, phase
+// `free_phase`; free_bar < 0: no MMA3 has read it yet). Keeping that order also
+// keeps the publish barrier at most one phase ahead of its waiter, since the Y
+// issuer waits for the publish before issuing the MMA3 that frees it.
 template <bool DECAY>
-__device__ __forceinline__ bool state_step(const Work& w, int c, int n, uint32_t taddr, const Shared& sh,
-                                           float* S, float* z) {
-    if (!mbar_wait(&sh.bars[BAR_DS], c & 1, sh.abort_flag, sh.status)) return false;
+__device__ __forceinline__ bool state_step(const Work& w, int r, bool last, int free_bar, uint32_t free_phase,
+                                           uint32_t sb_off, int pub_bar, int next_tile, int n, uint32_t taddr,
+                                           const Shared& sh, float* S, float* z) {
+    if (!mbar_wait(&sh.bars[BAR_DS], r & 1, sh.abort_flag, sh.status)) return false;
     tc_fence_after();
-    const bool last = c + 1 == w.nchunks;
-    // Publish for MMA3_{c+1} only once MMA3_c has completed (PQF phase c). That
-    // frees the buffer (last read by MMA3_c) and, because the Y issuer waits
-    // for SBR phase c-1 before issuing MMA3_c, keeps SBR at most one phase ahead
-    // of its waiter: a barrier two phases ahead would look unfinished to it.
-    if (!last && !mbar_wait(&sh.bars[BAR_PQF], c & 1, sh.abort_flag, sh.status)) return false;
-    // Coarse decay: chunk c+1 reads gamma_{c+1} S_c, and its state update adds to
-    // gamma_{c+1} S_c, so the state is scaled in tensor memory before MMA4_{c+1}
-    // (which waits for DSF) and published scaled.
+    if (!last && free_bar >= 0 && !mbar_wait(&sh.bars[free_bar], free_phase, sh.abort_flag, sh.status)) return false;
+    // Coarse decay (CL = 128): tile c+1 reads gamma_{c+1} S_c, and its state update
+    // adds to gamma_{c+1} S_c, so the state is scaled in tensor memory before the
+    // next MMA4 (which waits for DSF) and published scaled.
     const bool decay = DECAY && !last;
-    const float g = decay ? w.gamma[c + 1] : 1.0f;
-    float r[80];
+    const float g = decay ? w.gamma[next_tile] : 1.0f;
+    float v[80];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
 #pragma unroll
-        for (int m = 0; m < 5; ++m) tmem_ld16(taddr + 80 * half + 16 * m, r + 16 * m);
+        for (int m = 0; m < 5; ++m) tmem_ld16(taddr + 80 * half + 16 * m, v + 16 * m);
         tmem_ld_wait();
         if (decay) {                                     // compiled only into the DECAY kernel
 #pragma unroll
-            for (int i = 0; i < 80; ++i) r[i] *= g;
+            for (int i = 0; i < 80; ++i) v[i] *= g;
 #pragma unroll
             for (int m = 0; m < 5; ++m)
-                tmem_st16(taddr + 80 * half + 16 * m, reinterpret_cast<const uint32_t*>(r + 16 * m));
+                tmem_st16(taddr + 80 * half + 16 * m, reinterpret_cast<const uint32_t*>(v + 16 * m));
             if (half == 1) tmem_st_wait();
         }
         if (half == 1 && !last) {
@@ -439,7 +487,7 @@ __device__ __forceinline__ bool state_step(const Work& w, int c, int n, uint32_t
         if (n >= NV) continue;
         if (!last) {
 #pragma unroll
-            for (int m = 0; m < 5; ++m) store_sb16(sh.sbase, n, 5 * half + m, r + 16 * m);
+            for (int m = 0; m < 5; ++m) store_sb16(sh.sbase, sb_off, n, 5 * half + m, v + 16 * m);
         } else if (w.final_state && S != nullptr && n <= DV) {
             // Stage the final state for the whole-CTA write-out (write_final_state):
             // stage[f][n], rows of kStageStride floats, over the phi(K) tiles,
@@ -448,13 +496,13 @@ __device__ __forceinline__ bool state_step(const Work& w, int c, int n, uint32_t
 #pragma unroll
             for (int i = 0; i < 80; ++i) {
                 const int f = 80 * half + i;
-                if (f < DS) stage[f * kStageStride + n] = r[i];
+                if (f < DS) stage[f * kStageStride + n] = v[i];
             }
         }
     }
     if (!last) {
         fence_proxy_async_smem();
-        mbar_arrive(&sh.bars[BAR_SBR]);
+        mbar_arrive(&sh.bars[pub_bar]);
     }
     return true;
 }
@@ -485,22 +533,27 @@ __device__ __forceinline__ void load_token(Raw& r, const __nv_bfloat16* q, const
 }
 
 // ------------------------------------------------------------------ producers (warps 0-3)
+template <int CL>
 __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint32_t tmem, int warp, int tid,
                                           const __nv_bfloat16* q, const __nv_bfloat16* k,
                                           const __nv_bfloat16* v, int N) {
-    const int t = tid;                                   // token within chunk == TMEM lane
+    const int t = tid;                                   // token within the tile == TMEM lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const uint32_t cm = (t & 7) * 16;                    // row within a core matrix
     const size_t row0 = w.bh * (size_t)N;
     const bool with_q = !w.totals;
+    // CL = 64: the first MMA3 pass of a tile reads phi(Q) of rows 0-63 only, the
+    // second of rows 64-127 only; the other half's rows hold zeros.
+    const bool first_half = CL != 64 || warp < 2;
+    const uint32_t zeros[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
     Raw nxt;
     load_token(nxt, q, k, v, row0 + w.t_begin + t, w.t_begin + t < w.t_end, with_q);
-    for (int c = 0; c < w.nchunks; ++c) {
+    for (int c = 0; c < w.ntiles; ++c) {
         const int b = c & 1;
         const int tok = w.t_begin + c * C + t;
         const bool valid = tok < w.t_end;
         const Raw cur = nxt;
-        if (c + 1 < w.nchunks) load_token(nxt, q, k, v, row0 + tok + C, tok + C < w.t_end, with_q);
+        if (c + 1 < w.ntiles) load_token(nxt, q, k, v, row0 + tok + C, tok + C < w.t_end, with_q);
         if (c >= 2 && !mbar_wait(&sh.bars[BAR_FREE0 + b], ((c >> 1) - 1) & 1, sh.abort_flag, sh.status)) return;
         // [V | 1] (MN-major: a 16-byte piece is 8 columns of token t)
         const uint32_t va = sh.sbase + OFF_VA + b * VA_BYTES + cm + (t >> 3) * VA_LBO;
@@ -515,8 +568,9 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
             st_shared_v4(sh.sbase + OFF_Q + qk + QK_LBO, cur.q[1]);
             st_shared_v4(sh.sbase + OFF_K + qk, cur.k[0]);
             st_shared_v4(sh.sbase + OFF_K + qk + QK_LBO, cur.k[1]);
-            // phi(Q) goes to TMEM once MMA3 of the previous chunk has read it.
-            if (c >= 1 && !mbar_wait(&sh.bars[BAR_PQF], (c - 1) & 1, sh.abort_flag, sh.status)) return;
+            // phi(Q) goes to TMEM once the last MMA3 of the previous tile has read it.
+            const int pqf = CL == 64 ? BAR_PQF_HI : BAR_PQF;
+            if (c >= 1 && !mbar_wait(&sh.bars[pqf], (c - 1) & 1, sh.abort_flag, sh.status)) return;
             tc_fence_after();
         }
         // phi(K) (MN-major: a 16-byte piece is 8 features of token t; padded
@@ -526,7 +580,7 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 st_shared_v4(pk + (4 * g + j) * PK_SBO, make_uint4(uk[4 * j], uk[4 * j + 1], uk[4 * j + 2], uk[4 * j + 3]));
-            if (with_q) tmem_st16(lane_base + COL_PQ + 16 * g, uq);
+            if (with_q) tmem_st16(lane_base + COL_PQ + 16 * g, first_half ? uq : zeros);
         });
         fence_proxy_async_smem();
         mbar_arrive(&sh.bars[BAR_IN0 + b]);
@@ -534,25 +588,47 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&sh.bars[BAR_PQIN]);
+        if constexpr (CL == 64) {
+            // Second pass: once the MMA3 of rows 0-63 has completed, rows 64-127
+            // take their phi(Q) and rows 0-63 zeros.
+            if (!mbar_wait(&sh.bars[BAR_PQF], c & 1, sh.abort_flag, sh.status)) return;
+            tc_fence_after();
+            if (first_half) {
+#pragma unroll
+                for (int g = 0; g < KF / 32; ++g) tmem_st16(lane_base + COL_PQ + 16 * g, zeros);
+            } else {
+                emit_phi2(cur.q, 0x3F80u, cur.q, 0x3F80u, [&](int g, const uint32_t* uq, const uint32_t*) {
+                    tmem_st16(lane_base + COL_PQ + 16 * g, uq);
+                });
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sh.bars[BAR_PQIN]);
+        }
     }
 }
 
 // ------------------------------------------------------------------ intra (warps 4-7)
-// Thread = token i of the chunk = TMEM lane i; WQ = the warp's lane quadrant.
-// Row i of A in bf16, by blocks of 32 keys: blocks below the quadrant's
-// diagonal are unmasked, the diagonal block keeps keys j <= i, blocks above are
-// zero and are neither loaded nor computed. Block kb goes to the 16 TMEM
-// columns col_a(kb) of lane i; the first store waits for MMA2 of the previous
-// chunk to have read them. Arriving on BAR_A also releases s to MMA1 of the
-// next chunk.
-__device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, int lane, int c) {
+// Thread = token i of the tile = TMEM lane i; WQ = the warp's lane quadrant.
+// Row i of A in bf16, by blocks of 32 keys, for intra block number kb. `mode`:
+//   0  diagonal block: keys j <= i (blocks above the quadrant's diagonal are
+//      zero and are neither loaded nor computed);
+//   1  an earlier key tile of the same chunk: every key;
+//   2  diagonal block of a tile holding two 64-token chunks: keys j <= i of
+//      the query's own chunk (rows 64-127 drop keys 0-63).
+// Block kb goes to the 16 TMEM columns col_a(kb) of lane i; the first store
+// waits for the previous block's MMA2 to have read them. Arriving on BAR_A
+// also releases s to the next block's MMA1.
+__device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, int lane, int kb, int mode) {
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
-    if (!mbar_wait(&sh.bars[BAR_S], c & 1, sh.abort_flag, sh.status)) return false;
+    if (!mbar_wait(&sh.bars[BAR_S], kb & 1, sh.abort_flag, sh.status)) return false;
     tc_fence_after();
+    const bool full = mode == 1;
+    const int first_blk = (mode == 2 && wq >= 2) ? 2 : 0;       // key blocks below this one are another chunk's
 #pragma unroll 1
     for (int h = 0; h < 2; ++h) {
         uint32_t pw[32];                                         // keys 64h .. 64h+63, two per word
-        if (2 * h > wq) {                                        // every key of this batch is in the future
+        if ((!full && 2 * h > wq) || 2 * h + 1 < first_blk) {   // every key of this batch is masked
 #pragma unroll
             for (int p = 0; p < 32; ++p) pw[p] = 0u;
         } else {
@@ -563,7 +639,7 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
 #pragma unroll
             for (int p = 0; p < 8; ++p) {
                 const int blk = 2 * h + p / 4;                  // key block of this piece (warp-uniform)
-                if (blk > wq) {
+                if ((!full && blk > wq) || blk < first_blk) {
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) pw[4 * p + q2] = 0u;
                     continue;
@@ -575,7 +651,7 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
                     taylor_pair(sv[8 * p + 2 * q2], sv[8 * p + 2 * q2 + 1], a0, a1);
                     wd[q2] = pack_bf16x2(a0, a1);
                 }
-                if (blk == wq) {                                // diagonal block: keep keys j <= i
+                if (!full && blk == wq) {                       // diagonal block: keep keys j <= i
 #pragma unroll
                     for (int q2 = 0; q2 < 4; ++q2) {
                         const int kk = (8 * p + 2 * q2) & 31;   // key of the pair's low half, within the block
@@ -588,7 +664,7 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
         }
         if (h == 0) {
             tc_fence_before();                                  // s has been read
-            if (c > 0 && !mbar_wait(&sh.bars[BAR_AF], (c - 1) & 1, sh.abort_flag, sh.status)) return false;
+            if (kb > 0 && !mbar_wait(&sh.bars[BAR_AF], (kb - 1) & 1, sh.abort_flag, sh.status)) return false;
             tc_fence_after();
         }
         tmem_st16(lane_base + col_a(2 * h), pw);
@@ -600,17 +676,54 @@ __device__ __forceinline__ bool intra(const Shared& sh, uint32_t tmem, int wq, i
     return true;
 }
 
+// Warps 4-7 of the main pass: for every tile, its intra blocks, then (warps
+// 4-6, lanes = value columns) its state read-outs.
+template <int CL, bool DECAY>
+__device__ __forceinline__ void intra_and_state(const Work& w, const Shared& sh, uint32_t tmem, int wq, int lane,
+                                                float* S, float* z) {
+    using P = Plan<CL>;
+    const int n = wq * 32 + lane;                        // value column == TMEM lane (state role)
+    const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + COL_ST;
+    const bool state = wq < 3;
+    if (state && w.has_init) init_state<DECAY>(w, n, taddr, sh);
+    int kb = 0, r = 0;
+    for (int c = 0; c < w.ntiles; ++c) {
+        const int nb = P::blocks(c);
+        for (int j = 0; j < nb; ++j, ++kb) {
+            const int mode = CL == 64 ? 2 : (j + 1 < nb ? 1 : 0);
+            if (!intra(sh, tmem, wq, lane, kb, mode)) return;
+        }
+        if (!state) continue;
+        const bool last_tile = c + 1 == w.ntiles;
+        if constexpr (CL == 64) {
+            // After the first 64 tokens: publish into the second buffer, which the
+            // previous tile's second MMA3 read.
+            if (!state_step<DECAY>(w, r++, false, c >= 1 ? BAR_PQF_HI : -1, (c - 1) & 1, OFF_SB1, BAR_SBR1, c + 1, n,
+                                   taddr, sh, S, z))
+                return;
+            if (!state_step<DECAY>(w, r++, last_tile, BAR_PQF, c & 1, OFF_SB, BAR_SBR, c + 1, n, taddr, sh, S, z))
+                return;
+        } else {
+            if (!P::reads_after(c, w.ntiles)) continue;
+            if (!state_step<DECAY>(w, r++, last_tile, BAR_PQF, c & 1, OFF_SB, BAR_SBR, c + 1, n, taddr, sh, S, z))
+                return;
+        }
+    }
+}
+
 // ------------------------------------------------------------------ epilogue (warps 8-11)
 // Thread = token i = TMEM lane i (wq = the warp's lane quadrant). Y -> y =
 // Y[:, :64] / Y[:, 64] in bf16, into the 128-byte swizzled tile b = c & 1 (row
 // i, 16-byte piece p at slot p ^ (i & 7)), which the store thread (quadrant 0,
 // lane 0) writes out with one TMA store; rows past the end of the sequence are
 // clipped by the tensor map.
+template <int CL>
 __device__ __forceinline__ bool epilogue(const Work& w, const Shared& sh, uint32_t tmem, int c, int wq, int lane,
                                          const CUtensorMap* ty) {
     const int t = wq * 32 + lane;
     const bool store_thread = wq == 0 && lane == 0;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
+    const uint32_t ys = off_ys(CL);
     const int b = c & 1;
     if (!mbar_wait(&sh.bars[BAR_Y], c & 1, sh.abort_flag, sh.status)) return false;
     tc_fence_after();
@@ -620,15 +733,15 @@ __device__ __forceinline__ bool epilogue(const Work& w, const Shared& sh, uint32
     tmem_ld_wait();
     tc_fence_before();
     mbar_arrive(&sh.bars[BAR_YF]);
-    // The store of chunk c-1 has been issued; once it has read its tile, that
-    // tile is free for chunk c+1.
+    // The store of tile c-1 has been issued; once it has read its tile, that
+    // tile is free for tile c+1.
     if (store_thread && c >= 1) {
         bulk_wait_read_all();
         mbar_arrive(&sh.bars[BAR_YSF0 + ((c - 1) & 1)]);
     }
     if (c >= 2 && !mbar_wait(&sh.bars[BAR_YSF0 + b], ((c >> 1) - 1) & 1, sh.abort_flag, sh.status)) return false;
     const float inv = 1.0f / yv[DV];
-    const uint32_t row = sh.sbase + OFF_YS + b * YS_BYTES + t * 128;
+    const uint32_t row = sh.sbase + ys + b * YS_BYTES + t * 128;
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
         float o[8];
@@ -640,7 +753,7 @@ __device__ __forceinline__ bool epilogue(const Work& w, const Shared& sh, uint32
     mbar_arrive(&sh.bars[BAR_YSR0 + b]);
     if (store_thread) {
         if (!mbar_wait(&sh.bars[BAR_YSR0 + b], (c >> 1) & 1, sh.abort_flag, sh.status)) return false;
-        tma_store_3d(ty, sh.sbase + OFF_YS + b * YS_BYTES, 0, w.t_begin + c * C, (int)w.bh);
+        tma_store_3d(ty, sh.sbase + ys + b * YS_BYTES, 0, w.t_begin + c * C, (int)w.bh);
         bulk_commit();
     }
     return true;
@@ -655,70 +768,124 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ Y issuer (warp 13, lane 0)
+// Per tile c: MMA3 (phi(Q) against the state at its chunk's start), MMA2 of each
+// intra block (A formed from the s of that block's MMA1), MMA1 of the next
+// block. At CL = 256 the even tile's buffer is still read by the odd tile's
+// first block, so the Y issuer releases it (FREE) only after that block's MMA2.
+// At CL = 64 the tile's second MMA3 (rows 64-127, the state after its first
+// chunk) comes after MMA2.
+template <int CL>
 __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32_t tmem) {
     const uint32_t sb = sh.sbase;
     const uint64_t dq0 = smem_desc(sb + OFF_Q, QK_LBO, QK_SBO);
     const uint64_t dk0 = smem_desc(sb + OFF_K, QK_LBO, QK_SBO);
     const uint64_t dva0 = smem_desc(sb + OFF_VA, VA_LBO, VA_SBO);
     const uint64_t dsb0 = smem_desc(sb + OFF_SB, SB_LBO, SB_SBO);
+    const uint64_t dsb1 = smem_desc(sb + OFF_SB1, SB_LBO, SB_SBO);
     uint64_t* bars = sh.bars;
     uint64_t* last_bar = nullptr;
     uint32_t last_parity = 0;
+    int kb = 0;                                          // blocks issued (MMA1 commits on BAR_S)
     auto wait = [&](int bar, uint32_t parity) { return mbar_wait(&bars[bar], parity, sh.abort_flag, sh.status); };
-    auto mma1 = [&](int c) {
-        const int b = c & 1;
-        mma_bf16(tmem + COL_S, dq0 + ((b * QK_BYTES) >> 4), dk0 + ((b * QK_BYTES) >> 4), ID_QK, 0);
-        mma_commit(&bars[BAR_S]);
-        last_bar = &bars[BAR_S];
-        last_parity = c & 1;
+    auto commit = [&](int bar, uint32_t parity) {
+        mma_commit(&bars[bar]);
+        last_bar = &bars[bar];
+        last_parity = parity;
+    };
+    // s = Q_qt K_kt^T (query tile qt's buffer, key tile kt's buffer)
+    auto mma1 = [&](int qt, int kt) {
+        mma_bf16(tmem + COL_S, dq0 + (((qt & 1) * QK_BYTES) >> 4), dk0 + (((kt & 1) * QK_BYTES) >> 4), ID_QK, 0);
+        commit(BAR_S, kb & 1);
+        ++kb;
+    };
+    // Y (+)= phi(Q) [S|z] from the buffer `dsb`
+    auto mma3 = [&](uint64_t dsb, bool acc) {
+#pragma unroll
+        for (int j = 0; j < KF / 16; ++j)
+            mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j, dsb + ((j * 2 * SB_LBO) >> 4), ID_INT, (acc || j > 0) ? 1u : 0u);
+    };
+    // Y (+)= A [V_kt | 1] once A of block `blk` is formed
+    auto mma2 = [&](int blk, int kt, bool acc) {
+        if (!wait(BAR_A, blk & 1)) return false;
+        tc_fence_after();
+        const uint64_t dva = dva0 + (((kt & 1) * VA_BYTES) >> 4);
+#pragma unroll
+        for (int j = 0; j < C / 16; ++j)
+            mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
+                        (acc || j > 0) ? 1u : 0u);
+        commit(BAR_AF, blk & 1);
+        return true;
     };
     bool ok = wait(BAR_IN0, 0);
     if (ok) {
         tc_fence_after();
-        mma1(0);
+        mma1(0, 0);
     }
-    for (int c = 0; ok && c < w.nchunks; ++c) {
+    for (int c = 0; ok && c < w.ntiles; ++c) {
         const int b = c & 1;
-        const bool did3 = c > 0 || w.has_init;
-        if (!wait(BAR_PQIN, c & 1)) break;
-        if (c > 0) {
-            if (!wait(BAR_YF, (c - 1) & 1) || !wait(BAR_SBR, (c - 1) & 1)) break;
-        } else if (w.has_init && !wait(BAR_INIT, 0)) {
-            break;
+        const int blk0 = Plan<CL>::blocks_before(c);     // first block of this tile
+        if (!wait(BAR_PQIN, (CL == 64 ? 2 * c : c) & 1)) break;
+        if (c > 0 && !wait(BAR_YF, (c - 1) & 1)) break;
+        // The state MMA3 reads: the state at the tile's chunk start (CL >= 128), or
+        // before the tile (CL = 64, rows 0-63). Zero (no MMA3) at a segment's start
+        // without an initial state.
+        const int chunk_first_tile = CL == 256 ? (c & ~1) : c;
+        const bool did3 = chunk_first_tile > 0 || w.has_init;
+        if (chunk_first_tile == c) {                     // a new state to wait for
+            if (chunk_first_tile > 0) {
+                const int pub = CL == 256 ? (c >> 1) - 1 : c - 1;
+                if (!wait(BAR_SBR, pub & 1)) break;
+            } else if (w.has_init && !wait(BAR_INIT, 0)) {
+                break;
+            }
         }
         tc_fence_after();
-        // MMA3: Y = phi(Q) [S|z]_{c-1}
-        if (did3) {
-#pragma unroll
-            for (int j = 0; j < KF / 16; ++j)
-                mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j, dsb0 + ((j * 2 * SB_LBO) >> 4), ID_INT, j > 0);
+        if (did3) mma3(dsb0, false);
+        commit(BAR_PQF, c & 1);
+        if constexpr (CL == 256) {
+            if (c & 1) {
+                // block (c, c-1): the whole previous tile of the chunk, then release its buffer
+                if (!mma2(blk0, c - 1, did3)) break;
+                commit(BAR_FREE0 + (b ^ 1), 0);
+                mma1(c, c);                              // s was read when A of block (c, c-1) was formed
+                if (!mma2(blk0 + 1, c, true)) break;
+                commit(BAR_FREE0 + b, 0);
+            } else {
+                if (!mma2(blk0, c, did3)) break;
+                if (c + 1 == w.ntiles) commit(BAR_FREE0 + b, 0);   // no odd tile reads this buffer
+            }
+        } else {
+            if (!mma2(blk0, c, did3)) break;
+            commit(BAR_FREE0 + b, 0);
         }
-        mma_commit(&bars[BAR_PQF]);
-        // MMA2: Y += A [V|1], as soon as A_c is formed.
-        if (!wait(BAR_A, c & 1)) break;
-        tc_fence_after();
-        const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
-#pragma unroll
-        for (int j = 0; j < C / 16; ++j)
-            mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
-                     (did3 || j > 0) ? 1u : 0u);
-        mma_commit(&bars[BAR_FREE0 + b]);
-        mma_commit(&bars[BAR_AF]);
-        mma_commit(&bars[BAR_Y]);
-        last_bar = &bars[BAR_Y];
-        last_parity = c & 1;
-        // MMA1 of the next chunk (s was freed when A_c was formed).
-        if (c + 1 < w.nchunks) {
+        if constexpr (CL == 64) {
+            // rows 64-127: phi(Q) of the second chunk against the state after the first
+            if (!wait(BAR_PQIN, (2 * c + 1) & 1) || !wait(BAR_SBR1, c & 1)) break;
+            tc_fence_after();
+            mma3(dsb1, true);
+            commit(BAR_PQF_HI, c & 1);
+        }
+        commit(BAR_Y, c & 1);
+        // MMA1 of the next tile's first block (s was freed when the last A was formed).
+        if (c + 1 < w.ntiles) {
             if (!wait(BAR_IN0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
             tc_fence_after();
-            mma1(c + 1);
+            // CL = 256, next tile odd: its first block is against this tile's keys
+            mma1(c + 1, (CL == 256 && ((c + 1) & 1)) ? c : c + 1);
         }
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
 
 // ------------------------------------------------------------------ state issuer (warp 12, lane 0)
+// MMA4 of every tile, in Plan::kSteps steps of 128 / kSteps tokens; a DS commit
+// after every step that a read-out follows, and before the next step the wait
+// for that read-out (DSF).
+template <int CL>
 __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, uint32_t tmem) {
+    using P = Plan<CL>;
+    constexpr int kSteps = P::kSteps;
+    constexpr int kJ = C / 16 / kSteps;                  // K steps of 16 tokens per MMA4 step
     const uint32_t sb = sh.sbase;
     const uint64_t dva0 = smem_desc(sb + OFF_VA, VA_LBO, VA_SBO);    // [V|1]^T: M = column, MN-major
     const uint64_t dpk0 = smem_desc(sb + OFF_PK, PK_LBO, PK_SBO);    // phi(K): N = feature, MN-major
@@ -726,45 +893,63 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     uint64_t* last_bar = nullptr;
     uint32_t last_parity = 0;
     auto wait = [&](int bar, uint32_t parity) { return mbar_wait(&bars[bar], parity, sh.abort_flag, sh.status); };
+    // Read-outs: every step in the main pass (at CL = 256 after odd tiles and
+    // the last); in the totals pass only after the last tile, or every tile
+    // with decay (the state is rescaled per tile).
+    const bool decay_totals = w.totals && w.gamma != nullptr;
+    int r = 0;                                           // read-outs committed so far
+    bool pending = false;                                // a read-out follows the previous step
     bool ok = !w.has_init || wait(BAR_INIT, 0);
-    for (int c = 0; ok && c < w.nchunks; ++c) {
+    for (int c = 0; ok && c < w.ntiles; ++c) {
         const int b = c & 1;
         if (!wait(BAR_IN0 + b, (c >> 1) & 1)) break;
-        const bool per_chunk = !w.totals || w.gamma != nullptr;   // the state warps step every chunk
-        if (c > 0 && per_chunk && !wait(BAR_DSF, (c - 1) & 1)) break;
-        tc_fence_after();
-        const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
-        const uint64_t dpk = dpk0 + ((b * PK_BYTES) >> 4);
+        for (int h = 0; h < kSteps; ++h) {
+            if (pending && !wait(BAR_DSF, (r - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
+            const uint64_t dpk = dpk0 + ((b * PK_BYTES) >> 4);
 #pragma unroll
-        for (int j = 0; j < C / 16; ++j)
-            mma_bf16(tmem + COL_ST, dva + ((j * 2 * VA_LBO) >> 4), dpk + ((j * 2 * PK_LBO) >> 4), ID_UPD,
-                     (c > 0 || j > 0 || w.has_init) ? 1u : 0u);
-        mma_commit(&bars[BAR_FREE0 + b]);
-        last_bar = &bars[BAR_FREE0 + b];
-        last_parity = (c >> 1) & 1;
-        // Undecayed totals pass: the state is read once, after the last chunk (phase 0).
-        if (per_chunk || c + 1 == w.nchunks) {
-            mma_commit(&bars[BAR_DS]);
-            last_bar = &bars[BAR_DS];
-            last_parity = per_chunk ? (uint32_t)(c & 1) : 0u;
+            for (int jj = 0; jj < kJ; ++jj) {
+                const int j = h * kJ + jj;
+                mma_bf16(tmem + COL_ST, dva + ((j * 2 * VA_LBO) >> 4), dpk + ((j * 2 * PK_LBO) >> 4), ID_UPD,
+                         (c > 0 || j > 0 || w.has_init) ? 1u : 0u);
+            }
+            if (h + 1 == kSteps) {
+                mma_commit(&bars[BAR_FREE0 + b]);
+                last_bar = &bars[BAR_FREE0 + b];
+                last_parity = (c >> 1) & 1;
+            }
+            const bool last = c + 1 == w.ntiles && h + 1 == kSteps;
+            bool readout;
+            if (w.totals) readout = last || decay_totals;
+            else readout = CL == 64 || P::reads_after(c, w.ntiles);
+            if (readout) {
+                mma_commit(&bars[BAR_DS]);
+                last_bar = &bars[BAR_DS];
+                last_parity = (uint32_t)(w.totals && !decay_totals ? 0 : r & 1);
+                ++r;
+            }
+            pending = readout && !last && (!w.totals || decay_totals);
         }
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
 
 // mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2.
-template <bool DECAY>
+template <int CL, bool DECAY>
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
-                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_chunks, int mode,
+                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int mode,
                      int packed, float* __restrict__ ws, const float* __restrict__ gamma, unsigned* status,
                      unsigned debug) {
+    static_assert(!DECAY || CL == 128, "coarse decay is per 128-token tile, with 128-token chunks");
     extern __shared__ __align__(1024) unsigned char smem[];
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + OFF_BAR + 8 * NUM_BARS);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_BAR + 8 * NUM_BARS + 4);
+    constexpr uint32_t kOffBar = off_bar(CL);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
+    uint32_t* tmem_base_slot = reinterpret_cast<uint32_t*>(smem + kOffBar + 8 * NUM_BARS);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffBar + 8 * NUM_BARS + 4);
     const Shared sh{smem_u32(smem), bars, abort_flag, status};
 
     const int tid = threadIdx.x;
@@ -777,16 +962,16 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     w.bh = blockIdx.x / per_head;
     w.seg = blockIdx.x % per_head;
     w.nseg = nseg;
-    w.t_begin = w.seg * seg_chunks * C;
-    w.t_end = min(N, w.t_begin + seg_chunks * C);
-    w.nchunks = (w.t_end - w.t_begin + C - 1) / C;
+    w.t_begin = w.seg * seg_tiles * C;
+    w.t_end = min(N, w.t_begin + seg_tiles * C);
+    w.ntiles = (w.t_end - w.t_begin + C - 1) / C;
     w.has_init = !w.totals && w.seg > 0;
     w.final_state = !w.totals && w.seg == nseg - 1;
     w.packed = packed != 0;
     w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) + w.seg) * kTotalFloats : nullptr;
     w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
     w.c0 = w.t_begin / C;
-    w.seg_chunks = seg_chunks;
+    w.seg_tiles = seg_tiles;
     w.gamma_head = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
     w.gamma = gamma != nullptr ? w.gamma_head + w.c0 : nullptr;
 
@@ -796,7 +981,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
             if (i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A || i == BAR_YF || i == BAR_YSR0 ||
                 i == BAR_YSR1)
                 count = 128;                                 // one warpgroup
-            if (i == BAR_DSF || i == BAR_SBR || i == BAR_INIT) count = kStateLanes;
+            if (i == BAR_DSF || i == BAR_SBR || i == BAR_SBR1 || i == BAR_INIT) count = kStateLanes;
             if ((i == BAR_FREE0 || i == BAR_FREE1) && !w.totals) count = 2;   // both issuers read the buffer
             mbar_init(&bars[i], count);
         }
@@ -812,33 +997,27 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;   // testing: issue nothing, every waiter times out
 
     if (warp < 4) {
-        producers(w, sh, tmem, warp, tid, q, k, v, N);
+        producers<CL>(w, sh, tmem, warp, tid, q, k, v, N);
     } else if (warp < 8) {
         const int wq = warp & 3;
-        const int n = wq * 32 + lane;                        // value column == TMEM lane (state role)
-        const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + COL_ST;
-        const bool state = wq < 3;
         if (w.totals) {
-            if (state && (w.gamma == nullptr || totals_decay_steps(w, n, taddr, sh))) store_total(w, n, taddr, sh);
+            const int n = wq * 32 + lane;
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + COL_ST;
+            if (wq < 3 && (w.gamma == nullptr || totals_decay_steps(w, n, taddr, sh))) store_total(w, n, taddr, sh);
         } else {
-            if (state && w.has_init) init_state<DECAY>(w, n, taddr, sh);
-            bool ok = intra(sh, tmem, wq, lane, 0);
-            for (int c = 0; ok && c < w.nchunks; ++c) {
-                if (state) ok = state_step<DECAY>(w, c, n, taddr, sh, S, z);
-                if (ok && c + 1 < w.nchunks) ok = intra(sh, tmem, wq, lane, c + 1);
-            }
+            intra_and_state<CL, DECAY>(w, sh, tmem, wq, lane, S, z);
         }
     } else if (warp < 12) {
         if (!w.totals) {
             const int wq = warp & 3;
-            for (int c = 0; c < w.nchunks; ++c)
-                if (!epilogue(w, sh, tmem, c, wq, lane, &ty)) break;
+            for (int c = 0; c < w.ntiles; ++c)
+                if (!epilogue<CL>(w, sh, tmem, c, wq, lane, &ty)) break;
             if (wq == 0 && lane == 0) bulk_wait_all();      // the y stores have completed
         }
     } else if (warp == 12) {
-        if (lane == 0 && !skip_mma) state_issuer(w, sh, tmem);
+        if (lane == 0 && !skip_mma) state_issuer<CL>(w, sh, tmem);
     } else {
-        if (lane == 0 && !w.totals && !skip_mma) y_issuer(w, sh, tmem);
+        if (lane == 0 && !w.totals && !skip_mma) y_issuer<CL>(w, sh, tmem);
     }
 
     tc_fence_before();
@@ -851,54 +1030,71 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     }
 }
 
-// Segments per sequence: enough CTAs to cover the SMs once, whole chunks each.
-void plan_segments(int BH, int N, int num_sms, int* nseg, int* seg_chunks) {
-    const int nchunks = (N + C - 1) / C;
+// Segments per sequence: enough CTAs to cover the SMs once, whole chunks each
+// (tiles_per_chunk tiles of 128 tokens per chunk).
+void plan_segments(int BH, int N, int num_sms, int tiles_per_chunk, int* nseg, int* seg_tiles) {
+    const int chunk_tokens = C * tiles_per_chunk;
+    const int nchunks = (N + chunk_tokens - 1) / chunk_tokens;
     int n = 1;
     if (BH < num_sms) n = std::min(nchunks, std::max(1, num_sms / BH));
     const int per = (nchunks + n - 1) / n;
-    *seg_chunks = per;
+    *seg_tiles = per * tiles_per_chunk;
     *nseg = (nchunks + per - 1) / per;
 }
 
-}  // namespace
+int tiles_per_chunk(int chunk) { return chunk > C ? chunk / C : 1; }
 
-bool la_prefill_tc_supported(int d_feat, int d_v, int chunk) {
-    return d_feat == DF && d_v == DV && chunk == C;
-}
-
-size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms) {
-    if (!la_prefill_tc_supported(d_feat, d_v, chunk)) return 0;
-    int nseg, seg_chunks;
-    plan_segments(B * H, N, num_sms, &nseg, &seg_chunks);
-    return (size_t)B * H * (nseg - 1) * kTotalFloats * sizeof(float);
-}
-
-cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
-    if (!la_prefill_tc_supported(a.d_feat, a.d_v, a.chunk) || !a.bf16) return cudaErrorInvalidValue;
-    auto kern = a.gamma != nullptr ? la_prefill_tc_kernel<true> : la_prefill_tc_kernel<false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+template <int CL>
+cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
+    auto kern = la_prefill_tc_kernel<CL, false>;
+    if constexpr (CL == 128)
+        if (a.gamma != nullptr) kern = la_prefill_tc_kernel<128, true>;
+    constexpr uint32_t kSmem = smem_bytes(CL);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
     const int BH = a.B * a.H;
-    int nseg, seg_chunks;
-    plan_segments(BH, a.N, num_sms, &nseg, &seg_chunks);
+    int nseg, seg_tiles;
+    plan_segments(BH, a.N, num_sms, tiles_per_chunk(CL), &nseg, &seg_tiles);
     using bf = __nv_bfloat16;
     auto q = static_cast<const bf*>(a.q);
     auto k = static_cast<const bf*>(a.k);
     auto v = static_cast<const bf*>(a.v);
     auto y = static_cast<bf*>(a.y);
     float* ws = static_cast<float*>(a.workspace);
-    if (nseg > 1 && (ws == nullptr || a.ws_bytes < la_prefill_tc_workspace(a.B, a.H, a.N, a.d_feat, a.d_v, C, num_sms)))
+    if (nseg > 1 && (ws == nullptr || a.ws_bytes < la_prefill_tc_workspace(a.B, a.H, a.N, a.d_feat, a.d_v, CL, num_sms)))
         return cudaErrorInvalidValue;                    // the segment totals need their workspace
     CUtensorMap ty;
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {
-        e = launch_pdl(kern, dim3(BH * (nseg - 1)), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v,
-                       y, a.S, a.z, a.N, nseg, seg_chunks, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+        e = launch_pdl(kern, dim3(BH * (nseg - 1)), dim3(kThreads), kSmem, stream, ty, q, k, v,
+                       y, a.S, a.z, a.N, nseg, seg_tiles, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), SMEM_BYTES, stream, ty, q, k, v, y, a.S,
-                      a.z, a.N, nseg, seg_chunks, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+    return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, q, k, v, y, a.S,
+                      a.z, a.N, nseg, seg_tiles, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+}
+
+}  // namespace
+
+bool la_prefill_tc_supported(int d_feat, int d_v, int chunk) {
+    return d_feat == DF && d_v == DV && (chunk == 64 || chunk == 128 || chunk == 256);
+}
+
+size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms) {
+    if (!la_prefill_tc_supported(d_feat, d_v, chunk)) return 0;
+    int nseg, seg_tiles;
+    plan_segments(B * H, N, num_sms, tiles_per_chunk(chunk), &nseg, &seg_tiles);
+    return (size_t)B * H * (nseg - 1) * kTotalFloats * sizeof(float);
+}
+
+cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
+    if (!la_prefill_tc_supported(a.d_feat, a.d_v, a.chunk) || !a.bf16) return cudaErrorInvalidValue;
+    if (a.gamma != nullptr && a.chunk != 128) return cudaErrorInvalidValue;   // decay tiles are the 128-token chunks
+    switch (a.chunk) {
+        case 64: return launch_cl<64>(a, num_sms, stream);
+        case 256: return launch_cl<256>(a, num_sms, stream);
+        default: return launch_cl<128>(a, num_sms, stream);
+    }
 }
 
 }  // namespace based

@@ -75,6 +75,46 @@ def test_bf16_chunks_agree_with_oracle():
         _check_full(inp, torch.bfloat16, y, S, z)
 
 
+# Chunk lengths of the chunked tensor-core kernel (d'=16, dv=64, bf16): 128-token
+# MMA tiles holding two 64-token chunks, one 128-token chunk, or half of a
+# 256-token chunk.
+TC_CHUNKS = [64, 128, 256]
+
+
+@pytest.mark.parametrize("chunk", TC_CHUNKS)
+@pytest.mark.parametrize("N", [1, 7, 63, 64, 65, 127, 128, 129, 191, 255, 256, 257, 300, 513])
+def test_tc_chunks_ragged(chunk, N):
+    """Every output and the final state, for lengths that end inside a chunk,
+    on a chunk boundary, inside the second tile of a 256-token chunk and inside
+    the second half of a tile holding two 64-token chunks."""
+    inp = synthetic.la_inputs(2, 3, N, 16, 64, "bf16", seed=N + chunk)
+    y, S, z = _run_prefill(inp, chunk)
+    _check_full(inp, torch.bfloat16, y, S, z)
+
+
+@pytest.mark.parametrize("chunk", TC_CHUNKS)
+@pytest.mark.parametrize("B,H,N", [(1, 1, 300), (1, 2, 3000), (2, 3, 1000), (1, 1, 2500), (1, 1, 129)])
+def test_tc_chunks_segmented(chunk, B, H, N):
+    """Few (b, h) pairs, so sequences are split into segments of whole chunks
+    (at 256 tokens, segments whose last one has an odd number of tiles)."""
+    inp = synthetic.la_inputs(B, H, N, 16, 64, "bf16", seed=3 * N + chunk)
+    y, S, z = _run_prefill(inp, chunk)
+    _check_full(inp, torch.bfloat16, y, S, z)
+
+
+@pytest.mark.parametrize("chunk", TC_CHUNKS)
+def test_tc_chunks_repeated_calls_agree(chunk):
+    """Repeated calls complete (no expired wait) and agree bit for bit."""
+    inp = synthetic.la_inputs(3, 5, 1200, 16, 64, "bf16", seed=chunk)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y0, S0, z0 = based.la_prefill(q, k, v, chunk=chunk)
+    assert based.get_last_error() == 0
+    for _ in range(4):
+        y, S, z = based.la_prefill(q, k, v, chunk=chunk)
+        assert based.get_last_error() == 0
+        assert torch.equal(y, y0) and torch.equal(S, S0) and torch.equal(z, z0)
+
+
 def test_no_state_output():
     inp = synthetic.la_inputs(2, 2, 100, 16, 64, "bf16", seed=6)
     y, S, z = _run_prefill(inp, want_state=False)
@@ -146,15 +186,17 @@ def test_outputs_stay_in_bounds_and_deterministic():
 # ------------------------------------------------------------ full-size workloads (sampled)
 
 def _sampled_check(inp, dtype, y, S, z, heads, rows, state_heads):
+    """y of `heads` at `rows` (a list, or a function (b, h) -> rows) against the
+    oracle row by row; the final S and z of `state_heads` in full."""
     y64, S64, z64 = to64(y), to64(S), to64(z)
     for (b, h) in heads:
-        ref = oracle.la_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], rows)
-        assert_y(y64[b, h, rows], ref, dtype, f"y[{b},{h}]")
-    bs = [b for b, _ in state_heads]
-    hs = [h for _, h in state_heads]
-    ref_S, ref_z = oracle.la_state(inp.k64[bs, hs], inp.v64[bs, hs])
-    assert_state(S64[bs, hs], ref_S, dtype, "S")
-    assert_state(z64[bs, hs], ref_z, dtype, "z")
+        rr = rows(b, h) if callable(rows) else rows
+        ref = oracle.la_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], rr)
+        assert_y(y64[b, h, rr], ref, dtype, f"y[{b},{h}]")
+    for (b, h) in state_heads:                  # one head at a time: phi(K) of a long head is large
+        ref_S, ref_z = oracle.la_state(inp.k64[b, h], inp.v64[b, h])
+        assert_state(S64[b, h], ref_S, dtype, f"S[{b},{h}]")
+        assert_state(z64[b, h], ref_z, dtype, f"z[{b},{h}]")
     assert np.all(z64[..., 0] == inp.k64.shape[-2])
 
 
@@ -163,39 +205,50 @@ def _rows(N, rng, n=48):
     return sorted(set([r for r in fixed if r < N] + rng.integers(0, N, n).tolist()))
 
 
-def test_360m_prefill_sampled():
-    """B=8, H=16, N=2048, d'=16, dv=64, bf16, library's default chunk."""
+def _every_head(B, H):
+    return [(b, h) for b in range(B) for h in range(H)]
+
+
+def _head_rows(N, seed, n=16):
+    """Rows for one head: chunk, tile and segment boundaries plus n random rows.
+    Every head gets its own random rows (a boundary bug confined to some heads
+    or segments still meets a checked row)."""
+    edges = [0, 1, 63, 64, 65, 127, 128, 129, 255, 256, 257, N // 4, N // 2, 3 * N // 4, N - 2, N - 1]
+    def rows(b, h):
+        rng = np.random.default_rng(seed + 1000 * b + h)
+        return sorted(set([r for r in edges if 0 <= r < N] + rng.integers(0, N, n).tolist()))
+    return rows
+
+
+@pytest.mark.parametrize("chunk", [0, 64, 128, 256])
+def test_360m_prefill_sampled(chunk):
+    """B=8, H=16, N=2048, d'=16, dv=64, bf16: every head at 16+ rows (chunk,
+    tile and random rows of its own) and every head's final state."""
     inp = synthetic.la_inputs(8, 16, 2048, 16, 64, "bf16", seed=0)
-    y, S, z = _run_prefill(inp)
-    rng = np.random.default_rng(0)
-    heads = [(0, 0), (7, 15), (3, 9), (5, 2)]
-    _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(2048, rng),
-                   [(b, h) for b in range(8) for h in (0, 5, 11, 15)])
+    y, S, z = _run_prefill(inp, chunk)
+    _sampled_check(inp, torch.bfloat16, y, S, z, _every_head(8, 16), _head_rows(2048, 0), _every_head(8, 16))
     # all outputs finite, in a sane range (y is a convex-ish average of v)
     assert torch.isfinite(y.float()).all()
 
 
 @pytest.mark.parametrize("chunk", [0, 64, 128, 256])
 def test_long_prefill_sampled(chunk):
-    """B=2, H=16, N=16384, chunk length swept; final S and z of sampled heads checked."""
+    """B=2, H=16, N=16384, chunk length swept over 64/128/256 (each on the
+    tensor cores; none may be refused): every head at 16+ rows including
+    segment boundaries, every head's final S and z."""
     inp = synthetic.la_inputs(2, 16, 16384, 16, 64, "bf16", seed=0)
-    try:
-        y, S, z = _run_prefill(inp, chunk)
-    except based.BasedError as e:
-        assert e.status == 2, e
-        pytest.skip(f"chunk {chunk} not built for bf16")
-    rng = np.random.default_rng(1)
-    _sampled_check(inp, torch.bfloat16, y, S, z, [(0, 0), (1, 15), (1, 7)], _rows(16384, rng, 24),
-                   [(0, 0), (0, 8), (1, 3), (1, 15)])
+    y, S, z = _run_prefill(inp, chunk)
+    _sampled_check(inp, torch.bfloat16, y, S, z, _every_head(2, 16), _head_rows(16384, 1, 24),
+                   _every_head(2, 16))
 
 
 def test_large_state_prefill_sampled():
-    """d'=32 (D=1057), H=8, dv=128, B=4, N=8192, bf16."""
+    """d'=32 (D=1057), H=8, dv=128, B=4, N=8192, bf16: every head at 16+ rows,
+    the final state of eight heads."""
     inp = synthetic.la_inputs(4, 8, 8192, 32, 128, "bf16", seed=0)
     y, S, z = _run_prefill(inp)
-    rng = np.random.default_rng(2)
-    _sampled_check(inp, torch.bfloat16, y, S, z, [(0, 0), (3, 7)], _rows(8192, rng, 16),
-                   [(0, 0), (2, 5), (3, 7)])
+    _sampled_check(inp, torch.bfloat16, y, S, z, _every_head(4, 8), _head_rows(8192, 2),
+                   [(0, 0), (0, 7), (1, 3), (1, 4), (2, 5), (2, 1), (3, 6), (3, 7)])
 
 
 # ------------------------------------------------------------ decode

@@ -27,7 +27,7 @@ def _dev(inp):
 
 # (d', dv, dtype, chunk): every prefill path -- chunked tensor cores (16, 64,
 # bf16, 0), CUDA cores (explicit chunks, fp32), quadratic tensor cores (the rest).
-PATHS = [(16, 64, "bf16", 0), (16, 64, "bf16", 64), (16, 64, "f32", 0), (16, 128, "bf16", 0),
+PATHS = [(16, 64, "bf16", 0), (16, 64, "bf16", 64), (16, 64, "bf16", 256), (16, 64, "f32", 0), (16, 128, "bf16", 0),
          (32, 64, "bf16", 0), (32, 128, "bf16", 0), (32, 128, "f32", 32)]
 
 
@@ -48,11 +48,12 @@ def test_packed_prefill_state(d_feat, d_v, dtype, chunk):
     assert np.all(to64(z)[..., 0] == 200)
 
 
-def test_packed_prefill_segmented():
+@pytest.mark.parametrize("chunk", [0, 64, 256])
+def test_packed_prefill_segmented(chunk):
     """Few long sequences: the chunked tensor-core path splits them into segments."""
     inp = synthetic.la_inputs(1, 2, 3000, 16, 64, "bf16", seed=4)
     q, k, v = _dev(inp)
-    _, S, z = based.la_prefill(q, k, v, packed=True)
+    _, S, z = based.la_prefill(q, k, v, chunk=chunk, packed=True)
     assert based.get_last_error() == 0
     ref_S, ref_z = oracle.la_state_packed(inp.k64, inp.v64)
     assert_state(to64(S), ref_S, torch.bfloat16, "S packed")
