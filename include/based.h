@@ -90,19 +90,23 @@ typedef enum {
  *   chunk   tokens per chunk (on-diagonal tile): 0 (library's choice) or one
  *           of the values built for the call. BASED_BF16 at d_feat 16, d_v 64:
  *           64, 128 or 256 on the tensor cores, the chunked form with the state
- *           in tensor memory. BASED_BF16, other shapes (whose state does not
- *           fit one SM's tensor memory): 128, the quadratic masked form in
- *           128-token tiles with the final state from a separate contraction.
- *           Both dtypes: 16, 32 (and 64 at d_feat 16 for BASED_F32) on the
- *           CUDA cores in fp32 arithmetic. 0 picks 128 for bf16 and the largest
- *           CUDA-core chunk for fp32. Other values return
- *           BASED_ERR_UNSUPPORTED. The result does not depend on the chunk
- *           beyond rounding.
+ *           in tensor memory (0 picks 128). BASED_BF16, other shapes (whose
+ *           state does not fit one SM's tensor memory): any multiple of 128 on
+ *           the tensor cores; the start state of every chunk is computed first
+ *           into the workspace, then each chunk's outputs from the masked
+ *           quadratic form within the chunk plus phi(q) against that state (0
+ *           picks 1024; a chunk of at least N is the plain quadratic form and
+ *           needs no workspace). Both dtypes: 16, 32 (and 64 at d_feat 16 for
+ *           BASED_F32) on the CUDA cores in fp32 arithmetic (0 picks the
+ *           largest for fp32). Other values return BASED_ERR_UNSUPPORTED. The
+ *           result does not depend on the chunk beyond rounding.
  *   workspace, workspace_bytes
  *           device scratch of at least based_la_prefill_workspace(...) bytes
- *           (NULL allowed when that size is 0). Used to split long sequences
- *           into segments whose start states are summed from the preceding
- *           segments' totals; its contents on entry do not matter.
+ *           (NULL allowed when that size is 0). Holds the chunk start states
+ *           of the shapes whose state does not fit tensor memory (bf16, (d_feat
+ *           x d_v) x (chunks - 1) x 128-feature tiles), or the segment totals
+ *           that let long sequences of the d_feat 16, d_v 64 kernel run in
+ *           segments at once; its contents on entry do not matter.
  * Returns BASED_ERR_INVALID_ARG for null or misaligned pointers, non-positive
  * sizes, or a workspace smaller than required; BASED_ERR_UNSUPPORTED for a
  * (d_feat, d_v, dtype, chunk) combination outside the built set.

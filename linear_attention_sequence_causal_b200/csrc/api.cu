@@ -156,19 +156,26 @@ enum class LaPath { None, Simt, TensorCore, Quad };
 
 // Kernel choice for a prefill. bf16: the chunked tcgen05 kernel where it is
 // built (d' = 16, dv = 64; chunks of 64, 128 or 256 tokens, 128 by default),
-// else the tcgen05 quadratic-form kernel (128-token tiles; the state of the
-// other shapes does not fit one SM's tensor memory); other explicit chunks
-// (16, 32, and 64 for those shapes) and every fp32 call take the CUDA-core kernel.
+// else the tcgen05 chunked quadratic path (any multiple of 128 tokens,
+// kQuadDefaultChunk by default: the state of the other shapes does not fit one
+// SM's tensor memory, so chunk start states go through the workspace); other
+// explicit chunks (16, 32, and 64 for those shapes) and every fp32 call take
+// the CUDA-core kernel.
 LaPath choose_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk) {
     const bool bf16 = dtype == BASED_BF16;
     if (*chunk == 0) {
         if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, 128)) { *chunk = 128; return LaPath::TensorCore; }
-        if (bf16 && based::la_prefill_quad_supported(d_feat, d_v)) { *chunk = 128; return LaPath::Quad; }
+        if (bf16 && based::la_prefill_quad_supported(d_feat, d_v)) {
+            *chunk = based::kQuadDefaultChunk;
+            return LaPath::Quad;
+        }
         *chunk = d_feat == 16 ? 64 : 32;
         return LaPath::Simt;
     }
     if (bf16 && based::la_prefill_tc_supported(d_feat, d_v, *chunk)) return LaPath::TensorCore;
-    if (bf16 && *chunk == 128 && based::la_prefill_quad_supported(d_feat, d_v)) return LaPath::Quad;
+    if (bf16 && based::la_prefill_quad_supported(d_feat, d_v) && !based::la_prefill_tc_supported(d_feat, d_v, 128) &&
+        based::la_prefill_quad_chunk_ok(*chunk))
+        return LaPath::Quad;
     if (simt_chunk_ok(d_feat, *chunk)) return LaPath::Simt;
     return LaPath::None;
 }
@@ -213,6 +220,7 @@ size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int d_v, base
     int dev;
     if (!current_device(&dev)) return 0;
     const LaPath path = choose_la_path(d_feat, d_v, dtype, &chunk);
+    if (path == LaPath::Quad) return based::la_prefill_quad_workspace(B, H, N, d_feat, d_v, chunk);
     if (path != LaPath::TensorCore) return 0;
     return based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, num_sms(dev));
 }
@@ -245,6 +253,8 @@ based_status_t la_prefill_impl(const void* q, const void* k, const void* v, void
         if (workspace_bytes < need || (need > 0 && !ok_ptr(workspace))) return BASED_ERR_INVALID_ARG;
         e = based::launch_la_prefill_tc(a, sms, stream);
     } else if (path == LaPath::Quad) {
+        const size_t need = based::la_prefill_quad_workspace(B, H, N, d_feat, d_v, chunk);
+        if (workspace_bytes < need || (need > 0 && !ok_ptr(workspace))) return BASED_ERR_INVALID_ARG;
         e = based::launch_la_prefill_quad(a, sms, stream);
     } else {
         e = based::launch_la_prefill_simt(a, stream);

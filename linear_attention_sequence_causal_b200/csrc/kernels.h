@@ -34,10 +34,18 @@ bool la_prefill_tc_supported(int d_feat, int d_v, int chunk);
 size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms);
 cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
 
-// Tensor-core quadratic-form path (bf16, any built d', dv): y from the masked
-// quadratic form, the final state from phi(K)^T [V|1] over all tokens.
+// Tensor-core chunked path for the shapes whose state does not fit one SM's
+// tensor memory (bf16, any built d', dv): the start state of every chunk by a
+// sweep over the tokens (into the workspace), then y from the masked quadratic
+// form within each chunk plus phi(q) against its chunk's start state. chunk: a
+// multiple of 128 tokens; 0 (LaPrefillArgs) or >= N: one chunk, the plain
+// quadratic form, no workspace.
 bool la_prefill_quad_supported(int d_feat, int d_v);
+bool la_prefill_quad_chunk_ok(int chunk);
+size_t la_prefill_quad_workspace(int B, int H, int N, int d_feat, int d_v, int chunk);
 cudaError_t launch_la_prefill_quad(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
+// Chunk of the chunked quadratic path when the caller leaves the choice to the library.
+constexpr int kQuadDefaultChunk = 1024;
 
 // Backward (training) pass of the causal Taylor linear attention, bf16 tensor
 // cores: dq, dk, dv from q, k, v, the forward's y and the upstream dy.

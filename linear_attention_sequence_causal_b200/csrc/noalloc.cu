@@ -51,9 +51,16 @@ extern "C" based_status_t based_la_prefill_noalloc(const void* q, const void* k,
     const int sms = based::device_sm_count(dev);
     unsigned* status = based::device_status_word(dev);
     if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
+    const bool library_chunk = chunk == 0;
     const int path = based::resolve_la_path(d_feat, d_v, dtype, &chunk);
     if (path == 0) return BASED_ERR_UNSUPPORTED;
-    const size_t need = path == 2 ? based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms) : 0;
+    size_t need = path == 2 ? based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms)
+                : path == 3 ? based::la_prefill_quad_workspace(B, H, N, d_feat, d_v, chunk)
+                            : 0;
+    if (path == 3 && need > kScratchBytes && library_chunk) {
+        chunk = 0;          // the library's choice: one chunk (the quadratic form) needs no scratch
+        need = 0;
+    }
     if (need > kScratchBytes) return BASED_ERR_UNSUPPORTED;         // beyond the fixed scratch
     void* scratch = scratch_address(dev);
     if (scratch == nullptr) return BASED_ERR_CUDA;

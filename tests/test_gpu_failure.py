@@ -36,6 +36,21 @@ def test_stalled_la_prefill_reports_timeout(monkeypatch):
     assert_y(to64(y), oracle.la_quadratic(inp.q64, inp.k64, inp.v64), torch.bfloat16)
 
 
+def test_stalled_chunked_state_path_reports_timeout(monkeypatch):
+    """d'=32, dv=128 in 128-token chunks: the chunk start-state sweep and the
+    output kernel both stall and report; the next call is correct."""
+    import torch
+    inp = synthetic.la_inputs(1, 2, 300, 32, 128, "bf16", seed=9)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    monkeypatch.setenv("BASED_DEBUG_SKIP_MMA", "1")
+    based.la_prefill(q, k, v, chunk=128)
+    assert based.get_last_error() == TIMEOUT
+    monkeypatch.delenv("BASED_DEBUG_SKIP_MMA")
+    y, S, z = based.la_prefill(q, k, v, chunk=128)
+    assert based.get_last_error() == 0
+    assert_y(to64(y), oracle.la_quadratic(inp.q64, inp.k64, inp.v64), torch.bfloat16)
+
+
 def test_stalled_swa_prefill_reports_timeout(monkeypatch):
     import torch
     inp = synthetic.swa_inputs(1, 2, 200, 64, "bf16", seed=4)

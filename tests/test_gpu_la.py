@@ -154,6 +154,43 @@ def test_quadratic_path_many_units(d_feat, d_v):
     _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(N, rng, 24), heads)
 
 
+# Chunks of the chunked quadratic path (the shapes whose state does not fit one
+# SM's tensor memory): chunk start states go through the workspace.
+@pytest.mark.parametrize("d_feat,d_v", [(16, 128), (32, 64), (32, 128)])
+@pytest.mark.parametrize("chunk", [128, 256, 512])
+@pytest.mark.parametrize("N", [129, 300, 700, 1100])
+def test_chunked_state_path(d_feat, d_v, chunk, N):
+    """Every output and the final state; N from just past one chunk of 128 to
+    several chunks with a ragged last tile."""
+    inp = synthetic.la_inputs(1, 3, N, d_feat, d_v, "bf16", seed=N + chunk + d_feat)
+    y, S, z = _run_prefill(inp, chunk)
+    _check_full(inp, torch.bfloat16, y, S, z)
+
+
+@pytest.mark.parametrize("d_feat,d_v", [(16, 128), (32, 64), (32, 128)])
+def test_chunked_state_path_many_units(d_feat, d_v):
+    """More (query tile, head) units than SMs in 256-token chunks: units with
+    and without chunk start states, of different lengths, on every CTA; the
+    result agrees with the one-chunk quadratic form and with the oracle."""
+    B, H, N = 2, 40, 1100
+    inp = synthetic.la_inputs(B, H, N, d_feat, d_v, "bf16", seed=13)
+    y, S, z = _run_prefill(inp, 256)
+    y1, S1, z1 = _run_prefill(inp, 1152)             # one chunk: no start states
+    assert_y(to64(y), to64(y1), torch.bfloat16, "chunked vs one chunk")
+    assert_state(to64(S), to64(S1), torch.bfloat16, "S")
+    rng = np.random.default_rng(4)
+    heads = [(0, 0), (0, 17), (1, 39), (1, 2)]
+    _sampled_check(inp, torch.bfloat16, y, S, z, heads, _rows(N, rng, 24), heads)
+
+
+def test_chunked_state_path_rejects_bad_chunks():
+    inp = synthetic.la_inputs(1, 1, 300, 32, 128, "bf16", seed=1)
+    for chunk in (100, 192 + 1, -128):
+        with pytest.raises(based.BasedError) as e:
+            _run_prefill(inp, chunk)
+        assert e.value.status in (1, 2)
+
+
 def test_quadratic_path_repeated_calls_agree():
     """Two O issuers (dv = 64) hand P buffers back and forth across many steps:
     repeated calls must all complete (no expired wait) and agree bit for bit."""

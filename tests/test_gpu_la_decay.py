@@ -42,12 +42,14 @@ def test_prefill_decay(d_feat, d_v):
 
 
 def test_prefill_decay_of_one_is_the_undecayed_kernel():
-    """gamma = 1 gives weights of exactly 1: the same bits as the undecayed quadratic path."""
+    """gamma = 1 gives weights of exactly 1: the same bits as the undecayed
+    quadratic form (one chunk of at least the sequence, which the decayed path
+    of this shape always uses)."""
     inp = synthetic.la_inputs(2, 2, 700, 32, 128, "bf16", seed=9)
     q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
     ones = torch.ones((2, 2, oracle.decay_chunks(700)), dtype=torch.float32, device=DEV)
     y1, S1, z1 = based.la_prefill_decay(q, k, v, ones)
-    y0, S0, z0 = based.la_prefill(q, k, v)
+    y0, S0, z0 = based.la_prefill(q, k, v, chunk=768)
     assert based.get_last_error() == 0
     assert torch.equal(y1, y0) and torch.equal(S1, S0) and torch.equal(z1, z0)
 

@@ -28,7 +28,7 @@ def _dev(inp):
 # (d', dv, dtype, chunk): every prefill path -- chunked tensor cores (16, 64,
 # bf16, 0), CUDA cores (explicit chunks, fp32), quadratic tensor cores (the rest).
 PATHS = [(16, 64, "bf16", 0), (16, 64, "bf16", 64), (16, 64, "bf16", 256), (16, 64, "f32", 0), (16, 128, "bf16", 0),
-         (32, 64, "bf16", 0), (32, 128, "bf16", 0), (32, 128, "f32", 32)]
+         (32, 64, "bf16", 0), (32, 128, "bf16", 0), (32, 128, "bf16", 128), (32, 128, "f32", 32)]
 
 
 @pytest.mark.parametrize("d_feat,d_v,dtype,chunk", PATHS)
