@@ -444,6 +444,8 @@ def run_mine(args):
         "e2e": e2e,
         "clocks": clk,
     }
+    if not args.no_workloads:
+        result["workloads"] = run_workloads(based, dev, stream, peaks, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0:
@@ -472,7 +474,9 @@ def run_e2e(based, dev, stream, B, H, N, df, dv, Hs, ds, w, scale, chunk, y, S, 
         host[name] = t[:, :, :N].contiguous().pin_memory()
         host[name + "1"] = t[:, :, N].contiguous().pin_memory()
     dev_in = [{n: torch.empty_like(t, device=dev) for n, t in host.items()} for _ in range(2)]
-    dev_out = [{"y": y, "ys": ys, "y1": y1, "ys1": ys1}]
+    # Every result of the step's calls: y, the final state S and z (updated by the
+    # decode step), the sliding-window outputs and ring caches, the decode outputs.
+    dev_out = [{"y": y, "S": S, "z": z, "ys": ys, "kc": kc, "vc": vc, "y1": y1, "ys1": ys1}]
     dev_out.append({n: torch.empty_like(t) for n, t in dev_out[0].items()})
     host_out = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in dev_out[0].items()}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
@@ -495,10 +499,11 @@ def run_e2e(based, dev, stream, B, H, N, df, dv, Hs, ds, w, scale, chunk, y, S, 
             stream.wait_event(ev_in[b])
             if i >= 2:
                 stream.wait_event(ev_read[b])            # step i-2's outputs have been read back
-            based.la_prefill(d["q"], d["k"], d["v"], chunk=chunk, y=o["y"], S=S, z=z, workspace=ws)
-            based.swa_prefill(d["sq"], d["sk"], d["sv"], w=w, scale=scale, y=o["ys"], k_cache=kc, v_cache=vc)
-            based.la_decode_step(S, z, d["q1"], d["k1"], d["v1"], y=o["y1"])
-            based.swa_decode(kc, vc, N, d["sq1"], d["sk1"], d["sv1"], w=w, scale=scale, y=o["ys1"])
+            based.la_prefill(d["q"], d["k"], d["v"], chunk=chunk, y=o["y"], S=o["S"], z=o["z"], workspace=ws)
+            based.swa_prefill(d["sq"], d["sk"], d["sv"], w=w, scale=scale, y=o["ys"], k_cache=o["kc"],
+                              v_cache=o["vc"])
+            based.la_decode_step(o["S"], o["z"], d["q1"], d["k1"], d["v1"], y=o["y1"])
+            based.swa_decode(o["kc"], o["vc"], N, d["sq1"], d["sk1"], d["sv1"], w=w, scale=scale, y=o["ys1"])
             ev_done[b].record(stream)
         with torch.cuda.stream(down):
             down.wait_event(ev_done[b])
@@ -522,7 +527,165 @@ def run_e2e(based, dev, stream, B, H, N, df, dv, Hs, ds, w, scale, chunk, y, S, 
     ms = max_over_ranks(a.elapsed_time(b), world, dev)
     return {"value": world * (B * N + B) * steps / (ms / 1e3), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "returned": sorted(host_out),
             "overlap": "uploads and downloads of neighbouring steps on their own streams"}
+
+
+# ---------------------------------------------------------------- the other configurations
+
+def graph_time_ms(fns, reps, dev, stream):
+    """Average device time of one call of a list of calls (run in turn) captured in a
+    CUDA graph and replayed `reps` times; CUDA events on the launching stream."""
+    import torch
+    for f in fns:
+        f()
+    torch.cuda.synchronize(dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side):
+        for f in fns:
+            f()
+    stream.wait_stream(side)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    del g
+    return a.elapsed_time(b) / (reps * len(fns))
+
+
+def _frac(flops, byts, ms, peaks):
+    """Fraction of the roofline: the slower of flops at the tensor peak and bytes at the
+    HBM peak, over the measured time."""
+    return max(flops / (peaks["bf16_tflops"] * 1e12), byts / (peaks["hbm_gbs"] * 1e9)) / (ms / 1e3)
+
+
+def run_workloads(based, dev, stream, peaks, world):
+    """The other configurations of the workload list, each against its roofline:
+      decode: H=16, d'=16, dv=64 (LA) and 16 SWA heads of 64 with w=64, batch
+        1/16/64/128/256, states prefilled from a 512-token prompt; steps in a CUDA
+        graph cycling over three state sets (three batch-64 LA states are 437 MB,
+        so a step does not find the previous step's state in the 126 MB L2);
+      long prefill: B=2, H=16, N=16384, d'=16, dv=64 at chunk 64, 128 and 256;
+      large state: d'=32, dv=128, H=8, B=4, N=8192 prefill (the library's chunk),
+        then decode at batch 64 (256 steps, two state sets of 277 MB).
+    Prefill inputs are rotated over two sets (2 x 100 MB). Tokens/s are whole-job
+    (all ranks; every rank runs its own copy)."""
+    import torch
+    from linear_attention_sequence_causal_b200 import synthetic
+
+    out = {}
+    H, df, dv, Hs, ds, w = 16, 16, 64, 16, 64, 64
+    D = _feature_dim(df)
+    scale = 1.0 / math.sqrt(ds)
+    prompt, nsets, steps_per_set = 512, 3, 32
+    dec = {}
+    for batch in (1, 16, 64, 128, 256):
+        sets = []
+        for si in range(nsets):
+            q, k, v = synthetic.device_la_inputs(batch, H, prompt + steps_per_set, df, dv, dev, seed=900 + si)
+            sq, sk, sv = synthetic.device_swa_inputs(batch, Hs, prompt + steps_per_set, ds, dev, seed=950 + si)
+            _, S, z = based.la_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                                       v[:, :, :prompt].contiguous())
+            _, kc, vc = based.swa_prefill(sq[:, :, :prompt].contiguous(), sk[:, :, :prompt].contiguous(),
+                                          sv[:, :, :prompt].contiguous(), w=w, scale=scale)
+            step_in = [tuple(x[:, :, prompt + t].contiguous() for x in (q, k, v, sq, sk, sv))
+                       for t in range(steps_per_set)]
+            sets.append(dict(S=S, z=z, kc=kc, vc=vc, inp=step_in,
+                             y=torch.empty(batch, H, dv, dtype=torch.bfloat16, device=dev),
+                             ys=torch.empty(batch, Hs, ds, dtype=torch.bfloat16, device=dev)))
+            del q, k, v, sq, sk, sv
+        torch.cuda.synchronize(dev)
+
+        def la_step(st, t):
+            qi, ki, vi = st["inp"][t][:3]
+            return lambda: based.la_decode_step(st["S"], st["z"], qi, ki, vi, y=st["y"])
+
+        def swa_step(st, t):
+            qi, ki, vi = st["inp"][t][3:]
+            return lambda: based.swa_decode(st["kc"], st["vc"], prompt + t, qi, ki, vi, w=w, scale=scale, y=st["ys"])
+
+        order = [(t, si) for t in range(steps_per_set) for si in range(nsets)]
+        la_ms = graph_time_ms([la_step(sets[si], t) for t, si in order], 3, dev, stream)
+        swa_ms = graph_time_ms([swa_step(sets[si], t) for t, si in order], 3, dev, stream)
+        both = []
+        for t, si in order:
+            both += [la_step(sets[si], t), swa_step(sets[si], t)]
+        step_ms = graph_time_ms(both, 3, dev, stream) * 2        # per step of both layer types
+        lf, lb = la_decode_work(batch, H, df, dv)
+        sf, sb = swa_decode_work(batch, Hs, ds, w)
+        dec[str(batch)] = {
+            "la": {"us_per_step": round(la_ms * 1e3, 2), "tokens_per_s": world * batch / (la_ms / 1e3),
+                   "roofline_frac": round(_frac(lf, lb, la_ms, peaks), 3)},
+            "swa": {"us_per_step": round(swa_ms * 1e3, 2), "tokens_per_s": world * batch / (swa_ms / 1e3),
+                    "roofline_frac": round(_frac(sf, sb, swa_ms, peaks), 3)},
+            "based_step": {"us_per_step": round(step_ms * 1e3, 2), "tokens_per_s": world * batch / (step_ms / 1e3),
+                           "roofline_frac": round(_frac(lf + sf, lb + sb, step_ms, peaks), 3)},
+        }
+        del sets
+    out["decode"] = {"workload": f"H=16 d'=16 dv=64 LA + 16 SWA heads d=64 w=64; {prompt}-token prompt "
+                                 f"prefilled; {nsets} state sets rotated per step", "bound": "hbm",
+                     "batches": dec}
+
+    # long prefill
+    B, N = 2, 16384
+    ins = [synthetic.device_la_inputs(B, H, N, df, dv, dev, seed=30 + i) for i in range(2)]
+    y = torch.empty(B, H, N, dv, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(B, H, D, dv, device=dev)
+    z = torch.empty(B, H, D, device=dev)
+    lp = {}
+    for chunk in (64, 128, 256):
+        wsb = based.la_prefill_workspace(B, H, N, df, dv, torch.bfloat16, chunk)
+        ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+        ms = graph_time_ms([lambda qkv=qkv: based.la_prefill(*qkv, chunk=chunk, y=y, S=S, z=z, workspace=ws)
+                            for qkv in ins], 5, dev, stream)
+        fl, by = la_prefill_work(B, H, N, df, dv, chunk)
+        lp[str(chunk)] = {"us": round(ms * 1e3, 2), "tokens_per_s": world * B * N / (ms / 1e3),
+                          "TFLOP_s": round(fl / (ms / 1e3) / 1e12, 1),
+                          "roofline_frac": round(_frac(fl, by, ms, peaks), 3)}
+    out["long_prefill"] = {"workload": "B=2 H=16 N=16384 d'=16 dv=64 bf16, final S and z", "chunks": lp}
+    del ins, y, S, z
+
+    # large state
+    Bl, Hl, Nl, dfl, dvl = 4, 8, 8192, 32, 128
+    Dl = _feature_dim(dfl)
+    ins = [synthetic.device_la_inputs(Bl, Hl, Nl, dfl, dvl, dev, seed=40 + i) for i in range(2)]
+    y = torch.empty(Bl, Hl, Nl, dvl, dtype=torch.bfloat16, device=dev)
+    S = torch.empty(Bl, Hl, Dl, dvl, device=dev)
+    z = torch.empty(Bl, Hl, Dl, device=dev)
+    wsb = based.la_prefill_workspace(Bl, Hl, Nl, dfl, dvl, torch.bfloat16, 0)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev)
+    ms = graph_time_ms([lambda qkv=qkv: based.la_prefill(*qkv, y=y, S=S, z=z, workspace=ws) for qkv in ins],
+                       5, dev, stream)
+    # flops at the survey's C=64 count (the smallest of the chunk-dependent counts)
+    fl, by = la_prefill_work(Bl, Hl, Nl, dfl, dvl, 64)
+    large = {"prefill": {"us": round(ms * 1e3, 2), "tokens_per_s": world * Bl * Nl / (ms / 1e3),
+                         "TFLOP_s": round(fl / (ms / 1e3) / 1e12, 1),
+                         "roofline_frac": round(_frac(fl, by, ms, peaks), 3),
+                         "chunk": "library default (1024)", "flops_counted_at_chunk": 64}}
+    del ins, y, S, z, ws
+    lsets = []
+    for si in range(2):
+        q, k, v = synthetic.device_la_inputs(64, Hl, 512 + 8, dfl, dvl, dev, seed=60 + si)
+        _, S, z = based.la_prefill(q[:, :, :512].contiguous(), k[:, :, :512].contiguous(), v[:, :, :512].contiguous())
+        lsets.append(dict(S=S, z=z, inp=[tuple(x[:, :, 512 + t].contiguous() for x in (q, k, v)) for t in range(8)],
+                          y=torch.empty(64, Hl, dvl, dtype=torch.bfloat16, device=dev)))
+        del q, k, v
+    fns = [lambda st=lsets[t % 2], t8=(t // 2) % 8: based.la_decode_step(st["S"], st["z"], *st["inp"][t8], y=st["y"])
+           for t in range(256)]
+    ms = graph_time_ms(fns, 2, dev, stream)
+    fl, by = la_decode_work(64, Hl, dfl, dvl)
+    large["decode"] = {"batch": 64, "steps": 256, "us_per_step": round(ms * 1e3, 2),
+                       "tokens_per_s": world * 64 / (ms / 1e3), "roofline_frac": round(_frac(fl, by, ms, peaks), 3)}
+    del lsets
+    out["large_state"] = dict(workload="d'=32 dv=128 H=8: B=4 N=8192 prefill; decode batch 64, 256 steps", **large)
+    return out
 
 
 # ---------------------------------------------------------------- the CPU oracle arm
@@ -792,8 +955,10 @@ def run_sweep(reps, only=None):
     y = torch.empty(Bl, Hl, Nl, dvl, dtype=torch.bfloat16, device=dev)
     S = torch.empty(Bl, Hl, Dl, dvl, device=dev)
     z = torch.empty(Bl, Hl, Dl, device=dev)
-    ms = timed(lambda: based.la_prefill(q, k, v, y=y, S=S, z=z), 1)
-    flops, byts = la_prefill_work(Bl, Hl, Nl, dfl, dvl, 32)
+    wsl = torch.empty(max(16, based.la_prefill_workspace(Bl, Hl, Nl, dfl, dvl, torch.bfloat16, 0)),
+                      dtype=torch.uint8, device=dev)
+    ms = timed(lambda: based.la_prefill(q, k, v, y=y, S=S, z=z, workspace=wsl), 1)
+    flops, byts = la_prefill_work(Bl, Hl, Nl, dfl, dvl, 64)
     print(json.dumps({"sweep": "la_prefill_large_state", "us": ms * 1e3, "tokens_per_s": Bl * Nl / (ms / 1e3),
                       "TFLOP_s": flops / (ms / 1e3) / 1e12,
                       "tensor_frac": flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
@@ -883,6 +1048,7 @@ def main(argv=None):
     p.add_argument("--impl", choices=("mine", "reference"), default="mine")
     p.add_argument("--cpu-seconds", type=float, default=15.0, help="CPU oracle sample size")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-workloads", action="store_true", help="skip the other configurations' lines")
     p.add_argument("--preroll-s", type=float, default=1.0, help="loaded seconds before the timed region")
     p.add_argument("--profile", choices=sorted(PROFILE_CASES), help="run one kernel on its ncu capture case")
     p.add_argument("--profile-reps", type=int, default=3)

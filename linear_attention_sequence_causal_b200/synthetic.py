@@ -65,6 +65,26 @@ def swa_inputs(B, H, N, d, dtype="bf16", seed=0, qk_scale=16 ** -0.25) -> Triple
     return qkv((B, H, N, d), (B, H, N, d), qk_scale, dtype, seed)
 
 
+def device_qkv(shape_qk, shape_v, qk_scale: float, device, seed: int = 0):
+    """The same distribution as qkv (q, k ~ N(0,1)*qk_scale, v ~ N(0,1), bf16),
+    drawn on the device by a seeded torch generator: for timing-only workloads
+    too large to draw on the host in seconds. No float64 copies (not a parity case)."""
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    q = (torch.randn(shape_qk, generator=g, device=device) * qk_scale).to(torch.bfloat16)
+    k = (torch.randn(shape_qk, generator=g, device=device) * qk_scale).to(torch.bfloat16)
+    v = torch.randn(shape_v, generator=g, device=device).to(torch.bfloat16)
+    return q, k, v
+
+
+def device_la_inputs(B, H, N, d_feat, d_v, device, seed=0):
+    return device_qkv((B, H, N, d_feat), (B, H, N, d_v), d_feat ** -0.25, device, seed)
+
+
+def device_swa_inputs(B, H, N, d, device, seed=0):
+    return device_qkv((B, H, N, d), (B, H, N, d), 16 ** -0.25, device, seed)
+
+
 WORKLOADS = {
     "tiny": dict(B=1, H=1, N=256, d_feat=16, d_v=64, dtype="f32", swa_heads=1),
     "360M": dict(B=8, H=16, N=2048, d_feat=16, d_v=64, dtype="bf16", swa_heads=16),
