@@ -158,7 +158,8 @@ constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 constexpr size_t kTotalFloats = (size_t)KF * NV;
 
 enum {
-    BAR_IN0, BAR_IN1,        // producers -> issuers: Q, K, [V|1], phi(K) of a tile are in buffer b
+    BAR_QK0, BAR_QK1,        // producers -> Y issuer: Q, K, [V|1] of a tile are in buffer b
+    BAR_IN0, BAR_IN1,        // producers -> state issuer: phi(K) (and [V|1]) of a tile are in buffer b
     BAR_FREE0, BAR_FREE1,    // both issuers' commits: every MMA reading buffer b has completed
     BAR_PQIN,                // producers -> Y issuer: phi(Q) (one MMA3 pass's rows) is in TMEM
     BAR_PQF,                 // Y-issuer commit: MMA3 (CL = 64: of rows 0-63) done; phi(Q) and the [S|z] buffer it read are free
@@ -568,11 +569,15 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
             st_shared_v4(sh.sbase + OFF_Q + qk + QK_LBO, cur.q[1]);
             st_shared_v4(sh.sbase + OFF_K + qk, cur.k[0]);
             st_shared_v4(sh.sbase + OFF_K + qk + QK_LBO, cur.k[1]);
-            // phi(Q) goes to TMEM once the last MMA3 of the previous tile has read it.
-            const int pqf = CL == 64 ? BAR_PQF_HI : BAR_PQF;
-            if (c >= 1 && !mbar_wait(&sh.bars[pqf], (c - 1) & 1, sh.abort_flag, sh.status)) return;
-            tc_fence_after();
+            // Q, K and [V|1] are all the MMA1 and MMA2 of this tile read: release them
+            // now, before the wait below for the previous tile's MMA3.
+            fence_proxy_async_smem();
+            mbar_arrive(&sh.bars[BAR_QK0 + b]);
         }
+        // phi(Q) goes to TMEM once the last MMA3 of the previous tile has read it.
+        const int pqf = CL == 64 ? BAR_PQF_HI : BAR_PQF;
+        if (with_q && c >= 1 && !mbar_wait(&sh.bars[pqf], (c - 1) & 1, sh.abort_flag, sh.status)) return;
+        tc_fence_after();
         // phi(K) (MN-major: a 16-byte piece is 8 features of token t; padded
         // tokens contribute nothing) and phi(Q) (TMEM lane t), in one pass.
         const uint32_t pk = sh.sbase + OFF_PK + b * PK_BYTES + cm + (t >> 3) * PK_LBO;
@@ -768,12 +773,13 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
 }
 
 // ------------------------------------------------------------------ Y issuer (warp 13, lane 0)
-// Per tile c: MMA3 (phi(Q) against the state at its chunk's start), MMA2 of each
-// intra block (A formed from the s of that block's MMA1), MMA1 of the next
-// block. At CL = 256 the even tile's buffer is still read by the odd tile's
-// first block, so the Y issuer releases it (FREE) only after that block's MMA2.
-// At CL = 64 the tile's second MMA3 (rows 64-127, the state after its first
-// chunk) comes after MMA2.
+// Per tile c: MMA3 (phi(Q) against the state at its chunk's start), then for
+// each intra block: once its A has been formed (which frees s), MMA1 of the
+// next block -- so that the next A is formed while this block's MMA2 and the
+// next MMA3 run -- then this block's MMA2. At CL = 256 the even tile's buffer
+// is still read by the odd tile's first block, so the Y issuer releases it
+// (FREE) only after that block's MMA2. At CL = 64 the tile's second MMA3 (rows
+// 64-127, the state after its first chunk) comes after MMA2.
 template <int CL>
 __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32_t tmem) {
     const uint32_t sb = sh.sbase;
@@ -804,25 +810,26 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
         for (int j = 0; j < KF / 16; ++j)
             mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j, dsb + ((j * 2 * SB_LBO) >> 4), ID_INT, (acc || j > 0) ? 1u : 0u);
     };
-    // Y (+)= A [V_kt | 1] once A of block `blk` is formed
+    // Y (+)= A [V_kt | 1]
     auto mma2 = [&](int blk, int kt, bool acc) {
-        if (!wait(BAR_A, blk & 1)) return false;
-        tc_fence_after();
         const uint64_t dva = dva0 + (((kt & 1) * VA_BYTES) >> 4);
 #pragma unroll
         for (int j = 0; j < C / 16; ++j)
             mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
                         (acc || j > 0) ? 1u : 0u);
         commit(BAR_AF, blk & 1);
-        return true;
     };
-    bool ok = wait(BAR_IN0, 0);
+    // The first block of tile t: against t's own keys, or (CL = 256, t odd) the
+    // previous tile's.
+    auto first_kt = [](int t) { return (CL == 256 && (t & 1)) ? t - 1 : t; };
+    bool ok = wait(BAR_QK0, 0);
     if (ok) {
         tc_fence_after();
         mma1(0, 0);
     }
     for (int c = 0; ok && c < w.ntiles; ++c) {
         const int b = c & 1;
+        const int nb = Plan<CL>::blocks(c);
         const int blk0 = Plan<CL>::blocks_before(c);     // first block of this tile
         if (!wait(BAR_PQIN, (CL == 64 ? 2 * c : c) & 1)) break;
         if (c > 0 && !wait(BAR_YF, (c - 1) & 1)) break;
@@ -842,22 +849,26 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
         tc_fence_after();
         if (did3) mma3(dsb0, false);
         commit(BAR_PQF, c & 1);
-        if constexpr (CL == 256) {
-            if (c & 1) {
-                // block (c, c-1): the whole previous tile of the chunk, then release its buffer
-                if (!mma2(blk0, c - 1, did3)) break;
-                commit(BAR_FREE0 + (b ^ 1), 0);
-                mma1(c, c);                              // s was read when A of block (c, c-1) was formed
-                if (!mma2(blk0 + 1, c, true)) break;
-                commit(BAR_FREE0 + b, 0);
-            } else {
-                if (!mma2(blk0, c, did3)) break;
-                if (c + 1 == w.ntiles) commit(BAR_FREE0 + b, 0);   // no odd tile reads this buffer
+        for (int j = 0; ok && j < nb; ++j) {
+            const int blk = blk0 + j;
+            if (!wait(BAR_A, blk & 1)) { ok = false; break; }   // A formed: s has been read
+            tc_fence_after();
+            // MMA1 of the next block: the second block of this tile, or the next tile's first.
+            if (j + 1 < nb) {
+                mma1(c, c);
+            } else if (c + 1 < w.ntiles) {
+                if (!wait(BAR_QK0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) { ok = false; break; }
+                tc_fence_after();
+                mma1(c + 1, first_kt(c + 1));
             }
-        } else {
-            if (!mma2(blk0, c, did3)) break;
-            commit(BAR_FREE0 + b, 0);
+            const int kt = j == 0 ? first_kt(c) : c;
+            mma2(blk, kt, did3 || j > 0);
+            if (CL == 256 && (c & 1) && j == 0) commit(BAR_FREE0 + (b ^ 1), ((c - 1) >> 1) & 1);
         }
+        if (!ok) break;
+        // Release this tile's buffer -- at CL = 256 an even tile's only after the odd
+        // tile's first block has read it (or when no odd tile follows).
+        if (CL != 256 || (c & 1) || c + 1 == w.ntiles) commit(BAR_FREE0 + b, (c >> 1) & 1);
         if constexpr (CL == 64) {
             // rows 64-127: phi(Q) of the second chunk against the state after the first
             if (!wait(BAR_PQIN, (2 * c + 1) & 1) || !wait(BAR_SBR1, c & 1)) break;
@@ -866,13 +877,6 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
             commit(BAR_PQF_HI, c & 1);
         }
         commit(BAR_Y, c & 1);
-        // MMA1 of the next tile's first block (s was freed when the last A was formed).
-        if (c + 1 < w.ntiles) {
-            if (!wait(BAR_IN0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) break;
-            tc_fence_after();
-            // CL = 256, next tile odd: its first block is against this tile's keys
-            mma1(c + 1, (CL == 256 && ((c + 1) & 1)) ? c : c + 1);
-        }
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
@@ -978,8 +982,8 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) {
             uint32_t count = 1;
-            if (i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A || i == BAR_YF || i == BAR_YSR0 ||
-                i == BAR_YSR1)
+            if (i == BAR_QK0 || i == BAR_QK1 || i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A ||
+                i == BAR_YF || i == BAR_YSR0 || i == BAR_YSR1)
                 count = 128;                                 // one warpgroup
             if (i == BAR_DSF || i == BAR_SBR || i == BAR_SBR1 || i == BAR_INIT) count = kStateLanes;
             if ((i == BAR_FREE0 || i == BAR_FREE1) && !w.totals) count = 2;   // both issuers read the buffer
