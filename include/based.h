@@ -60,7 +60,10 @@ typedef enum {
     BASED_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size, workspace too small */
     BASED_ERR_UNSUPPORTED = 2,   /* valid but not built: d', dv, d, w, chunk or dtype outside the set */
     BASED_ERR_CUDA = 3,          /* a CUDA runtime call failed (launch, device query, sync) */
-    BASED_ERR_TIMEOUT = 4        /* a bounded wait inside a kernel expired; outputs are undefined */
+    BASED_ERR_TIMEOUT = 4,       /* a bounded wait inside a kernel expired; outputs are undefined */
+    BASED_ERR_BOUNDS = 5         /* debug library only (built with BASED_DEBUG_BOUNDS): a kernel
+                                    computed a store index outside its buffer; the store was
+                                    skipped and the outputs are undefined */
 } based_status_t;
 
 typedef enum {
@@ -377,8 +380,9 @@ BASED_API based_status_t based_baseconv_decode(void* state, const void* u_gate, 
 /*
  * based_get_last_error -- synchronises `stream`, then reports and clears the
  * device status word of the current device: BASED_ERR_TIMEOUT if a bounded
- * wait in a kernel expired since the last call, BASED_ERR_CUDA if the stream
- * reported a CUDA error, else BASED_OK.
+ * wait in a kernel expired since the last call, BASED_ERR_BOUNDS (debug
+ * library only) if a kernel's store index check failed, BASED_ERR_CUDA if the
+ * stream reported a CUDA error, else BASED_OK.
  */
 BASED_API based_status_t based_get_last_error(cudaStream_t stream);
 

@@ -211,6 +211,7 @@ const char* based_status_string(based_status_t s) {
         case BASED_ERR_UNSUPPORTED: return "BASED_ERR_UNSUPPORTED";
         case BASED_ERR_CUDA: return "BASED_ERR_CUDA";
         case BASED_ERR_TIMEOUT: return "BASED_ERR_TIMEOUT";
+        case BASED_ERR_BOUNDS: return "BASED_ERR_BOUNDS";
     }
     return "BASED_ERR_UNKNOWN";
 }
@@ -273,9 +274,10 @@ based_status_t la_decode_impl(float* S, float* z, const void* q, const void* k, 
     int dev;
     if (!current_device(&dev)) return BASED_ERR_CUDA;
     const int sms = num_sms(dev);
-    if (sms <= 0) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
     const cudaError_t e = based::launch_la_decode(S, z, q, k, v, y, gamma, B, H, d_feat, d_v, dtype == BASED_BF16,
-                                                  packed, sms, stream);
+                                                  packed, sms, status, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
@@ -432,9 +434,11 @@ based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t, const v
     if (d != 64 || w > 64 || (long long)B * H > (1LL << 30)) return BASED_ERR_UNSUPPORTED;
     int dev;
     if (!current_device(&dev)) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (status == nullptr) return BASED_ERR_CUDA;
     const bool preload = !take_ring_fresh(k_cache, dev);
     const cudaError_t e = based::launch_swa_decode(k_cache, v_cache, t, q, k, v, y, B, H, d, w, scale,
-                                                   dtype == BASED_BF16, preload, stream);
+                                                   dtype == BASED_BF16, preload, status, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
@@ -450,9 +454,10 @@ based_status_t based_baseconv_prefill(const void* u_gate, const void* u_conv, co
     int dev;
     if (!current_device(&dev)) return BASED_ERR_CUDA;
     const int sms = num_sms(dev);
-    if (sms <= 0) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (sms <= 0 || status == nullptr) return BASED_ERR_CUDA;
     const cudaError_t e = based::launch_baseconv_prefill(u_gate, u_conv, h, bias, y, state, B, N, d, K,
-                                                         dtype == BASED_BF16, sms, stream);
+                                                         dtype == BASED_BF16, sms, status, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
@@ -465,8 +470,12 @@ based_status_t based_baseconv_decode(void* state, const void* u_gate, const void
     if (B <= 0 || d <= 0 || K <= 0 || !ok_dtype(dtype)) return BASED_ERR_INVALID_ARG;
     if (d % 4 != 0 || K > based::kMaxConvTaps || (long long)B * (d / 4) > (1LL << 30))
         return BASED_ERR_UNSUPPORTED;
+    int dev;
+    if (!current_device(&dev)) return BASED_ERR_CUDA;
+    unsigned* status = status_word(dev);
+    if (status == nullptr) return BASED_ERR_CUDA;
     const cudaError_t e = based::launch_baseconv_decode(state, u_gate, u_conv, h, bias, y, B, d, K,
-                                                        dtype == BASED_BF16, stream);
+                                                        dtype == BASED_BF16, status, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 
@@ -482,7 +491,8 @@ based_status_t based_get_last_error(cudaStream_t stream) {
         const unsigned zero = 0;
         if (cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return BASED_ERR_CUDA;
     }
-    return (word & based::DEV_ERR_TIMEOUT) ? BASED_ERR_TIMEOUT : BASED_OK;
+    if (word & based::DEV_ERR_TIMEOUT) return BASED_ERR_TIMEOUT;
+    return (word & based::DEV_ERR_BOUNDS) ? BASED_ERR_BOUNDS : BASED_OK;
 }
 
 }  // extern "C"

@@ -34,6 +34,7 @@
 #include <algorithm>
 #include <atomic>
 
+#include "common.cuh"
 #include "kernels.h"
 
 namespace based {
@@ -169,7 +170,8 @@ template <int K, bool BF16, int V>
 __global__ void __launch_bounds__(kThreads, prefill_min_blocks(K, BF16, V))
 baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ conv,
                         const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
-                        void* __restrict__ state, int N, int d, int seg, int nseg, int groups, int items) {
+                        void* __restrict__ state, int N, int d, int seg, int nseg, int groups, int items,
+                        unsigned* status, size_t y_elems, size_t state_elems) {
     constexpr int S = kStages<BF16, V>;
     const int item = blockIdx.x * kThreads + threadIdx.x;
     if (item >= items) return;
@@ -242,7 +244,7 @@ baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ 
                     c = fmaf(hr[K - 1][e], x[e], c);
                     out[e] = g[e] * silu(c);
                 }
-                store<BF16, V>(y, (row0 + t) * d + c0, out);
+                if (in_bounds((row0 + t) * d + c0 + V - 1, y_elems, status)) store<BF16, V>(y, (row0 + t) * d + c0, out);
 #pragma unroll
                 for (int j = 0; j + 1 < K - 1; ++j)
 #pragma unroll
@@ -258,7 +260,9 @@ baseconv_prefill_kernel(const void* __restrict__ gate, const void* __restrict__ 
     // The window now holds tokens N-K+1 .. N-1 (zeros before token 0).
     if (state != nullptr && t1 == N) {
 #pragma unroll
-        for (int j = 0; j < K - 1; ++j) store<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, win[j]);
+        for (int j = 0; j < K - 1; ++j)
+            if (in_bounds(((size_t)b * (K - 1) + j) * d + c0 + V - 1, state_elems, status))
+                store<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, win[j]);
     }
 }
 
@@ -268,7 +272,7 @@ template <int K, bool BF16>
 __global__ void __launch_bounds__(kDecodeThreads)
 baseconv_decode_kernel(void* __restrict__ state, const void* __restrict__ gate, const void* __restrict__ conv,
                        const float* __restrict__ h, const float* __restrict__ bias, void* __restrict__ y,
-                       int d, int groups, int items) {
+                       int d, int groups, int items, unsigned* status, size_t y_elems, size_t state_elems) {
     constexpr int V = kDecodeVec;
     const int item = blockIdx.x * kDecodeThreads + threadIdx.x;
     if (item >= items) return;
@@ -295,8 +299,9 @@ baseconv_decode_kernel(void* __restrict__ state, const void* __restrict__ gate, 
         c = fmaf(hr[K - 1][e], x[e], c);
         out[e] = g[e] * silu(c);
     }
-    store<BF16, V>(y, (size_t)b * d + c0, out);
+    if (in_bounds((size_t)b * d + c0 + V - 1, y_elems, status)) store<BF16, V>(y, (size_t)b * d + c0, out);
     if constexpr (K > 1) {
+        if (!in_bounds(((size_t)b * (K - 1) + (K - 2)) * d + c0 + V - 1, state_elems, status)) return;
 #pragma unroll
         for (int j = 0; j + 1 < K - 1; ++j) store<BF16, V>(state, ((size_t)b * (K - 1) + j) * d + c0, st[j + 1]);
         store<BF16, V>(state, ((size_t)b * (K - 1) + (K - 2)) * d + c0, x);
@@ -314,7 +319,7 @@ int prefill_segment(int B, int N, int groups, long long slots) {
 
 template <int K, bool BF16, int V>
 cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
-                      void* y, void* state, int B, int N, int d, int num_sms) {
+                      void* y, void* state, int B, int N, int d, int num_sms, unsigned* status) {
     // Resident blocks per SM, a property of the compiled kernel on a device:
     // looked up once per device (the carveout attribute is set per device too).
     constexpr int kDevices = 64;
@@ -341,19 +346,21 @@ cudaError_t prefill_k(cudaStream_t st, const void* gate, const void* conv, const
     if (items > 0x7fffffffLL - kThreads) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((items + kThreads - 1) / kThreads));
     baseconv_prefill_kernel<K, BF16, V><<<grid, kThreads, 0, st>>>(gate, conv, h, bias, y, state, N, d, seg,
-                                                                    nseg, groups, (int)items);
+                                                                    nseg, groups, (int)items, status,
+                                                                    (size_t)B * N * d, (size_t)B * (K - 1) * d);
     return cudaGetLastError();
 }
 
 template <int K, bool BF16>
 cudaError_t decode_k(cudaStream_t st, void* state, const void* gate, const void* conv, const float* h,
-                     const float* bias, void* y, int B, int d) {
+                     const float* bias, void* y, int B, int d, unsigned* status) {
     const int groups = d / kDecodeVec;
     const long long items = (long long)B * groups;
     if (items > 0x7fffffffLL - kDecodeThreads) return cudaErrorInvalidValue;
     const dim3 grid((unsigned)((items + kDecodeThreads - 1) / kDecodeThreads));
     baseconv_decode_kernel<K, BF16><<<grid, kDecodeThreads, 0, st>>>(state, gate, conv, h, bias, y, d, groups,
-                                                                      (int)items);
+                                                                      (int)items, status, (size_t)B * d,
+                                                                      (size_t)B * (K - 1) * d);
     return cudaGetLastError();
 }
 
@@ -362,41 +369,42 @@ cudaError_t decode_k(cudaStream_t st, void* state, const void* gate, const void*
 // 4 channels.
 template <int K, bool BF16>
 cudaError_t prefill_v(cudaStream_t st, const void* gate, const void* conv, const float* h, const float* bias,
-                      void* y, void* state, int B, int N, int d, int num_sms) {
+                      void* y, void* state, int B, int N, int d, int num_sms, unsigned* status) {
     if constexpr (BF16 && K <= 5) {
-        if (d % 8 == 0) return prefill_k<K, true, 8>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        if (d % 8 == 0) return prefill_k<K, true, 8>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
     }
-    return prefill_k<K, BF16, 4>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+    return prefill_k<K, BF16, 4>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
 }
 
 template <bool BF16>
 cudaError_t prefill_any(int K, cudaStream_t st, const void* gate, const void* conv, const float* h,
-                        const float* bias, void* y, void* state, int B, int N, int d, int num_sms) {
+                        const float* bias, void* y, void* state, int B, int N, int d, int num_sms,
+                        unsigned* status) {
     switch (K) {
-        case 1: return prefill_v<1, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 2: return prefill_v<2, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 3: return prefill_v<3, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 4: return prefill_v<4, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 5: return prefill_v<5, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 6: return prefill_v<6, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 7: return prefill_v<7, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
-        case 8: return prefill_v<8, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms);
+        case 1: return prefill_v<1, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 2: return prefill_v<2, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 3: return prefill_v<3, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 4: return prefill_v<4, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 5: return prefill_v<5, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 6: return prefill_v<6, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 7: return prefill_v<7, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
+        case 8: return prefill_v<8, BF16>(st, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
         default: return cudaErrorInvalidValue;
     }
 }
 
 template <bool BF16>
 cudaError_t decode_any(int K, cudaStream_t st, void* state, const void* gate, const void* conv, const float* h,
-                       const float* bias, void* y, int B, int d) {
+                       const float* bias, void* y, int B, int d, unsigned* status) {
     switch (K) {
-        case 1: return decode_k<1, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 2: return decode_k<2, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 3: return decode_k<3, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 4: return decode_k<4, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 5: return decode_k<5, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 6: return decode_k<6, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 7: return decode_k<7, BF16>(st, state, gate, conv, h, bias, y, B, d);
-        case 8: return decode_k<8, BF16>(st, state, gate, conv, h, bias, y, B, d);
+        case 1: return decode_k<1, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 2: return decode_k<2, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 3: return decode_k<3, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 4: return decode_k<4, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 5: return decode_k<5, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 6: return decode_k<6, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 7: return decode_k<7, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
+        case 8: return decode_k<8, BF16>(st, state, gate, conv, h, bias, y, B, d, status);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -405,19 +413,19 @@ cudaError_t decode_any(int K, cudaStream_t st, void* state, const void* gate, co
 
 cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const float* h, const float* bias,
                                     void* y, void* state, int B, int N, int d, int K, bool bf16, int num_sms,
-                                    cudaStream_t stream) {
+                                    unsigned* status, cudaStream_t stream) {
     if (B <= 0 || N <= 0 || d <= 0 || d % 4 != 0 || K < 1 || K > kMaxConvTaps || num_sms <= 0)
         return cudaErrorInvalidValue;
-    return bf16 ? prefill_any<true>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms)
-                : prefill_any<false>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms);
+    return bf16 ? prefill_any<true>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms, status)
+                : prefill_any<false>(K, stream, gate, conv, h, bias, y, state, B, N, d, num_sms, status);
 }
 
 cudaError_t launch_baseconv_decode(void* state, const void* gate, const void* conv, const float* h,
                                    const float* bias, void* y, int B, int d, int K, bool bf16,
-                                   cudaStream_t stream) {
+                                   unsigned* status, cudaStream_t stream) {
     if (B <= 0 || d <= 0 || d % kDecodeVec != 0 || K < 1 || K > kMaxConvTaps) return cudaErrorInvalidValue;
-    return bf16 ? decode_any<true>(K, stream, state, gate, conv, h, bias, y, B, d)
-                : decode_any<false>(K, stream, state, gate, conv, h, bias, y, B, d);
+    return bf16 ? decode_any<true>(K, stream, state, gate, conv, h, bias, y, B, d, status)
+                : decode_any<false>(K, stream, state, gate, conv, h, bias, y, B, d, status);
 }
 
 }  // namespace based

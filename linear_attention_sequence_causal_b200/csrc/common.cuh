@@ -12,7 +12,25 @@ namespace based {
 // Bits of the per-device status word (read and cleared by based_get_last_error).
 enum : unsigned {
     DEV_ERR_TIMEOUT = 1u,   // a bounded wait expired
+    DEV_ERR_BOUNDS = 2u,    // debug builds: a store's index fell outside its buffer
 };
+
+// Index check of a hand-indexed global store. In a build with
+// BASED_DEBUG_BOUNDS defined (the debug library), an index outside [0, extent)
+// records DEV_ERR_BOUNDS in the status word and the store is skipped; in the
+// regular build it compiles to nothing.
+__device__ __forceinline__ bool in_bounds(size_t idx, size_t extent, unsigned* status) {
+#ifdef BASED_DEBUG_BOUNDS
+    if (idx < extent) return true;
+    if (status != nullptr) atomicOr(status, DEV_ERR_BOUNDS);
+    return false;
+#else
+    (void)idx;
+    (void)extent;
+    (void)status;
+    return true;
+#endif
+}
 
 // Inputs are read as fp32 regardless of storage type.
 __device__ __forceinline__ float to_f32(float x) { return x; }

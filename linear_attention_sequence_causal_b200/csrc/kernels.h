@@ -66,7 +66,7 @@ cudaError_t launch_la_backward(const LaBackwardArgs& a, int num_sms, cudaStream_
 // gamma: [B, H] fp32 decay applied to S, z before the token (nullptr: none).
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
                              void* y, const float* gamma, int B, int H, int d_feat, int d_v, bool bf16,
-                             bool packed, int num_sms, cudaStream_t stream);
+                             bool packed, int num_sms, unsigned* status, cudaStream_t stream);
 
 cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void* y,
                                void* k_cache, void* v_cache, int B, int H, int N, int d, int w,
@@ -83,15 +83,15 @@ cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, v
 // false when the kernel before it may have written any slot of this ring.
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q,
                               const void* k, const void* v, void* y, int B, int H, int d, int w,
-                              float scale, bool bf16, bool preload, cudaStream_t stream);
+                              float scale, bool bf16, bool preload, unsigned* status, cudaStream_t stream);
 
 // Short gated convolution: filter taps K in [1, kMaxConvTaps], d a multiple of 4.
 constexpr int kMaxConvTaps = 8;
 cudaError_t launch_baseconv_prefill(const void* gate, const void* conv, const float* h, const float* bias,
                                     void* y, void* state, int B, int N, int d, int K, bool bf16, int num_sms,
-                                    cudaStream_t stream);
+                                    unsigned* status, cudaStream_t stream);
 cudaError_t launch_baseconv_decode(void* state, const void* gate, const void* conv, const float* h,
                                    const float* bias, void* y, int B, int d, int K, bool bf16,
-                                   cudaStream_t stream);
+                                   unsigned* status, cudaStream_t stream);
 
 }  // namespace based

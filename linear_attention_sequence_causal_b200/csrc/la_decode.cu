@@ -68,7 +68,7 @@ template <typename T, int DF, int DV, bool PACKED>
 __global__ void __launch_bounds__(kThreads)
 la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restrict__ q,
                  const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y,
-                 const float* __restrict__ gamma, int P) {
+                 const float* __restrict__ gamma, int P, unsigned* status) {
     constexpr int D = PACKED ? sym_feature_dim(DF) : feature_dim(DF);
     constexpr int G = DV / 4;              // float4 column groups per row
     constexpr int RPS = kThreads / G;      // rows per sweep of the CTA
@@ -91,6 +91,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     const int r_thr = tid / G;
 
     float* Sp = S + (bh * D) * (size_t)DV + 4 * g;
+    const size_t n_heads = gridDim.x / (unsigned)P;       // extents of S, z and y for the index checks
     grid_dependency_wait();
 
     // First batch of state rows: in flight before anything else.
@@ -138,7 +139,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
         const int f = f0 + tid + i * kThreads;
         if (f < f1) {
             const float zn = fmaf(gdec, zr[i], phi(s_x[1], f));
-            zbh[f] = zn;
+            if (in_bounds(bh * D + f, n_heads * D, status)) zbh[f] = zn;
             dpart = fmaf(phi(s_x[0], f), zn, dpart);
         }
     }
@@ -152,7 +153,8 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
             if (f < f1) {
                 float4 s = make_float4(gdec * buf[u].x, gdec * buf[u].y, gdec * buf[u].z, gdec * buf[u].w);
                 fma4(s, phi(s_x[1], f), vv);
-                *reinterpret_cast<float4*>(Sp + (size_t)f * DV) = s;
+                if (in_bounds((bh * D + f) * DV + 4 * g + 3, n_heads * D * DV, status))
+                    *reinterpret_cast<float4*>(Sp + (size_t)f * DV) = s;
                 fma4(acc, phi(s_x[0], f), s);
             }
         }
@@ -201,7 +203,7 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
             num += o[tid];
             den += o[DV];
         }
-        y[bh * DV + tid] = from_f32<T>(num / den);
+        if (in_bounds(bh * DV + tid, n_heads * DV, status)) y[bh * DV + tid] = from_f32<T>(num / den);
     }
     cluster.sync();   // keep every rank's shared memory alive until rank 0 has read it
 }
@@ -219,7 +221,7 @@ int ranks_per_head(int BH, int D, int num_sms) {
 
 template <typename T, int DF, int DV, bool PACKED>
 cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const void* v, void* y,
-                         const float* gamma, int BH, int num_sms, cudaStream_t stream) {
+                         const float* gamma, int BH, int num_sms, unsigned* status, cudaStream_t stream) {
     const int P = ranks_per_head(BH, PACKED ? sym_feature_dim(DF) : feature_dim(DF), num_sms);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)BH * P);
@@ -238,16 +240,22 @@ cudaError_t launch_typed(float* S, float* z, const void* q, const void* k, const
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, la_decode_kernel<T, DF, DV, PACKED>, S, z, static_cast<const T*>(q),
-                              static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), gamma, P);
+                              static_cast<const T*>(k), static_cast<const T*>(v), static_cast<T*>(y), gamma, P,
+                              status);
 }
 
 template <typename T, bool PACKED>
 cudaError_t dispatch(float* S, float* z, const void* q, const void* k, const void* v, void* y,
-                     const float* gamma, int BH, int d_feat, int d_v, int num_sms, cudaStream_t stream) {
-    if (d_feat == 16 && d_v == 64) return launch_typed<T, 16, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
-    if (d_feat == 16 && d_v == 128) return launch_typed<T, 16, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 64) return launch_typed<T, 32, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
-    if (d_feat == 32 && d_v == 128) return launch_typed<T, 32, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, stream);
+                     const float* gamma, int BH, int d_feat, int d_v, int num_sms, unsigned* status,
+                     cudaStream_t stream) {
+    if (d_feat == 16 && d_v == 64)
+        return launch_typed<T, 16, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, status, stream);
+    if (d_feat == 16 && d_v == 128)
+        return launch_typed<T, 16, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, status, stream);
+    if (d_feat == 32 && d_v == 64)
+        return launch_typed<T, 32, 64, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, status, stream);
+    if (d_feat == 32 && d_v == 128)
+        return launch_typed<T, 32, 128, PACKED>(S, z, q, k, v, y, gamma, BH, num_sms, status, stream);
     return cudaErrorInvalidValue;
 }
 
@@ -255,13 +263,13 @@ cudaError_t dispatch(float* S, float* z, const void* q, const void* k, const voi
 
 cudaError_t launch_la_decode(float* S, float* z, const void* q, const void* k, const void* v,
                              void* y, const float* gamma, int B, int H, int d_feat, int d_v, bool bf16, bool packed,
-                             int num_sms, cudaStream_t stream) {
+                             int num_sms, unsigned* status, cudaStream_t stream) {
     const int BH = B * H;
     if (packed)
-        return bf16 ? dispatch<__nv_bfloat16, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream)
-                    : dispatch<float, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream);
-    return bf16 ? dispatch<__nv_bfloat16, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream)
-                : dispatch<float, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, stream);
+        return bf16 ? dispatch<__nv_bfloat16, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, status, stream)
+                    : dispatch<float, true>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, status, stream);
+    return bf16 ? dispatch<__nv_bfloat16, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, status, stream)
+                : dispatch<float, false>(S, z, q, k, v, y, gamma, BH, d_feat, d_v, num_sms, status, stream);
 }
 
 }  // namespace based

@@ -440,7 +440,8 @@ __device__ __forceinline__ void quad_rows(const QuadCtx& cx, uint32_t tmem, int 
                 tmem_ld16(ob + DV + 32 * h + 16, o1 + 16);
             }
             tmem_ld_wait();
-            if (tok < cx.N) {
+            const size_t y_at = ((size_t)bh * cx.N + tok) * DV + 32 * h;
+            if (tok < cx.N && in_bounds(y_at + 31, (size_t)cx.BH * cx.N * DV, cx.status)) {
 #pragma unroll
                 for (int p8 = 0; p8 < 4; ++p8) {
                     float t8[8];
@@ -734,6 +735,7 @@ la_prefix_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__
     const int f0 = ft * 128;
     const int nsteps = (N + CS - 1) / CS;
     const int nqt = (N + 127) / 128;                      // 128-token decay tiles
+    const size_t n_heads = gridDim.x / L::NFT;            // extents for the index checks
     // A chunk boundary follows step c when (c + 1) is a multiple of snap_steps
     // and another step comes after it.
     auto boundary_after = [&](int c) { return (c + 1) % snap_steps == 0 && c + 1 < nsteps; };
@@ -795,14 +797,18 @@ la_prefix_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__
                 if (!mbar_wait(&bars[SB_SNAP], snaps & 1, abort_flag, status)) { ok = false; break; }
                 tc_fence_after();
                 const int chunk = (c * CS) / (snap_steps * CS);        // the chunk that starts here
-                uint4* dst = reinterpret_cast<uint4*>(spre + (((size_t)bh * (nch - 1) + chunk - 1) * (L::NFT * 128) + f) * DV);
+                const size_t row = ((size_t)bh * (nch - 1) + chunk - 1) * (L::NFT * 128) + f;
+                const bool row_ok = in_bounds(row, n_heads * (nch - 1) * (L::NFT * 128), status);
+                uint4* dst = reinterpret_cast<uint4*>(spre + row * DV);
 #pragma unroll 1
                 for (int m = 0; m < DV / 16; ++m) {
                     float r[16];
                     tmem_ld16(taddr + 16 * m, r);
                     tmem_ld_wait();
-                    dst[2 * m] = pack_bf16x8(r);
-                    dst[2 * m + 1] = pack_bf16x8(r + 8);
+                    if (row_ok) {
+                        dst[2 * m] = pack_bf16x8(r);
+                        dst[2 * m + 1] = pack_bf16x8(r + 8);
+                    }
                 }
                 tc_fence_before();
                 mbar_arrive(&bars[SB_SNAPF]);
@@ -819,7 +825,8 @@ la_prefix_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__
 #pragma unroll
                 for (int e = 0; e < 64; ++e) zacc[e] = 0.0f;
                 const int chunk = ((c + 1) * CS) / (snap_steps * CS);
-                zpre[((size_t)bh * (nch - 1) + chunk - 1) * (L::NFT * 128) + f] = zrun;
+                const size_t at = ((size_t)bh * (nch - 1) + chunk - 1) * (L::NFT * 128) + f;
+                if (in_bounds(at, n_heads * (nch - 1) * (L::NFT * 128), status)) zpre[at] = zrun;
             }
         }
         // Epilogue: thread = feature f (TMEM lane), rows of the full or the symmetric layout.
@@ -849,7 +856,9 @@ la_prefix_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__
                 float r[16];
                 tmem_ld16(taddr + 16 * m, r);
                 tmem_ld_wait();
-                if (f >= L::DS) continue;
+                if (f >= L::DS || !in_bounds((hb * D + (r1 >= 0 ? max(r0, r1) : r0)) * DV + 16 * m + 15,
+                                             n_heads * D * DV, status))
+                    continue;
                 float4* row0 = reinterpret_cast<float4*>(S + (hb * D + r0) * DV + 16 * m);
                 float4* row1 = reinterpret_cast<float4*>(S + (hb * D + (r1 >= 0 ? r1 : r0)) * DV + 16 * m);
 #pragma unroll
@@ -860,7 +869,7 @@ la_prefix_kernel(const __grid_constant__ CUtensorMap tk, const __grid_constant__
                     if (r1 >= 0) row1[e] = val;
                 }
             }
-            if (f < L::DS) {
+            if (f < L::DS && in_bounds(hb * D + (r1 >= 0 ? max(r0, r1) : r0), n_heads * D, status)) {
                 z[hb * D + r0] = zrun * coef;
                 if (r1 >= 0) z[hb * D + r1] = zrun * coef;
             }

@@ -284,6 +284,9 @@ struct Work {
     const float* gamma_head; // coarse decay: gamma of the sequence's tiles (index = global tile)
     int c0;                  // global index of this segment's first tile
     int seg_tiles;           // tiles per segment
+    const float* ws_base;    // the workspace and its size (floats), for the index checks
+    size_t ws_floats;
+    unsigned* status;
 };
 
 struct Shared {
@@ -344,17 +347,19 @@ __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase,
     };
     const int D = w.packed ? DS : feature_dim(DF);
     float4* Sd = reinterpret_cast<float4*>(S + w.bh * D * DV);
+    const size_t n_heads = gridDim.x / w.nseg;          // extents of S and z for the index checks
     for (int idx = tid; idx < D * (DV / 4); idx += kThreads) {
         const int r = idx / (DV / 4), g = idx % (DV / 4);
         float coef = 1.0f;
         const int f = w.packed ? source_packed(r) : source(r, coef);
         const float4 x = *reinterpret_cast<const float4*>(stage + f * kStageStride + 4 * g);
-        Sd[idx] = make_float4(x.x * coef, x.y * coef, x.z * coef, x.w * coef);
+        if (in_bounds(w.bh * D * DV + 4 * (size_t)idx + 3, n_heads * D * DV, w.status))
+            Sd[idx] = make_float4(x.x * coef, x.y * coef, x.z * coef, x.w * coef);
     }
     for (int r = tid; r < D; r += kThreads) {
         float coef = 1.0f;
         const int f = w.packed ? source_packed(r) : source(r, coef);
-        z[w.bh * D + r] = stage[f * kStageStride + DV] * coef;
+        if (in_bounds(w.bh * D + r, n_heads * D, w.status)) z[w.bh * D + r] = stage[f * kStageStride + DV] * coef;
     }
 }
 
@@ -440,7 +445,9 @@ __device__ __forceinline__ void store_total(const Work& w, int n, uint32_t taddr
 #pragma unroll
         for (int m = 0; m < 5; ++m) tmem_ld16(taddr + 80 * half + 16 * m, r + 16 * m);
         tmem_ld_wait();
-        if (n >= NV) continue;
+        if (n >= NV || !in_bounds((size_t)(w.ws_out - w.ws_base) + (size_t)n * KF + 80 * half + 79, w.ws_floats,
+                                  w.status))
+            continue;
         float4* dst = reinterpret_cast<float4*>(w.ws_out + (size_t)n * KF + 80 * half);
 #pragma unroll
         for (int j = 0; j < 20; ++j) dst[j] = make_float4(r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
@@ -976,6 +983,9 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
     w.c0 = w.t_begin / C;
     w.seg_tiles = seg_tiles;
+    w.ws_base = ws;
+    w.ws_floats = (size_t)(gridDim.x / per_head) * (nseg - 1) * kTotalFloats;
+    w.status = status;
     w.gamma_head = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
     w.gamma = gamma != nullptr ? w.gamma_head + w.c0 : nullptr;
 

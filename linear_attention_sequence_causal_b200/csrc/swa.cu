@@ -135,7 +135,7 @@ template <typename T>
 __global__ void __launch_bounds__(kMaxW)
 swa_decode_kernel(T* __restrict__ kc, T* __restrict__ vc, long long t, const T* __restrict__ q,
                   const T* __restrict__ k, const T* __restrict__ v, T* __restrict__ y, int w,
-                  float scale) {
+                  float scale, unsigned* status) {
     __shared__ float s_q[kHead], s_k[kHead], s_v[kHead];
     __shared__ float s_p[kMaxW];
     __shared__ float s_red[2][2];
@@ -192,9 +192,13 @@ swa_decode_kernel(T* __restrict__ kc, T* __restrict__ vc, long long t, const T* 
             acc = fmaf(pj, vj, acc);
         }
     }
-    y[bh * kHead + tid] = from_f32<T>(acc * inv);
-    kc[(bh * w + new_slot) * kHead + tid] = knew;
-    vc[(bh * w + new_slot) * kHead + tid] = vnew;
+    const size_t n_heads = gridDim.x;                // extents of y and the ring for the index checks
+    if (in_bounds(bh * kHead + tid, n_heads * kHead, status)) y[bh * kHead + tid] = from_f32<T>(acc * inv);
+    const size_t slot_at = (bh * w + new_slot) * kHead + tid;
+    if (in_bounds(slot_at, n_heads * w * kHead, status)) {
+        kc[slot_at] = knew;
+        vc[slot_at] = vnew;
+    }
 }
 
 template <typename T>
@@ -231,7 +235,7 @@ __global__ void __launch_bounds__(128)
 swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, int new_slot,
-                       float scale, int preload) {
+                       float scale, int preload, unsigned* status) {
     __shared__ float s_sc[kMaxW];
     __shared__ float s_part[4][kHead];
     const int tid = threadIdx.x;
@@ -278,7 +282,8 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
             }
         }
     }
-    if (tid < 8) {
+    const size_t n_heads = gridDim.x;                // extents of y and the ring for the index checks
+    if (tid < 8 && in_bounds((bh * w + new_slot) * kHead + 8 * c + 7, n_heads * w * kHead, status)) {
         reinterpret_cast<uint4*>(kc + (bh * w + new_slot) * kHead)[c] = knew;
         reinterpret_cast<uint4*>(vc + (bh * w + new_slot) * kHead)[c] = vnew;
     }
@@ -350,7 +355,8 @@ swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict
         packed.y = pack2(o[2], o[3]);
         packed.z = pack2(o[4], o[5]);
         packed.w = pack2(o[6], o[7]);
-        reinterpret_cast<uint4*>(y + bh * kHead)[tid] = packed;
+        if (in_bounds(bh * kHead + 8 * tid + 7, n_heads * kHead, status))
+            reinterpret_cast<uint4*>(y + bh * kHead)[tid] = packed;
     }
 }
 
@@ -366,7 +372,7 @@ cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void
 
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
                               const void* v, void* y, int B, int H, int d, int w, float scale,
-                              bool bf16, bool preload, cudaStream_t stream) {
+                              bool bf16, bool preload, unsigned* status, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
     if (bf16) {
         // Programmatic dependent launch: a step's CTAs are scheduled while the
@@ -384,13 +390,13 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
                                            static_cast<__nv_bfloat16*>(v_cache), (long long)t,
                                            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w,
-                                           (int)(t % w), scale, preload ? 1 : 0);   // the new token's slot
+                                           (int)(t % w), scale, preload ? 1 : 0, status);   // the new token's slot
         if (e != cudaSuccess) return e;
     } else {
         swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(
             static_cast<float*>(k_cache), static_cast<float*>(v_cache), (long long)t,
             static_cast<const float*>(q), static_cast<const float*>(k), static_cast<const float*>(v),
-            static_cast<float*>(y), w, scale);
+            static_cast<float*>(y), w, scale, status);
     }
     return cudaGetLastError();
 }

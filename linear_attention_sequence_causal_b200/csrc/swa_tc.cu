@@ -251,7 +251,8 @@ __device__ __forceinline__ void softmax_wg(const Ctx& cx, uint32_t tmem, int g, 
         if (k_cache != nullptr && i0 + QT > N - w) {
             const int n = 2 * kk + g, s = n % kStages;
             if (!wait_bar(cx, BAR_FULL0 + s, (n / kStages) & 1)) return;
-            if (qi < N && qi >= N - w) {
+            if (qi < N && qi >= N - w && in_bounds(((size_t)bh * w + qi % w) * HD + HD - 1,
+                                                   (size_t)(cx.ntiles / cx.nqb) * w * HD, cx.status)) {
                 const uint32_t kr = cx.sbase + OFF_STAGE + s * STAGE_BYTES + Q_BYTES + (i + 64) * 128;
                 const uint32_t sw = (uint32_t)((i + 64) & 7);
                 uint4* kd = reinterpret_cast<uint4*>(k_cache + ((size_t)bh * w + qi % w) * HD);
@@ -303,7 +304,8 @@ __device__ __forceinline__ void softmax_wg(const Ctx& cx, uint32_t tmem, int g, 
         // w never fills (the filled slots were written before PF).
         if (k_cache != nullptr) {
             const size_t ring = (size_t)bh * w;
-            if (i0 == 0 && N + i < w) {
+            if (i0 == 0 && N + i < w &&
+                in_bounds((ring + N + i) * HD + HD - 1, (size_t)(cx.ntiles / cx.nqb) * w * HD, cx.status)) {
                 uint4* kd = reinterpret_cast<uint4*>(k_cache + (ring + N + i) * HD);
                 uint4* vd = reinterpret_cast<uint4*>(v_cache + (ring + N + i) * HD);
 #pragma unroll
