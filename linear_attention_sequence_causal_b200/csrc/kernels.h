@@ -31,7 +31,11 @@ cudaError_t launch_la_prefill_simt(const LaPrefillArgs& a, cudaStream_t stream);
 
 // Tensor-core (tcgen05/TMEM) path: bf16 inputs, d' = 16, dv = 64, chunk = 128.
 bool la_prefill_tc_supported(int d_feat, int d_v, int chunk);
+// Workspace for the segment totals: the size that lets the totals pass split
+// every total into the pieces that fill the SMs best, and the least it can run
+// with (one piece per total); the launcher splits as finely as ws_bytes allows.
 size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms);
+size_t la_prefill_tc_workspace_min(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms);
 cudaError_t launch_la_prefill_tc(const LaPrefillArgs& a, int num_sms, cudaStream_t stream);
 
 // Tensor-core chunked path for the shapes whose state does not fit one SM's

@@ -278,8 +278,10 @@ struct Work {
     bool has_init;           // main pass, segment > 0: starts from the workspace prefix sum
     bool final_state;        // main pass, last segment: writes S and z
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
-    float* ws_out;           // totals pass: this segment's total
-    const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1
+    float* ws_out;           // totals pass: this part's total
+    const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1 (parts each)
+    int parts;               // totals per segment (each segment's total is split into parts)
+    int sub_tiles;           // tiles per part (the last part of a segment may have fewer)
     const float* gamma;      // coarse decay: gamma of this segment's tiles (index = local tile), or nullptr
     const float* gamma_head; // coarse decay: gamma of the sequence's tiles (index = global tile)
     int c0;                  // global index of this segment's first tile
@@ -363,11 +365,12 @@ __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase,
     }
 }
 
-// Segment start state: row n = sum of the totals of segments 0..seg-1, placed in
-// the TMEM accumulator (fp32) and in the [S|z] buffer (bf16) for the first MMA3.
-// With coarse decay (DECAY), the total of segment s' (its own state, started from
-// zero) counts with the product of gamma over the tiles from segment s'+1 up to
-// and including this segment's first tile, whose gamma scales the state it enters.
+// Segment start state: row n = sum of the totals of segments 0..seg-1 (each
+// segment's total in `parts` pieces of consecutive tiles), placed in the TMEM
+// accumulator (fp32) and in the [S|z] buffer (bf16) for the first MMA3. With
+// coarse decay (DECAY), the total of a piece (its own state, started from zero)
+// counts with the product of gamma over the tiles after it up to and including
+// this segment's first tile, whose gamma scales the state it enters.
 template <bool DECAY>
 __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr, const Shared& sh) {
     const bool real = n < NV;
@@ -377,9 +380,9 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
 #pragma unroll
         for (int i = 0; i < 16; ++i) r[i] = 0.f;
         if (real) {
-            float ws = DECAY ? w.gamma_head[w.c0] : 1.0f;   // weight of segment s, nearest first
-            for (int s = w.seg - 1; s >= 0; --s) {
-                const float4* src = reinterpret_cast<const float4*>(w.ws_in + s * kTotalFloats + (size_t)n * KF + 16 * m);
+            float ws = DECAY ? w.gamma_head[w.c0] : 1.0f;   // weight of part j, nearest first
+            for (int j = w.seg * w.parts - 1; j >= 0; --j) {
+                const float4* src = reinterpret_cast<const float4*>(w.ws_in + j * kTotalFloats + (size_t)n * KF + 16 * m);
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
                     const float4 t = __ldg(src + j);
@@ -388,8 +391,12 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
                     r[4 * j + 2] = fmaf(ws, t.z, r[4 * j + 2]);
                     r[4 * j + 3] = fmaf(ws, t.w, r[4 * j + 3]);
                 }
-                if constexpr (DECAY)
-                    for (int c = s * w.seg_tiles; c < (s + 1) * w.seg_tiles; ++c) ws *= w.gamma_head[c];
+                if constexpr (DECAY) {
+                    const int s = j / w.parts, p = j % w.parts;
+                    const int c_lo = s * w.seg_tiles + p * w.sub_tiles;
+                    const int c_hi = s * w.seg_tiles + min((p + 1) * w.sub_tiles, w.seg_tiles);
+                    for (int c = c_lo; c < c_hi; ++c) ws *= w.gamma_head[c];
+                }
             }
         }
         uint32_t u[16];
@@ -946,13 +953,14 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
 
-// mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2.
+// mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2,
+// each split into `parts` pieces of at most sub_tiles = ceil(seg_tiles / parts) tiles.
 template <int CL, bool DECAY>
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
                      const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                      const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
-                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int mode,
+                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int parts, int mode,
                      int packed, float* __restrict__ ws, const float* __restrict__ gamma, unsigned* status,
                      unsigned debug) {
     static_assert(!DECAY || CL == 128, "coarse decay is per 128-token tile, with 128-token chunks");
@@ -969,22 +977,31 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
 
     Work w;
     w.totals = mode == 1;
-    const int per_head = w.totals ? nseg - 1 : nseg;
+    w.parts = parts;
+    w.sub_tiles = (seg_tiles + parts - 1) / parts;
+    const int per_head = w.totals ? (nseg - 1) * parts : nseg;
     w.bh = blockIdx.x / per_head;
-    w.seg = blockIdx.x % per_head;
+    const int j = blockIdx.x % per_head;
+    w.seg = w.totals ? j / parts : j;
     w.nseg = nseg;
-    w.t_begin = w.seg * seg_tiles * C;
-    w.t_end = min(N, w.t_begin + seg_tiles * C);
+    if (w.totals) {                                      // part j % parts of segment seg
+        const int p = j % parts;
+        w.t_begin = (w.seg * seg_tiles + p * w.sub_tiles) * C;
+        w.t_end = min(N, (w.seg * seg_tiles + min((p + 1) * w.sub_tiles, seg_tiles)) * C);
+    } else {
+        w.t_begin = w.seg * seg_tiles * C;
+        w.t_end = min(N, w.t_begin + seg_tiles * C);
+    }
     w.ntiles = (w.t_end - w.t_begin + C - 1) / C;
     w.has_init = !w.totals && w.seg > 0;
     w.final_state = !w.totals && w.seg == nseg - 1;
     w.packed = packed != 0;
-    w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) + w.seg) * kTotalFloats : nullptr;
-    w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * kTotalFloats : nullptr;
+    w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) * parts + j) * kTotalFloats : nullptr;
+    w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * parts * kTotalFloats : nullptr;
     w.c0 = w.t_begin / C;
     w.seg_tiles = seg_tiles;
     w.ws_base = ws;
-    w.ws_floats = (size_t)(gridDim.x / per_head) * (nseg - 1) * kTotalFloats;
+    w.ws_floats = (size_t)(gridDim.x / per_head) * (nseg - 1) * parts * kTotalFloats;
     w.status = status;
     w.gamma_head = gamma != nullptr ? gamma + w.bh * (size_t)((N + C - 1) / C) : nullptr;
     w.gamma = gamma != nullptr ? w.gamma_head + w.c0 : nullptr;
@@ -1058,6 +1075,30 @@ void plan_segments(int BH, int N, int num_sms, int tiles_per_chunk, int* nseg, i
 
 int tiles_per_chunk(int chunk) { return chunk > C ? chunk / C : 1; }
 
+// Pieces per segment total in the totals pass: the most even use of the SMs.
+// A total splits into `parts` pieces of consecutive tiles (each its own CTA);
+// the pass takes about ceil(CTAs / SMs) rounds of (tiles per piece + ~2 tiles of
+// start-up and store). Only splits whose totals fit `ws_cap` bytes, and whose
+// last piece is not empty, are considered.
+int plan_parts(int BH, int nseg, int seg_tiles, int num_sms, size_t ws_cap) {
+    if (nseg <= 1) return 1;
+    const long long units = (long long)BH * (nseg - 1);
+    int best = 1;
+    double best_cost = 1e30;
+    for (int p = 1; p <= std::min(seg_tiles, 16); ++p) {
+        const int sub = (seg_tiles + p - 1) / p;
+        if ((p - 1) * sub >= seg_tiles) continue;
+        if ((size_t)units * p * kTotalFloats * sizeof(float) > ws_cap) break;
+        const long long waves = (units * p + num_sms - 1) / num_sms;
+        const double cost = (double)waves * (sub + 2.0);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
+            best = p;
+        }
+    }
+    return best;
+}
+
 template <int CL>
 cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
     auto kern = la_prefill_tc_kernel<CL, false>;
@@ -1075,17 +1116,22 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
     auto v = static_cast<const bf*>(a.v);
     auto y = static_cast<bf*>(a.y);
     float* ws = static_cast<float*>(a.workspace);
-    if (nseg > 1 && (ws == nullptr || a.ws_bytes < la_prefill_tc_workspace(a.B, a.H, a.N, a.d_feat, a.d_v, CL, num_sms)))
+    // Split the totals as finely as helps and as the given workspace holds (the
+    // workspace query sizes it for the best split; a smaller one, as the
+    // allocation-free entry point has, takes fewer pieces).
+    const int parts = plan_parts(BH, nseg, seg_tiles, num_sms, a.ws_bytes);
+    if (nseg > 1 && (ws == nullptr || a.ws_bytes < (size_t)BH * (nseg - 1) * parts * kTotalFloats * sizeof(float)))
         return cudaErrorInvalidValue;                    // the segment totals need their workspace
     CUtensorMap ty;
     if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
     if (nseg > 1) {
-        e = launch_pdl(kern, dim3(BH * (nseg - 1)), dim3(kThreads), kSmem, stream, ty, q, k, v,
-                       y, a.S, a.z, a.N, nseg, seg_tiles, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+        e = launch_pdl(kern, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, q, k, v,
+                       y, a.S, a.z, a.N, nseg, seg_tiles, parts, 1, a.packed ? 1 : 0, ws, a.gamma, a.status,
+                       a.debug);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, q, k, v, y, a.S,
-                      a.z, a.N, nseg, seg_tiles, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+                      a.z, a.N, nseg, seg_tiles, parts, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
 }
 
 }  // namespace
@@ -1095,6 +1141,14 @@ bool la_prefill_tc_supported(int d_feat, int d_v, int chunk) {
 }
 
 size_t la_prefill_tc_workspace(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms) {
+    if (!la_prefill_tc_supported(d_feat, d_v, chunk)) return 0;
+    int nseg, seg_tiles;
+    plan_segments(B * H, N, num_sms, tiles_per_chunk(chunk), &nseg, &seg_tiles);
+    const int parts = plan_parts(B * H, nseg, seg_tiles, num_sms, ~(size_t)0);
+    return (size_t)B * H * (nseg - 1) * parts * kTotalFloats * sizeof(float);
+}
+
+size_t la_prefill_tc_workspace_min(int B, int H, int N, int d_feat, int d_v, int chunk, int num_sms) {
     if (!la_prefill_tc_supported(d_feat, d_v, chunk)) return 0;
     int nseg, seg_tiles;
     plan_segments(B * H, N, num_sms, tiles_per_chunk(chunk), &nseg, &seg_tiles);

@@ -16,9 +16,11 @@ int resolve_la_path(int d_feat, int d_v, based_dtype_t dtype, int* chunk);   // 
 
 namespace {
 
-// Largest scratch the prefill can need: segment totals of at most one CTA per
-// SM (148 x 160 x 80 fp32 = 7.6 MB on a B200), rounded up to 8 MiB. Every GPU
-// that loads the library holds this array until the process exits.
+// Largest scratch the prefill needs at the least: segment totals of at most one
+// CTA per SM (148 x 160 x 80 fp32 = 7.6 MB on a B200), rounded up to 8 MiB. (The
+// chunked kernel splits each total into pieces when its scratch has room for
+// them; with this array it takes as many as fit.) Every GPU that loads the
+// library holds this array until the process exits.
 constexpr size_t kScratchBytes = size_t(8) << 20;
 static __device__ __align__(256) unsigned char g_prefill_scratch[kScratchBytes];
 
@@ -54,7 +56,7 @@ extern "C" based_status_t based_la_prefill_noalloc(const void* q, const void* k,
     const bool library_chunk = chunk == 0;
     const int path = based::resolve_la_path(d_feat, d_v, dtype, &chunk);
     if (path == 0) return BASED_ERR_UNSUPPORTED;
-    size_t need = path == 2 ? based::la_prefill_tc_workspace(B, H, N, d_feat, d_v, chunk, sms)
+    size_t need = path == 2 ? based::la_prefill_tc_workspace_min(B, H, N, d_feat, d_v, chunk, sms)
                 : path == 3 ? based::la_prefill_quad_workspace(B, H, N, d_feat, d_v, chunk)
                             : 0;
     if (path == 3 && need > kScratchBytes && library_chunk) {

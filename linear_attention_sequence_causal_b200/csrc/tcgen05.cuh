@@ -300,6 +300,13 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
+// Prefetch `bytes` (a multiple of 16) of global memory from `src` (16-byte
+// aligned) into L2, with no completion to wait for.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
+                 : "memory");
+}
+
 // Prefetch the 3-D tile at (x, y, z) of a tensor map into L2 (no shared
 // memory, no completion to wait for): later TMA loads of it hit L2.
 __device__ __forceinline__ void tma_prefetch_3d(const void* tmap, int x, int y, int z) {
