@@ -56,12 +56,18 @@
 // phi(Q)) in tensor memory matters: an MMA of N = 80 with both operands in
 // shared memory is bound by shared-memory bandwidth (6.5 KB per 40 tensor cycles).
 //
-// Other roles (448 threads, one CTA per (b, h, segment)); a warp reaches the
+// Other roles (480 threads, one CTA per (b, h, segment)); a warp reaches the
 // TMEM lanes of quadrant (warp mod 4):
-//   warps 0-3   producers: thread t loads token t of tile c+1 (prefetched in
-//               registers a tile ahead) and writes Q, K, [V|1] and phi(K) into
-//               the free half of the double-buffered shared-memory tiles, then
-//               phi(Q) into TMEM once MMA3 has consumed the previous one.
+//   warp 14     input loader: TMA loads of the Q, K and V tiles into a ring of
+//               stages, in the layouts the MMAs read (Q, K rows of 32 bytes
+//               under the 32-byte swizzle; V rows of 128 bytes under the
+//               128-byte swizzle, with a constant ones block as the second
+//               atom that makes it [V | 1]), a stage at a time as the MMAs
+//               reading it complete.
+//   warps 0-3   producers: thread t reads q_t and k_t from the landed stage
+//               and writes phi(K) into the free one of two shared-memory
+//               tiles, and phi(Q) into TMEM once MMA3 has consumed the
+//               previous one.
 //   warps 4-7   intra + state: turn s into A (TMEM lane = token); warps 4-6
 //               also read the fp32 state after MMA4 (lane = value column,
 //               0..79) and publish it as the bf16 B operand of the next MMA3,
@@ -77,9 +83,9 @@
 // workspace; the main launch then starts segment s from the sum of the totals
 // of segments 0..s-1, so all segments of a sequence run at once.
 //
-// Shared-memory operands use the canonical no-swizzle layouts (8-row x 16-byte
-// core matrices, each a contiguous 128-byte block); each thread writes whole
-// 16-byte rows of core matrices, so eight consecutive threads fill one block.
+// phi(K) and the bf16 state use the canonical no-swizzle layouts (8-row x
+// 16-byte core matrices, each a contiguous 128-byte block); each thread writes
+// whole 16-byte rows of core matrices, so eight consecutive threads fill one block.
 #include <algorithm>
 
 #include "common.cuh"
@@ -98,39 +104,44 @@ constexpr int C = 128;           // tokens per tile (the M of every MMA)
 constexpr int DS = 153;          // distinct (symmetric) features
 constexpr int KF = 160;          // DS padded to the MMA K step
 constexpr int NV = 80;           // [V | 1] padded to the MMA N step
-constexpr int kThreads = 448;
+constexpr int kThreads = 480;
 constexpr int kStateLanes = 96;  // warps 4-6 read state lanes 0..95 (0..79 hold data)
 
 // ------------------------------------------------------------------ shared memory
-// [b] tiles are double-buffered by tile parity.
-constexpr uint32_t PK_BYTES = C * KF * 2;       // phi(K): K = token, N = feature, MN-major
-constexpr uint32_t VA_BYTES = C * NV * 2;       // [V|1]:  K = token, N = column, MN-major
-constexpr uint32_t QK_BYTES = C * DF * 2;       // Q, K:   M/N = token, K = d', K-major
-constexpr uint32_t SB_BYTES = KF * NV * 2;      // [S|z] bf16: N = column, K = feature, K-major
-constexpr uint32_t OFF_PK = 0;
-constexpr uint32_t OFF_VA = OFF_PK + 2 * PK_BYTES;
-constexpr uint32_t OFF_Q = OFF_VA + 2 * VA_BYTES;
-constexpr uint32_t OFF_K = OFF_Q + 2 * QK_BYTES;
+// phi(K) tiles are double-buffered by tile parity; the inputs Q, K, V arrive by
+// TMA in a ring of stages(CL) stages, in the layouts the MMAs read directly.
+__host__ __device__ constexpr int stages(int cl) { return cl == 64 ? 2 : 3; }
+constexpr uint32_t PK_BYTES = C * KF * 2;       // phi(K): K = token, N = feature, MN-major (no swizzle)
+constexpr uint32_t V_BYTES = C * DV * 2;        // V: rows = tokens of 64 values (128 B), 128-byte swizzle
+constexpr uint32_t QK_BYTES = C * DF * 2;       // Q, K: rows = tokens of d' values (32 B), 32-byte swizzle
+constexpr uint32_t SB_BYTES = KF * NV * 2;      // [S|z] bf16: N = column, K = feature, K-major (no swizzle)
 constexpr uint32_t YS_BYTES = C * DV * 2;       // y tile, 128-byte swizzled rows (TMA store source)
-constexpr uint32_t OFF_SB = OFF_K + 2 * QK_BYTES;               // [S|z] of the state before the tile
+constexpr uint32_t QK_SBO = 8 * DF * 2;         // 8-row atoms of the 32-byte swizzle
+constexpr uint32_t OFF_PK = 0;                                  // [2]
+constexpr uint32_t OFF_SB = OFF_PK + 2 * PK_BYTES;              // [S|z] of the state before the tile
 constexpr uint32_t OFF_SB1 = OFF_SB + SB_BYTES;                 // CL = 64: the state after its first chunk
-// The rest depends on whether the second [S|z] buffer is used (CL = 64).
-__host__ __device__ constexpr uint32_t off_ys(int cl) {       // [2], 1024-aligned for the swizzle
-    return ((cl == 64 ? OFF_SB1 + SB_BYTES : OFF_SB + SB_BYTES) + 1023) & ~1023u;
+// The rest depends on the chunk length (a second [S|z] buffer and two input
+// stages at CL = 64, three stages otherwise). The 128-byte swizzled tiles start
+// on 1024-byte boundaries, the 32-byte swizzled ones on 256-byte boundaries.
+__host__ __device__ constexpr uint32_t off_v(int cl) { return OFF_SB + (cl == 64 ? 2 : 1) * SB_BYTES; }
+// The ones block: V's second 64-column atom (column 64 = 1, the rest 0, for
+// every token), shared by all stages. With it, a V stage read as an operand of
+// N (or M) > 64 is [V | 1 | 0...]: the descriptor's atom stride points here.
+__host__ __device__ constexpr uint32_t off_ones(int cl) { return off_v(cl) + stages(cl) * V_BYTES; }
+__host__ __device__ constexpr uint32_t off_q(int cl) { return off_ones(cl) + V_BYTES; }
+__host__ __device__ constexpr uint32_t off_k(int cl) { return off_q(cl) + stages(cl) * QK_BYTES; }
+__host__ __device__ constexpr uint32_t off_ys(int cl) {        // [2], 1024-aligned for the swizzle
+    return (off_k(cl) + stages(cl) * QK_BYTES + 1023) & ~1023u;
 }
 __host__ __device__ constexpr uint32_t off_bar(int cl) { return off_ys(cl) + 2 * YS_BYTES; }
 __host__ __device__ constexpr uint32_t smem_bytes(int cl) { return off_bar(cl) + 256; }
 static_assert(smem_bytes(64) <= 227 * 1024 && smem_bytes(128) <= 227 * 1024, "shared memory");
+static_assert(off_v(64) % 1024 == 0 && off_v(128) % 1024 == 0 && off_q(64) % 256 == 0 && off_q(128) % 256 == 0,
+              "swizzled tiles aligned");
 
-// Core-matrix strides (bytes): LBO along K, SBO along M/N.
+// Core-matrix strides (bytes) of the no-swizzle operands: LBO along K, SBO along M/N.
 constexpr uint32_t PK_LBO = (KF / 8) * 128, PK_SBO = 128;
-constexpr uint32_t VA_LBO = (NV / 8) * 128, VA_SBO = 128;
-constexpr uint32_t QK_LBO = 128, QK_SBO = (DF / 8) * 128;
 constexpr uint32_t SB_LBO = 128, SB_SBO = (KF / 8) * 128;
-// MMA4 reads [V|1]^T as a 128-row A operand: rows 80..127 (never-read output
-// lanes) alias the next 768 bytes, which must lie inside the allocation.
-static_assert(OFF_VA + VA_BYTES + (C / 8 - 1) * VA_LBO + 15 * VA_SBO + 128 <= OFF_Q + 2 * QK_BYTES,
-              "MMA4 A-operand rows past [V|1] stay inside shared memory");
 
 // ------------------------------------------------------------------ tensor memory
 // Every region starts on a multiple of 32 columns (an accumulator at an
@@ -150,7 +161,7 @@ static_assert(COL_Y + NV + 16 <= COL_PQ && COL_PQ + KF / 2 + 16 <= COL_ST && COL
               "A columns");
 
 constexpr uint32_t ID_QK = idesc_bf16_f32(128, C, false, false);
-constexpr uint32_t ID_AV = idesc_bf16_f32(128, NV, false, true);   // A in TMEM, [V|1] MN-major
+constexpr uint32_t ID_AV = idesc_bf16_f32(128, NV, false, true);   // A in TMEM, [V|1] MN-major (V stage + ones)
 constexpr uint32_t ID_INT = idesc_bf16_f32(128, NV, false, false);
 constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 
@@ -158,9 +169,10 @@ constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 constexpr size_t kTotalFloats = (size_t)KF * NV;
 
 enum {
-    BAR_QK0, BAR_QK1,        // producers -> Y issuer: Q, K, [V|1] of a tile are in buffer b
-    BAR_IN0, BAR_IN1,        // producers -> state issuer: phi(K) (and [V|1]) of a tile are in buffer b
-    BAR_FREE0, BAR_FREE1,    // both issuers' commits: every MMA reading buffer b has completed
+    BAR_RF0, BAR_RF1, BAR_RF2,   // TMA: Q, K, V of a tile landed in input stage s
+    BAR_RE0, BAR_RE1, BAR_RE2,   // both issuers' commits: every MMA reading input stage s has completed
+    BAR_PKF0, BAR_PKF1,          // state-issuer commit: MMA4 has read phi(K) buffer b
+    BAR_IN0, BAR_IN1,            // producers -> state issuer: phi(K) of a tile is in buffer b
     BAR_PQIN,                // producers -> Y issuer: phi(Q) (one MMA3 pass's rows) is in TMEM
     BAR_PQF,                 // Y-issuer commit: MMA3 (CL = 64: of rows 0-63) done; phi(Q) and the [S|z] buffer it read are free
     BAR_PQF_HI,              // CL = 64: the same for the MMA3 of rows 64-127
@@ -188,7 +200,6 @@ static_assert(8 * NUM_BARS + 8 <= 256, "barrier area");
 template <int CL>
 struct Plan {
     static_assert(CL == 64 || CL == 128 || CL == 256, "chunk length");
-    static constexpr int kTilesPerChunk = CL > C ? CL / C : 1;
     static constexpr int kSteps = CL < C ? 2 : 1;       // MMA4 steps (and read-outs) per tile
     // Intra blocks of tile c: key tiles c - blocks(c) + 1 .. c.
     __device__ static int blocks(int c) { return CL == 256 ? 1 + (c & 1) : 1; }
@@ -384,12 +395,12 @@ __device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr,
             for (int j = w.seg * w.parts - 1; j >= 0; --j) {
                 const float4* src = reinterpret_cast<const float4*>(w.ws_in + j * kTotalFloats + (size_t)n * KF + 16 * m);
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const float4 t = __ldg(src + j);
-                    r[4 * j] = fmaf(ws, t.x, r[4 * j]);
-                    r[4 * j + 1] = fmaf(ws, t.y, r[4 * j + 1]);
-                    r[4 * j + 2] = fmaf(ws, t.z, r[4 * j + 2]);
-                    r[4 * j + 3] = fmaf(ws, t.w, r[4 * j + 3]);
+                for (int i = 0; i < 4; ++i) {
+                    const float4 t = __ldg(src + i);
+                    r[4 * i] = fmaf(ws, t.x, r[4 * i]);
+                    r[4 * i + 1] = fmaf(ws, t.y, r[4 * i + 1]);
+                    r[4 * i + 2] = fmaf(ws, t.z, r[4 * i + 2]);
+                    r[4 * i + 3] = fmaf(ws, t.w, r[4 * i + 3]);
                 }
                 if constexpr (DECAY) {
                     const int s = j / w.parts, p = j % w.parts;
@@ -522,80 +533,45 @@ __device__ __forceinline__ bool state_step(const Work& w, int r, bool last, int 
     return true;
 }
 
-struct Raw {          // one token's inputs: q, k (2 x 16 B each), v (8 x 16 B)
-    uint4 q[2], k[2], v[8];
-};
-
-__device__ __forceinline__ void load_token(Raw& r, const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                           const __nv_bfloat16* v, size_t row, bool valid, bool with_qk) {
-    if (valid) {
-        const uint4* qp = reinterpret_cast<const uint4*>(q + row * DF);
-        const uint4* kp = reinterpret_cast<const uint4*>(k + row * DF);
-        const uint4* vp = reinterpret_cast<const uint4*>(v + row * DV);
-        if (with_qk) {
-            r.q[0] = __ldg(qp); r.q[1] = __ldg(qp + 1);
-        } else {
-            r.q[0] = r.q[1] = make_uint4(0, 0, 0, 0);
-        }
-        r.k[0] = __ldg(kp); r.k[1] = __ldg(kp + 1);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) r.v[i] = __ldg(vp + i);
-    } else {
-        r.q[0] = r.q[1] = r.k[0] = r.k[1] = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) r.v[i] = make_uint4(0, 0, 0, 0);
-    }
+// ------------------------------------------------------------------ producers (warps 0-3)
+// Row t of a Q or K stage (32-byte swizzle: the two 16-byte halves of row t
+// swap places when bit 2 of t is set).
+__device__ __forceinline__ void ld_row32(uint32_t tile, int t, uint4* x) {
+    const uint32_t sw = ((t >> 2) & 1) << 4;
+    x[0] = ld_shared_v4(tile + t * 32 + sw);
+    x[1] = ld_shared_v4(tile + t * 32 + (16 ^ sw));
 }
 
-// ------------------------------------------------------------------ producers (warps 0-3)
+// Thread t = token t of the tile = TMEM lane t. Once the tile's inputs have
+// landed (stage s), form phi(k_t) into phi(K) buffer b and phi(q_t) into TMEM.
 template <int CL>
-__device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint32_t tmem, int warp, int tid,
-                                          const __nv_bfloat16* q, const __nv_bfloat16* k,
-                                          const __nv_bfloat16* v, int N) {
-    const int t = tid;                                   // token within the tile == TMEM lane
+__device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint32_t tmem, int warp, int tid) {
+    constexpr int KS = stages(CL);
+    const int t = tid;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const uint32_t cm = (t & 7) * 16;                    // row within a core matrix
-    const size_t row0 = w.bh * (size_t)N;
     const bool with_q = !w.totals;
     // CL = 64: the first MMA3 pass of a tile reads phi(Q) of rows 0-63 only, the
     // second of rows 64-127 only; the other half's rows hold zeros.
     const bool first_half = CL != 64 || warp < 2;
     const uint32_t zeros[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-    Raw nxt;
-    load_token(nxt, q, k, v, row0 + w.t_begin + t, w.t_begin + t < w.t_end, with_q);
     for (int c = 0; c < w.ntiles; ++c) {
-        const int b = c & 1;
-        const int tok = w.t_begin + c * C + t;
-        const bool valid = tok < w.t_end;
-        const Raw cur = nxt;
-        if (c + 1 < w.ntiles) load_token(nxt, q, k, v, row0 + tok + C, tok + C < w.t_end, with_q);
-        if (c >= 2 && !mbar_wait(&sh.bars[BAR_FREE0 + b], ((c >> 1) - 1) & 1, sh.abort_flag, sh.status)) return;
-        // [V | 1] (MN-major: a 16-byte piece is 8 columns of token t)
-        const uint32_t va = sh.sbase + OFF_VA + b * VA_BYTES + cm + (t >> 3) * VA_LBO;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) st_shared_v4(va + i * VA_SBO, cur.v[i]);
-        st_shared_v4(va + 8 * VA_SBO, make_uint4(valid ? 0x3F80u : 0u, 0u, 0u, 0u));  // bf16 1.0, column 64
-        st_shared_v4(va + 9 * VA_SBO, make_uint4(0, 0, 0, 0));
-        if (with_q) {
-            // Q, K (K-major, 2 core matrices along d')
-            const uint32_t qk = cm + (t >> 3) * QK_SBO + b * QK_BYTES;
-            st_shared_v4(sh.sbase + OFF_Q + qk, cur.q[0]);
-            st_shared_v4(sh.sbase + OFF_Q + qk + QK_LBO, cur.q[1]);
-            st_shared_v4(sh.sbase + OFF_K + qk, cur.k[0]);
-            st_shared_v4(sh.sbase + OFF_K + qk + QK_LBO, cur.k[1]);
-            // Q, K and [V|1] are all the MMA1 and MMA2 of this tile read: release them
-            // now, before the wait below for the previous tile's MMA3.
-            fence_proxy_async_smem();
-            mbar_arrive(&sh.bars[BAR_QK0 + b]);
-        }
-        // phi(Q) goes to TMEM once the last MMA3 of the previous tile has read it.
+        const int b = c & 1, s = c % KS;
+        const bool valid = w.t_begin + c * C + t < w.t_end;
+        if (!mbar_wait(&sh.bars[BAR_RF0 + s], (c / KS) & 1, sh.abort_flag, sh.status)) return;
+        uint4 kx[2], qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
+        ld_row32(sh.sbase + off_k(CL) + s * QK_BYTES, t, kx);
+        if (with_q) ld_row32(sh.sbase + off_q(CL) + s * QK_BYTES, t, qx);
+        // phi(K) buffer b is free once MMA4 of tile c-2 has read it; phi(Q) goes
+        // to TMEM once the last MMA3 of the previous tile has read it.
+        if (c >= 2 && !mbar_wait(&sh.bars[BAR_PKF0 + b], ((c >> 1) - 1) & 1, sh.abort_flag, sh.status)) return;
         const int pqf = CL == 64 ? BAR_PQF_HI : BAR_PQF;
         if (with_q && c >= 1 && !mbar_wait(&sh.bars[pqf], (c - 1) & 1, sh.abort_flag, sh.status)) return;
         tc_fence_after();
-        // phi(K) (MN-major: a 16-byte piece is 8 features of token t; padded
-        // tokens contribute nothing) and phi(Q) (TMEM lane t), in one pass.
+        // phi(K) (MN-major: a 16-byte piece is 8 features of token t; tokens past
+        // the end contribute nothing) and phi(Q) (TMEM lane t), in one pass.
         const uint32_t pk = sh.sbase + OFF_PK + b * PK_BYTES + cm + (t >> 3) * PK_LBO;
-        emit_phi2(cur.k, valid ? 0x3F80u : 0u, cur.q, 0x3F80u, [&](int g, const uint32_t* uk, const uint32_t* uq) {
+        emit_phi2(kx, valid ? 0x3F80u : 0u, qx, 0x3F80u, [&](int g, const uint32_t* uk, const uint32_t* uq) {
 #pragma unroll
             for (int j = 0; j < 4; ++j)
                 st_shared_v4(pk + (4 * g + j) * PK_SBO, make_uint4(uk[4 * j], uk[4 * j + 1], uk[4 * j + 2], uk[4 * j + 3]));
@@ -616,7 +592,7 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
 #pragma unroll
                 for (int g = 0; g < KF / 32; ++g) tmem_st16(lane_base + COL_PQ + 16 * g, zeros);
             } else {
-                emit_phi2(cur.q, 0x3F80u, cur.q, 0x3F80u, [&](int g, const uint32_t* uq, const uint32_t*) {
+                emit_phi2(qx, 0x3F80u, qx, 0x3F80u, [&](int g, const uint32_t* uq, const uint32_t*) {
                     tmem_st16(lane_base + COL_PQ + 16 * g, uq);
                 });
             }
@@ -625,6 +601,34 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
             mbar_arrive(&sh.bars[BAR_PQIN]);
         }
     }
+}
+
+// ------------------------------------------------------------------ input loader (warp 14, lane 0)
+// Q, K and V of tile c into stage c mod KS by TMA (Q not in the totals pass),
+// once every MMA reading the stage's previous tile has completed. Rows past
+// the end of the sequence are zero-filled.
+template <int CL>
+__device__ __forceinline__ void loader(const Work& w, const Shared& sh, const CUtensorMap* tq, const CUtensorMap* tk,
+                                       const CUtensorMap* tv) {
+    constexpr int KS = stages(CL);
+    const uint32_t bytes = (w.totals ? 0u : QK_BYTES) + QK_BYTES + V_BYTES;
+    int issued = 0;
+    for (int c = 0; c < w.ntiles; ++c, ++issued) {
+        const int s = c % KS;
+        if (c >= KS && !mbar_wait(&sh.bars[BAR_RE0 + s], ((c / KS) - 1) & 1, sh.abort_flag, sh.status)) break;
+        uint64_t* full = &sh.bars[BAR_RF0 + s];
+        const int row = w.t_begin + c * C;
+        mbar_expect_tx(full, bytes);
+        if (!w.totals) tma_load_3d(sh.sbase + off_q(CL) + s * QK_BYTES, tq, full, 0, row, (int)w.bh);
+        tma_load_3d(sh.sbase + off_k(CL) + s * QK_BYTES, tk, full, 0, row, (int)w.bh);
+        tma_load_3d(sh.sbase + off_v(CL) + s * V_BYTES, tv, full, 0, row, (int)w.bh);
+    }
+    // Nothing may land in shared memory after the CTA exits: wait (bounded) for
+    // the last load issued into each stage (already complete unless the CTA is
+    // giving up early).
+    const uint64_t t0 = global_ns();
+    for (int c = max(0, issued - KS); c < issued; ++c)
+        while (!mbar_try_wait(&sh.bars[BAR_RF0 + c % KS], (c / KS) & 1) && global_ns() - t0 < kWaitLimitNs) {}
 }
 
 // ------------------------------------------------------------------ intra (warps 4-7)
@@ -796,10 +800,8 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
 // 64-127, the state after its first chunk) comes after MMA2.
 template <int CL>
 __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32_t tmem) {
+    constexpr int KS = stages(CL);
     const uint32_t sb = sh.sbase;
-    const uint64_t dq0 = smem_desc(sb + OFF_Q, QK_LBO, QK_SBO);
-    const uint64_t dk0 = smem_desc(sb + OFF_K, QK_LBO, QK_SBO);
-    const uint64_t dva0 = smem_desc(sb + OFF_VA, VA_LBO, VA_SBO);
     const uint64_t dsb0 = smem_desc(sb + OFF_SB, SB_LBO, SB_SBO);
     const uint64_t dsb1 = smem_desc(sb + OFF_SB1, SB_LBO, SB_SBO);
     uint64_t* bars = sh.bars;
@@ -812,9 +814,11 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
         last_bar = &bars[bar];
         last_parity = parity;
     };
-    // s = Q_qt K_kt^T (query tile qt's buffer, key tile kt's buffer)
+    // s = Q_qt K_kt^T (query tile qt's stage, key tile kt's stage)
     auto mma1 = [&](int qt, int kt) {
-        mma_bf16(tmem + COL_S, dq0 + (((qt & 1) * QK_BYTES) >> 4), dk0 + (((kt & 1) * QK_BYTES) >> 4), ID_QK, 0);
+        const uint64_t dq = smem_desc_swizzled(sb + off_q(CL) + (qt % KS) * QK_BYTES, 16, QK_SBO, 32);
+        const uint64_t dk = smem_desc_swizzled(sb + off_k(CL) + (kt % KS) * QK_BYTES, 16, QK_SBO, 32);
+        mma_bf16(tmem + COL_S, dq, dk, ID_QK, 0);
         commit(BAR_S, kb & 1);
         ++kb;
     };
@@ -824,25 +828,26 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
         for (int j = 0; j < KF / 16; ++j)
             mma_bf16_ts(tmem + COL_Y, tmem + COL_PQ + 8 * j, dsb + ((j * 2 * SB_LBO) >> 4), ID_INT, (acc || j > 0) ? 1u : 0u);
     };
-    // Y (+)= A [V_kt | 1]
+    // Y (+)= A [V_kt | 1]: key tile kt's V stage with the ones block as its
+    // second atom; a K step of 16 tokens is 2048 bytes.
     auto mma2 = [&](int blk, int kt, bool acc) {
-        const uint64_t dva = dva0 + (((kt & 1) * VA_BYTES) >> 4);
+        const uint32_t va = sb + off_v(CL) + (kt % KS) * V_BYTES;
+        const uint64_t dva = smem_desc_sw128(va, sb + off_ones(CL) - va, 1024);
 #pragma unroll
         for (int j = 0; j < C / 16; ++j)
-            mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2 * VA_LBO) >> 4), ID_AV,
+            mma_bf16_ts(tmem + COL_Y, tmem + col_a(j >> 1) + 8 * (j & 1), dva + ((j * 2048) >> 4), ID_AV,
                         (acc || j > 0) ? 1u : 0u);
         commit(BAR_AF, blk & 1);
     };
     // The first block of tile t: against t's own keys, or (CL = 256, t odd) the
     // previous tile's.
     auto first_kt = [](int t) { return (CL == 256 && (t & 1)) ? t - 1 : t; };
-    bool ok = wait(BAR_QK0, 0);
+    bool ok = wait(BAR_RF0, 0);
     if (ok) {
         tc_fence_after();
         mma1(0, 0);
     }
     for (int c = 0; ok && c < w.ntiles; ++c) {
-        const int b = c & 1;
         const int nb = Plan<CL>::blocks(c);
         const int blk0 = Plan<CL>::blocks_before(c);     // first block of this tile
         if (!wait(BAR_PQIN, (CL == 64 ? 2 * c : c) & 1)) break;
@@ -871,18 +876,18 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
             if (j + 1 < nb) {
                 mma1(c, c);
             } else if (c + 1 < w.ntiles) {
-                if (!wait(BAR_QK0 + ((c + 1) & 1), ((c + 1) >> 1) & 1)) { ok = false; break; }
+                if (!wait(BAR_RF0 + (c + 1) % KS, ((c + 1) / KS) & 1)) { ok = false; break; }
                 tc_fence_after();
                 mma1(c + 1, first_kt(c + 1));
             }
             const int kt = j == 0 ? first_kt(c) : c;
             mma2(blk, kt, did3 || j > 0);
-            if (CL == 256 && (c & 1) && j == 0) commit(BAR_FREE0 + (b ^ 1), ((c - 1) >> 1) & 1);
+            if (CL == 256 && (c & 1) && j == 0) commit(BAR_RE0 + (c - 1) % KS, ((c - 1) / KS) & 1);
         }
         if (!ok) break;
-        // Release this tile's buffer -- at CL = 256 an even tile's only after the odd
-        // tile's first block has read it (or when no odd tile follows).
-        if (CL != 256 || (c & 1) || c + 1 == w.ntiles) commit(BAR_FREE0 + b, (c >> 1) & 1);
+        // Release this tile's input stage -- at CL = 256 an even tile's only after
+        // the odd tile's first block has read it (or when no odd tile follows).
+        if (CL != 256 || (c & 1) || c + 1 == w.ntiles) commit(BAR_RE0 + c % KS, (c / KS) & 1);
         if constexpr (CL == 64) {
             // rows 64-127: phi(Q) of the second chunk against the state after the first
             if (!wait(BAR_PQIN, (2 * c + 1) & 1) || !wait(BAR_SBR1, c & 1)) break;
@@ -904,8 +909,8 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     using P = Plan<CL>;
     constexpr int kSteps = P::kSteps;
     constexpr int kJ = C / 16 / kSteps;                  // K steps of 16 tokens per MMA4 step
+    constexpr int KS = stages(CL);
     const uint32_t sb = sh.sbase;
-    const uint64_t dva0 = smem_desc(sb + OFF_VA, VA_LBO, VA_SBO);    // [V|1]^T: M = column, MN-major
     const uint64_t dpk0 = smem_desc(sb + OFF_PK, PK_LBO, PK_SBO);    // phi(K): N = feature, MN-major
     uint64_t* bars = sh.bars;
     uint64_t* last_bar = nullptr;
@@ -919,23 +924,26 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     bool pending = false;                                // a read-out follows the previous step
     bool ok = !w.has_init || wait(BAR_INIT, 0);
     for (int c = 0; ok && c < w.ntiles; ++c) {
-        const int b = c & 1;
-        if (!wait(BAR_IN0 + b, (c >> 1) & 1)) break;
+        const int b = c & 1, s = c % KS;
+        if (!wait(BAR_RF0 + s, (c / KS) & 1) || !wait(BAR_IN0 + b, (c >> 1) & 1)) break;
+        // [V|1]^T as the A operand (M = column: V's atom, then the ones block; K = token)
+        const uint32_t va = sb + off_v(CL) + s * V_BYTES;
+        const uint64_t dva = smem_desc_sw128(va, sb + off_ones(CL) - va, 1024);
         for (int h = 0; h < kSteps; ++h) {
             if (pending && !wait(BAR_DSF, (r - 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            const uint64_t dva = dva0 + ((b * VA_BYTES) >> 4);
             const uint64_t dpk = dpk0 + ((b * PK_BYTES) >> 4);
 #pragma unroll
             for (int jj = 0; jj < kJ; ++jj) {
                 const int j = h * kJ + jj;
-                mma_bf16(tmem + COL_ST, dva + ((j * 2 * VA_LBO) >> 4), dpk + ((j * 2 * PK_LBO) >> 4), ID_UPD,
+                mma_bf16(tmem + COL_ST, dva + ((j * 2048) >> 4), dpk + ((j * 2 * PK_LBO) >> 4), ID_UPD,
                          (c > 0 || j > 0 || w.has_init) ? 1u : 0u);
             }
             if (h + 1 == kSteps) {
-                mma_commit(&bars[BAR_FREE0 + b]);
-                last_bar = &bars[BAR_FREE0 + b];
-                last_parity = (c >> 1) & 1;
+                mma_commit(&bars[BAR_PKF0 + b]);
+                mma_commit(&bars[BAR_RE0 + s]);
+                last_bar = &bars[BAR_RE0 + s];
+                last_parity = (c / KS) & 1;
             }
             const bool last = c + 1 == w.ntiles && h + 1 == kSteps;
             bool readout;
@@ -957,9 +965,8 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
 // each split into `parts` pieces of at most sub_tiles = ceil(seg_tiles / parts) tiles.
 template <int CL, bool DECAY>
 __global__ void __launch_bounds__(kThreads, 1)
-la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
-                     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                     const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y,
+la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_constant__ CUtensorMap tq,
+                     const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
                      float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int parts, int mode,
                      int packed, float* __restrict__ ws, const float* __restrict__ gamma, unsigned* status,
                      unsigned debug) {
@@ -1009,17 +1016,27 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     if (tid == 0) {
         for (int i = 0; i < NUM_BARS; ++i) {
             uint32_t count = 1;
-            if (i == BAR_QK0 || i == BAR_QK1 || i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A ||
-                i == BAR_YF || i == BAR_YSR0 || i == BAR_YSR1)
+            if (i == BAR_IN0 || i == BAR_IN1 || i == BAR_PQIN || i == BAR_A || i == BAR_YF || i == BAR_YSR0 ||
+                i == BAR_YSR1)
                 count = 128;                                 // one warpgroup
             if (i == BAR_DSF || i == BAR_SBR || i == BAR_SBR1 || i == BAR_INIT) count = kStateLanes;
-            if ((i == BAR_FREE0 || i == BAR_FREE1) && !w.totals) count = 2;   // both issuers read the buffer
+            if (i >= BAR_RE0 && i <= BAR_RE2 && !w.totals) count = 2;   // both issuers read an input stage
             mbar_init(&bars[i], count);
         }
         *abort_flag = 0;
         mbar_fence_init();
     }
     if (warp == 13) tmem_alloc(tmem_base_slot, TMEM_COLS);
+    {
+        // The ones block: row t (token) holds bf16 1.0 in column 64, i.e. in its
+        // 16-byte piece 0, which the 128-byte swizzle stores at slot (t mod 8).
+        const uint32_t ones = sh.sbase + off_ones(CL);
+        for (int i = tid; i < C * 8; i += kThreads) {
+            const int row = i >> 3, slot = i & 7;
+            st_shared_v4(ones + row * 128 + slot * 16, make_uint4(slot == (row & 7) ? 0x3F80u : 0u, 0u, 0u, 0u));
+        }
+        fence_proxy_async_smem();
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -1028,7 +1045,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
     const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;   // testing: issue nothing, every waiter times out
 
     if (warp < 4) {
-        producers<CL>(w, sh, tmem, warp, tid, q, k, v, N);
+        producers<CL>(w, sh, tmem, warp, tid);
     } else if (warp < 8) {
         const int wq = warp & 3;
         if (w.totals) {
@@ -1047,8 +1064,10 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty,
         }
     } else if (warp == 12) {
         if (lane == 0 && !skip_mma) state_issuer<CL>(w, sh, tmem);
-    } else {
+    } else if (warp == 13) {
         if (lane == 0 && !w.totals && !skip_mma) y_issuer<CL>(w, sh, tmem);
+    } else {
+        if (lane == 0) loader<CL>(w, sh, &tq, &tk, &tv);
     }
 
     tc_fence_before();
@@ -1110,11 +1129,6 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
     const int BH = a.B * a.H;
     int nseg, seg_tiles;
     plan_segments(BH, a.N, num_sms, tiles_per_chunk(CL), &nseg, &seg_tiles);
-    using bf = __nv_bfloat16;
-    auto q = static_cast<const bf*>(a.q);
-    auto k = static_cast<const bf*>(a.k);
-    auto v = static_cast<const bf*>(a.v);
-    auto y = static_cast<bf*>(a.y);
     float* ws = static_cast<float*>(a.workspace);
     // Split the totals as finely as helps and as the given workspace holds (the
     // workspace query sizes it for the best split; a smaller one, as the
@@ -1122,15 +1136,18 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
     const int parts = plan_parts(BH, nseg, seg_tiles, num_sms, a.ws_bytes);
     if (nseg > 1 && (ws == nullptr || a.ws_bytes < (size_t)BH * (nseg - 1) * parts * kTotalFloats * sizeof(float)))
         return cudaErrorInvalidValue;                    // the segment totals need their workspace
-    CUtensorMap ty;
-    if (!make_tmap_bf16_3d(&ty, y, DV, a.N, BH, DV, C)) return cudaErrorInvalidValue;
+    CUtensorMap ty, tq, tk, tv;
+    if (!make_tmap_bf16_3d(&ty, a.y, DV, a.N, BH, DV, C) ||
+        !make_tmap_bf16_3d_swizzle(&tq, a.q, DF, a.N, BH, DF, C, 32) ||
+        !make_tmap_bf16_3d_swizzle(&tk, a.k, DF, a.N, BH, DF, C, 32) ||
+        !make_tmap_bf16_3d_swizzle(&tv, a.v, DV, a.N, BH, DV, C, 128))
+        return cudaErrorInvalidValue;
     if (nseg > 1) {
-        e = launch_pdl(kern, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, q, k, v,
-                       y, a.S, a.z, a.N, nseg, seg_tiles, parts, 1, a.packed ? 1 : 0, ws, a.gamma, a.status,
-                       a.debug);
+        e = launch_pdl(kern, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
+                       a.z, a.N, nseg, seg_tiles, parts, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, q, k, v, y, a.S,
+    return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
                       a.z, a.N, nseg, seg_tiles, parts, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
 }
 

@@ -231,6 +231,16 @@ __device__ __forceinline__ void st_shared_v4(uint32_t saddr, uint4 v) {
                  : "memory");
 }
 
+__device__ __forceinline__ void st_shared_f32(uint32_t saddr, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(saddr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ float ld_shared_f32(uint32_t saddr) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(saddr) : "memory");
+    return v;
+}
+
 }  // namespace tc
 }  // namespace based
 
