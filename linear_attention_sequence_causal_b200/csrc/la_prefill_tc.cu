@@ -80,8 +80,9 @@
 // there are fewer (b, h) pairs than SMs, each sequence is cut into segments of
 // whole chunks. A first launch (totals pass) runs only the state chain over
 // every segment but the last and stores each segment's [S | z] total in the
-// workspace; the main launch then starts segment s from the sum of the totals
-// of segments 0..s-1, so all segments of a sequence run at once.
+// workspace; a small launch turns them into running sums (the state entering
+// each segment) and the main launch then starts segment s from that state, so
+// all segments of a sequence run at once.
 //
 // phi(K) and the bf16 state use the canonical no-swizzle layouts (8-row x
 // 16-byte core matrices, each a contiguous 128-byte block); each thread writes
@@ -186,6 +187,7 @@ enum {
     BAR_SBR,                 // state warps -> Y issuer: [S|z] bf16 written (buffer OFF_SB)
     BAR_SBR1,                // CL = 64: the same for buffer OFF_SB1
     BAR_INIT,                // state warps -> issuers: start state of the segment is in TMEM and the [S|z] buffer
+    BAR_INITLD,              // copy of the segment's start state (main pass, segment > 0) landed
     BAR_YSR0, BAR_YSR1,      // epilogue warps -> store thread: y tile b written
     BAR_YSF0, BAR_YSF1,      // store thread -> epilogue warps: the TMA store has read y tile b
     NUM_BARS
@@ -290,7 +292,7 @@ struct Work {
     bool final_state;        // main pass, last segment: writes S and z
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this part's total
-    const float* ws_in;      // main pass: totals of this sequence's segments 0..seg-1 (parts each)
+    const float* ws_in;      // main pass: the state entering this segment (rows of KF floats)
     int parts;               // totals per segment (each segment's total is split into parts)
     int sub_tiles;           // tiles per part (the last part of a segment may have fewer)
     const float* gamma;      // coarse decay: gamma of this segment's tiles (index = local tile), or nullptr
@@ -376,43 +378,37 @@ __device__ __forceinline__ void write_final_state(const Work& w, uint32_t sbase,
     }
 }
 
-// Segment start state: row n = sum of the totals of segments 0..seg-1 (each
-// segment's total in `parts` pieces of consecutive tiles), placed in the TMEM
-// accumulator (fp32) and in the [S|z] buffer (bf16) for the first MMA3. With
-// coarse decay (DECAY), the total of a piece (its own state, started from zero)
-// counts with the product of gamma over the tiles after it up to and including
-// this segment's first tile, whose gamma scales the state it enters.
-template <bool DECAY>
-__device__ __forceinline__ void init_state(const Work& w, int n, uint32_t taddr, const Shared& sh) {
+// Segment start state. Between the totals pass and the main pass a small
+// kernel (la_segment_prefix_kernel) turns the totals into running sums: the
+// state entering segment s (s >= 1) replaces the first piece of segment s-1 in
+// the workspace. The main pass's loader copies that state, row by row, into a
+// staging area over the phi(K) tiles, at kInitStride floats per row (padded so
+// that the row reads below are free of bank conflicts).
+constexpr int kInitStride = KF + 4;
+static_assert(NV * kInitStride * 4 <= 2 * PK_BYTES, "segment start state fits in the phi(K) tiles");
+constexpr uint32_t kRowBytes = KF * 4;              // one row of a total / start state
+
+// State warps: once the copy has landed, row n of the staged start state into
+// the TMEM accumulator (fp32) and into the [S|z] buffer (bf16) for the first
+// MMA3; the arrival on INIT also releases the staging area to the producers.
+__device__ __forceinline__ void init_state(int n, uint32_t taddr, const Shared& sh) {
     const bool real = n < NV;
+    const uint32_t stage = sh.sbase + OFF_PK;
+    if (!mbar_wait(&sh.bars[BAR_INITLD], 0, sh.abort_flag, sh.status)) return;
 #pragma unroll 1
     for (int m = 0; m < KF / 16; ++m) {
+        uint32_t u[16];
         float r[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) r[i] = 0.f;
-        if (real) {
-            float ws = DECAY ? w.gamma_head[w.c0] : 1.0f;   // weight of part j, nearest first
-            for (int j = w.seg * w.parts - 1; j >= 0; --j) {
-                const float4* src = reinterpret_cast<const float4*>(w.ws_in + j * kTotalFloats + (size_t)n * KF + 16 * m);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float4 t = __ldg(src + i);
-                    r[4 * i] = fmaf(ws, t.x, r[4 * i]);
-                    r[4 * i + 1] = fmaf(ws, t.y, r[4 * i + 1]);
-                    r[4 * i + 2] = fmaf(ws, t.z, r[4 * i + 2]);
-                    r[4 * i + 3] = fmaf(ws, t.w, r[4 * i + 3]);
-                }
-                if constexpr (DECAY) {
-                    const int s = j / w.parts, p = j % w.parts;
-                    const int c_lo = s * w.seg_tiles + p * w.sub_tiles;
-                    const int c_hi = s * w.seg_tiles + min((p + 1) * w.sub_tiles, w.seg_tiles);
-                    for (int c = c_lo; c < c_hi; ++c) ws *= w.gamma_head[c];
-                }
-            }
+        for (int i = 0; i < 4; ++i) {
+            const uint4 t = real ? ld_shared_v4(stage + (n * kInitStride + 16 * m + 4 * i) * 4) : make_uint4(0, 0, 0, 0);
+            u[4 * i] = t.x;
+            u[4 * i + 1] = t.y;
+            u[4 * i + 2] = t.z;
+            u[4 * i + 3] = t.w;
         }
-        uint32_t u[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) u[i] = __float_as_uint(r[i]);
+        for (int i = 0; i < 16; ++i) r[i] = __uint_as_float(u[i]);
         tmem_st16(taddr + 16 * m, u);
         if (real) store_sb16(sh.sbase, OFF_SB, n, m, r);
     }
@@ -555,6 +551,8 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
     // second of rows 64-127 only; the other half's rows hold zeros.
     const bool first_half = CL != 64 || warp < 2;
     const uint32_t zeros[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    // A segment's start state is staged over the phi(K) tiles until INIT.
+    if (w.has_init && !mbar_wait(&sh.bars[BAR_INIT], 0, sh.abort_flag, sh.status)) return;
     for (int c = 0; c < w.ntiles; ++c) {
         const int b = c & 1, s = c % KS;
         const bool valid = w.t_begin + c * C + t < w.t_end;
@@ -612,6 +610,11 @@ __device__ __forceinline__ void loader(const Work& w, const Shared& sh, const CU
                                        const CUtensorMap* tv) {
     constexpr int KS = stages(CL);
     const uint32_t bytes = (w.totals ? 0u : QK_BYTES) + QK_BYTES + V_BYTES;
+    if (w.has_init) {                                    // the segment's start state, row n at kInitStride floats
+        mbar_expect_tx(&sh.bars[BAR_INITLD], NV * kRowBytes);
+        for (int n = 0; n < NV; ++n)
+            bulk_load(sh.sbase + OFF_PK + n * kInitStride * 4, w.ws_in + (size_t)n * KF, kRowBytes, &sh.bars[BAR_INITLD]);
+    }
     int issued = 0;
     for (int c = 0; c < w.ntiles; ++c, ++issued) {
         const int s = c % KS;
@@ -629,6 +632,8 @@ __device__ __forceinline__ void loader(const Work& w, const Shared& sh, const CU
     const uint64_t t0 = global_ns();
     for (int c = max(0, issued - KS); c < issued; ++c)
         while (!mbar_try_wait(&sh.bars[BAR_RF0 + c % KS], (c / KS) & 1) && global_ns() - t0 < kWaitLimitNs) {}
+    if (w.has_init)
+        while (!mbar_try_wait(&sh.bars[BAR_INITLD], 0) && global_ns() - t0 < kWaitLimitNs) {}
 }
 
 // ------------------------------------------------------------------ intra (warps 4-7)
@@ -708,7 +713,7 @@ __device__ __forceinline__ void intra_and_state(const Work& w, const Shared& sh,
     const int n = wq * 32 + lane;                        // value column == TMEM lane (state role)
     const uint32_t taddr = tmem + (static_cast<uint32_t>(wq * 32) << 16) + COL_ST;
     const bool state = wq < 3;
-    if (state && w.has_init) init_state<DECAY>(w, n, taddr, sh);
+    if (state && w.has_init) init_state(n, taddr, sh);
     int kb = 0, r = 0;
     for (int c = 0; c < w.ntiles; ++c) {
         const int nb = P::blocks(c);
@@ -963,7 +968,9 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
 
 // mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2,
 // each split into `parts` pieces of at most sub_tiles = ceil(seg_tiles / parts) tiles.
-template <int CL, bool DECAY>
+// SEG: compiled for more than one segment per sequence (a segment may start from
+// a state); without it, every CTA starts from zero and none of that code exists.
+template <int CL, bool DECAY, bool SEG>
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
@@ -1000,11 +1007,11 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
         w.t_end = min(N, w.t_begin + seg_tiles * C);
     }
     w.ntiles = (w.t_end - w.t_begin + C - 1) / C;
-    w.has_init = !w.totals && w.seg > 0;
+    w.has_init = SEG && !w.totals && w.seg > 0;
     w.final_state = !w.totals && w.seg == nseg - 1;
     w.packed = packed != 0;
     w.ws_out = w.totals ? ws + (w.bh * (nseg - 1) * parts + j) * kTotalFloats : nullptr;
-    w.ws_in = w.has_init ? ws + w.bh * (nseg - 1) * parts * kTotalFloats : nullptr;
+    w.ws_in = w.has_init ? ws + (w.bh * (nseg - 1) * parts + (size_t)(w.seg - 1) * parts) * kTotalFloats : nullptr;
     w.c0 = w.t_begin / C;
     w.seg_tiles = seg_tiles;
     w.ws_base = ws;
@@ -1042,6 +1049,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
     tc_fence_after();
     const uint32_t tmem = *tmem_base_slot;
     grid_dependency_wait();                              // inputs and workspace may come from the previous kernel
+
     const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;   // testing: issue nothing, every waiter times out
 
     if (warp < 4) {
@@ -1077,6 +1085,42 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+// Running sums of the segment totals, in place. Thread = one float4 column of a
+// total (16 rows x 4 features of the KF-wide rows), blockIdx.y = the sequence.
+// Walking the pieces of segments 0..nseg-2 in order, the state entering
+// segment s+1 replaces the first piece of segment s, which this thread has
+// read by then (each thread touches only its own column). With coarse decay
+// (DECAY) a piece's total counts with the product of gamma over its own tiles
+// on the state before it, and the state handed to segment s+1 takes the gamma
+// of that segment's first tile.
+template <bool DECAY>
+__global__ void __launch_bounds__(256)
+la_segment_prefix_kernel(float* __restrict__ ws, int nseg, int parts, int seg_tiles, const float* __restrict__ gamma,
+                         int seq_tiles) {
+    grid_dependency_wait();                              // the totals pass has written the pieces
+    constexpr int kCols = (int)(kTotalFloats / 4);
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= kCols) return;
+    float4* base = reinterpret_cast<float4*>(ws) + (size_t)blockIdx.y * (nseg - 1) * parts * kCols;
+    const float* g = DECAY ? gamma + (size_t)blockIdx.y * seq_tiles : nullptr;
+    const int sub = (seg_tiles + parts - 1) / parts;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int sg = 0; sg + 1 < nseg; ++sg) {
+        for (int p = 0; p < parts; ++p) {
+            const float4 t = base[(size_t)(sg * parts + p) * kCols + i];
+            if constexpr (DECAY) {
+                float d = 1.0f;
+                const int c_hi = sg * seg_tiles + min((p + 1) * sub, seg_tiles);
+                for (int c = sg * seg_tiles + p * sub; c < c_hi; ++c) d *= g[c];
+                acc = make_float4(acc.x * d, acc.y * d, acc.z * d, acc.w * d);
+            }
+            acc = make_float4(acc.x + t.x, acc.y + t.y, acc.z + t.z, acc.w + t.w);
+        }
+        const float g0 = DECAY ? g[(sg + 1) * seg_tiles] : 1.0f;
+        base[(size_t)(sg * parts) * kCols + i] = make_float4(acc.x * g0, acc.y * g0, acc.z * g0, acc.w * g0);
     }
 }
 
@@ -1120,15 +1164,15 @@ int plan_parts(int BH, int nseg, int seg_tiles, int num_sms, size_t ws_cap) {
 
 template <int CL>
 cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) {
-    auto kern = la_prefill_tc_kernel<CL, false>;
-    if constexpr (CL == 128)
-        if (a.gamma != nullptr) kern = la_prefill_tc_kernel<128, true>;
-    constexpr uint32_t kSmem = smem_bytes(CL);
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    if (e != cudaSuccess) return e;
     const int BH = a.B * a.H;
     int nseg, seg_tiles;
     plan_segments(BH, a.N, num_sms, tiles_per_chunk(CL), &nseg, &seg_tiles);
+    auto kern = nseg > 1 ? la_prefill_tc_kernel<CL, false, true> : la_prefill_tc_kernel<CL, false, false>;
+    if constexpr (CL == 128)
+        if (a.gamma != nullptr) kern = nseg > 1 ? la_prefill_tc_kernel<128, true, true> : la_prefill_tc_kernel<128, true, false>;
+    constexpr uint32_t kSmem = smem_bytes(CL);
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e != cudaSuccess) return e;
     float* ws = static_cast<float*>(a.workspace);
     // Split the totals as finely as helps and as the given workspace holds (the
     // workspace query sizes it for the best split; a smaller one, as the
@@ -1145,6 +1189,14 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
     if (nseg > 1) {
         e = launch_pdl(kern, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
                        a.z, a.N, nseg, seg_tiles, parts, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+        if (e != cudaSuccess) return e;
+        const dim3 pgrid((unsigned)((kTotalFloats / 4 + 255) / 256), (unsigned)BH);
+        const int seq_tiles = (a.N + C - 1) / C;
+        e = a.gamma != nullptr
+                ? launch_pdl(la_segment_prefix_kernel<true>, pgrid, dim3(256), 0, stream, ws, nseg, parts, seg_tiles,
+                             a.gamma, seq_tiles)
+                : launch_pdl(la_segment_prefix_kernel<false>, pgrid, dim3(256), 0, stream, ws, nseg, parts, seg_tiles,
+                             a.gamma, seq_tiles);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
