@@ -438,7 +438,7 @@ based_status_t based_swa_decode(void* k_cache, void* v_cache, int64_t t, const v
     if (status == nullptr) return BASED_ERR_CUDA;
     const bool preload = !take_ring_fresh(k_cache, dev);
     const cudaError_t e = based::launch_swa_decode(k_cache, v_cache, t, q, k, v, y, B, H, d, w, scale,
-                                                   dtype == BASED_BF16, preload, status, stream);
+                                                   dtype == BASED_BF16, preload, num_sms(dev), status, stream);
     return e == cudaSuccess ? BASED_OK : BASED_ERR_CUDA;
 }
 

@@ -87,7 +87,8 @@ cudaError_t launch_swa_prefill_tc(const void* q, const void* k, const void* v, v
 // false when the kernel before it may have written any slot of this ring.
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q,
                               const void* k, const void* v, void* y, int B, int H, int d, int w,
-                              float scale, bool bf16, bool preload, unsigned* status, cudaStream_t stream);
+                              float scale, bool bf16, bool preload, int num_sms, unsigned* status,
+                              cudaStream_t stream);
 
 // Short gated convolution: filter taps K in [1, kMaxConvTaps], d a multiple of 4.
 constexpr int kMaxConvTaps = 8;

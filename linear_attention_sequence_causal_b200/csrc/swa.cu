@@ -16,12 +16,13 @@
 // (running max and sum, rescaling the accumulator), in fp32 with expf.
 //
 // Decode: one CTA per (b, h); the new key/value go to slot t mod w. bf16 uses
-// 16-byte loads (see swa_decode_bf16_kernel); the fp32 kernel scores slot j on
+// 16-byte loads (see the two swa_decode_bf16 kernels); the fp32 kernel scores slot j on
 // thread j, reduces max and sum, then accumulates output dim e on thread e.
 #include <math.h>
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tcgen05.cuh"
 
 namespace based {
 namespace {
@@ -29,6 +30,13 @@ namespace {
 constexpr int kQTile = 64;
 constexpr int kHead = 64;        // head dim d
 constexpr int kMaxW = 64;
+
+// 16-byte asynchronous copy global -> shared (through L2, not L1), and the wait
+// for all of this thread's copies.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 // Two floats as a bf16x2 word (round to nearest even), low half first.
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -223,7 +231,154 @@ cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void
     }
 }
 
-// bf16 decode: 128 threads per (b, h), one memory round trip. Thread (warp,
+// bf16 decode, shared-memory variant (more heads than one wave of the register
+// variant; bound by bytes in flight): 128 threads per (b, h). The valid slots of the head's key and
+// value rings (slots 0..min(t, w-1)) are copied into shared memory with 16-byte
+// asynchronous copies, so the data in flight costs no registers and many
+// heads' copies are in flight per SM. Thread (warp, lane) owns the 16-byte
+// piece c = lane % 8 (dims 8c..8c+7) of slots 16p + 4*warp + lane/8, p = 0..3,
+// and copies that piece of the key and the value of its slots. Slots that
+// neither this step (t) nor the previous one (t - 1) writes are copied before
+// the wait for the previous kernel in the stream (griddepcontrol): only that
+// kernel can still be running, and consecutive decode steps on one cache write
+// slot (t - 1) mod w at most. Slot (t - 1) mod w is copied after the wait, and
+// slot t mod w takes the new key and value (and is written back to the ring).
+// Without `preload` (the ring was just written whole, by a prefill, or the
+// kernel is launched in plain stream order) every slot is copied after the
+// wait. The eight lanes of a slot combine their partial dot
+// products by shuffles; every warp then reduces the 64 scores itself (max,
+// exp, sum) from shared memory; the four warps' partial outputs are added
+// through shared memory.
+__global__ void __launch_bounds__(128)
+swa_decode_bf16_smem_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
+                       const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                       const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, int new_slot,
+                       float scale, int preload, unsigned* status) {
+    __shared__ __align__(128) uint4 s_k[kMaxW * 8];      // slot rows of 128 bytes
+    __shared__ __align__(128) uint4 s_v[kMaxW * 8];
+    __shared__ float s_sc[kMaxW];
+    __shared__ float s_part[4][kHead];
+    const int tid = threadIdx.x;
+    const int warp = tid >> 5, lane = tid & 31;
+    const int c = lane & 7;
+    const size_t bh = blockIdx.x;
+    const size_t n_heads = gridDim.x;                    // extents of y and the ring for the index checks
+    const int nvalid = t >= w ? w : (int)t + 1;          // slots holding a token: 0 .. nvalid-1
+    const uint4* kring = reinterpret_cast<const uint4*>(kc + bh * w * kHead);
+    const uint4* vring = reinterpret_cast<const uint4*>(vc + bh * w * kHead);
+    const int prev_slot = new_slot == 0 ? w - 1 : new_slot - 1;
+    auto copy_slot = [&](int slot) {
+        cp_async16(tc::smem_u32(&s_k[slot * 8 + c]), kring + slot * 8 + c);
+        cp_async16(tc::smem_u32(&s_v[slot * 8 + c]), vring + slot * 8 + c);
+    };
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        if (preload && slot < nvalid && slot != new_slot && slot != prev_slot) copy_slot(slot);
+    }
+    grid_dependency_wait();
+    const uint4 knew = __ldg(reinterpret_cast<const uint4*>(k + bh * kHead) + c);
+    const uint4 vnew = __ldg(reinterpret_cast<const uint4*>(v + bh * kHead) + c);
+    const uint4 qu = __ldg(reinterpret_cast<const uint4*>(q + bh * kHead) + c);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        if (slot >= nvalid) continue;
+        if (slot == new_slot) {
+            s_k[slot * 8 + c] = knew;
+            s_v[slot * 8 + c] = vnew;
+        } else if (!preload || slot == prev_slot) {
+            copy_slot(slot);
+        }
+    }
+    if (tid < 8 && in_bounds((bh * w + new_slot) * kHead + 8 * c + 7, n_heads * w * kHead, status)) {
+        reinterpret_cast<uint4*>(kc + (bh * w + new_slot) * kHead)[c] = knew;
+        reinterpret_cast<uint4*>(vc + (bh * w + new_slot) * kHead)[c] = vnew;
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // No early trigger for the next kernel: with more CTAs than one wave, its
+    // CTAs would become resident and wait while this grid still has CTAs to run.
+    float qv[8];
+    {
+        const uint32_t wd[4] = {qu.x, qu.y, qu.z, qu.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            qv[2 * e] = __uint_as_float(wd[e] << 16) * scale;
+            qv[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u) * scale;
+        }
+    }
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        const bool valid = slot < nvalid;
+        const uint4 kr = valid ? s_k[slot * 8 + c] : make_uint4(0, 0, 0, 0);
+        const uint32_t wd[4] = {kr.x, kr.y, kr.z, kr.w};
+        float part = 0.f;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            part = fmaf(qv[2 * e], __uint_as_float(wd[e] << 16), part);
+            part = fmaf(qv[2 * e + 1], __uint_as_float(wd[e] & 0xFFFF0000u), part);
+        }
+        part += __shfl_xor_sync(0xffffffffu, part, 1);
+        part += __shfl_xor_sync(0xffffffffu, part, 2);
+        part += __shfl_xor_sync(0xffffffffu, part, 4);
+        if (c == 0) s_sc[slot] = valid ? part : -INFINITY;
+    }
+    __syncthreads();
+    // Softmax statistics, computed by every warp (slot 0 always holds a token).
+    const float a = s_sc[lane], bsc = s_sc[lane + 32];
+    float m = fmaxf(a, bsc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = (a == -INFINITY ? 0.f : expf(a - m)) + (bsc == -INFINITY ? 0.f : expf(bsc - m));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv = 1.f / sum;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        const int slot = 16 * p + 4 * warp + (lane >> 3);
+        if (slot >= nvalid) continue;
+        const float pr = expf(s_sc[slot] - m) * inv;
+        const uint4 vr = s_v[slot * 8 + c];
+        const uint32_t wd[4] = {vr.x, vr.y, vr.z, vr.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            acc[2 * e] = fmaf(pr, __uint_as_float(wd[e] << 16), acc[2 * e]);
+            acc[2 * e + 1] = fmaf(pr, __uint_as_float(wd[e] & 0xFFFF0000u), acc[2 * e + 1]);
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
+        acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
+    }
+    if (lane < 8) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) s_part[warp][8 * c + e] = acc[e];
+    }
+    __syncthreads();
+    if (tid < 8) {
+        float o[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            o[e] = s_part[0][8 * tid + e] + s_part[1][8 * tid + e] + s_part[2][8 * tid + e] + s_part[3][8 * tid + e];
+        uint4 packed;
+        packed.x = pack2(o[0], o[1]);
+        packed.y = pack2(o[2], o[3]);
+        packed.z = pack2(o[4], o[5]);
+        packed.w = pack2(o[6], o[7]);
+        if (in_bounds(bh * kHead + 8 * tid + 7, n_heads * kHead, status))
+            reinterpret_cast<uint4*>(y + bh * kHead)[tid] = packed;
+    }
+}
+
+// bf16 decode, register variant (used while every head's CTA fits one wave at
+// eight CTAs per SM, where the step is bound by latency): 128 threads per
+// (b, h), one memory round trip. Thread (warp,
 // lane) owns the 16-byte piece c = lane % 8 (dims 8c..8c+7) of slots
 // 16p + 4*warp + lane/8, p = 0..3, and loads that piece of both the key and the
 // value of its four slots up front, together with q and the new key/value. The
@@ -232,7 +387,7 @@ cudaError_t prefill_t(const void* q, const void* k, const void* v, void* y, void
 // the weights are applied to values already in registers; the four warps'
 // partial outputs are added through shared memory.
 __global__ void __launch_bounds__(128)
-swa_decode_bf16_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
+swa_decode_bf16_reg_kernel(__nv_bfloat16* __restrict__ kc, __nv_bfloat16* __restrict__ vc, long long t,
                        const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
                        const __nv_bfloat16* __restrict__ v, __nv_bfloat16* __restrict__ y, int w, int new_slot,
                        float scale, int preload, unsigned* status) {
@@ -372,11 +527,18 @@ cudaError_t launch_swa_prefill(const void* q, const void* k, const void* v, void
 
 cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const void* q, const void* k,
                               const void* v, void* y, int B, int H, int d, int w, float scale,
-                              bool bf16, bool preload, unsigned* status, cudaStream_t stream) {
+                              bool bf16, bool preload, int num_sms, unsigned* status, cudaStream_t stream) {
     if (d != kHead || w < 1 || w > kMaxW) return cudaErrorInvalidValue;
     if (bf16) {
-        // Programmatic dependent launch: a step's CTAs are scheduled while the
-        // previous kernel drains and wait (griddepcontrol) before reading.
+        // Every head's CTA in one wave of the register variant (8 per SM): bound by
+        // latency, where the register variant is quicker, launched as a
+        // programmatic dependent (its CTAs are scheduled while the previous kernel
+        // drains, and wait with griddepcontrol before reading what it wrote).
+        // Beyond one wave the shared-memory variant keeps more bytes in flight; it
+        // is launched in plain stream order, since CTAs that became resident early
+        // and then waited would hold shared memory the previous kernel's last
+        // CTAs need (every slot is then copied at once).
+        const bool one_wave = (long long)B * H <= 8LL * num_sms;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3((unsigned)(B * H));
         cfg.blockDim = dim3(128);
@@ -385,12 +547,13 @@ cudaError_t launch_swa_decode(void* k_cache, void* v_cache, int64_t t, const voi
         attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr[0].val.programmaticStreamSerializationAllowed = 1;
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        cudaError_t e = cudaLaunchKernelEx(&cfg, swa_decode_bf16_kernel, static_cast<__nv_bfloat16*>(k_cache),
+        cfg.numAttrs = one_wave ? 1 : 0;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, one_wave ? swa_decode_bf16_reg_kernel : swa_decode_bf16_smem_kernel,
+                                           static_cast<__nv_bfloat16*>(k_cache),
                                            static_cast<__nv_bfloat16*>(v_cache), (long long)t,
                                            static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
                                            static_cast<const __nv_bfloat16*>(v), static_cast<__nv_bfloat16*>(y), w,
-                                           (int)(t % w), scale, preload ? 1 : 0, status);   // the new token's slot
+                                           (int)(t % w), scale, (preload && one_wave) ? 1 : 0, status);
         if (e != cudaSuccess) return e;
     } else {
         swa_decode_kernel<float><<<B * H, kMaxW, 0, stream>>>(

@@ -120,14 +120,15 @@ def test_decode_steps_back_to_back(w, prompt):
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
 
-@pytest.mark.parametrize("w", [64, 16])
-def test_prefill_then_decode_back_to_back(w):
+@pytest.mark.parametrize("w,batch,prompt", [(64, 64, 2048), (16, 64, 2048), (64, 128, 256), (16, 128, 256)])
+def test_prefill_then_decode_back_to_back(w, batch, prompt):
     """based_swa_prefill immediately followed by based_swa_decode on the same
     stream, every buffer allocated beforehand, so no other kernel runs between
     them. The ring holds stale values (a large constant) before each prefill:
     a decode that read any slot before the prefill had finished would attend
-    to them."""
-    batch, H, prompt = 64, 16, 2048
+    to them. Batch 64 x 16 heads fits one wave of decode CTAs, batch 128 x 16
+    does not (the decode then stages the rings in shared memory)."""
+    H = 16
     inp = synthetic.swa_inputs(batch, H, prompt + 2, 64, "bf16", seed=31 + w)
     q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
     qp, kp, vp = (x[:, :, :prompt].contiguous() for x in (q, k, v))
