@@ -753,7 +753,10 @@ __device__ __forceinline__ bool epilogue(const Work& w, const Shared& sh, uint32
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(wq * 32) << 16);
     const uint32_t ys = off_ys(CL);
     const int b = c & 1;
-    if (!mbar_wait(&sh.bars[BAR_Y], c & 1, sh.abort_flag, sh.status)) return false;
+    // At CL = 128 a tile is one intra block whose MMA2 completes Y: its AF commit
+    // (phase c) stands for BAR_Y. (The epilogue cannot fall two phases behind:
+    // the next tile's MMA2 waits for this epilogue's YF.)
+    if (!mbar_wait(&sh.bars[CL == 128 ? BAR_AF : BAR_Y], c & 1, sh.abort_flag, sh.status)) return false;
     tc_fence_after();
     float yv[NV];
 #pragma unroll
@@ -900,7 +903,7 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
             mma3(dsb1, true);
             commit(BAR_PQF_HI, c & 1);
         }
-        commit(BAR_Y, c & 1);
+        if (CL != 128) commit(BAR_Y, c & 1);         // CL = 128: the epilogue waits for AF
     }
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
