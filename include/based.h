@@ -109,7 +109,8 @@ typedef enum {
  *           of the shapes whose state does not fit tensor memory (bf16, (d_feat
  *           x d_v) x (chunks - 1) x 128-feature tiles), or the segment totals
  *           that let long sequences of the d_feat 16, d_v 64 kernel run in
- *           segments at once; its contents on entry do not matter.
+ *           segments at once (overwritten in place by the state entering each
+ *           segment); its contents on entry do not matter.
  * Returns BASED_ERR_INVALID_ARG for null or misaligned pointers, non-positive
  * sizes, or a workspace smaller than required; BASED_ERR_UNSUPPORTED for a
  * (d_feat, d_v, dtype, chunk) combination outside the built set.
@@ -123,7 +124,9 @@ BASED_API based_status_t based_la_prefill(const void* q, const void* k, const vo
 
 /*
  * based_la_prefill_workspace -- bytes of device scratch based_la_prefill needs
- * for these arguments on the current device (0 when no segment split is used).
+ * for these arguments on the current device (0 when the call needs none: one
+ * segment per sequence on the d_feat 16, d_v 64 kernel, one chunk on the
+ * others, or the CUDA-core path).
  * Returns 0 for arguments based_la_prefill would reject.
  */
 BASED_API size_t based_la_prefill_workspace(int B, int H, int N, int d_feat, int d_v,

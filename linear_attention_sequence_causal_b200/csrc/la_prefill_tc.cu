@@ -288,7 +288,7 @@ struct Work {
     int t_begin, t_end;      // tokens [t_begin, t_end) of the sequence
     int ntiles;              // 128-token tiles of the segment
     bool totals;             // totals pass: state chain only, result to the workspace
-    bool has_init;           // main pass, segment > 0: starts from the workspace prefix sum
+    bool has_init;           // main pass, segment > 0: starts from the state the prefix launch wrote
     bool final_state;        // main pass, last segment: writes S and z
     bool packed;             // S and z in the symmetric layout (1 + d' + d'(d'+1)/2 rows)
     float* ws_out;           // totals pass: this part's total
