@@ -137,6 +137,24 @@ __host__ __device__ constexpr uint32_t off_ys(int cl) {        // [2], 1024-alig
 __host__ __device__ constexpr uint32_t off_bar(int cl) { return off_ys(cl) + 2 * YS_BYTES; }
 __host__ __device__ constexpr uint32_t smem_bytes(int cl) { return off_bar(cl) + 256; }
 static_assert(smem_bytes(64) <= 227 * 1024 && smem_bytes(128) <= 227 * 1024, "shared memory");
+// The totals pass reads neither Q nor an [S|z] operand, and its ring is the
+// chain's latency: a tile's stage comes free only once its MMA4 has completed,
+// and the next load into it then takes about a microsecond to land. So it runs
+// kTotalsStages stages, the extra ones (K and V) in the idle [S|z] region.
+constexpr int kTotalsStages = 4;
+__host__ __device__ constexpr int ring(int cl, bool totals) { return totals ? kTotalsStages : stages(cl); }
+__host__ __device__ constexpr int extra_stages(int cl) { return kTotalsStages - stages(cl); }
+__device__ __forceinline__ uint32_t stage_v(int cl, bool totals, int s) {
+    return !totals || s < stages(cl) ? off_v(cl) + s * V_BYTES : OFF_SB + (s - stages(cl)) * V_BYTES;
+}
+__device__ __forceinline__ uint32_t stage_k(int cl, bool totals, int s) {
+    return !totals || s < stages(cl) ? off_k(cl) + s * QK_BYTES
+                                     : OFF_SB + extra_stages(cl) * V_BYTES + (s - stages(cl)) * QK_BYTES;
+}
+static_assert(extra_stages(64) * (V_BYTES + QK_BYTES) <= 2 * SB_BYTES &&
+                  extra_stages(128) * (V_BYTES + QK_BYTES) <= SB_BYTES && OFF_SB % 1024 == 0 &&
+                  (OFF_SB + extra_stages(64) * V_BYTES) % 256 == 0 && (OFF_SB + extra_stages(128) * V_BYTES) % 256 == 0,
+              "the totals pass's extra stages fit the [S|z] region (below the ones block), aligned");
 static_assert(off_v(64) % 1024 == 0 && off_v(128) % 1024 == 0 && off_q(64) % 256 == 0 && off_q(128) % 256 == 0,
               "swizzled tiles aligned");
 
@@ -170,8 +188,8 @@ constexpr uint32_t ID_UPD = idesc_bf16_f32(128, KF, true, true);
 constexpr size_t kTotalFloats = (size_t)KF * NV;
 
 enum {
-    BAR_RF0, BAR_RF1, BAR_RF2,   // TMA: Q, K, V of a tile landed in input stage s
-    BAR_RE0, BAR_RE1, BAR_RE2,   // both issuers' commits: every MMA reading input stage s has completed
+    BAR_RF0, BAR_RF1, BAR_RF2, BAR_RF3,   // TMA: Q, K, V of a tile landed in input stage s
+    BAR_RE0, BAR_RE1, BAR_RE2, BAR_RE3,   // both issuers' commits: every MMA reading input stage s has completed
     BAR_PKF0, BAR_PKF1,          // state-issuer commit: MMA4 has read phi(K) buffer b
     BAR_IN0, BAR_IN1,            // producers -> state issuer: phi(K) of a tile is in buffer b
     BAR_PQIN,                // producers -> Y issuer: phi(Q) (one MMA3 pass's rows) is in TMEM
@@ -540,9 +558,9 @@ __device__ __forceinline__ void ld_row32(uint32_t tile, int t, uint4* x) {
 
 // Thread t = token t of the tile = TMEM lane t. Once the tile's inputs have
 // landed (stage s), form phi(k_t) into phi(K) buffer b and phi(q_t) into TMEM.
-template <int CL>
+template <int CL, bool TOT>
 __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint32_t tmem, int warp, int tid) {
-    constexpr int KS = stages(CL);
+    constexpr int KS = ring(CL, TOT);
     const int t = tid;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
     const uint32_t cm = (t & 7) * 16;                    // row within a core matrix
@@ -558,7 +576,7 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
         const bool valid = w.t_begin + c * C + t < w.t_end;
         if (!mbar_wait(&sh.bars[BAR_RF0 + s], (c / KS) & 1, sh.abort_flag, sh.status)) return;
         uint4 kx[2], qx[2] = {make_uint4(0, 0, 0, 0), make_uint4(0, 0, 0, 0)};
-        ld_row32(sh.sbase + off_k(CL) + s * QK_BYTES, t, kx);
+        ld_row32(sh.sbase + stage_k(CL, TOT, s), t, kx);
         if (with_q) ld_row32(sh.sbase + off_q(CL) + s * QK_BYTES, t, qx);
         // phi(K) buffer b is free once MMA4 of tile c-2 has read it; phi(Q) goes
         // to TMEM once the last MMA3 of the previous tile has read it.
@@ -602,13 +620,13 @@ __device__ __forceinline__ void producers(const Work& w, const Shared& sh, uint3
 }
 
 // ------------------------------------------------------------------ input loader (warp 14, lane 0)
-// Q, K and V of tile c into stage c mod KS by TMA (Q not in the totals pass),
+// Q, K and V of tile c into stage c mod KS (the ring's length) by TMA (Q not in the totals pass),
 // once every MMA reading the stage's previous tile has completed. Rows past
 // the end of the sequence are zero-filled.
-template <int CL>
+template <int CL, bool TOT>
 __device__ __forceinline__ void loader(const Work& w, const Shared& sh, const CUtensorMap* tq, const CUtensorMap* tk,
                                        const CUtensorMap* tv) {
-    constexpr int KS = stages(CL);
+    constexpr int KS = ring(CL, TOT);
     const uint32_t bytes = (w.totals ? 0u : QK_BYTES) + QK_BYTES + V_BYTES;
     if (w.has_init) {                                    // the segment's start state, row n at kInitStride floats
         mbar_expect_tx(&sh.bars[BAR_INITLD], NV * kRowBytes);
@@ -623,8 +641,8 @@ __device__ __forceinline__ void loader(const Work& w, const Shared& sh, const CU
         const int row = w.t_begin + c * C;
         mbar_expect_tx(full, bytes);
         if (!w.totals) tma_load_3d(sh.sbase + off_q(CL) + s * QK_BYTES, tq, full, 0, row, (int)w.bh);
-        tma_load_3d(sh.sbase + off_k(CL) + s * QK_BYTES, tk, full, 0, row, (int)w.bh);
-        tma_load_3d(sh.sbase + off_v(CL) + s * V_BYTES, tv, full, 0, row, (int)w.bh);
+        tma_load_3d(sh.sbase + stage_k(CL, TOT, s), tk, full, 0, row, (int)w.bh);
+        tma_load_3d(sh.sbase + stage_v(CL, TOT, s), tv, full, 0, row, (int)w.bh);
     }
     // Nothing may land in shared memory after the CTA exits: wait (bounded) for
     // the last load issued into each stage (already complete unless the CTA is
@@ -912,12 +930,12 @@ __device__ __forceinline__ void y_issuer(const Work& w, const Shared& sh, uint32
 // MMA4 of every tile, in Plan::kSteps steps of 128 / kSteps tokens; a DS commit
 // after every step that a read-out follows, and before the next step the wait
 // for that read-out (DSF).
-template <int CL>
+template <int CL, bool TOT>
 __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, uint32_t tmem) {
     using P = Plan<CL>;
     constexpr int kSteps = P::kSteps;
     constexpr int kJ = C / 16 / kSteps;                  // K steps of 16 tokens per MMA4 step
-    constexpr int KS = stages(CL);
+    constexpr int KS = ring(CL, TOT);
     const uint32_t sb = sh.sbase;
     const uint64_t dpk0 = smem_desc(sb + OFF_PK, PK_LBO, PK_SBO);    // phi(K): N = feature, MN-major
     uint64_t* bars = sh.bars;
@@ -935,7 +953,7 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
         const int b = c & 1, s = c % KS;
         if (!wait(BAR_RF0 + s, (c / KS) & 1) || !wait(BAR_IN0 + b, (c >> 1) & 1)) break;
         // [V|1]^T as the A operand (M = column: V's atom, then the ones block; K = token)
-        const uint32_t va = sb + off_v(CL) + s * V_BYTES;
+        const uint32_t va = sb + stage_v(CL, TOT, s);
         const uint64_t dva = smem_desc_sw128(va, sb + off_ones(CL) - va, 1024);
         for (int h = 0; h < kSteps; ++h) {
             if (pending && !wait(BAR_DSF, (r - 1) & 1)) { ok = false; break; }
@@ -969,18 +987,20 @@ __device__ __forceinline__ void state_issuer(const Work& w, const Shared& sh, ui
     if (*sh.abort_flag) drain(last_bar, last_parity);
 }
 
-// mode 0: main pass over every segment; mode 1: totals pass over segments 0..nseg-2,
-// each split into `parts` pieces of at most sub_tiles = ceil(seg_tiles / parts) tiles.
+// TOT false: main pass over every segment; TOT true: totals pass over segments
+// 0..nseg-2, each split into `parts` pieces of at most sub_tiles = ceil(seg_tiles /
+// parts) tiles (only the state chain and its read-out are compiled in).
 // SEG: compiled for more than one segment per sequence (a segment may start from
 // a state); without it, every CTA starts from zero and none of that code exists.
-template <int CL, bool DECAY, bool SEG>
+template <int CL, bool DECAY, bool SEG, bool TOT>
 __global__ void __launch_bounds__(kThreads, 1)
 la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_constant__ CUtensorMap tq,
                      const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int parts, int mode,
+                     float* __restrict__ S, float* __restrict__ z, int N, int nseg, int seg_tiles, int parts,
                      int packed, float* __restrict__ ws, const float* __restrict__ gamma, unsigned* status,
                      unsigned debug) {
     static_assert(!DECAY || CL == 128, "coarse decay is per 128-token tile, with 128-token chunks");
+    static_assert(!TOT || SEG, "the totals pass exists only with segments");
     extern __shared__ __align__(1024) unsigned char smem[];
     constexpr uint32_t kOffBar = off_bar(CL);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kOffBar);
@@ -992,8 +1012,17 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
     const int warp = tid >> 5;
     const int lane = tid & 31;
 
+    if (warp == 14 && lane == 0) {                       // the loader's maps (and the y stores')
+        prefetch_tensormap(&tk);
+        prefetch_tensormap(&tv);
+        if (!TOT) {
+            prefetch_tensormap(&tq);
+            prefetch_tensormap(&ty);
+        }
+    }
+
     Work w;
-    w.totals = mode == 1;
+    w.totals = TOT;
     w.parts = parts;
     w.sub_tiles = (seg_tiles + parts - 1) / parts;
     const int per_head = w.totals ? (nseg - 1) * parts : nseg;
@@ -1030,7 +1059,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
                 i == BAR_YSR1)
                 count = 128;                                 // one warpgroup
             if (i == BAR_DSF || i == BAR_SBR || i == BAR_SBR1 || i == BAR_INIT) count = kStateLanes;
-            if (i >= BAR_RE0 && i <= BAR_RE2 && !w.totals) count = 2;   // both issuers read an input stage
+            if (i >= BAR_RE0 && i <= BAR_RE3 && !w.totals) count = 2;   // both issuers read an input stage
             mbar_init(&bars[i], count);
         }
         *abort_flag = 0;
@@ -1056,7 +1085,7 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
     const bool skip_mma = (debug & DEBUG_SKIP_MMA) != 0;   // testing: issue nothing, every waiter times out
 
     if (warp < 4) {
-        producers<CL>(w, sh, tmem, warp, tid);
+        producers<CL, TOT>(w, sh, tmem, warp, tid);
     } else if (warp < 8) {
         const int wq = warp & 3;
         if (w.totals) {
@@ -1074,11 +1103,11 @@ la_prefill_tc_kernel(const __grid_constant__ CUtensorMap ty, const __grid_consta
             if (wq == 0 && lane == 0) bulk_wait_all();      // the y stores have completed
         }
     } else if (warp == 12) {
-        if (lane == 0 && !skip_mma) state_issuer<CL>(w, sh, tmem);
+        if (lane == 0 && !skip_mma) state_issuer<CL, TOT>(w, sh, tmem);
     } else if (warp == 13) {
         if (lane == 0 && !w.totals && !skip_mma) y_issuer<CL>(w, sh, tmem);
     } else {
-        if (lane == 0) loader<CL>(w, sh, &tq, &tk, &tv);
+        if (lane == 0) loader<CL, TOT>(w, sh, &tq, &tk, &tv);
     }
 
     tc_fence_before();
@@ -1170,11 +1199,17 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
     const int BH = a.B * a.H;
     int nseg, seg_tiles;
     plan_segments(BH, a.N, num_sms, tiles_per_chunk(CL), &nseg, &seg_tiles);
-    auto kern = nseg > 1 ? la_prefill_tc_kernel<CL, false, true> : la_prefill_tc_kernel<CL, false, false>;
+    auto kern = nseg > 1 ? la_prefill_tc_kernel<CL, false, true, false> : la_prefill_tc_kernel<CL, false, false, false>;
+    auto ktot = la_prefill_tc_kernel<CL, false, true, true>;
     if constexpr (CL == 128)
-        if (a.gamma != nullptr) kern = nseg > 1 ? la_prefill_tc_kernel<128, true, true> : la_prefill_tc_kernel<128, true, false>;
+        if (a.gamma != nullptr) {
+            kern = nseg > 1 ? la_prefill_tc_kernel<128, true, true, false> : la_prefill_tc_kernel<128, true, false, false>;
+            ktot = la_prefill_tc_kernel<128, true, true, true>;
+        }
     constexpr uint32_t kSmem = smem_bytes(CL);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (e == cudaSuccess && nseg > 1)
+        e = cudaFuncSetAttribute(ktot, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
     if (e != cudaSuccess) return e;
     float* ws = static_cast<float*>(a.workspace);
     // Split the totals as finely as helps and as the given workspace holds (the
@@ -1190,8 +1225,8 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
         !make_tmap_bf16_3d_swizzle(&tv, a.v, DV, a.N, BH, DV, C, 128))
         return cudaErrorInvalidValue;
     if (nseg > 1) {
-        e = launch_pdl(kern, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
-                       a.z, a.N, nseg, seg_tiles, parts, 1, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+        e = launch_pdl(ktot, dim3(BH * (nseg - 1) * parts), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
+                       a.z, a.N, nseg, seg_tiles, parts, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
         if (e != cudaSuccess) return e;
         const dim3 pgrid((unsigned)((kTotalFloats / 4 + 255) / 256), (unsigned)BH);
         const int seq_tiles = (a.N + C - 1) / C;
@@ -1203,7 +1238,7 @@ cudaError_t launch_cl(const LaPrefillArgs& a, int num_sms, cudaStream_t stream) 
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(kern, dim3(BH * nseg), dim3(kThreads), kSmem, stream, ty, tq, tk, tv, a.S,
-                      a.z, a.N, nseg, seg_tiles, parts, 0, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
+                      a.z, a.N, nseg, seg_tiles, parts, a.packed ? 1 : 0, ws, a.gamma, a.status, a.debug);
 }
 
 }  // namespace

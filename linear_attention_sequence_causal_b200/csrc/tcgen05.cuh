@@ -310,6 +310,12 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const void* tmap, uint
         : "memory");
 }
 
+// Fetch a tensor map (a __grid_constant__ kernel parameter) into the TMA unit
+// ahead of its first copy, which would otherwise wait for it.
+__device__ __forceinline__ void prefetch_tensormap(const void* tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
 // Prefetch `bytes` (a multiple of 16) of global memory from `src` (16-byte
 // aligned) into L2, with no completion to wait for.
 __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
