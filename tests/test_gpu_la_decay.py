@@ -118,6 +118,24 @@ def test_prefill_decay_long_sampled_heads(d_feat, d_v):
         assert_state(to64(S[0, h]), rS, torch.bfloat16, f"S head {h}")
 
 
+def test_prefill_decay_segments_of_many_tiles():
+    """32 (b, h) pairs of 4096 tokens: each sequence is cut into four segments of
+    eight 128-token tiles, so the totals CTA of a segment rescales its state
+    tile by tile over eight tiles, more than its ring of input stages holds."""
+    B, H, N = 2, 16, 4096
+    inp = synthetic.la_inputs(B, H, N, 16, 64, "bf16", seed=21)
+    g, g64 = _gamma(B, H, N, seed=22, lo=0.9)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    y, S, z = based.la_prefill_decay(q, k, v, g.to(DEV))
+    assert based.get_last_error() == 0
+    for b, h in ((0, 0), (0, 15), (1, 6), (1, 15)):
+        ref = oracle.la_quadratic_decay(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], g64[b, h])
+        assert_y(to64(y[b, h]), ref, torch.bfloat16, f"y head ({b}, {h})")
+        rS, rz = oracle.la_state_decay(inp.k64[b, h], inp.v64[b, h], g64[b, h])
+        assert_state(to64(S[b, h]), rS, torch.bfloat16, f"S head ({b}, {h})")
+        assert_state(to64(z[b, h]), rz, torch.bfloat16, f"z head ({b}, {h})")
+
+
 @pytest.mark.parametrize("d_feat,d_v", [(16, 64), (32, 128)])
 def test_prefill_decay_fp32_cuda_cores(d_feat, d_v):
     """fp32 inputs: the CUDA-core kernel scales its state at every 128-token tile."""
