@@ -208,10 +208,12 @@ la_decode_kernel(float* __restrict__ S, float* __restrict__ z, const T* __restri
     cluster.sync();   // keep every rank's shared memory alive until rank 0 has read it
 }
 
-// Ranks per head: enough CTAs to cover every SM about twice, at least 16 rows
-// per CTA, a power of two up to the portable cluster size. (Measured at H=16,
-// d'=16, dv=64: covering the SMs four times split batch 8 and 16 into 8 and 4
-// ranks, 15 % slower than 2 and 1.)
+// Ranks per head: doubled while the grid is below twice the SM count, at least
+// 16 rows per CTA, a power of two up to the portable cluster size. At H=16,
+// d'=16, dv=64 that is 4 ranks at batch 8 and 2 at batch 16. A four-fold
+// cover (8 and 4 ranks) was ~15 % slower with L2 flushed between calls; in the
+// bench step's graph, stopping below twice the SMs (2 and 1 ranks) was 5-6 %
+// slower.
 int ranks_per_head(int BH, int D, int num_sms) {
     int P = 1;
     while (P < kMaxRanks && (long long)BH * P < 2LL * num_sms && D / (2 * P) >= 16) P *= 2;
