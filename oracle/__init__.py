@@ -54,6 +54,8 @@ from .taylor_la import (  # noqa: F401
     la_state_packed,
     la_recurrent_packed,
     la_backward,
+    feature_map_vjp,
+    la_backward_chunked,
     DECAY_CHUNK,
     decay_chunks,
     decay_per_step,

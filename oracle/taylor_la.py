@@ -313,6 +313,88 @@ def la_backward(q, k, v, dy):
     return dq, dk, dv
 
 
+def feature_map_vjp(x, u):
+    """u^T dphi/dx for phi(x) = [1, x, vec(x x^T)/sqrt2]: with u = [u_0, u_1, U_2]
+    (U_2 the d' x d' block, row-major), it is u_1 + (U_2 + U_2^T) x / sqrt2."""
+    x = np.asarray(x, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    d = x.shape[-1]
+    u2 = u[..., 1 + d:].reshape(u.shape[:-1] + (d, d))
+    sym = u2 + np.swapaxes(u2, -1, -2)
+    return u[..., 1:1 + d] + _SQRT_HALF * np.einsum("...ab,...b->...a", sym, x)
+
+
+def la_backward_chunked(q, k, v, dy, chunk: int):
+    """(dq, dk, dv) of the forward by chunks, with states instead of the full
+    causal square: the gradient of la_backward in the form a state-based
+    (reverse-scan) backward evaluates.
+
+    With a_ij = phi(q_i).phi(k_j), den_i = phi(q_i).z_i, g_i = dy_i / den_i,
+    c_i = g_i.y_i and da_ij = g_i.v_j - c_i (j <= i):
+      dphi(q_i) = sum_{j<=i} da_ij phi(k_j) = S_i g_i - c_i z_i,
+      dphi(k_j) = sum_{i>=j} da_ij phi(q_i) = R_j v_j - r_j,
+      dv_j      = sum_{i>=j} a_ij g_i       = R_j^T phi(k_j),
+    where S_i, z_i sum phi(k) v^T and phi(k) over keys up to i (the forward
+    state), and R_j = sum_{i>=j} phi(q_i) g_i^T, r_j = sum_{i>=j} c_i phi(q_i)
+    sum over queries from j on (a state carried backwards). Within a chunk the
+    pairs are taken directly; the earlier chunks enter through the forward
+    state at the chunk's start, the later ones through the backward state at
+    its end (BASED App. B: quadratic on-diagonal tiles plus cumulative state,
+    here for the derivative of that forward). dq, dk follow by the chain rule
+    through phi (feature_map_vjp).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    *lead, n, d_feat = q.shape
+    dv_dim = v.shape[-1]
+    D = feature_dim(d_feat)
+    fq, fk = feature_map(q), feature_map(k)
+    bounds = [(c0, min(n, c0 + chunk)) for c0 in range(0, n, chunk)]
+    masks = {c1 - c0: np.tril(np.ones((c1 - c0, c1 - c0), dtype=bool)) for c0, c1 in bounds}
+
+    # Forward pass over the chunks: y, den, and the state entering each chunk.
+    S = np.zeros(tuple(lead) + (D, dv_dim))
+    z = np.zeros(tuple(lead) + (D,))
+    S_in, z_in, a_in = [], [], []
+    g = np.empty(tuple(lead) + (n, dv_dim))
+    cc = np.empty(tuple(lead) + (n,))
+    for c0, c1 in bounds:
+        a = np.where(masks[c1 - c0], fq[..., c0:c1, :] @ np.swapaxes(fk[..., c0:c1, :], -1, -2), 0.0)
+        num = a @ v[..., c0:c1, :] + fq[..., c0:c1, :] @ S
+        den = a.sum(axis=-1) + np.einsum("...tf,...f->...t", fq[..., c0:c1, :], z)
+        _check_den(den, np.arange(c0 + 1, c1 + 1, dtype=np.float64))
+        y = num / den[..., None]
+        g[..., c0:c1, :] = dy[..., c0:c1, :] / den[..., None]
+        cc[..., c0:c1] = np.sum(g[..., c0:c1, :] * y, axis=-1)
+        S_in.append(S)
+        z_in.append(z)
+        a_in.append(a)
+        S = S + np.swapaxes(fk[..., c0:c1, :], -1, -2) @ v[..., c0:c1, :]
+        z = z + fk[..., c0:c1, :].sum(axis=-2)
+
+    # Backward pass over the chunks, last first, carrying R and r.
+    R = np.zeros(tuple(lead) + (D, dv_dim))
+    r = np.zeros(tuple(lead) + (D,))
+    dfq = np.empty_like(fq)
+    dfk = np.empty_like(fk)
+    dv = np.empty_like(v)
+    for idx in range(len(bounds) - 1, -1, -1):
+        c0, c1 = bounds[idx]
+        m = masks[c1 - c0]
+        gc, ccc, vc = g[..., c0:c1, :], cc[..., c0:c1], v[..., c0:c1, :]
+        fqc, fkc = fq[..., c0:c1, :], fk[..., c0:c1, :]
+        da = np.where(m, gc @ np.swapaxes(vc, -1, -2) - ccc[..., None], 0.0)
+        dfq[..., c0:c1, :] = (da @ fkc + np.swapaxes(S_in[idx] @ np.swapaxes(gc, -1, -2), -1, -2)
+                              - ccc[..., None] * z_in[idx][..., None, :])
+        dfk[..., c0:c1, :] = np.swapaxes(da, -1, -2) @ fqc + vc @ np.swapaxes(R, -1, -2) - r[..., None, :]
+        dv[..., c0:c1, :] = np.swapaxes(a_in[idx], -1, -2) @ gc + fkc @ R
+        R = R + np.swapaxes(fqc, -1, -2) @ gc
+        r = r + np.einsum("...t,...tf->...f", ccc, fqc)
+    return feature_map_vjp(q, dfq), feature_map_vjp(k, dfk), dv
+
+
 # ---------------------------------------------------------------------------
 # Coarse input-dependent decay.
 #

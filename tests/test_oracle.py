@@ -449,6 +449,41 @@ def test_backward_of_first_token_only_touches_itself():
     assert np.allclose(dvv[..., 0, :], dy[..., 0, :]) and np.allclose(dvv[..., 1:, :], 0)
 
 
+def test_feature_map_vjp_matches_finite_differences():
+    rng = np.random.default_rng(31)
+    for d in (1, 3, 16):
+        x = rng.standard_normal(d)
+        u = rng.standard_normal(oracle.feature_dim(d))
+        h = 1e-6
+        fd = np.array([(u @ oracle.feature_map(x + h * e) - u @ oracle.feature_map(x - h * e)) / (2 * h)
+                       for e in np.eye(d)])
+        assert np.allclose(oracle.feature_map_vjp(x, u), fd, rtol=1e-7, atol=1e-8)
+
+
+@pytest.mark.parametrize("chunk", [1, 4, 16, 23, 64])
+def test_backward_by_chunks_matches_autograd(chunk):
+    """The state form (forward state at a chunk's start, backward state at its
+    end) gives autograd's gradients at every chunk length, ragged last chunks
+    and a single chunk (64 > N) included."""
+    N, d, dv = 23, 5, 4
+    q, k, v = _qkv(2, 1, N, d, dv, seed=chunk)
+    dy = np.random.default_rng(chunk + 7).standard_normal((2, 1, N, dv))
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    _torch_forward(tq, tk, tv).backward(torch.tensor(dy))
+    dq, dk, dvv = oracle.la_backward_chunked(q, k, v, dy, chunk)
+    for got, want in ((dq, tq.grad), (dk, tk.grad), (dvv, tv.grad)):
+        assert np.allclose(got, want.numpy(), rtol=1e-10, atol=1e-12)
+
+
+def test_backward_by_chunks_matches_the_quadratic_form_at_d16():
+    q, k, v = _qkv(1, 2, 150, 16, 8, seed=5)
+    dy = np.random.default_rng(6).standard_normal((1, 2, 150, 8))
+    ref = oracle.la_backward(q, k, v, dy)
+    for chunk in (7, 64, 128):
+        for got, want in zip(oracle.la_backward_chunked(q, k, v, dy, chunk), ref):
+            assert np.max(np.abs(got - want)) <= 1e-12 * np.max(np.abs(want))
+
+
 # ---------------------------------------------------------------- coarse decay (reading: one gamma per 128-token chunk)
 
 def _decay_case(B, H, N, d, dv, seed):
