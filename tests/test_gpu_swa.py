@@ -54,15 +54,19 @@ def test_large_scores_stay_finite():
 
 
 def test_360m_prefill_sampled():
-    """16 heads x d=64, B=8, N=2048, w=64, bf16."""
+    """16 heads x d=64, B=8, N=2048, w=64, bf16: every head at 18+ rows (the
+    window's first fill, 128-query tile edges, the end, and random rows of the
+    head's own), the ring of every head bit for bit."""
     inp = synthetic.swa_inputs(8, 16, 2048, 64, "bf16", seed=0)
     y, kc, vc = _prefill(inp, 64)
     y64 = to64(y)
-    rng = np.random.default_rng(0)
-    rows = sorted(set([0, 1, 62, 63, 64, 65, 127, 128, 1000, 2046, 2047] + rng.integers(0, 2048, 64).tolist()))
-    for b, h in [(0, 0), (7, 15), (2, 9), (5, 3)]:
-        ref = oracle.swa_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], 64, SCALE, rows)
-        assert_y(y64[b, h, rows], ref, torch.bfloat16, f"y[{b},{h}]")
+    edges = [0, 1, 62, 63, 64, 65, 127, 128, 129, 1023, 1024, 2046, 2047]
+    for b in range(8):
+        for h in range(16):
+            rng = np.random.default_rng(1000 * b + h)
+            rows = sorted(set(edges + rng.integers(0, 2048, 6).tolist()))
+            ref = oracle.swa_rows(inp.q64[b, h], inp.k64[b, h], inp.v64[b, h], 64, SCALE, rows)
+            assert_y(y64[b, h, rows], ref, torch.bfloat16, f"y[{b},{h}]")
     rk, rv = oracle.swa_ring_after_prefill(inp.k64, inp.v64, 64)
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
