@@ -98,6 +98,25 @@ def test_decode_continues_the_prompt(dtype, K, prompt):
     assert np.array_equal(to64(st), oracle.baseconv_state(inp.conv64, K))
 
 
+def test_decode_resume_from_copied_state_is_bit_identical():
+    """The shift-register state is the decode checkpoint: copied to the host and
+    back, it resumes bit for bit like the state that never left."""
+    K, prompt, steps = 4, 40, 12
+    inp = synthetic.conv_inputs(3, prompt + steps, 128, K, "bf16", seed=17)
+    g, x, h, b = _dev(inp)
+    _, st = based.baseconv_prefill(g[:, :prompt].contiguous(), x[:, :prompt].contiguous(), h, b)
+    saved = st.cpu().clone()
+    runs = []
+    for s in (st, saved.to(DEV), saved.to(DEV)):
+        torch.cuda.synchronize()
+        ys = torch.stack([based.baseconv_decode(s, g[:, t].contiguous(), x[:, t].contiguous(), h, b)
+                          for t in range(prompt, prompt + steps)])
+        runs.append((ys, s))
+    assert based.get_last_error() == 0
+    for ys, s in runs[1:]:
+        assert torch.equal(ys, runs[0][0]) and torch.equal(s, runs[0][1])
+
+
 def test_decode_single_tap_needs_no_state():
     inp = synthetic.conv_inputs(5, 1, 64, 1, "bf16", seed=11)
     g, x, h, b = _dev(inp)

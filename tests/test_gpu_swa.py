@@ -71,6 +71,27 @@ def test_360m_prefill_sampled():
     assert np.array_equal(to64(kc), rk) and np.array_equal(to64(vc), rv)
 
 
+def test_decode_resume_from_copied_ring_is_bit_identical():
+    """The ring cache and the position t are the decode checkpoint: a ring copied
+    to the host and back resumes bit for bit like the ring that never left."""
+    B, H, prompt, steps, w = 2, 4, 70, 30, 64
+    inp = synthetic.swa_inputs(B, H, prompt + steps, 64, "bf16", seed=13)
+    q, k, v = (t.to(DEV) for t in (inp.q, inp.k, inp.v))
+    _, kc, vc = based.swa_prefill(q[:, :, :prompt].contiguous(), k[:, :, :prompt].contiguous(),
+                                  v[:, :, :prompt].contiguous(), w=w, scale=SCALE)
+    saved = (kc.cpu().clone(), vc.cpu().clone())
+    qd, kd, vd = (x[:, :, prompt:].permute(2, 0, 1, 3).contiguous() for x in (q, k, v))
+    runs = []
+    for kr, vr in ((kc, vc), tuple(x.to(DEV) for x in saved), tuple(x.to(DEV) for x in saved)):
+        torch.cuda.synchronize()     # a ring written by a copy is settled before its first decode
+        ys = torch.stack([based.swa_decode(kr, vr, prompt + t, qd[t], kd[t], vd[t], w=w, scale=SCALE)
+                          for t in range(steps)])
+        runs.append((ys, kr, vr))
+    assert based.get_last_error() == 0
+    for ys, kr, vr in runs[1:]:
+        assert torch.equal(ys, runs[0][0]) and torch.equal(kr, runs[0][1]) and torch.equal(vr, runs[0][2])
+
+
 @pytest.mark.parametrize("dtype,batch,prompt,steps,w", [
     ("f32", 2, 0, 70, 16), ("f32", 2, 10, 70, 64), ("bf16", 3, 100, 80, 64),
     ("bf16", 64, 512, 1024, 64),
